@@ -1,0 +1,239 @@
+"""CPU oracle for the DDTree verification round (fp64, plain C + ctypes).
+
+TEST INFRASTRUCTURE ONLY.  The test-suite, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` are the only
+callers.  The product library (``block_draft_tree_b200``) never imports this
+package, and this package never imports the product: the two share no code.
+
+Each function restates one step of the DDTree page (Diffusion Draft Tree,
+curated summary of the authors' announcement), section "運作流程"
+(workflow):
+
+* :func:`topk`       -- step 1, per-position marginals q_i: log-sum-exp and
+  the top-k candidate tokens of each position;
+* :func:`build_tree` -- step 2 (best B prefixes of the factorised draft,
+  "核心創新" / "理論基礎" Propositions 1-2) and step 3's compilation into
+  token / parent / depth / position / ancestor-mask tensors;
+* :func:`tree_attn`  -- step 3, ancestor-only masked attention of each
+  tree row against the context KV cache and the tree's own KV;
+* :func:`tree_walk`  -- step 4, the greedy walk that accepts matching
+  children and returns the bonus token.
+
+Parity pins for every function live in ``tests/test_oracle_*.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ddt_oracle.c")
+_LIB = os.path.join(_HERE, "libddt_oracle.so")
+_lib = None
+
+i32p = np.ctypeslib.ndpointer(dtype=np.int32, flags="C_CONTIGUOUS")
+u32p = np.ctypeslib.ndpointer(dtype=np.uint32, flags="C_CONTIGUOUS")
+f64p = np.ctypeslib.ndpointer(dtype=np.float64, flags="C_CONTIGUOUS")
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (no FMA contraction, plain -O2)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
+               "-o", _LIB, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        lib.ddto_topk.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                  ctypes.c_int64, ctypes.c_int, ctypes.c_double,
+                                  i32p, f64p, f64p, f64p]
+        lib.ddto_build_tree.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                        ctypes.c_double, i32p, f64p, f64p, ctypes.c_int32,
+                                        ctypes.c_int32, ctypes.c_int, ctypes.c_int,
+                                        i32p, i32p, i32p, i32p, u32p,
+                                        ctypes.POINTER(ctypes.c_int32),
+                                        ctypes.POINTER(ctypes.c_double),
+                                        ctypes.POINTER(ctypes.c_double)]
+        lib.ddto_tree_attn.argtypes = [ctypes.c_int, i32p, ctypes.c_void_p, ctypes.c_int,
+                                       ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                       ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                       ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
+                                       i32p, ctypes.c_void_p, ctypes.c_void_p, u32p,
+                                       ctypes.c_int, i32p, ctypes.c_double, f64p, f64p]
+        lib.ddto_tree_walk.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64,
+                                       ctypes.c_int, i32p, i32p, i32p, ctypes.c_int,
+                                       ctypes.c_int, ctypes.POINTER(ctypes.c_int32),
+                                       i32p, i32p, ctypes.POINTER(ctypes.c_int32)]
+        for f in (lib.ddto_topk, lib.ddto_build_tree, lib.ddto_tree_attn, lib.ddto_tree_walk):
+            f.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _raw(x: np.ndarray):
+    """(pointer, is_bf16) for a bf16 (stored as uint16 bits) or float32 array."""
+    if x.dtype == np.uint16:
+        return x.ctypes.data_as(ctypes.c_void_p), 1
+    if x.dtype == np.float32:
+        return x.ctypes.data_as(ctypes.c_void_p), 0
+    raise TypeError("logits must be bf16 bits (uint16) or float32, got %s" % x.dtype)
+
+
+def topk(z: np.ndarray, k: int, inv_temperature: float = 1.0):
+    """Step 1 for every row of ``z`` (shape [..., V], bf16 bits or f32).
+
+    Returns ``ids`` int32 [..., k], ``zk`` f64 [..., k] (the raw logits of the
+    candidates), ``logp`` f64 [..., k] = invT*z - lse and ``lse`` f64 [...].
+    The order is logit descending, token id ascending.
+    """
+    z = np.ascontiguousarray(z)
+    lead = z.shape[:-1]
+    V = z.shape[-1]
+    rows = int(np.prod(lead)) if lead else 1
+    ids = np.empty(rows * k, np.int32)
+    zk = np.empty(rows * k, np.float64)
+    logp = np.empty(rows * k, np.float64)
+    lse = np.empty(rows, np.float64)
+    p, is_bf16 = _raw(z)
+    rc = _load().ddto_topk(p, is_bf16, rows, V, V, k, float(np.float32(inv_temperature)),
+                           ids, zk, logp, lse)
+    if rc != 0:
+        raise ValueError("ddto_topk failed (%d)" % rc)
+    return (ids.reshape(*lead, k), zk.reshape(*lead, k), logp.reshape(*lead, k),
+            lse.reshape(lead))
+
+
+def mask_words(n_max: int) -> int:
+    return (n_max + 31) // 32
+
+
+def build_tree(ids, zk, lse, budget, inv_temperature=1.0, root_token=None, ctx_len=None,
+               k_per_seq=None, n_max=None):
+    """Steps 2-3 for a batch.
+
+    ``ids``/``zk``: [batch, L, k] top-k ids and raw logits; ``lse``: [batch, L];
+    ``budget``: int or [batch] draft-node budgets; ``k_per_seq``: optional
+    [batch] number of candidates used per position (<= k).
+    Returns a dict of numpy arrays: tok, parent, depth, pos [batch, Nmax],
+    mask [batch, Nmax, W] uint32, n_nodes [batch], surrogate [batch],
+    delta_min [batch].
+    """
+    ids = np.ascontiguousarray(ids, np.int32)
+    zk = np.ascontiguousarray(zk, np.float64)
+    lse = np.ascontiguousarray(lse, np.float64)
+    bsz, L, kmax = ids.shape
+    budget = np.broadcast_to(np.asarray(budget, np.int64), (bsz,))
+    if k_per_seq is None:
+        k_per_seq = np.full(bsz, kmax, np.int64)
+    k_per_seq = np.broadcast_to(np.asarray(k_per_seq, np.int64), (bsz,))
+    root_token = np.zeros(bsz, np.int64) if root_token is None else np.broadcast_to(
+        np.asarray(root_token, np.int64), (bsz,))
+    ctx_len = np.zeros(bsz, np.int64) if ctx_len is None else np.broadcast_to(
+        np.asarray(ctx_len, np.int64), (bsz,))
+    if n_max is None:
+        n_max = int(budget.max()) + 1
+    W = mask_words(n_max)
+    out = {k_: np.empty((bsz, n_max), np.int32) for k_ in ("tok", "parent", "depth", "pos")}
+    out["mask"] = np.empty((bsz, n_max, W), np.uint32)
+    out["n_nodes"] = np.empty(bsz, np.int32)
+    out["surrogate"] = np.empty(bsz, np.float64)
+    out["delta_min"] = np.empty(bsz, np.float64)
+    lib = _load()
+    for b in range(bsz):
+        t, p, dp, ps = (np.empty(n_max, np.int32) for _ in range(4))
+        m = np.empty(n_max * W, np.uint32)
+        nn = ctypes.c_int32()
+        sg = ctypes.c_double()
+        dm = ctypes.c_double()
+        rc = lib.ddto_build_tree(L, int(k_per_seq[b]), kmax, int(budget[b]),
+                                 float(np.float32(inv_temperature)),
+                                 np.ascontiguousarray(ids[b]), np.ascontiguousarray(zk[b]),
+                                 np.ascontiguousarray(lse[b]), int(root_token[b]),
+                                 int(ctx_len[b]), n_max, W, t, p, dp, ps, m,
+                                 ctypes.byref(nn), ctypes.byref(sg), ctypes.byref(dm))
+        if rc != 0:
+            raise ValueError("ddto_build_tree failed (%d) for sequence %d" % (rc, b))
+        out["tok"][b], out["parent"][b], out["depth"][b], out["pos"][b] = t, p, dp, ps
+        out["mask"][b] = m.reshape(n_max, W)
+        out["n_nodes"][b] = nn.value
+        out["surrogate"][b] = sg.value
+        out["delta_min"][b] = dm.value
+    return out
+
+
+def tree_attn(items, q, k_cache, v_cache, ctx_len, k_tree, v_tree, mask, n_nodes, scale,
+              page_table=None, page_size=64):
+    """Step 3's attention for the listed (b, j, h) items.
+
+    ``q`` [batch, Nmax, Hq, d], ``k_tree``/``v_tree`` [batch, Nmax, Hkv, d] and the
+    cache are bf16 bits (uint16).  Dense cache: [batch, Tmax, Hkv, d]; paged
+    cache: [pages, page_size, Hkv, d] with ``page_table`` [batch, max_pages].
+    Returns (out f64 [n, d], lse f64 [n]).
+    """
+    items = np.ascontiguousarray(np.asarray(items, np.int32).reshape(-1, 3))
+    for a in (q, k_cache, v_cache, k_tree, v_tree):
+        if a.dtype != np.uint16 or not a.flags.c_contiguous:
+            raise TypeError("attention operands must be C-contiguous bf16 bits (uint16)")
+    bsz, n_max, hq, d = q.shape
+    hkv = k_tree.shape[2]
+    if page_table is None:
+        tmax = k_cache.shape[1]
+        pt = None
+        maxp = 0
+    else:
+        tmax = 0
+        pt = np.ascontiguousarray(page_table, np.int32)
+        maxp = pt.shape[1]
+    n = items.shape[0]
+    out = np.empty((n, d), np.float64)
+    lse = np.empty(n, np.float64)
+    W = mask.shape[-1]
+    rc = _load().ddto_tree_attn(
+        n, items, q.ctypes.data_as(ctypes.c_void_p), n_max, hq, hkv, d,
+        k_cache.ctypes.data_as(ctypes.c_void_p), v_cache.ctypes.data_as(ctypes.c_void_p),
+        tmax, None if pt is None else pt.ctypes.data_as(ctypes.c_void_p), page_size, maxp,
+        np.ascontiguousarray(ctx_len, np.int32), k_tree.ctypes.data_as(ctypes.c_void_p),
+        v_tree.ctypes.data_as(ctypes.c_void_p), np.ascontiguousarray(mask, np.uint32), W,
+        np.ascontiguousarray(n_nodes, np.int32), float(scale), out, lse)
+    if rc != 0:
+        raise ValueError("ddto_tree_attn failed (%d)" % rc)
+    return out, lse
+
+
+def tree_walk(logits, tok, parent, depth, n_nodes, L):
+    """Step 4 for a batch.  ``logits`` [batch, Nmax, V] f32 or bf16 bits.
+
+    Returns a dict: acc_len [batch], acc_nodes/acc_tok [batch, L], bonus [batch].
+    """
+    logits = np.ascontiguousarray(logits)
+    bsz, n_max, V = logits.shape
+    res = {"acc_len": np.empty(bsz, np.int32), "acc_nodes": np.empty((bsz, L), np.int32),
+           "acc_tok": np.empty((bsz, L), np.int32), "bonus": np.empty(bsz, np.int32)}
+    lib = _load()
+    for b in range(bsz):
+        row = np.ascontiguousarray(logits[b])
+        p, is_bf16 = _raw(row)
+        al = ctypes.c_int32()
+        bo = ctypes.c_int32()
+        an = np.empty(max(L, 1), np.int32)
+        at = np.empty(max(L, 1), np.int32)
+        rc = lib.ddto_tree_walk(p, is_bf16, V, V, np.ascontiguousarray(tok[b], np.int32),
+                                np.ascontiguousarray(parent[b], np.int32),
+                                np.ascontiguousarray(depth[b], np.int32), int(n_nodes[b]), L,
+                                ctypes.byref(al), an, at, ctypes.byref(bo))
+        if rc != 0:
+            raise ValueError("ddto_tree_walk failed (%d)" % rc)
+        res["acc_len"][b] = al.value
+        res["acc_nodes"][b] = an[:L]
+        res["acc_tok"][b] = at[:L]
+        res["bonus"][b] = bo.value
+    return res
