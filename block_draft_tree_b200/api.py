@@ -1,0 +1,317 @@
+"""ctypes binding of libddt.so (argument marshalling only).
+
+Every function here checks shapes and dtypes, allocates the output tensors
+with torch on the input's device, and calls the matching C entry point of
+``include/ddt.h`` on the current torch stream.  All arithmetic happens in the
+library's CUDA kernels; if ``libddt.so`` is missing or fails to load, every
+call raises :class:`DDTError` -- there is no other implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libddt.so")
+_lib = None
+_lock = threading.Lock()
+
+DDT_BF16, DDT_F32 = 0, 1
+DDT_TOPK_K_MAX = 32
+DDT_TREE_L_MAX = 64
+DDT_TREE_B_MAX = 1023
+
+EXPORTED = ("ddt_status_string", "ddt_mask_words", "ddt_topk_workspace_size", "ddt_topk",
+            "ddt_build_tree", "ddt_tree_attn_workspace_size", "ddt_tree_attn",
+            "ddt_tree_walk_workspace_size", "ddt_tree_walk")
+
+
+class DDTError(RuntimeError):
+    """A libddt call returned an error status (or the library is unavailable)."""
+
+
+class AttnArgs(ctypes.Structure):
+    """Mirror of ``ddt_attn_args`` (field order and types as in ddt.h)."""
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p),
+        ("page_table", ctypes.c_void_p), ("page_size", ctypes.c_int), ("max_pages", ctypes.c_int),
+        ("t_max", ctypes.c_int64), ("ctx_len", ctypes.c_void_p), ("max_ctx", ctypes.c_int),
+        ("k_tree", ctypes.c_void_p), ("v_tree", ctypes.c_void_p), ("mask", ctypes.c_void_p),
+        ("n_nodes", ctypes.c_void_p), ("batch", ctypes.c_int), ("n_max", ctypes.c_int),
+        ("hq", ctypes.c_int), ("hkv", ctypes.c_int), ("d", ctypes.c_int),
+        ("scale", ctypes.c_float), ("out", ctypes.c_void_p), ("lse_out", ctypes.c_void_p),
+        ("dev_status", ctypes.c_void_p),
+    ]
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load libddt.so (once).  Raises DDTError if it is missing or broken."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(_LIB_PATH):
+            raise DDTError("libddt.so is not built (python -m block_draft_tree_b200.build)")
+        try:
+            lib = ctypes.CDLL(_LIB_PATH)
+        except OSError as e:  # pragma: no cover - depends on the machine
+            raise DDTError("cannot load %s: %s" % (_LIB_PATH, e)) from e
+        vp, i32, i64, f32, sz = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float,
+                                 ctypes.c_size_t)
+        lib.ddt_status_string.restype = ctypes.c_char_p
+        lib.ddt_status_string.argtypes = [i32]
+        lib.ddt_mask_words.restype = i32
+        lib.ddt_mask_words.argtypes = [i32]
+        lib.ddt_topk_workspace_size.restype = sz
+        lib.ddt_topk_workspace_size.argtypes = [i32, i32, i32, i32]
+        lib.ddt_topk.restype = i32
+        lib.ddt_topk.argtypes = [vp, i32, i32, i32, i32, i64, i32, f32, vp, vp, vp, vp, vp, sz, vp]
+        lib.ddt_build_tree.restype = i32
+        lib.ddt_build_tree.argtypes = [vp, vp, vp, i32, i32, i32, f32, vp, vp, i32, vp, vp,
+                                       vp, vp, vp, vp, vp, vp, vp, vp, vp]
+        lib.ddt_tree_attn_workspace_size.restype = sz
+        lib.ddt_tree_attn_workspace_size.argtypes = [ctypes.POINTER(AttnArgs)]
+        lib.ddt_tree_attn.restype = i32
+        lib.ddt_tree_attn.argtypes = [ctypes.POINTER(AttnArgs), vp, sz, vp]
+        lib.ddt_tree_walk_workspace_size.restype = sz
+        lib.ddt_tree_walk_workspace_size.argtypes = [i32, i32, i32]
+        lib.ddt_tree_walk.restype = i32
+        lib.ddt_tree_walk.argtypes = [vp, i32, i32, i32, i32, i64, vp, vp, vp, vp, i32,
+                                      vp, vp, vp, vp, vp, sz, vp, vp]
+        _lib = lib
+        return lib
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        msg = load_library().ddt_status_string(rc).decode()
+        raise DDTError("%s failed: %s" % (what, msg))
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(dev: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _need_cuda(*ts):
+    dev = None
+    for t in ts:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise DDTError("libddt works on CUDA tensors only (got a %s tensor)" % t.device)
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise DDTError("all tensors must be on one device")
+    return dev
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return DDT_BF16
+    if t.dtype == torch.float32:
+        return DDT_F32
+    raise DDTError("logits must be bfloat16 or float32, got %s" % t.dtype)
+
+
+class _Workspaces:
+    """Zero-filled scratch per (device, stream, stage); grown on demand.
+
+    The kernels return every counter they use to zero, so a workspace stays
+    valid across calls that do not overlap on the GPU (same stream)."""
+
+    def __init__(self):
+        self._bufs = {}
+
+    def get(self, dev: torch.device, tag: str, nbytes: int) -> Optional[torch.Tensor]:
+        if nbytes == 0:
+            return None
+        key = (dev, torch.cuda.current_stream(dev).cuda_stream, tag)
+        buf = self._bufs.get(key)
+        if buf is None or buf.numel() < nbytes:
+            buf = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=dev)
+            self._bufs[key] = buf
+        return buf
+
+
+workspaces = _Workspaces()
+
+
+def topk_workspace_size(batch: int, L: int, V: int, k: int) -> int:
+    return int(load_library().ddt_topk_workspace_size(batch, L, V, k))
+
+
+def topk(logits: torch.Tensor, k: int, inv_temperature: float = 1.0, want_logp: bool = True):
+    """Stage 1.  ``logits`` [batch, L, V] bf16/f32 with unit stride on V and a
+    uniform row stride.  Returns (ids int32, zk f32, logp f32 or None) [batch, L, k]
+    and lse f32 [batch, L]."""
+    lib = load_library()
+    dev = _need_cuda(logits)
+    if logits.dim() != 3 or logits.stride(2) != 1 or logits.stride(0) != logits.stride(1) * logits.shape[1]:
+        raise DDTError("logits must be [batch, L, V] with contiguous rows and a uniform row stride")
+    b, L, V = logits.shape
+    ids = torch.empty((b, L, k), dtype=torch.int32, device=dev)
+    zk = torch.empty((b, L, k), dtype=torch.float32, device=dev)
+    logp = torch.empty((b, L, k), dtype=torch.float32, device=dev) if want_logp else None
+    lse = torch.empty((b, L), dtype=torch.float32, device=dev)
+    nb = int(lib.ddt_topk_workspace_size(b, L, V, k))
+    ws = workspaces.get(dev, "topk", nb)
+    with torch.cuda.device(dev):
+        rc = lib.ddt_topk(_ptr(logits), _dtype_code(logits), b, L, V, logits.stride(1), k,
+                          float(inv_temperature), _ptr(ids), _ptr(zk), _ptr(logp), _ptr(lse),
+                          _ptr(ws), nb, _stream(dev))
+    _check(rc, "ddt_topk")
+    return ids, zk, logp, lse
+
+
+def mask_words(n_max: int) -> int:
+    return (n_max + 31) // 32
+
+
+def build_tree(ids: torch.Tensor, zk: torch.Tensor, lse: torch.Tensor, B_max: int,
+               root_token: torch.Tensor, inv_temperature: float = 1.0,
+               k_per_seq: Optional[torch.Tensor] = None, budget: Optional[torch.Tensor] = None,
+               ctx_len: Optional[torch.Tensor] = None, dev_status: Optional[torch.Tensor] = None):
+    """Stages 2-3 (selection and compilation).  Returns a dict of tensors:
+    tok, parent, depth, pos [batch, B_max+1] int32, mask [batch, B_max+1, W]
+    int32 (bit pattern of the uint32 words), n_nodes [batch] int32,
+    surrogate [batch] float64."""
+    lib = load_library()
+    dev = _need_cuda(ids, zk, lse, root_token, k_per_seq, budget, ctx_len, dev_status)
+    for t, dt in ((ids, torch.int32), (zk, torch.float32), (lse, torch.float32),
+                  (root_token, torch.int32), (k_per_seq, torch.int32), (budget, torch.int32),
+                  (ctx_len, torch.int32), (dev_status, torch.int32)):
+        if t is not None and (t.dtype != dt or not t.is_contiguous()):
+            raise DDTError("build_tree: expected contiguous %s tensors" % dt)
+    b, L, k = ids.shape
+    n_max = B_max + 1
+    W = mask_words(n_max)
+    out = {n: torch.empty((b, n_max), dtype=torch.int32, device=dev)
+           for n in ("tok", "parent", "depth", "pos")}
+    out["mask"] = torch.empty((b, n_max, W), dtype=torch.int32, device=dev)
+    out["n_nodes"] = torch.empty(b, dtype=torch.int32, device=dev)
+    out["surrogate"] = torch.empty(b, dtype=torch.float64, device=dev)
+    with torch.cuda.device(dev):
+        rc = lib.ddt_build_tree(_ptr(ids), _ptr(zk), _ptr(lse), b, L, k, float(inv_temperature),
+                                _ptr(k_per_seq), _ptr(budget), B_max, _ptr(root_token),
+                                _ptr(ctx_len), _ptr(out["tok"]), _ptr(out["parent"]),
+                                _ptr(out["depth"]), _ptr(out["pos"]), _ptr(out["mask"]),
+                                _ptr(out["n_nodes"]), _ptr(out["surrogate"]), _ptr(dev_status),
+                                _stream(dev))
+    _check(rc, "ddt_build_tree")
+    return out
+
+
+def _attn_args(q, k_cache, v_cache, k_tree, v_tree, mask, n_nodes, ctx_len, max_ctx, scale,
+               page_table, out, lse_out, dev_status) -> AttnArgs:
+    b, n_max, hq, d = q.shape
+    hkv = k_tree.shape[2]
+    a = AttnArgs()
+    a.q = q.data_ptr()
+    a.k_cache = k_cache.data_ptr() if k_cache is not None and k_cache.numel() else None
+    a.v_cache = v_cache.data_ptr() if v_cache is not None and v_cache.numel() else None
+    if page_table is not None:
+        a.page_table = page_table.data_ptr()
+        a.page_size = k_cache.shape[1]
+        a.max_pages = page_table.shape[1]
+        a.t_max = 0
+    else:
+        a.page_table = None
+        a.page_size = 0
+        a.max_pages = 0
+        a.t_max = k_cache.shape[1] if k_cache is not None else 0
+    a.ctx_len = ctx_len.data_ptr()
+    a.max_ctx = int(max_ctx)
+    a.k_tree = k_tree.data_ptr()
+    a.v_tree = v_tree.data_ptr()
+    a.mask = mask.data_ptr()
+    a.n_nodes = n_nodes.data_ptr()
+    a.batch, a.n_max, a.hq, a.hkv, a.d = b, n_max, hq, hkv, d
+    a.scale = float(scale)
+    a.out = out.data_ptr() if out is not None else None
+    a.lse_out = lse_out.data_ptr() if lse_out is not None else None
+    a.dev_status = dev_status.data_ptr() if dev_status is not None else None
+    return a
+
+
+def tree_attn_workspace_size(q, k_cache, v_cache, k_tree, v_tree, mask, n_nodes, ctx_len,
+                             max_ctx, scale=None, page_table=None) -> int:
+    d = q.shape[-1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    a = _attn_args(q, k_cache, v_cache, k_tree, v_tree, mask, n_nodes, ctx_len, max_ctx, scale,
+                   page_table, None, None, None)
+    return int(load_library().ddt_tree_attn_workspace_size(ctypes.byref(a)))
+
+
+def tree_attn(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+              k_tree: torch.Tensor, v_tree: torch.Tensor, mask: torch.Tensor,
+              n_nodes: torch.Tensor, ctx_len: torch.Tensor, max_ctx: int,
+              scale: Optional[float] = None, page_table: Optional[torch.Tensor] = None,
+              want_lse: bool = False, dev_status: Optional[torch.Tensor] = None):
+    """Stage 3.  q [batch, n_max, hq, d] bf16; dense cache [batch, T_max, hkv, d]
+    or paged cache [pages, page_size, hkv, d] + page_table [batch, max_pages];
+    tree K/V [batch, n_max, hkv, d]; mask [batch, n_max, W].  Returns out bf16
+    [batch, n_max, hq, d] (and lse f32 [batch, n_max, hq] when asked)."""
+    lib = load_library()
+    dev = _need_cuda(q, k_cache, v_cache, k_tree, v_tree, mask, n_nodes, ctx_len, page_table,
+                     dev_status)
+    for t in (q, k_cache, v_cache, k_tree, v_tree):
+        if t is not None and (t.dtype != torch.bfloat16 or not t.is_contiguous()):
+            raise DDTError("tree_attn: q / caches / tree K,V must be contiguous bfloat16")
+    for t in (mask, n_nodes, ctx_len, page_table):
+        if t is not None and (t.dtype != torch.int32 or not t.is_contiguous()):
+            raise DDTError("tree_attn: mask / n_nodes / ctx_len / page_table must be contiguous int32")
+    b, n_max, hq, d = q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    out = torch.empty_like(q)
+    lse = torch.empty((b, n_max, hq), dtype=torch.float32, device=dev) if want_lse else None
+    a = _attn_args(q, k_cache, v_cache, k_tree, v_tree, mask, n_nodes, ctx_len, max_ctx, scale,
+                   page_table, out, lse, dev_status)
+    nb = int(lib.ddt_tree_attn_workspace_size(ctypes.byref(a)))
+    ws = workspaces.get(dev, "attn", nb)
+    with torch.cuda.device(dev):
+        rc = lib.ddt_tree_attn(ctypes.byref(a), _ptr(ws), nb, _stream(dev))
+    _check(rc, "ddt_tree_attn")
+    return (out, lse) if want_lse else out
+
+
+def tree_walk_workspace_size(batch: int, n_max: int, V: int) -> int:
+    return int(load_library().ddt_tree_walk_workspace_size(batch, n_max, V))
+
+
+def tree_walk(logits: torch.Tensor, tok: torch.Tensor, parent: torch.Tensor,
+              depth: torch.Tensor, n_nodes: torch.Tensor, L: int,
+              dev_status: Optional[torch.Tensor] = None):
+    """Stage 4.  ``logits`` [batch, n_max, V] f32/bf16 (rows contiguous, uniform
+    stride).  Returns dict acc_len [batch], acc_nodes/acc_tok [batch, L], bonus [batch]."""
+    lib = load_library()
+    dev = _need_cuda(logits, tok, parent, depth, n_nodes, dev_status)
+    if logits.dim() != 3 or logits.stride(2) != 1 or logits.stride(0) != logits.stride(1) * logits.shape[1]:
+        raise DDTError("logits must be [batch, n_max, V] with contiguous rows and a uniform row stride")
+    b, n_max, V = logits.shape
+    res = {"acc_len": torch.empty(b, dtype=torch.int32, device=dev),
+           "acc_nodes": torch.empty((b, L), dtype=torch.int32, device=dev),
+           "acc_tok": torch.empty((b, L), dtype=torch.int32, device=dev),
+           "bonus": torch.empty(b, dtype=torch.int32, device=dev)}
+    nb = int(lib.ddt_tree_walk_workspace_size(b, n_max, V))
+    ws = workspaces.get(dev, "walk", nb)
+    with torch.cuda.device(dev):
+        rc = lib.ddt_tree_walk(_ptr(logits), _dtype_code(logits), b, n_max, V, logits.stride(1),
+                               _ptr(tok), _ptr(parent), _ptr(depth), _ptr(n_nodes), L,
+                               _ptr(res["acc_len"]), _ptr(res["acc_nodes"]), _ptr(res["acc_tok"]),
+                               _ptr(res["bonus"]), _ptr(ws), nb, _ptr(dev_status), _stream(dev))
+    _check(rc, "ddt_tree_walk")
+    return res

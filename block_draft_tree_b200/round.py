@@ -1,0 +1,113 @@
+"""One verification round = the four C-ABI calls on preallocated buffers.
+
+:class:`VerifyRound` owns every output and workspace for one shape, so the
+round allocates nothing per call and can be captured once into a CUDA graph
+and replayed.  Inputs are bound by pointer (:meth:`bind`); the four calls
+read them in place.  Marshalling only -- all arithmetic is in libddt.so.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+from typing import Optional
+
+import torch
+
+from . import api
+
+
+class VerifyRound:
+    def __init__(self, *, batch: int, L: int, V: int, k: int, B_max: int, hq: int, hkv: int,
+                 d: int, max_ctx: int, draft_dtype: torch.dtype = torch.bfloat16,
+                 target_dtype: torch.dtype = torch.float32, inv_temperature: float = 1.0,
+                 paged: bool = False, page_size: int = 64, max_pages: int = 0,
+                 device: str = "cuda"):
+        self.lib = api.load_library()
+        self.dev = torch.device(device)
+        self.batch, self.L, self.V, self.k, self.B_max = batch, L, V, k, B_max
+        self.n_max = B_max + 1
+        self.hq, self.hkv, self.d, self.max_ctx = hq, hkv, d, max_ctx
+        self.inv_t = float(inv_temperature)
+        self.paged, self.page_size, self.max_pages = paged, page_size, max_pages
+        self.draft_code = api._dtype_code(torch.empty(0, dtype=draft_dtype))
+        self.target_code = api._dtype_code(torch.empty(0, dtype=target_dtype))
+        dev = self.dev
+        e = lambda *s, dt=torch.int32: torch.empty(s, dtype=dt, device=dev)
+        W = api.mask_words(self.n_max)
+        self.out = {
+            "ids": e(batch, L, k), "zk": e(batch, L, k, dt=torch.float32),
+            "lse": e(batch, L, dt=torch.float32),
+            "tok": e(batch, self.n_max), "parent": e(batch, self.n_max),
+            "depth": e(batch, self.n_max), "pos": e(batch, self.n_max),
+            "mask": e(batch, self.n_max, W), "n_nodes": e(batch),
+            "surrogate": e(batch, dt=torch.float64),
+            "attn": e(batch, self.n_max, hq, d, dt=torch.bfloat16),
+            "acc_len": e(batch), "acc_nodes": e(batch, L), "acc_tok": e(batch, L), "bonus": e(batch),
+            "status": torch.zeros(1, dtype=torch.int32, device=dev),
+        }
+        self.ws_topk_n = int(self.lib.ddt_topk_workspace_size(batch, L, V, k))
+        self.ws_walk_n = int(self.lib.ddt_tree_walk_workspace_size(batch, self.n_max, V))
+        self.ws_topk = torch.zeros(max(self.ws_topk_n, 256), dtype=torch.uint8, device=dev)
+        self.ws_walk = torch.zeros(max(self.ws_walk_n, 256), dtype=torch.uint8, device=dev)
+        self.ws_attn = None
+        self.attn_args = None
+        self.inputs = None
+
+    # ------------------------------------------------------------------
+    def bind(self, inputs: dict):
+        """Bind device input tensors: draft [b,L,V], root [b], ctx_len [b],
+        q [b,n,hq,d], k_cache/v_cache, optional page_table, k_tree/v_tree
+        [b,n,hkv,d], target [b,n,V]; optional k_per_seq / budget [b]."""
+        self.inputs = inputs
+        o = self.out
+        a = api._attn_args(inputs["q"], inputs["k_cache"], inputs["v_cache"], inputs["k_tree"],
+                           inputs["v_tree"], o["mask"], o["n_nodes"], inputs["ctx_len"],
+                           self.max_ctx, 1.0 / math.sqrt(self.d), inputs.get("page_table"),
+                           o["attn"], None, o["status"])
+        self.attn_args = a
+        n = int(self.lib.ddt_tree_attn_workspace_size(ctypes.byref(a)))
+        if self.ws_attn is None or self.ws_attn.numel() < n:
+            self.ws_attn = torch.zeros(max(n, 256), dtype=torch.uint8, device=self.dev)
+        self.ws_attn_n = n
+
+    def launch(self, stream: Optional[torch.cuda.Stream] = None, marks=None):
+        """Enqueue the four stages on ``stream``.  ``marks(i)`` is called
+        before stage i and after the last (i = 0..4), e.g. to record events."""
+        lib, o, x = self.lib, self.out, self.inputs
+        s = ctypes.c_void_p((stream or torch.cuda.current_stream(self.dev)).cuda_stream)
+        P = api._ptr
+        if marks:
+            marks(0)
+        rc = lib.ddt_topk(P(x["draft"]), self.draft_code, self.batch, self.L, self.V,
+                          x["draft"].stride(1), self.k, self.inv_t, P(o["ids"]), P(o["zk"]), None,
+                          P(o["lse"]), P(self.ws_topk), self.ws_topk_n, s)
+        api._check(rc, "ddt_topk")
+        if marks:
+            marks(1)
+        rc = lib.ddt_build_tree(P(o["ids"]), P(o["zk"]), P(o["lse"]), self.batch, self.L, self.k,
+                                self.inv_t, P(x.get("k_per_seq")), P(x.get("budget")),
+                                self.B_max, P(x["root"]), P(x["ctx_len"]), P(o["tok"]),
+                                P(o["parent"]), P(o["depth"]), P(o["pos"]), P(o["mask"]),
+                                P(o["n_nodes"]), P(o["surrogate"]), P(o["status"]), s)
+        api._check(rc, "ddt_build_tree")
+        if marks:
+            marks(2)
+        rc = lib.ddt_tree_attn(ctypes.byref(self.attn_args), P(self.ws_attn), self.ws_attn_n, s)
+        api._check(rc, "ddt_tree_attn")
+        if marks:
+            marks(3)
+        rc = lib.ddt_tree_walk(P(x["target"]), self.target_code, self.batch, self.n_max, self.V,
+                               x["target"].stride(1), P(o["tok"]), P(o["parent"]), P(o["depth"]),
+                               P(o["n_nodes"]), self.L, P(o["acc_len"]), P(o["acc_nodes"]),
+                               P(o["acc_tok"]), P(o["bonus"]), P(self.ws_walk), self.ws_walk_n,
+                               P(o["status"]), s)
+        api._check(rc, "ddt_tree_walk")
+        if marks:
+            marks(4)
+
+    def capture(self, marks=None) -> torch.cuda.CUDAGraph:
+        """Capture one round (with its current bindings) into a CUDA graph."""
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.launch(torch.cuda.current_stream(self.dev), marks)
+        return g

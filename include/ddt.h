@@ -1,0 +1,216 @@
+/*
+ * ddt.h -- C ABI of libddt.so: the DDTree verification round on B200 (sm_100a).
+ *
+ * The round (DDTree page, a curated summary of the authors' announcement of
+ * "Diffusion Draft Tree"; section 運作流程 "workflow", steps 1-4):
+ *   1. ddt_topk        per-position softmax normaliser and top-k candidates of
+ *                      the drafter's marginals q_i (step 1);
+ *   2. ddt_build_tree  the B most probable prefixes of the factorised draft
+ *                      (step 2; section 理論基礎 "theory", Propositions 1-2),
+ *                      compiled to token / parent / depth / position /
+ *                      ancestor-mask tensors (step 3);
+ *   3. ddt_tree_attn   one attention pass of every tree row against the KV
+ *                      cache and its own ancestors (step 3; section 核心創新
+ *                      "core innovation", ancestor-only attention mask);
+ *   4. ddt_tree_walk   the greedy walk over the target's logits that accepts
+ *                      matching children and returns the bonus token (step 4).
+ *
+ * Conventions shared by every entry point:
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller.  The
+ *     library allocates no device memory; scratch comes from a caller-owned
+ *     workspace sized by the matching *_workspace_size() function.
+ *   - A workspace must be zero-filled before its first use.  Every call that
+ *     returns DDT_OK leaves it zero-filled again when its kernels finish, so
+ *     it can be reused by the next call on the same stream.  Calls that
+ *     share one workspace must not overlap on the GPU.
+ *   - Calls are asynchronous on `stream` and perform no host synchronisation,
+ *     so they can be captured into a CUDA graph.
+ *   - Arguments are validated on the host before any launch: an invalid
+ *     argument returns DDT_ERR_INVALID_ARG / DDT_ERR_UNSUPPORTED /
+ *     DDT_ERR_WORKSPACE and launches nothing.  Problems only visible on the
+ *     device (e.g. a per-sequence budget above the maximum) are clamped and
+ *     reported through the optional `dev_status` word (0 = fine, otherwise a
+ *     ddt_status code); the word is only ever raised, never cleared.
+ *   - A launch failure returns DDT_ERR_CUDA.  No C++ exception crosses the ABI.
+ *   - "bf16" means IEEE bfloat16 stored in 2 bytes; all layouts are dense,
+ *     row-major, innermost index last.
+ */
+#ifndef DDT_H
+#define DDT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum ddt_status {
+  DDT_OK = 0,
+  DDT_ERR_INVALID_ARG = 1, /* null pointer, negative size, inconsistent shapes */
+  DDT_ERR_UNSUPPORTED = 2, /* valid but outside the implemented range (dtype, d, k, B, L) */
+  DDT_ERR_WORKSPACE = 3,   /* workspace missing, misaligned (256 B) or too small */
+  DDT_ERR_CUDA = 4,        /* a CUDA call failed; see cudaGetLastError() */
+  DDT_ERR_TIMEOUT = 5      /* a bounded device-side wait gave up (reported via dev_status) */
+} ddt_status;
+
+typedef enum ddt_dtype { DDT_BF16 = 0, DDT_F32 = 1 } ddt_dtype;
+
+/* Implementation limits. */
+#define DDT_TOPK_K_MAX 32     /* candidates per position */
+#define DDT_TREE_L_MAX 64     /* draft positions (tree depth) */
+#define DDT_TREE_B_MAX 1023   /* draft nodes; rows N = B + 1 <= 1024 */
+
+/* Human-readable name of a status code (static storage; never NULL). */
+const char* ddt_status_string(ddt_status s);
+
+/* Number of 32-bit mask words per tree row: ceil(n_max / 32). */
+int ddt_mask_words(int n_max);
+
+/* ------------------------------------------------------------------------
+ * Stage 1: per-position softmax normaliser and top-k.
+ * DDTree page, 運作流程 step 1: the drafter returns one marginal q_i per
+ * position i = 1..L (conditioned on the previous block only).  The tree's
+ * candidates at depth i are the k most likely tokens of q_i.
+ *
+ * logits   [batch][L] rows of V logits, row r = b*L + i starting at
+ *          logits + r*row_stride elements; dtype DDT_BF16 or DDT_F32.
+ *          row_stride >= V.  BF16 rows need logits and row_stride*2 bytes
+ *          aligned to 16 bytes for the vector path (otherwise a scalar path
+ *          is used).
+ * k        1..DDT_TOPK_K_MAX, k <= V.
+ * inv_temperature  > 0: q_i = softmax(inv_temperature * z).
+ * Outputs (all [batch][L][k] unless noted), in candidate order: logit
+ * descending, ties by smaller token id first:
+ *   ids  int32 token ids;   zk  float, the raw logit z (an exact copy);
+ *   logp float, inv_temperature*z - lse (may be NULL);
+ *   lse  float [batch][L], log sum_v exp(inv_temperature*z_v).
+ * The ordering is decided on raw z, so temperature never reorders it.
+ * ------------------------------------------------------------------------ */
+size_t ddt_topk_workspace_size(int batch, int L, int V, int k);
+ddt_status ddt_topk(const void* logits, ddt_dtype dtype, int batch, int L, int V,
+                    int64_t row_stride, int k, float inv_temperature, int32_t* ids, float* zk,
+                    float* logp, float* lse, void* workspace, size_t workspace_bytes,
+                    cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Stage 2: build and compile the draft tree (one CTA per sequence).
+ * DDTree page, 核心創新 and 運作流程 step 2: under a budget of B draft nodes
+ * the tree is the set of B most probable prefixes of the factorised draft
+ * prod_i q_i (it maximises the expected acceptance length under the draft,
+ * 理論基礎 Proposition 1, and is prefix-closed, Proposition 2).  Step 3: the
+ * tree is compiled into target-model inputs.
+ *
+ * Candidates: ids / zk / lse exactly as produced by ddt_topk
+ * ([batch][L][k], [batch][L]).  Sequence b uses the first k_b candidates of
+ * each position (k_per_seq[b], or k when k_per_seq is NULL) and the budget
+ * B_b (budget_per_seq[b], or B_max when NULL).  Out-of-range device values
+ * are clamped to [1,k] and [0,B_max] and flagged in dev_status.
+ *
+ * Total order (best first) on prefixes p of depth t with logit sum
+ * s(p) = sum of raw z along p and score(p) = inv_temperature*s(p) - sum_{i<=t} lse_i
+ * (fp64): at equal depth, larger s(p) first (exact: the lse terms cancel),
+ * then the smaller token id at the deepest position, then at the one above,
+ * and so on; at different depths, larger score first, then the shallower.
+ *
+ * Compiled outputs, N_max = B_max + 1 rows per sequence, breadth-first
+ * order (depth, parent row, candidate rank); row 0 is the root carrying
+ * root_token[b] (the bonus token of the previous round):
+ *   tok, parent (root: -1), depth (root: 0), pos = ctx_len[b] + depth
+ *        int32 [batch][N_max]; rows >= n_nodes[b] are -1;
+ *   mask uint32 [batch][N_max][W], W = ddt_mask_words(N_max): bit i of row j
+ *        set iff row i is row j or one of its ancestors; padding rows 0;
+ *   n_nodes int32 [batch] = 1 + number of selected prefixes;
+ *   surrogate double [batch] (may be NULL): sum of exp(score) over the
+ *        draft nodes, the expected acceptance length under the draft.
+ * ctx_len may be NULL (treated as 0).  Limits: L <= DDT_TREE_L_MAX,
+ * k <= DDT_TOPK_K_MAX, B_max <= DDT_TREE_B_MAX.
+ * ------------------------------------------------------------------------ */
+ddt_status ddt_build_tree(const int32_t* ids, const float* zk, const float* lse, int batch, int L,
+                          int k, float inv_temperature, const int32_t* k_per_seq,
+                          const int32_t* budget_per_seq, int B_max, const int32_t* root_token,
+                          const int32_t* ctx_len, int32_t* tok, int32_t* parent, int32_t* depth,
+                          int32_t* pos, uint32_t* mask, int32_t* n_nodes, double* surrogate,
+                          int32_t* dev_status, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Stage 3: tree attention.
+ * DDTree page, 核心創新 third bullet and 運作流程 step 3: one target forward
+ * scores the whole tree; each tree row attends to the committed context and
+ * to its own ancestors (and itself) only.
+ *
+ * For sequence b, tree row j < n_nodes[b] and query head h (kv head
+ * h / (hq/hkv)):  out = softmax(scale * q K^T) V  over the context
+ * positions 0..ctx_len[b]-1 and the tree rows i with mask bit (j, i) set.
+ * Accumulation is fp32; out is bf16.  Rows j >= n_nodes[b] are written as 0
+ * (and lse_out as -inf).
+ *
+ *   q       bf16 [batch][n_max][hq][d]
+ *   k_cache, v_cache  dense (page_table == NULL): bf16 [batch][t_max][hkv][d];
+ *           paged: bf16 [pages][page_size][hkv][d], context position t of
+ *           sequence b lives in page page_table[b*max_pages + t/page_size],
+ *           slot t % page_size.
+ *   k_tree, v_tree  bf16 [batch][n_max][hkv][d]  (the tree rows' own K/V)
+ *   mask    uint32 [batch][n_max][W] as produced by ddt_build_tree
+ *   out     bf16 [batch][n_max][hq][d];  lse_out optional f32 [batch][n_max][hq]
+ *           (natural log of the softmax normaliser of the scaled scores).
+ *   max_ctx host-side upper bound of ctx_len[] (sizes the KV-split grid);
+ *           a ctx_len above it is clamped and flagged in dev_status.
+ * Limits: d in {64, 128}; hq % hkv == 0; n_max <= 1024; all base pointers
+ * 16-byte aligned; page_size a multiple of 16.
+ * ------------------------------------------------------------------------ */
+typedef struct ddt_attn_args {
+  const void* q;
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* page_table; /* NULL: dense cache */
+  int page_size;
+  int max_pages;
+  int64_t t_max;             /* dense: tokens per sequence in k_cache/v_cache */
+  const int32_t* ctx_len;
+  int max_ctx;
+  const void* k_tree;
+  const void* v_tree;
+  const uint32_t* mask;
+  const int32_t* n_nodes;
+  int batch, n_max, hq, hkv, d;
+  float scale;
+  void* out;
+  float* lse_out;            /* may be NULL */
+  int32_t* dev_status;       /* may be NULL */
+} ddt_attn_args;
+
+size_t ddt_tree_attn_workspace_size(const ddt_attn_args* a);
+ddt_status ddt_tree_attn(const ddt_attn_args* a, void* workspace, size_t workspace_bytes,
+                         cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Stage 4: greedy tree walk.
+ * DDTree page, 運作流程 step 4: starting at the root, take the target's
+ * next token under its decoding rule (greedy: argmax, smaller token id on
+ * ties); if the current row has a child carrying that token, accept the
+ * child and continue from it; otherwise that token is the bonus token of
+ * the next round (also when the walk reaches a row of depth L).
+ *
+ *   logits  [batch][n_max] rows of V target logits, row (b, j) at
+ *           logits + (b*n_max + j)*row_stride elements; DDT_F32 or DDT_BF16.
+ *   tok, parent, depth, n_nodes: the compiled tree of ddt_build_tree.
+ *   L       the draft length (the deepest a row can be).
+ * Outputs: acc_len int32 [batch] (0..L), acc_nodes / acc_tok int32
+ * [batch][L] (accepted rows and their tokens in walk order; unused -1),
+ * bonus int32 [batch].  Tokens emitted this round = acc_len + 1.
+ * ------------------------------------------------------------------------ */
+size_t ddt_tree_walk_workspace_size(int batch, int n_max, int V);
+ddt_status ddt_tree_walk(const void* logits, ddt_dtype dtype, int batch, int n_max, int V,
+                         int64_t row_stride, const int32_t* tok, const int32_t* parent,
+                         const int32_t* depth, const int32_t* n_nodes, int L, int32_t* acc_len,
+                         int32_t* acc_nodes, int32_t* acc_tok, int32_t* bonus, void* workspace,
+                         size_t workspace_bytes, int32_t* dev_status, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DDT_H */

@@ -1,0 +1,117 @@
+"""The C ABI without a GPU: libddt.so builds, loads, exports every function
+include/ddt.h declares, and rejects bad arguments on the host before any
+launch (no compute call is made here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from block_draft_tree_b200 import api, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", f)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(ddt_[a-z0-9_]+)\s*\(", src))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return api.load_library()
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = _declared()
+    assert {"ddt_topk", "ddt_build_tree", "ddt_tree_attn", "ddt_tree_walk"} <= declared
+    raw = ctypes.CDLL(api.library_path())
+    for name in sorted(declared):
+        assert hasattr(raw, name), name
+    assert set(api.EXPORTED) <= declared
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        assert lib.ddt_status_string(code).startswith(b"DDT_")
+    assert lib.ddt_mask_words(513) == 17 and lib.ddt_mask_words(32) == 1
+
+
+def test_topk_rejects_bad_arguments(lib):
+    f = lib.ddt_topk
+    dummy = ctypes.c_void_p(16)
+    args = dict(logits=dummy, dt=0, b=1, L=4, V=64, stride=64, k=4, it=1.0)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return f(a["logits"], a["dt"], a["b"], a["L"], a["V"], a["stride"], a["k"], a["it"],
+                 dummy, dummy, dummy, dummy, None, 0, None)
+
+    assert call(k=33) == 2           # above DDT_TOPK_K_MAX
+    assert call(k=65) in (1, 2)      # k > V
+    assert call(stride=10) == 1      # row stride < V
+    assert call(it=0.0) == 1 and call(it=-1.0) == 1 and call(it=float("inf")) == 1
+    assert call(dt=7) == 2
+    assert call(logits=None) == 1
+    assert call(V=200000, stride=200000) == 3  # needs a workspace, none given
+    assert call(b=100, L=1000) == 2  # more rows than the grid holds
+
+
+def test_build_tree_rejects_bad_arguments(lib):
+    f = lib.ddt_build_tree
+    d = ctypes.c_void_p(16)
+
+    def call(b=1, L=4, k=4, B=8, it=1.0, ids=d):
+        return f(ids, d, d, b, L, k, it, None, None, B, d, None, d, d, d, d, d, d, None, None, None)
+
+    assert call(L=65) == 2 and call(k=33) == 2 and call(B=1024) == 2
+    assert call(L=0) == 1 and call(B=-1) == 1 and call(it=0.0) == 1
+    assert call(ids=None) == 1
+
+
+def test_attn_rejects_bad_arguments(lib):
+    a = api.AttnArgs()
+    a.q = a.k_cache = a.v_cache = a.k_tree = a.v_tree = a.mask = a.n_nodes = a.ctx_len = a.out = 256
+    a.batch, a.n_max, a.hq, a.hkv, a.d, a.max_ctx, a.t_max = 1, 9, 4, 1, 64, 128, 128
+    a.scale = 0.125
+    f = lib.ddt_tree_attn
+    base = dict((n, getattr(a, n)) for n, _ in api.AttnArgs._fields_)
+
+    def call(**kw):
+        b = api.AttnArgs(**dict(base, **kw))
+        return f(ctypes.byref(b), None, 0, None)
+
+    assert call(d=96) == 2
+    assert call(hq=6, hkv=4) == 1
+    assert call(n_max=1025) == 2
+    assert call(q=None) == 1
+    assert call(q=258) == 1              # misaligned
+    assert call(t_max=100) == 1          # dense cache shorter than max_ctx
+    assert call(page_table=512, page_size=10, max_pages=20) == 2
+    assert call(page_table=512, page_size=16, max_pages=2) == 1
+    assert call(scale=0.0) == 1
+    assert f(None, None, 0, None) == 1
+
+
+def test_walk_rejects_bad_arguments(lib):
+    f = lib.ddt_tree_walk
+    d = ctypes.c_void_p(16)
+
+    def call(b=1, n=9, V=64, stride=64, L=4, dt=1, logits=d):
+        return f(logits, dt, b, n, V, stride, d, d, d, d, L, d, d, d, d, None, 0, None, None)
+
+    assert call(stride=3) == 1 and call(dt=5) == 2 and call(n=2000) == 2 and call(L=65) == 2
+    assert call(logits=None) == 1
+    assert call(V=10 ** 6, stride=10 ** 6) == 3  # workspace required
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    with pytest.raises(api.DDTError):
+        api.topk(torch.zeros(1, 2, 64), 4)
