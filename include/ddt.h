@@ -96,6 +96,32 @@ ddt_status ddt_topk(const void* logits, ddt_dtype dtype, int batch, int L, int V
                     cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
+ * ddt_topk_noalloc: ddt_topk for callers that cannot allocate device memory.
+ * The DDTree page has no counterpart to this entry point; it is a service of
+ * this library for code that runs where obtaining device memory is not
+ * allowed at the point of the call (an allocator-free region under a custom
+ * memory manager that owns the heap, an embedded runtime with a fixed memory
+ * plan, a plug-in whose host forbids cudaMalloc), so that it cannot supply
+ * the workspace ddt_topk needs.
+ *
+ * Same arguments, outputs and results as ddt_topk, minus the workspace.
+ * Its scratch is a fixed array in device global memory owned by libddt.so:
+ * DDT_TOPK_NOALLOC_SCRATCH_BYTES on every GPU that loads the library, held
+ * until the process exits.  Shapes whose ddt_topk_workspace_size exceeds it
+ * are rejected with DDT_ERR_WORKSPACE before anything is launched.
+ * The first call on a device (with that device current) looks up the array's
+ * device address once; make that first call before any stream capture.
+ * Every call on a device shares the array; each call clears the part it uses
+ * (an asynchronous memset on `stream`), so consecutive calls on one stream
+ * are independent, while calls that overlap on the GPU race on the array.
+ * Never calls cudaMalloc, cudaFree or any allocating library routine.
+ * ------------------------------------------------------------------------ */
+#define DDT_TOPK_NOALLOC_SCRATCH_BYTES (4u << 20)
+ddt_status ddt_topk_noalloc(const void* logits, ddt_dtype dtype, int batch, int L, int V,
+                            int64_t row_stride, int k, float inv_temperature, int32_t* ids,
+                            float* zk, float* logp, float* lse, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
  * Stage 2: build and compile the draft tree (one CTA per sequence).
  * DDTree page, 核心創新 and 運作流程 step 2: under a budget of B draft nodes
  * the tree is the set of B most probable prefixes of the factorised draft
