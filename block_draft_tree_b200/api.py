@@ -40,6 +40,7 @@ class AttnArgs(ctypes.Structure):
     _fields_ = [
         ("q", ctypes.c_void_p), ("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p),
         ("page_table", ctypes.c_void_p), ("page_size", ctypes.c_int), ("max_pages", ctypes.c_int),
+        ("num_pages", ctypes.c_int),
         ("t_max", ctypes.c_int64), ("ctx_len", ctypes.c_void_p), ("max_ctx", ctypes.c_int),
         ("k_tree", ctypes.c_void_p), ("v_tree", ctypes.c_void_p), ("mask", ctypes.c_void_p),
         ("n_nodes", ctypes.c_void_p), ("batch", ctypes.c_int), ("n_max", ctypes.c_int),
@@ -227,11 +228,13 @@ def _attn_args(q, k_cache, v_cache, k_tree, v_tree, mask, n_nodes, ctx_len, max_
         a.page_table = page_table.data_ptr()
         a.page_size = k_cache.shape[1]
         a.max_pages = page_table.shape[1]
+        a.num_pages = k_cache.shape[0]
         a.t_max = 0
     else:
         a.page_table = None
         a.page_size = 0
         a.max_pages = 0
+        a.num_pages = 0
         a.t_max = k_cache.shape[1] if k_cache is not None else 0
     a.ctx_len = ctx_len.data_ptr()
     a.max_ctx = int(max_ctx)

@@ -46,6 +46,9 @@ bool ws_ok(const void* ws, size_t have, size_t need) {
 
 ddt_status launch_attn_simt(AttnParams& p, cudaStream_t stream);
 int attn_simt_rows_per_cta();
+bool attn_tc_eligible(const ddt_attn_args* a);
+size_t attn_tc_workspace_size(const ddt_attn_args* a, int sms);
+ddt_status launch_attn_tc(const ddt_attn_args* a, void* ws, int sms, cudaStream_t stream);
 
 // KV-split plan shared by the workspace query and the launch.
 static void attn_plan(const ddt_attn_args* a, int rows_per_cta, int* row_tiles, int* nsplit,
@@ -67,13 +70,24 @@ static void attn_plan(const ddt_attn_args* a, int rows_per_cta, int* row_tiles, 
 }
 
 size_t attn_workspace_size(const ddt_attn_args* a) {
+  if (attn_tc_eligible(a)) {
+    const size_t n = attn_tc_workspace_size(a, sm_count());
+    return n ? (size_t)DDT_WS_COUNTER_BYTES + n : 0;
+  }
   int rt, ns, tps;
   attn_plan(a, attn_simt_rows_per_cta(), &rt, &ns, &tps);
   if (ns <= 1) return 0;
   const size_t groups = (size_t)a->batch * a->hkv;
   const size_t R = (size_t)a->n_max * (a->hq / a->hkv);
-  return align256(sizeof(unsigned) * groups * rt) + align256(sizeof(float2) * groups * ns * R) +
+  return (size_t)DDT_WS_COUNTER_BYTES + align256(sizeof(float2) * groups * ns * R) +
          align256(sizeof(float) * groups * ns * R * a->d);
+}
+
+// Counters the CUDA-core attention needs (one ticket per row tile and kv head).
+static size_t attn_simt_counters(const ddt_attn_args* a) {
+  int rt, ns, tps;
+  attn_plan(a, attn_simt_rows_per_cta(), &rt, &ns, &tps);
+  return ns > 1 ? (size_t)a->batch * a->hkv * rt : 0;
 }
 
 ddt_status launch_attn(const ddt_attn_args* a, void* ws, size_t ws_bytes, cudaStream_t stream) {
@@ -102,13 +116,16 @@ ddt_status launch_attn(const ddt_attn_args* a, void* ws, size_t ws_bytes, cudaSt
   p.out = (uint16_t*)a->out;
   p.lse_out = a->lse_out;
   p.status = a->dev_status;
+  if (a->batch == 0) return DDT_OK;
+  if (attn_tc_eligible(a))
+    return launch_attn_tc(a, ws ? (char*)ws + DDT_WS_COUNTER_BYTES : nullptr, sm_count(), stream);
   attn_plan(a, attn_simt_rows_per_cta(), &p.row_tiles, &p.nsplit, &p.tok_per_split);
   const size_t groups = (size_t)a->batch * a->hkv;
   const size_t R = (size_t)a->n_max * p.g;
   char* w = (char*)ws;
-  p.tickets = (unsigned*)w;
+  p.tickets = (unsigned*)w;  // counter region
   if (p.nsplit > 1) {
-    w += align256(sizeof(unsigned) * groups * p.row_tiles);
+    w += DDT_WS_COUNTER_BYTES;
     p.part_ml = (float2*)w;
     w += align256(sizeof(float2) * groups * p.nsplit * R);
     p.part_o = (float*)w;
@@ -116,7 +133,6 @@ ddt_status launch_attn(const ddt_attn_args* a, void* ws, size_t ws_bytes, cudaSt
     p.part_ml = nullptr;
     p.part_o = nullptr;
   }
-  if (a->batch == 0) return DDT_OK;
   return launch_attn_simt(p, stream);
 }
 
@@ -201,6 +217,7 @@ static ddt_status check_attn(const ddt_attn_args* a) {
     if (a->page_table) {
       if (a->page_size < 16 || a->page_size % 16 != 0) return DDT_ERR_UNSUPPORTED;
       if ((long)a->max_pages * a->page_size < a->max_ctx) return DDT_ERR_INVALID_ARG;
+      if (a->num_pages < 0) return DDT_ERR_INVALID_ARG;
     } else if (a->t_max < a->max_ctx) {
       return DDT_ERR_INVALID_ARG;
     }
@@ -213,10 +230,13 @@ size_t ddt_tree_attn_workspace_size(const ddt_attn_args* a) {
   return attn_workspace_size(a);
 }
 
+static const size_t kMaxCounters = DDT_WS_COUNTER_BYTES / sizeof(unsigned);
+
 ddt_status ddt_tree_attn(const ddt_attn_args* a, void* workspace, size_t workspace_bytes,
                          cudaStream_t stream) {
   const ddt_status st = check_attn(a);
   if (st != DDT_OK) return st;
+  if (!attn_tc_eligible(a) && attn_simt_counters(a) > kMaxCounters) return DDT_ERR_UNSUPPORTED;
   if (!ws_ok(workspace, workspace_bytes, attn_workspace_size(a))) return DDT_ERR_WORKSPACE;
   return launch_attn(a, workspace, workspace_bytes, stream);
 }
@@ -234,6 +254,7 @@ ddt_status ddt_tree_walk(const void* logits, ddt_dtype dtype, int batch, int n_m
   if (batch < 0 || n_max < 1 || V < 1 || row_stride < V || L < 0) return DDT_ERR_INVALID_ARG;
   if (dtype != DDT_BF16 && dtype != DDT_F32) return DDT_ERR_UNSUPPORTED;
   if (n_max > DDT_TREE_B_MAX + 1 || batch > 65535 || L > DDT_TREE_L_MAX) return DDT_ERR_UNSUPPORTED;
+  if ((size_t)batch * n_max + batch > kMaxCounters) return DDT_ERR_UNSUPPORTED;
   if (batch > 0 && (!logits || !tok || !parent || !depth || !n_nodes || !acc_len || !bonus ||
                     (L > 0 && (!acc_nodes || !acc_tok))))
     return DDT_ERR_INVALID_ARG;

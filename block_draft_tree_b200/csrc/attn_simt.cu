@@ -205,16 +205,7 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnParams p) {
     const int qr = rt * kRows + warp * 4 + r;
     if (qr < R) combine_row<DV>(p, grp, b, kvh, qr, lane);
   }
-  // leave the workspace as it was found: all zero
-  __syncthreads();
-  const int r0 = rt * kRows, nr = min(kRows, R - r0);
-  for (int s = 0; s < p.nsplit; ++s) {
-    float* po = p.part_o + ((grp * p.nsplit + s) * R + r0) * D;
-    for (int i = tid; i < nr * D; i += kThreads) po[i] = 0.f;
-    for (int i = tid; i < nr; i += kThreads)
-      p.part_ml[(grp * p.nsplit + s) * R + r0 + i] = make_float2(0.f, 0.f);
-  }
-  if (tid == 0) p.tickets[grp * p.row_tiles + rt] = 0u;
+  if (tid == 0) p.tickets[grp * p.row_tiles + rt] = 0u;  // the counter region is left zero
 }
 
 }  // namespace

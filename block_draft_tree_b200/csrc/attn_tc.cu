@@ -1,0 +1,754 @@
+// attn_tc.cu -- stage 3 of the verification round on the 5th-generation tensor
+// cores: tcgen05 MMAs with TMEM accumulators, K/V tiles staged by TMA.
+//
+// DDTree page, section 核心創新 third bullet and 運作流程 step 3: the target
+// scores every tree row in one pass; each row attends to the committed
+// context and to its own ancestors (and itself) only.
+//
+// Once the tree has N*g >= 64 query rows per kv head (g = hq/hkv) the
+// attention is a dense contraction Q[rows x d] K^T[d x tokens] followed by
+// P[rows x tokens] V[tokens x d], so it runs as tiles of 128 query rows x 128
+// tokens (d = 128):
+//   * grid = (query tiles, KV splits, batch*hkv); one CTA per SM (TMEM: 512
+//     columns = S double buffer 2x128, O 128, P 64; smem 224 KB: Q + a 3-deep K/V ring);
+//   * warp 0 issues TMA loads (Q once; K and V per token tile, 128B-swizzled,
+//     dense rows, 64-token pages, or the tree's own rows), warp 1 issues the
+//     MMAs from one thread, warps 2-5 own one TMEM lane (one query row) each;
+//   * S = Q K^T lands in TMEM; the softmax warps read it, apply the
+//     context-length / ancestor-bitset mask, keep a base-2 running max that
+//     only moves (and rescales O) when it grows by more than 2^8, write
+//     P = 2^(S - m) as bf16 back into TMEM, and the MMA warp computes
+//     O += P V with P as the TMEM-resident A operand and V as an MN-major
+//     shared-memory B operand;
+//   * with one split the CTA normalises and writes bf16 rows; with several
+//     it writes (O, m, l) partials and a second kernel merges them.
+// Every mbarrier wait is bounded (about one second); a wait that gives up
+// raises DDT_ERR_TIMEOUT in the status word and the CTA stops issuing work.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "attn_common.cuh"
+#include "common.cuh"
+#include "launch.h"
+
+namespace ddt {
+namespace tc {
+
+constexpr int BM = 128;                   // query rows per tile (MMA M)
+constexpr int BN = 128;                   // tokens per tile (MMA N of QK^T, K of PV)
+constexpr int D = 128;                    // head dim
+constexpr int kStages = 3;                // K/V ring depth
+constexpr int kThreads = 192;             // warp 0 TMA, warp 1 MMA, warps 2-5 softmax
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP = 384;
+constexpr int kHalf = BN * 128;           // one 64-wide d half: 128 rows x 128 B
+constexpr int kTile = 2 * kHalf;          // 32 KB
+constexpr long long kWaitCycles = 2000000000LL;
+constexpr float kRescaleLog2 = 8.f;       // move the running max only when it grows by > 2^8
+
+struct Params {
+  int batch, n_max, hq, hkv, g, W, max_ctx;
+  int paged, page_size, max_pages, rows_per_box, boxes_per_tile;
+  int64_t t_max;
+  float scale_log2;
+  const int32_t* ctx_len;
+  const int32_t* n_nodes;
+  const uint32_t* mask;
+  const int32_t* page_table;
+  uint16_t* out;
+  float* lse_out;
+  int32_t* status;
+  int nsplit, tiles_per_split, qtiles;
+  float* part_o;    // [grp][qtile][split][BM][D]
+  float2* part_ml;  // [grp][qtile][split][BM]
+};
+
+struct __align__(8) Bars {
+  uint64_t q_full;
+  uint64_t kv_full[kStages];
+  uint64_t kv_empty[kStages];
+  uint64_t s_full[2];
+  uint64_t p_full;
+  uint64_t pv_done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+// ---------------------------------------------------------------- PTX helpers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait: false (and the CTA-wide abort flag set) if the phase does not
+// complete within kWaitCycles or another role already aborted.
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, Bars* bars) {
+  if (mbar_try_wait(b, parity)) return true;
+  const long long t0 = clock64();
+  for (;;) {
+    if (mbar_try_wait(b, parity)) return true;
+    if (*(volatile int*)&bars->abort) return false;
+    if (clock64() - t0 > kWaitCycles) {
+      *(volatile int*)&bars->abort = 1;
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int c0, int c1, int c2,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, "
+      "%4}], [%5];" ::"r"(smem_u32(dst)),
+      "l"((uint64_t)map), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int c0, int c1, int c2,
+                                            int c3, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, "
+      "%4, %5}], [%6];" ::"r"(smem_u32(dst)),
+      "l"((uint64_t)map), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                       uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+      "%13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, "
+      "[%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, "
+      "%31, %32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+      "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]),
+      "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]),
+      "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version bits.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1u << 46;  // descriptor version for sm_100
+  d |= (uint64_t)2u << 61;  // SWIZZLE_128B
+  return d;
+}
+// Instruction descriptor, kind::f16: bf16 x bf16 -> f32, M = 128, N = 128,
+// A K-major; B K-major (QK^T) or MN-major (PV).
+__host__ __device__ constexpr uint32_t idesc_bf16(bool b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+         ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+
+struct TileInfo {
+  int tree;   // 0: context tile, 1: tree tile
+  int base;   // first token (context position or tree row)
+  int cnt;    // valid tokens in the tile
+};
+
+__device__ __forceinline__ TileInfo tile_info(int t, int nct, int T, int n) {
+  TileInfo ti;
+  if (t < nct) {
+    ti.tree = 0;
+    ti.base = t * BN;
+    ti.cnt = min(BN, T - ti.base);
+  } else {
+    ti.tree = 1;
+    ti.base = (t - nct) * BN;
+    ti.cnt = min(BN, n - ti.base);
+  }
+  return ti;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kt,
+                   const __grid_constant__ CUtensorMap tm_vt, const Params p) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // 1024-byte alignment for the swizzle atoms
+  unsigned char* smem = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  unsigned char* sQ = smem;                              // [2][128][128 B]
+  unsigned char* sK = smem + kTile;                      // [kStages][2][128][128 B]
+  unsigned char* sV = sK + kStages * kTile;              // [kStages][2][128][128 B]
+  Bars* bars = (Bars*)(sV + kStages * kTile);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int qtile = blockIdx.x, split = blockIdx.y, grp = blockIdx.z;
+  const int b = grp / p.hkv, kvh = grp % p.hkv;
+  const int g = p.g;
+  const int R = p.n_max * g;
+  const int q0 = qtile * BM;
+  int n = p.n_nodes[b];
+  n = min(max(n, 1), p.n_max);
+  int T = p.ctx_len[b];
+  if (T < 0 || T > p.max_ctx) {
+    if (qtile == 0 && split == 0 && kvh == 0 && tid == 0) raise_status(p.status, DDT_ERR_INVALID_ARG);
+    T = min(max(T, 0), p.max_ctx);
+  }
+  const int nct = (T + BN - 1) / BN;
+  const int ntt = (n + BN - 1) / BN;
+  const int t_lo = min(split * p.tiles_per_split, nct + ntt);
+  const int t_hi = min(t_lo + p.tiles_per_split, nct + ntt);
+  const int ntiles = t_hi - t_lo;
+  const int64_t part_row0 = (((int64_t)grp * p.qtiles + qtile) * p.nsplit + split) * BM;
+
+  if (ntiles == 0) {  // nothing in this split: an empty partial (or zero rows)
+    if (tid >= 64) {
+      const int row = tid - 64;
+      const int qr = q0 + row;
+      if (p.nsplit > 1) {
+        float4* po = (float4*)(p.part_o + (part_row0 + row) * D);
+        for (int i = 0; i < D / 4; ++i) po[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        p.part_ml[part_row0 + row] = make_float2(-INFINITY, 0.f);
+      } else if (qr < R) {
+        const int j = qr / g, h = kvh * g + qr % g;
+        uint4* dst = (uint4*)(p.out + (((int64_t)b * p.n_max + j) * p.hq + h) * D);
+        for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(0, 0, 0, 0);
+        if (p.lse_out) p.lse_out[((int64_t)b * p.n_max + j) * p.hq + h] = -INFINITY;
+      }
+    }
+    return;
+  }
+
+  if (tid == 0) {
+    mbar_init(&bars->q_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bars->kv_full[s], 1);
+      mbar_init(&bars->kv_empty[s], 1);
+    }
+    mbar_init(&bars->s_full[0], 1);
+    mbar_init(&bars->s_full[1], 1);
+    mbar_init(&bars->p_full, 128);
+    mbar_init(&bars->pv_done, 1);
+    bars->abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&bars->tmem_base)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const int j0 = q0 / g;
+      mbar_expect_tx(&bars->q_full, (uint32_t)kTile);
+      tma_load_3d(sQ, &tm_q, 0, kvh * g, b * p.n_max + j0, &bars->q_full);
+      tma_load_3d(sQ + kHalf, &tm_q, 64, kvh * g, b * p.n_max + j0, &bars->q_full);
+      for (int i = 0; i < ntiles; ++i) {
+        const int s = i % kStages;
+        const uint32_t ph = (uint32_t)(i / kStages) & 1u;
+        if (!mbar_wait(&bars->kv_empty[s], ph ^ 1u, bars)) break;
+        const TileInfo ti = tile_info(t_lo + i, nct, T, n);
+        unsigned char* k_dst = sK + s * kTile;
+        unsigned char* v_dst = sV + s * kTile;
+        if (ti.tree) {
+          const int row = b * p.n_max + ti.base;
+          mbar_expect_tx(&bars->kv_full[s], (uint32_t)(2 * kTile));
+          for (int h = 0; h < 2; ++h) {
+            tma_load_3d(k_dst + h * kHalf, &tm_kt, 64 * h, kvh, row, &bars->kv_full[s]);
+            tma_load_3d(v_dst + h * kHalf, &tm_vt, 64 * h, kvh, row, &bars->kv_full[s]);
+          }
+        } else if (!p.paged) {
+          const int row = (int)((int64_t)b * p.t_max + ti.base);
+          mbar_expect_tx(&bars->kv_full[s], (uint32_t)(2 * kTile));
+          for (int h = 0; h < 2; ++h) {
+            tma_load_3d(k_dst + h * kHalf, &tm_k, 64 * h, kvh, row, &bars->kv_full[s]);
+            tma_load_3d(v_dst + h * kHalf, &tm_v, 64 * h, kvh, row, &bars->kv_full[s]);
+          }
+        } else {
+          // boxes of rows_per_box tokens; boxes past the context are not loaded
+          const int rpb = p.rows_per_box;
+          int nbox = 0;
+          for (int bx = 0; bx < p.boxes_per_tile; ++bx)
+            if (ti.base + bx * rpb < T) ++nbox;
+          mbar_expect_tx(&bars->kv_full[s], (uint32_t)(nbox * rpb * 128 * 2 * 2));
+          for (int bx = 0; bx < nbox; ++bx) {
+            const int tok = ti.base + bx * rpb;
+            const int page = p.page_table[(int64_t)b * p.max_pages + tok / p.page_size];
+            const int slot = tok % p.page_size;
+            for (int h = 0; h < 2; ++h) {
+              tma_load_4d(k_dst + h * kHalf + bx * rpb * 128, &tm_k, 64 * h, kvh, slot, page,
+                          &bars->kv_full[s]);
+              tma_load_4d(v_dst + h * kHalf + bx * rpb * 128, &tm_v, 64 * h, kvh, slot, page,
+                          &bars->kv_full[s]);
+            }
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdQK = idesc_bf16(false);
+      constexpr uint32_t kIdPV = idesc_bf16(true);
+      const uint32_t q_addr = smem_u32(sQ);
+      bool ok = mbar_wait(&bars->q_full, 0, bars);
+      for (int i = 0; ok && i <= ntiles; ++i) {
+        if (i < ntiles) {
+          const int s = i % kStages;
+          if (!mbar_wait(&bars->kv_full[s], (uint32_t)(i / kStages) & 1u, bars)) break;
+          fence_after();
+          const uint32_t k_addr = smem_u32(sK + s * kTile);
+          const uint32_t d_tm = tmem + ((i & 1) ? kColS1 : kColS0);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (uint32_t)((kk >> 2) * kHalf + (kk & 3) * 32);
+            mma_ss(d_tm, sdesc(q_addr + off, 16, 1024), sdesc(k_addr + off, 16, 1024), kIdQK,
+                   kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&bars->s_full[i & 1]);
+        }
+        if (i > 0) {
+          const int ip = i - 1;
+          if (!mbar_wait(&bars->p_full, (uint32_t)ip & 1u, bars)) break;
+          fence_after();
+          const int sp = ip % kStages;
+          const uint32_t v_addr = smem_u32(sV + sp * kTile);
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk)
+            mma_ts(tmem + kColO, tmem + kColP + kk * 8, sdesc(v_addr + kk * 2048, kHalf, 1024), kIdPV,
+                   (ip > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&bars->pv_done);
+          mma_commit(&bars->kv_empty[sp]);
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warps
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    const int qr = q0 + row;
+    const int j = qr / g;
+    const bool row_valid = qr < R && j < n;
+    const uint32_t* mrow = p.mask + ((int64_t)b * p.n_max + (j < p.n_max ? j : 0)) * p.W;
+    float m_used = -INFINITY, l = 0.f;
+    uint32_t r[BN];
+    bool ok = true;
+    for (int i = 0; i < ntiles && ok; ++i) {
+      const TileInfo ti = tile_info(t_lo + i, nct, T, n);
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->s_full[i & 1], (uint32_t)(i >> 1) & 1u, bars));
+      if (!ok) break;
+      fence_after();
+      const uint32_t s_col = (i & 1) ? kColS1 : kColS0;
+#pragma unroll
+      for (int c = 0; c < BN / 32; ++c) tmem_ld32(lane_base + s_col + 32 * c, r + 32 * c);
+      tmem_ld_wait();
+      // Row maximum in the raw score domain (scale > 0 commutes with max).
+      // Full context tiles need no masking; partial and tree tiles mask with
+      // -inf, which the exp below turns into 0.
+      const float c_log2 = p.scale_log2;
+      const bool full_tile = !ti.tree && ti.cnt == BN && row_valid;
+      if (!full_tile) {
+        uint32_t mw[4] = {0u, 0u, 0u, 0u};
+        if (ti.tree && row_valid) {
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const int word = (ti.base >> 5) + w;
+            mw[w] = word < p.W ? mrow[word] : 0u;
+          }
+        } else if (!ti.tree && row_valid) {
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const int lo = 32 * w;
+            mw[w] = ti.cnt >= lo + 32 ? 0xFFFFFFFFu : (ti.cnt > lo ? ((1u << (ti.cnt - lo)) - 1u) : 0u);
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < BN; ++c)
+          if (!((mw[c >> 5] >> (c & 31)) & 1u)) r[c] = 0xFF800000u;  // -inf
+      }
+      float mx8[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(r[e]);
+#pragma unroll
+      for (int c = 8; c < BN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(r[c]));
+      const float mx_raw = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      const float mx = mx_raw * c_log2;
+      const float m_new = fmaxf(m_used, mx);
+      const bool move = m_new > m_used + kRescaleLog2 || (m_used == -INFINITY && m_new != -INFINITY);
+      const float m_tgt = move ? m_new : m_used;
+      float rs8[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) rs8[e] = 0.f;
+      if (m_tgt == -INFINITY) {
+#pragma unroll
+        for (int c = 0; c < BN / 2; ++c) r[c] = 0u;
+      } else {
+        // p = 2^(s*c - m): one FFMA and one MUFU per score; bf16 pairs packed in place
+#pragma unroll
+        for (int c = 0; c < BN; c += 2) {
+          const float a = ex2(fmaf(__uint_as_float(r[c]), c_log2, -m_tgt));
+          const float bb = ex2(fmaf(__uint_as_float(r[c + 1]), c_log2, -m_tgt));
+          rs8[(c >> 1) & 7] += a + bb;
+          __nv_bfloat162 pk = __floats2bfloat162_rn(a, bb);
+          r[c >> 1] = *(uint32_t*)&pk;
+        }
+      }
+      const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+      // PV of the previous tile must be done before P and O are touched
+      if (i > 0) {
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->pv_done, (uint32_t)(i - 1) & 1u, bars));
+        if (!ok) break;
+      }
+      fence_after();
+      if (move) {
+        if (i > 0 && m_used != -INFINITY) {
+          const float alpha = ex2(m_used - m_new);
+          uint32_t o[32];
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            tmem_ld32(lane_base + kColO + 32 * c, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(lane_base + kColO + 32 * c, o);
+          }
+          l *= alpha;
+        }
+        m_used = m_new;
+      }
+      l += rs;
+      tmem_st32(lane_base + kColP, r);
+      tmem_st32(lane_base + kColP + 32, r + 32);
+      // token row `row` of a partial tile: zero its V row so that 0 * garbage cannot
+      // turn into NaN in the PV product
+      if (row >= ti.cnt) {
+        uint4* vrow0 = (uint4*)(sV + (i % kStages) * kTile + row * 128);
+        uint4* vrow1 = (uint4*)(sV + (i % kStages) * kTile + kHalf + row * 128);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          vrow0[e] = make_uint4(0, 0, 0, 0);
+          vrow1[e] = make_uint4(0, 0, 0, 0);
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      }
+      tmem_st_wait();
+      fence_before();
+      mbar_arrive(&bars->p_full);
+    }
+    if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->pv_done, (uint32_t)(ntiles - 1) & 1u, bars));
+    fence_after();
+    // epilogue: O row -> partial or final output
+    float* po = p.part_o + (part_row0 + row) * D;
+    const bool final_out = p.nsplit == 1;
+    const float inv = (l > 0.f) ? 1.f / l : 0.f;
+    uint16_t* dst = nullptr;
+    if (final_out && qr < R)
+      dst = p.out + (((int64_t)b * p.n_max + j) * p.hq + (kvh * g + qr % g)) * D;
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t o[32];
+      tmem_ld32(lane_base + kColO + 32 * c, o);
+      tmem_ld_wait();
+      if (!ok || !row_valid) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[e] = 0u;
+      }
+      if (!final_out) {
+        float4* q4 = (float4*)(po + 32 * c);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          q4[e] = make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
+                              __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]));
+      } else if (dst) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(o[2 * e]) * inv,
+                                                   __uint_as_float(o[2 * e + 1]) * inv);
+          pk[e] = *(uint32_t*)&h2;
+        }
+        uint4* d4 = (uint4*)(dst + 32 * c);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) d4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+      }
+    }
+    const bool has = ok && row_valid && l > 0.f;
+    if (!final_out) {
+      p.part_ml[part_row0 + row] = has ? make_float2(m_used, l) : make_float2(-INFINITY, 0.f);
+    } else if (dst && p.lse_out) {
+      p.lse_out[((int64_t)b * p.n_max + j) * p.hq + (kvh * g + qr % g)] =
+          has ? (m_used + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+    }
+  }
+
+  fence_before();
+  __syncthreads();
+  if (bars->abort && tid == 0) raise_status(p.status, DDT_ERR_TIMEOUT);
+  if (warp == 0) {
+    __syncwarp();
+    fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// Merge the per-split partials: one warp per query row, 4 dims per lane.
+__global__ void __launch_bounds__(256) attn_tc_combine(const Params p) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 8 + warp;          // row within the query tile
+  const int qtile = row / BM, r = row % BM;
+  const int grp = blockIdx.y;
+  const int b = grp / p.hkv, kvh = grp % p.hkv;
+  const int g = p.g;
+  const int R = p.n_max * g;
+  const int qr = qtile * BM + r;
+  if (qtile >= p.qtiles || qr >= R) return;
+  int n = p.n_nodes[b];
+  n = min(max(n, 1), p.n_max);
+  const int j = qr / g, h = kvh * g + qr % g;
+  const int64_t base = (((int64_t)grp * p.qtiles + qtile) * p.nsplit) * BM + r;
+  float M = -INFINITY;
+  for (int s = 0; s < p.nsplit; ++s) M = fmaxf(M, p.part_ml[base + (int64_t)s * BM].x);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float L = 0.f;
+  if (M != -INFINITY && j < n) {
+    for (int s = 0; s < p.nsplit; ++s) {
+      const float2 ml = p.part_ml[base + (int64_t)s * BM];
+      if (ml.x == -INFINITY) continue;
+      const float w = ex2(ml.x - M);
+      L += ml.y * w;
+      const float4 v = ((const float4*)(p.part_o + (base + (int64_t)s * BM) * D))[lane];
+      acc.x = fmaf(w, v.x, acc.x);
+      acc.y = fmaf(w, v.y, acc.y);
+      acc.z = fmaf(w, v.z, acc.z);
+      acc.w = fmaf(w, v.w, acc.w);
+    }
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  __nv_bfloat162 h0 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+  __nv_bfloat162 h1 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+  uint2* dst = (uint2*)(p.out + (((int64_t)b * p.n_max + j) * p.hq + h) * D);
+  dst[lane] = make_uint2(*(uint32_t*)&h0, *(uint32_t*)&h1);
+  if (lane == 0 && p.lse_out)
+    p.lse_out[((int64_t)b * p.n_max + j) * p.hq + h] =
+        L > 0.f ? (M + __log2f(L)) * 0.69314718055994531f : -INFINITY;
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (PFN_cuTensorMapEncodeTiled_v12000)f;
+  });
+  return fn;
+}
+
+bool encode(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
+            const cuuint64_t* strides, const cuuint32_t* box) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), dims,
+            strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+size_t smem_bytes() { return 1024 + (size_t)(1 + 2 * kStages) * kTile + sizeof(Bars) + 64; }
+
+}  // namespace tc
+
+// Can the tensor-core path serve this call?
+bool attn_tc_eligible(const ddt_attn_args* a) {
+  if (a->d != 128) return false;
+  const int g = a->hq / a->hkv;
+  if (g > 128 || 128 % g != 0) return false;
+  if ((long)a->n_max * g < 64) return false;
+  if (a->page_table) {
+    const int ps = a->page_size;
+    if (a->num_pages <= 0) return false;
+    if (ps <= 128 ? (128 % ps != 0) : (ps % 128 != 0)) return false;
+  }
+  return tc::encode_fn() != nullptr;
+}
+
+// KV-split plan of the tensor-core path: one CTA per SM, as few waves and
+// splits as possible.
+void attn_tc_plan(const ddt_attn_args* a, int sms, int* qtiles, int* nsplit, int* tps) {
+  const int g = a->hq / a->hkv;
+  const long R = (long)a->n_max * g;
+  *qtiles = (int)((R + tc::BM - 1) / tc::BM);
+  const long base = (long)*qtiles * a->batch * a->hkv;
+  const int tiles = (a->max_ctx + tc::BN - 1) / tc::BN + (a->n_max + tc::BN - 1) / tc::BN;
+  int best = 1;
+  double best_eff = 0.0;
+  for (int s = 1; s <= 16 && s <= tiles; ++s) {
+    const long ctas = base * s;
+    const long waves = (ctas + sms - 1) / sms;
+    const double eff = (double)ctas / (double)(waves * sms);
+    if (eff > best_eff + 0.02) {
+      best_eff = eff;
+      best = s;
+    }
+  }
+  int t = (tiles + best - 1) / best;
+  *tps = t;
+  *nsplit = (tiles + t - 1) / t;
+}
+
+size_t attn_tc_workspace_size(const ddt_attn_args* a, int sms) {
+  int qt, ns, tps;
+  attn_tc_plan(a, sms, &qt, &ns, &tps);
+  if (ns <= 1) return 0;
+  const size_t rows = (size_t)a->batch * a->hkv * qt * ns * tc::BM;
+  return ((rows * tc::D * sizeof(float) + 255) & ~(size_t)255) + rows * sizeof(float2);
+}
+
+ddt_status launch_attn_tc(const ddt_attn_args* a, void* ws, int sms, cudaStream_t stream) {
+  using namespace tc;
+  Params p;
+  p.batch = a->batch;
+  p.n_max = a->n_max;
+  p.hq = a->hq;
+  p.hkv = a->hkv;
+  p.g = a->hq / a->hkv;
+  p.W = (a->n_max + 31) / 32;
+  p.max_ctx = a->max_ctx;
+  p.paged = a->page_table != nullptr;
+  p.page_size = a->page_size;
+  p.max_pages = a->max_pages;
+  p.rows_per_box = p.paged ? (a->page_size < 128 ? a->page_size : 128) : 128;
+  p.boxes_per_tile = 128 / p.rows_per_box;
+  p.t_max = a->t_max;
+  p.scale_log2 = a->scale * kLog2e;
+  p.ctx_len = a->ctx_len;
+  p.n_nodes = a->n_nodes;
+  p.mask = a->mask;
+  p.page_table = a->page_table;
+  p.out = (uint16_t*)a->out;
+  p.lse_out = a->lse_out;
+  p.status = a->dev_status;
+  attn_tc_plan(a, sms, &p.qtiles, &p.nsplit, &p.tiles_per_split);
+  if (p.nsplit > 1) {
+    const size_t rows = (size_t)a->batch * a->hkv * p.qtiles * p.nsplit * BM;
+    p.part_o = (float*)ws;
+    p.part_ml = (float2*)((char*)ws + ((rows * D * sizeof(float) + 255) & ~(size_t)255));
+  } else {
+    p.part_o = nullptr;
+    p.part_ml = nullptr;
+  }
+  const int g = p.g;
+  const cuuint64_t hkv = (cuuint64_t)a->hkv;
+  CUtensorMap mq, mk, mv, mkt, mvt;
+  {
+    cuuint64_t dims[3] = {D, (cuuint64_t)a->hq, (cuuint64_t)a->batch * a->n_max};
+    cuuint64_t str[2] = {D * 2, (cuuint64_t)a->hq * D * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)g, (cuuint32_t)(BM / g)};
+    if (!encode(&mq, a->q, 3, dims, str, box)) return DDT_ERR_CUDA;
+  }
+  {
+    cuuint64_t dims[3] = {D, hkv, (cuuint64_t)a->batch * a->n_max};
+    cuuint64_t str[2] = {D * 2, hkv * D * 2};
+    cuuint32_t box[3] = {64, 1, BN};
+    if (!encode(&mkt, a->k_tree, 3, dims, str, box)) return DDT_ERR_CUDA;
+    if (!encode(&mvt, a->v_tree, 3, dims, str, box)) return DDT_ERR_CUDA;
+  }
+  if (a->max_ctx > 0 && !p.paged) {
+    cuuint64_t dims[3] = {D, hkv, (cuuint64_t)a->batch * a->t_max};
+    cuuint64_t str[2] = {D * 2, hkv * D * 2};
+    cuuint32_t box[3] = {64, 1, BN};
+    if (!encode(&mk, a->k_cache, 3, dims, str, box)) return DDT_ERR_CUDA;
+    if (!encode(&mv, a->v_cache, 3, dims, str, box)) return DDT_ERR_CUDA;
+  } else if (a->max_ctx > 0) {
+    cuuint64_t dims[4] = {D, hkv, (cuuint64_t)a->page_size, (cuuint64_t)a->num_pages};
+    cuuint64_t str[3] = {D * 2, hkv * D * 2, (cuuint64_t)a->page_size * hkv * D * 2};
+    cuuint32_t box[4] = {64, 1, (cuuint32_t)p.rows_per_box, 1};
+    if (!encode(&mk, a->k_cache, 4, dims, str, box)) return DDT_ERR_CUDA;
+    if (!encode(&mv, a->v_cache, 4, dims, str, box)) return DDT_ERR_CUDA;
+  } else {
+    mk = mkt;  // no context: never read
+    mv = mvt;
+  }
+  const size_t smem = smem_bytes();
+  if (ensure_smem_attr((const void*)attn_tc_kernel, smem) != cudaSuccess) return DDT_ERR_CUDA;
+  dim3 grid(p.qtiles, p.nsplit, a->batch * a->hkv);
+  attn_tc_kernel<<<grid, kThreads, smem, stream>>>(mq, mk, mv, mkt, mvt, p);
+  if (cudaGetLastError() != cudaSuccess) return DDT_ERR_CUDA;
+  if (p.nsplit > 1) {
+    attn_tc_combine<<<dim3(p.qtiles * BM / 8, a->batch * a->hkv), 256, 0, stream>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return DDT_ERR_CUDA;
+  }
+  return DDT_OK;
+}
+
+}  // namespace ddt

@@ -1,6 +1,7 @@
 // common.cuh -- small device helpers shared by the libddt kernels.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 

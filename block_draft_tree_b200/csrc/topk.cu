@@ -114,11 +114,12 @@ __device__ void write_row(const TopkParams& p, int row, const uint64_t* s_top, f
 }
 
 template <bool BF16>
-__global__ void __launch_bounds__(kThreads) topk_kernel(TopkParams p) {
+__global__ void __launch_bounds__(kThreads, 3) topk_kernel(TopkParams p) {
   constexpr int EPV = BF16 ? 8 : 4;           // elements per 16-byte vector
   constexpr int EPT = kChunk / kThreads;      // 32 elements per thread
   constexpr int VPT = EPT / EPV;
   constexpr int ES = BF16 ? 2 : 4;
+  constexpr int NW = EPT * ES / 4;            // 32-bit words held per thread
 
   __shared__ uint64_t s_cand[kCandCap];
   __shared__ uint64_t s_top[DDT_TOPK_K_MAX];
@@ -131,74 +132,74 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkParams p) {
   const int64_t c0 = (int64_t)chunk * kChunk;
   const char* rowp = (const char*)p.logits + (int64_t)row * p.row_stride * ES;
 
-  // element e of vector j of this thread has index c0 + (j*kThreads + tid)*EPV + e
-  float x[EPT];
+  // word j of vector q of this thread holds elements starting at index
+  // c0 + (q*kThreads + tid)*EPV + j*(EPV/4); out-of-range elements read as -inf
+  uint32_t w[NW];
   const bool full = p.vec_ok && (c0 + kChunk <= p.V);
   if (full) {
-    uint4 v[VPT];
 #pragma unroll
-    for (int j = 0; j < VPT; ++j)
-      v[j] = ld_stream_v4(rowp + (c0 + (int64_t)(j * kThreads + tid) * EPV) * ES);
+    for (int q = 0; q < VPT; ++q) {
+      const uint4 v = ld_stream_v4(rowp + (c0 + (int64_t)(q * kThreads + tid) * EPV) * ES);
+      w[4 * q] = v.x;
+      w[4 * q + 1] = v.y;
+      w[4 * q + 2] = v.z;
+      w[4 * q + 3] = v.w;
+    }
+  } else {
 #pragma unroll
-    for (int j = 0; j < VPT; ++j) {
-      const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+    for (int q = 0; q < VPT; ++q)
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int j = 0; j < 4; ++j) {
+        const int64_t e0 = c0 + (int64_t)(q * kThreads + tid) * EPV + j * (EPV / 4);
         if (BF16) {
-          x[j * EPV + 2 * q] = bf16_lo(w[q]);
-          x[j * EPV + 2 * q + 1] = bf16_hi(w[q]);
+          const uint32_t lo = e0 < p.V ? ((const uint16_t*)rowp)[e0] : 0xFF80u;
+          const uint32_t hi = e0 + 1 < p.V ? ((const uint16_t*)rowp)[e0 + 1] : 0xFF80u;
+          w[4 * q + j] = lo | (hi << 16);
         } else {
-          x[j * EPV + q] = __uint_as_float(w[q]);
+          w[4 * q + j] = e0 < p.V ? __float_as_uint(((const float*)rowp)[e0]) : 0xFF800000u;
         }
       }
-    }
-  } else {
-#pragma unroll
-    for (int j = 0; j < VPT; ++j) {
-#pragma unroll
-      for (int e = 0; e < EPV; ++e) {
-        const int64_t idx = c0 + (int64_t)(j * kThreads + tid) * EPV + e;
-        float val = -INFINITY;
-        if (idx < p.V) {
-          if (BF16)
-            val = bf16_to_f32(((const uint16_t*)rowp)[idx]);
-          else
-            val = ((const float*)rowp)[idx];
-        }
-        x[j * EPV + e] = val;
-      }
-    }
   }
-  auto index_of = [&](int i) -> int64_t {
-    return c0 + (int64_t)((i / EPV) * kThreads + tid) * EPV + (i % EPV);
+  const int ibase = (int)c0 + tid * EPV;
+  auto index_of = [&](int e) -> int {  // element e (0..EPT) of this thread
+    return ibase + (e / EPV) * kThreads * EPV + (e % EPV);
   };
-  int nvalid = 0;
-  if (full) {
-    nvalid = EPT;
-  } else {
+  auto value_of = [&](int e) -> float {
+    if (BF16) return (e & 1) ? bf16_hi(w[e >> 1]) : bf16_lo(w[e >> 1]);
+    return __uint_as_float(w[e]);
+  };
+  int nvalid = EPT;
+  if (!full) {
+    nvalid = 0;
 #pragma unroll
-    for (int i = 0; i < EPT; ++i) nvalid += (index_of(i) < p.V);
+    for (int e = 0; e < EPT; ++e) nvalid += (index_of(e) < p.V);
   }
 
-  // thread max and thread sum of exp2((z - max) * c)
-  float m = -INFINITY;
+  // thread max (packed bf16 pairs where possible) and sum of exp2((z-max)*c)
+  float m;
+  if (BF16) {
+    __nv_bfloat162 m2 = *(const __nv_bfloat162*)&w[0];
 #pragma unroll
-  for (int i = 0; i < EPT; ++i) m = fmaxf(m, x[i]);
+    for (int j = 1; j < NW; ++j) m2 = __hmax2(m2, *(const __nv_bfloat162*)&w[j]);
+    m = fmaxf(__low2float(m2), __high2float(m2));
+  } else {
+    m = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < EPT; ++e) m = fmaxf(m, value_of(e));
+  }
   float s = 0.f;
   if (m != -INFINITY) {
     const float mc = m * p.c;
+    float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int i = 0; i < EPT; ++i) s += ex2(fmaf(x[i], p.c, -mc));
+    for (int e = 0; e < EPT; ++e) s4[e & 3] += ex2(fmaf(value_of(e), p.c, -mc));
+    s = (s4[0] + s4[1]) + (s4[2] + s4[3]);
   }
   // order key of the thread maximum (0: thread holds no element)
   uint32_t tk = 0;
   if (nvalid > 0) {
-    float mx = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < EPT; ++i)
-      if (full || index_of(i) < p.V) mx = fmaxf(mx, x[i]);
-    tk = BF16 ? ord16(__float_as_uint(mx) >> 16) : ord32(mx);
-    if (tk == 0) tk = 1;  // keep "holds an element" distinct from "holds none"
+    tk = BF16 ? ord16(__float_as_uint(m) >> 16) : ord32(m);
+    if (tk == 0) tk = 1;
   }
   if (tid == 0) s_count = 0;
 
@@ -212,16 +213,23 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkParams p) {
   }
   if (tau == 0) tau = 1;  // fewer than k threads hold elements: take them all
 
-  // candidates: elements whose order key reaches tau
+  // candidates: elements whose order key reaches tau; with a float threshold
+  // this is one compare per element (ties included, -0 == +0 as in the keys)
+  {
+    const uint32_t tb = BF16 ? (tau & 0xFFFFu) : tau;
+    const uint32_t tbits = BF16 ? (((tb & 0x8000u) ? (tb & 0x7FFFu) : (~tb & 0xFFFFu)) << 16)
+                                : ((tb & 0x80000000u) ? (tb & 0x7FFFFFFFu) : ~tb);
+    // keys below the key of -inf only come from the take-everything sentinel
+    const float tf = tb < (BF16 ? 0x7Fu : 0x007FFFFFu) ? -INFINITY : __uint_as_float(tbits);
 #pragma unroll
-  for (int i = 0; i < EPT; ++i) {
-    const int64_t idx = index_of(i);
-    if (!full && idx >= p.V) continue;
-    uint32_t ok = BF16 ? ord16(__float_as_uint(x[i]) >> 16) : ord32(x[i]);
-    if (ok == 0) ok = 1;
-    if (ok >= tau) {
-      const int pos = atomicAdd(&s_count, 1);
-      if (pos < kCandCap) s_cand[pos] = cand_key(x[i], (uint32_t)idx);
+    for (int e = 0; e < EPT; ++e) {
+      const float v = value_of(e);
+      if (v >= tf) {
+        const int idx = index_of(e);
+        if (!full && idx >= p.V) continue;
+        const int pos = atomicAdd(&s_count, 1);
+        if (pos < kCandCap) s_cand[pos] = cand_key(v, (uint32_t)idx);
+      }
     }
   }
   block_ms_reduce(m, s, p.c, s_wm, s_wsum);  // contains __syncthreads
@@ -234,10 +242,10 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkParams p) {
     for (int r = 0; r < p.k; ++r) {
       uint64_t best = 0;
 #pragma unroll
-      for (int i = 0; i < EPT; ++i) {
-        const int64_t idx = index_of(i);
+      for (int e = 0; e < EPT; ++e) {
+        const int idx = index_of(e);
         if (!full && idx >= p.V) continue;
-        const uint64_t key = cand_key(x[i], (uint32_t)idx);
+        const uint64_t key = cand_key(value_of(e), (uint32_t)idx);
         if (key < prev && key > best) best = key;
       }
       best = block_max_u64(best, s_red);
@@ -305,11 +313,7 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkParams p) {
   }
   __syncthreads();
   write_row(p, row, s_top, row_lse_up(p.inv_t, M, Ssum));
-  // leave the workspace as it was found: all zero
-  for (int i = tid; i < tot; i += kThreads) p.part_keys[(int64_t)row * tot + i] = 0ull;
-  for (int cc = tid; cc < p.S; cc += kThreads)
-    p.part_ms[(int64_t)row * p.S + cc] = make_float2(0.f, 0.f);
-  if (tid == 0) p.tickets[row] = 0u;
+  if (tid == 0) p.tickets[row] = 0u;  // the counter region is left zero
 }
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -319,7 +323,7 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 size_t topk_workspace_size(int rows, int V, int k) {
   const int S = (V + kChunk - 1) / kChunk;
   if (S <= 1) return 0;
-  return align256(sizeof(unsigned) * rows) + align256(sizeof(float2) * (size_t)rows * S) +
+  return (size_t)DDT_WS_COUNTER_BYTES + align256(sizeof(float2) * (size_t)rows * S) +
          align256(sizeof(uint64_t) * (size_t)rows * S * k);
 }
 
@@ -337,8 +341,8 @@ ddt_status launch_topk(const void* logits, ddt_dtype dt, int rows, int V, int64_
   const int es = dt == DDT_BF16 ? 2 : 4;
   p.vec_ok = ((uintptr_t)logits % 16 == 0) && ((row_stride * es) % 16 == 0);
   char* w = (char*)ws;
-  p.tickets = (unsigned*)w;
-  w += align256(sizeof(unsigned) * rows);
+  p.tickets = (unsigned*)w;  // counter region: one ticket per row
+  w += DDT_WS_COUNTER_BYTES;
   p.part_ms = (float2*)w;
   w += align256(sizeof(float2) * (size_t)rows * p.S);
   p.part_keys = (uint64_t*)w;

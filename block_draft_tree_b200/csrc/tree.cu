@@ -7,33 +7,45 @@
 // which is prefix-closed), 理論基礎 Propositions 1-2, and step 3 (compile
 // the tree into target inputs with an ancestor-only mask).
 //
-// One CTA per sequence.  Instead of popping a heap one node at a time, the
-// selection proceeds in frontier rounds that are exact:
-//   * every selected node p keeps n_next[p], the number of its children
-//     already selected; they are always ranks 0..n_next[p]-1 because
+// One CTA of 256 threads per sequence.  Selection proceeds in frontier
+// rounds instead of popping a heap one node at a time, and selects exactly
+// the same set:
+//   * every selected node x keeps n_next[x], the number of its children
+//     already selected; they are always ranks 0..n_next[x]-1 because
 //     siblings come in the candidate order, which is the total order K;
-//   * the unselected children of selected nodes (the frontier) are, per p,
-//     the run of ranks n_next[p]..k-1, sorted by K;
-//   * theta = the K-best child any frontier node could have (the first child
-//     of each run head).  Every frontier item that precedes theta under K
-//     precedes everything not yet generated, so all of them are among the
-//     best remaining prefixes and are selected together;
-//   * when they would overshoot the budget, the final round sorts them
-//     (bitonic, shared memory) and keeps the best.
+//   * the unselected children of selected nodes (the frontier) are, per x,
+//     the run of ranks n_next[x]..k-1, sorted by K;
+//   * each round lays the frontier items out in shared memory, one thread
+//     per item: theta = the K-best child any of them could have; every item
+//     that precedes theta precedes everything not yet generated, so all of
+//     them are among the best remaining prefixes and are selected together;
+//   * when they would overshoot the budget, the last round keeps the R best
+//     of them: histograms of their fp64 scores narrow the cut to one bin,
+//     whose few items are ranked exactly under K.
 // Each round selects at least the K-best frontier item, so the loop ends.
-// The selected set is then numbered breadth-first, level by level.
+// A frontier too large for the item buffer is truncated per run, and the
+// first item cut from each run joins theta, so truncation never lets a
+// worse prefix in ahead of a better one.  The selected set is then numbered
+// breadth-first, level by level, and the ancestor masks are built level by
+// level (in shared memory when they fit).
 //
-// Order K (best first): equal depth -> larger exact fp64 sum of raw logits,
-// then reverse-lexicographic token ids; different depths -> larger fp64
-// score inv_t*sum(z) - sum(lse), then the shallower prefix.
+// Order K (best first): equal depth -> larger fp64 sum of raw logits, then
+// reverse-lexicographic token ids; different depths -> larger fp64 score
+// inv_t*sum(z) - sum(lse), then the shallower prefix.
 #include "common.cuh"
 #include "launch.h"
 
 namespace ddt {
 namespace {
 
-constexpr int kThreads = 512;
-constexpr int kSafeCap = 4096;
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kBins = 256;        // histogram bins of the final-round cut
+constexpr int kExactMax = 16;     // boundary items ranked exactly
+constexpr int kMaxPasses = 4;     // histogram passes before ranking what is left
+constexpr int kItemCapMax = 10240;
+constexpr size_t kSmemMax = 227 * 1024;
+constexpr unsigned kFull = 0xFFFFFFFFu;
 
 struct TreeParams {
   const int32_t* ids;
@@ -43,7 +55,7 @@ struct TreeParams {
   double inv_t;
   const int32_t* k_per_seq;
   const int32_t* budget;
-  int B_max, n_max, W;
+  int B_max, n_max, W, icap;
   const int32_t* root_token;
   const int32_t* ctx_len;
   int32_t *tok, *parent, *depth, *pos;
@@ -54,20 +66,24 @@ struct TreeParams {
 };
 
 struct Smem {
-  float* zt;      // [L*k] raw logits of the candidates
-  int* tt;        // [L*k] candidate token ids
-  double* S;      // [L+1] prefix sums of lse
-  double* nsz;    // [n_max] node logit sums
-  double* nsc;    // [n_max] node scores
-  int* npar;      // [n_max] parent node (creation index)
-  int* ndep;      // [n_max]
-  int* nrank;     // [n_max] candidate rank at the node's own position
-  int* nnext;     // [n_max] selected-children count
-  int* ncnt;      // [n_max] round scratch: safe-item count / BFS index
-  int* noff;      // [n_max] round scratch: scan / first-child index
-  int* ninv;      // [n_max] BFS row -> node
-  uint32_t* safe; // [kSafeCap] final-round list (node << 8 | rank)
-  int L, k;
+  double* zt;       // [L*k] raw logits of the candidates
+  int* tt;          // [L*k] candidate token ids
+  double* S;        // [L+1] prefix sums of lse
+  double* nsz;      // [n_max] node logit sums
+  double* nsc;      // [n_max] node scores
+  int* npar;        // [n_max] parent node (creation index)
+  int* ndep;        // [n_max]
+  int* nrank;       // [n_max] candidate rank at the node's own position
+  int* nnext;       // [n_max] selected-children count
+  int* nlen;        // [n_max] items of the run this round / BFS row
+  int* noff;        // [n_max] offset of the run's items / first-child row
+  int* ninv;        // [n_max] BFS row -> node
+  uint32_t* iown;   // [icap] item: node << 8 | rank
+  double* isc;      // [icap] item score
+  int* iflag;       // [icap] item selected this round
+  int* ipos;        // [icap] scan of iflag
+  int* hist;        // [kBins]
+  int k;
 };
 
 // A prefix given as a selected node plus up to two appended ranks.
@@ -86,7 +102,7 @@ __device__ __forceinline__ int vp_token(const Smem& s, const VP& v, int t) {
 }
 
 // true iff a strictly precedes b under K.  depth < 0 marks "no prefix" (last).
-__device__ bool vp_before(const Smem& s, const VP& a, const VP& b) {
+__device__ __forceinline__ bool vp_before(const Smem& s, const VP& a, const VP& b) {
   if (b.depth < 0) return a.depth >= 0;
   if (a.depth < 0) return false;
   if (a.depth == b.depth) {
@@ -105,15 +121,30 @@ __device__ __forceinline__ double score_of(const Smem& s, double inv_t, double s
   return __dsub_rn(__dmul_rn(inv_t, sz), s.S[t]);
 }
 
-__device__ __forceinline__ VP make_item(const Smem& s, double inv_t, int p, int r) {
+// Frontier item (x, r): the child of node x with candidate rank r.
+__device__ __forceinline__ VP make_item(const Smem& s, double inv_t, int x, int r) {
   VP v;
-  v.base = p;
+  v.base = x;
   v.r1 = r;
   v.r2 = -1;
-  const int d = s.ndep[p];
+  const int d = s.ndep[x];
   v.depth = d + 1;
-  v.sz = __dadd_rn(s.nsz[p], (double)s.zt[d * s.k + r]);
+  v.sz = __dadd_rn(s.nsz[x], s.zt[d * s.k + r]);
   v.sc = score_of(s, inv_t, v.sz, v.depth);
+  return v;
+}
+
+// Item i of the item buffer (its score already computed).
+__device__ __forceinline__ VP item_vp(const Smem& s, int i) {
+  VP v;
+  const uint32_t e = s.iown[i];
+  v.base = (int)(e >> 8);
+  v.r1 = (int)(e & 0xFFu);
+  v.r2 = -1;
+  const int d = s.ndep[v.base];
+  v.depth = d + 1;
+  v.sz = __dadd_rn(s.nsz[v.base], s.zt[d * s.k + v.r1]);
+  v.sc = s.isc[i];
   return v;
 }
 
@@ -126,74 +157,269 @@ __device__ __forceinline__ VP no_vp() {
   return v;
 }
 
-__device__ VP shfl_vp(const VP& v, int o) {
+__device__ __forceinline__ VP shfl_vp(const VP& v, int o) {
   VP r;
-  r.sz = __shfl_xor_sync(0xFFFFFFFFu, v.sz, o);
-  r.sc = __shfl_xor_sync(0xFFFFFFFFu, v.sc, o);
-  r.depth = __shfl_xor_sync(0xFFFFFFFFu, v.depth, o);
-  r.base = __shfl_xor_sync(0xFFFFFFFFu, v.base, o);
-  r.r1 = __shfl_xor_sync(0xFFFFFFFFu, v.r1, o);
-  r.r2 = __shfl_xor_sync(0xFFFFFFFFu, v.r2, o);
+  r.sz = __shfl_xor_sync(kFull, v.sz, o);
+  r.sc = __shfl_xor_sync(kFull, v.sc, o);
+  r.depth = __shfl_xor_sync(kFull, v.depth, o);
+  r.base = __shfl_xor_sync(kFull, v.base, o);
+  r.r1 = __shfl_xor_sync(kFull, v.r1, o);
+  r.r2 = __shfl_xor_sync(kFull, v.r2, o);
   return r;
 }
 
-// K-best over the block.  Every thread gets the result.
+// K-best over the block; every thread gets the result.
 __device__ VP block_best(const Smem& s, VP v, VP* red) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll 1
+#pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
-    VP u = shfl_vp(v, o);
+    const VP u = shfl_vp(v, o);
     if (vp_before(s, u, v)) v = u;
   }
-  __syncthreads();
-  if (lane == 0) red[warp] = v;
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
   __syncthreads();
   VP b = red[0];
-  for (int w = 1; w < kThreads / 32; ++w)
+  for (int w = 1; w < kWarps; ++w)
     if (vp_before(s, red[w], b)) b = red[w];
+  __syncthreads();
   return b;
 }
 
-// Exclusive scan of a[0..n) in place (n <= 2*kThreads); returns the total.
-__device__ int block_exscan(int* a, int n, int* red) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int i0 = 2 * threadIdx.x;
-  const int v0 = i0 < n ? a[i0] : 0;
-  const int v1 = i0 + 1 < n ? a[i0 + 1] : 0;
-  const int t = v0 + v1;
-  int inc = t;
+__device__ __forceinline__ int warp_incl_scan(int v, int lane) {
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const int u = __shfl_up_sync(0xFFFFFFFFu, inc, o);
-    if (lane >= o) inc += u;
+    const int u = __shfl_up_sync(kFull, v, o);
+    if (lane >= o) v += u;
   }
-  __syncthreads();
+  return v;
+}
+
+// out[i] = in[0] + ... + in[i-1] for i < n (out may alias in); returns the
+// total.  Thread t scans the contiguous block [t*c, (t+1)*c).
+__device__ int block_exscan(const int* in, int* out, int n, int* red) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int c = (n + kThreads - 1) / kThreads;
+  const int lo = min(tid * c, n), hi = min(lo + c, n);
+  int sum = 0;
+  for (int i = lo; i < hi; ++i) sum += in[i];
+  const int inc = warp_incl_scan(sum, lane);
   if (lane == 31) red[warp] = inc;
   __syncthreads();
-  int wofs = 0, total = 0;
-  for (int w = 0; w < kThreads / 32; ++w) {
-    if (w < warp) wofs += red[w];
+  int before = 0, total = 0;
+  for (int w = 0; w < kWarps; ++w) {
+    before += (w < warp) ? red[w] : 0;
     total += red[w];
   }
-  const int ex = wofs + inc - t;
-  if (i0 < n) a[i0] = ex;
-  if (i0 + 1 < n) a[i0 + 1] = ex + v0;
+  int run = before + inc - sum;
+  for (int i = lo; i < hi; ++i) {
+    const int v = in[i];
+    out[i] = run;
+    run += v;
+  }
   __syncthreads();
   return total;
 }
 
+__device__ int block_sum(int v, int* red) {
+  v = __reduce_add_sync(kFull, v);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  int t = 0;
+  for (int w = 0; w < kWarps; ++w) t += red[w];
+  __syncthreads();
+  return t;
+}
+
+// One histogram pass of the final-round cut.
+struct Pass {
+  double lo, scale;
+  int bstar;
+};
+
+// Position of a score relative to the cut: 1 above it (kept), -1 below it
+// (dropped), 0 in the boundary bin of every pass so far.  Each pass bins
+// with the same arithmetic, so an item's state never depends on rounding
+// of a recomputed bin edge.
+__device__ __forceinline__ int cut_state(double sc, const Pass* ps, int np) {
+  for (int q = 0; q < np; ++q) {
+    int bin = (int)((sc - ps[q].lo) * ps[q].scale);
+    bin = min(max(bin, 0), kBins - 1);
+    if (bin > ps[q].bstar) return 1;
+    if (bin < ps[q].bstar) return -1;
+  }
+  return 0;
+}
+
+struct CutShared {
+  Pass ps[kMaxPasses];
+  int np, above, in_cut, nb;
+  double lo, hi;
+  int list[kBins];
+};
+
+// Final round: among the F items with iflag set (more than R of them), keep
+// the R K-best (iflag cleared on the others).  The kept items of a run are a
+// prefix of it, since a run is K-ordered.
+__device__ void keep_best(const Smem& s, int F, int R, CutShared* cs, double* dred, int* red,
+                          VP* vred) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  double lo = INFINITY, hi = -INFINITY;
+  int in_cut = 0;
+  for (int i = tid; i < F; i += kThreads)
+    if (s.iflag[i]) {
+      lo = fmin(lo, s.isc[i]);
+      hi = fmax(hi, s.isc[i]);
+      ++in_cut;
+    }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = fmin(lo, __shfl_xor_sync(kFull, lo, o));
+    hi = fmax(hi, __shfl_xor_sync(kFull, hi, o));
+  }
+  if (lane == 0) {
+    dred[warp] = lo;
+    dred[kWarps + warp] = hi;
+  }
+  in_cut = block_sum(in_cut, red);  // its barriers also publish dred
+  if (tid == 0) {
+    double l = INFINITY, h = -INFINITY;
+    for (int w = 0; w < kWarps; ++w) {
+      l = fmin(l, dred[w]);
+      h = fmax(h, dred[kWarps + w]);
+    }
+    cs->lo = l;
+    cs->hi = h;
+    cs->np = 0;
+    cs->above = 0;
+    cs->in_cut = in_cut;
+  }
+  __syncthreads();
+  // narrow the cut with score histograms
+  for (;;) {
+    const int np = cs->np;
+    if (np >= kMaxPasses || cs->in_cut <= kExactMax || !(cs->hi > cs->lo)) break;
+    for (int bn = tid; bn < kBins; bn += kThreads) s.hist[bn] = 0;
+    __syncthreads();
+    Pass pass;
+    pass.lo = cs->lo;
+    pass.scale = (double)kBins / (cs->hi - cs->lo);
+    for (int i = tid; i < F; i += kThreads) {
+      if (!s.iflag[i]) continue;
+      const double sc = s.isc[i];
+      if (cut_state(sc, cs->ps, np) != 0) continue;
+      atomicAdd(&s.hist[min(max((int)((sc - pass.lo) * pass.scale), 0), kBins - 1)], 1);
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // lane l holds bins [8l, 8l+8); find the bin holding the R-th best from the top
+      int h[8], lt = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        h[e] = s.hist[8 * lane + e];
+        lt += h[e];
+      }
+      int suf = lt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_down_sync(kFull, suf, o);
+        if (lane + o < 32) suf += u;
+      }
+      const int above_lane = cs->above + suf - lt;
+      const bool mine = above_lane < R && above_lane + lt >= R;
+      const unsigned who = __ballot_sync(kFull, mine);
+      const int src = who ? __ffs(who) - 1 : 0;
+      if (lane == src) {
+        int acc = above_lane, bs = 0, cnt = 0;
+        for (int e = 7; e >= 0; --e) {
+          if (acc + h[e] >= R) {
+            bs = 8 * lane + e;
+            cnt = h[e];
+            break;
+          }
+          acc += h[e];
+        }
+        pass.bstar = bs;
+        cs->ps[np] = pass;
+        cs->np = np + 1;
+        cs->above = acc;
+        cs->in_cut = cnt;
+        cs->lo = pass.lo + bs / pass.scale;
+        cs->hi = pass.lo + (bs + 1) / pass.scale;
+      }
+    }
+    __syncthreads();
+  }
+  const int np = cs->np;
+  const int need = R - cs->above;
+  // gather the boundary items
+  if (tid == 0) cs->nb = 0;
+  __syncthreads();
+  for (int i = tid; i < F; i += kThreads)
+    if (s.iflag[i] && cut_state(s.isc[i], cs->ps, np) == 0) {
+      const int q = atomicAdd(&cs->nb, 1);
+      if (q < kBins) cs->list[q] = i;
+    }
+  __syncthreads();
+  const int nb = cs->nb;
+  if (nb <= kBins) {
+    // rank each boundary item among them; keep the `need` best
+    for (int t = tid; t < nb; t += kThreads) {
+      const int i = cs->list[t];
+      const VP vi = item_vp(s, i);
+      int rank = 0;
+      for (int u = 0; u < nb; ++u)
+        if (u != t) rank += vp_before(s, item_vp(s, cs->list[u]), vi);
+      s.ipos[i] = rank < need;  // verdict for boundary items
+    }
+    __syncthreads();
+    for (int i = tid; i < F; i += kThreads)
+      if (s.iflag[i]) {
+        const int st = cut_state(s.isc[i], cs->ps, np);
+        s.iflag[i] = st == 1 || (st == 0 && s.ipos[i]);
+      }
+    __syncthreads();
+  } else {
+    // many exact score ties: take the K-best undecided boundary item, need times
+    for (int i = tid; i < F; i += kThreads)
+      if (s.iflag[i]) {
+        const int st = cut_state(s.isc[i], cs->ps, np);
+        s.iflag[i] = st == 1 ? 1 : (st == 0 ? 2 : 0);  // 2: boundary, undecided
+      }
+    __syncthreads();
+    for (int t = 0; t < need; ++t) {
+      VP best = no_vp();
+      int bi = -1;
+      for (int i = tid; i < F; i += kThreads)
+        if (s.iflag[i] == 2) {
+          const VP v = item_vp(s, i);
+          if (vp_before(s, v, best)) {
+            best = v;
+            bi = i;
+          }
+        }
+      const VP bb = block_best(s, best, vred);
+      if (bi >= 0 && bb.base == best.base && bb.r1 == best.r1 && bb.depth == best.depth)
+        s.iflag[bi] = 3;  // taken
+      __syncthreads();
+    }
+    for (int i = tid; i < F; i += kThreads) s.iflag[i] = (s.iflag[i] == 1 || s.iflag[i] == 3);
+    __syncthreads();
+  }
+}
+
 __global__ void __launch_bounds__(kThreads) build_tree_kernel(TreeParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  __shared__ VP s_red_vp[kThreads / 32];
-  __shared__ int s_red_i[kThreads / 32];
-  __shared__ double s_red_d[kThreads / 32];
   __shared__ int s_lvl[DDT_TREE_L_MAX + 2];
+  __shared__ int s_red[kWarps + 1];
+  __shared__ double s_dred[2 * kWarps];
+  __shared__ VP s_vred[kWarps];
+  __shared__ CutShared s_cut;
+  __shared__ int s_maxd;
 
-  const int b = blockIdx.x, tid = threadIdx.x;
-  const int L = p.L, k = p.k, NM = p.n_max;
+  const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int L = p.L, k = p.k, NM = p.n_max, icap = p.icap;
+  const double inv_t = p.inv_t;
 
   Smem s;
-  s.L = L;
   s.k = k;
   {
     unsigned char* q = smem_raw;
@@ -203,20 +429,23 @@ __global__ void __launch_bounds__(kThreads) build_tree_kernel(TreeParams p) {
       return r;
     };
     s.S = (double*)take(sizeof(double) * (L + 1));
+    s.zt = (double*)take(sizeof(double) * L * k);
     s.nsz = (double*)take(sizeof(double) * NM);
     s.nsc = (double*)take(sizeof(double) * NM);
-    s.zt = (float*)take(sizeof(float) * L * k);
+    s.isc = (double*)take(sizeof(double) * icap);
     s.tt = (int*)take(sizeof(int) * L * k);
     s.npar = (int*)take(sizeof(int) * NM);
     s.ndep = (int*)take(sizeof(int) * NM);
     s.nrank = (int*)take(sizeof(int) * NM);
     s.nnext = (int*)take(sizeof(int) * NM);
-    s.ncnt = (int*)take(sizeof(int) * NM);
+    s.nlen = (int*)take(sizeof(int) * NM);
     s.noff = (int*)take(sizeof(int) * NM);
     s.ninv = (int*)take(sizeof(int) * NM);
-    s.safe = (uint32_t*)take(sizeof(uint32_t) * kSafeCap);
+    s.iown = (uint32_t*)take(sizeof(uint32_t) * icap);
+    s.iflag = (int*)take(sizeof(int) * icap);
+    s.ipos = (int*)take(sizeof(int) * icap);
+    s.hist = (int*)take(sizeof(int) * kBins);
   }
-  const double inv_t = p.inv_t;
 
   // per-sequence candidate count and budget (clamped, flagged)
   int kb = p.k_per_seq ? p.k_per_seq[b] : k;
@@ -226,18 +455,19 @@ __global__ void __launch_bounds__(kThreads) build_tree_kernel(TreeParams p) {
     kb = min(max(kb, 1), k);
     Bb = min(max(Bb, 0), p.B_max);
   }
-
   for (int i = tid; i < L * k; i += kThreads) {
-    s.zt[i] = p.zk[(int64_t)b * L * k + i];
+    s.zt[i] = (double)p.zk[(int64_t)b * L * k + i];
     s.tt[i] = p.ids[(int64_t)b * L * k + i];
   }
-  if (tid == 0) {
+  if (tid == 32) {
     double acc = 0.0;
     s.S[0] = 0.0;
     for (int t = 1; t <= L; ++t) {
       acc = __dadd_rn(acc, (double)p.lse[(int64_t)b * L + t - 1]);
       s.S[t] = acc;
     }
+  }
+  if (tid == 0) {
     s.nsz[0] = 0.0;
     s.nsc[0] = 0.0;
     s.npar[0] = -1;
@@ -247,181 +477,125 @@ __global__ void __launch_bounds__(kThreads) build_tree_kernel(TreeParams p) {
   }
   __syncthreads();
 
-  int nn = 1;       // nodes including the root
-  int nsel = 0;     // draft nodes
-  // ---------------- frontier rounds ----------------
+  // ---------------- selection ----------------
+  int nn = 1, nsel = 0;
+  if (kb == 1) {
+    // one candidate per position: the tree is the chain of the first B positions
+    const int len = min(Bb, L);
+    for (int t = 1 + tid; t <= len; t += kThreads) {
+      double sz = 0.0;
+      for (int u = 0; u < t; ++u) sz = __dadd_rn(sz, s.zt[u * k]);
+      s.nsz[t] = sz;
+      s.nsc[t] = score_of(s, inv_t, sz, t);
+      s.npar[t] = t - 1;
+      s.ndep[t] = t;
+      s.nrank[t] = 0;
+      s.nnext[t] = t < len ? 1 : 0;
+    }
+    if (tid == 0) s.nnext[0] = len > 0 ? 1 : 0;
+    nn = 1 + len;
+    nsel = Bb;  // no other prefix exists
+    __syncthreads();
+  }
 #pragma unroll 1
   while (nsel < Bb) {
-    // theta: the K-best first child of any run head
+    // runs of this round, truncated to fit the item buffer
+    int tot = 0;
+    for (int x = tid; x < nn; x += kThreads) {
+      const int len = (s.ndep[x] < L) ? max(0, kb - s.nnext[x]) : 0;
+      s.nlen[x] = len;
+      tot += len;
+    }
+    tot = block_sum(tot, s_red);
+    if (tot == 0) break;
+    const int cap = tot <= icap ? DDT_TOPK_K_MAX : max(1, icap / nn);
     VP th = no_vp();
-    int has_head = 0;
-    for (int x = tid; x < nn; x += kThreads) {
-      const int d = s.ndep[x], r = s.nnext[x];
-      if (d < L && r < kb) {
-        has_head = 1;
-        if (d + 1 < L) {
-          VP c;
-          c.base = x;
-          c.r1 = r;
-          c.r2 = 0;
-          c.depth = d + 2;
-          c.sz = __dadd_rn(__dadd_rn(s.nsz[x], (double)s.zt[d * k + r]),
-                           (double)s.zt[(d + 1) * k + 0]);
-          c.sc = score_of(s, inv_t, c.sz, c.depth);
-          if (vp_before(s, c, th)) th = c;
-        }
-      }
-    }
-    if (!__syncthreads_or(has_head)) break;
-    th = block_best(s, th, s_red_vp);
-
-    // safe items per run: ranks n_next[x].. that precede theta
-    for (int x = tid; x < nn; x += kThreads) {
-      const int d = s.ndep[x];
-      int c = 0;
-      if (d < L) {
-        for (int r = s.nnext[x]; r < kb; ++r) {
-          if (!vp_before(s, make_item(s, inv_t, x, r), th)) break;
-          ++c;
-        }
-      }
-      s.ncnt[x] = c;
-      s.noff[x] = c;
-    }
-    __syncthreads();
-    int total = block_exscan(s.noff, nn, s_red_i);
-    const int R = Bb - nsel;
-    if (total == 0) {
-      // Only reachable when a candidate scores above its parent (inputs whose
-      // lse is below some inv_t*z): take the K-best run head so that every
-      // round selects something and the loop ends.
-      VP best = no_vp();
-      int bx = -1;
-      for (int x = tid; x < nn; x += kThreads)
-        if (s.ndep[x] < L && s.nnext[x] < kb) {
-          const VP v = make_item(s, inv_t, x, s.nnext[x]);
-          if (vp_before(s, v, best)) best = v;
-        }
-      best = block_best(s, best, s_red_vp);
-      bx = best.base;
+    if (tot > icap) {
       for (int x = tid; x < nn; x += kThreads) {
-        s.ncnt[x] = (x == bx) ? 1 : 0;
-        s.noff[x] = (x == bx) ? 1 : 0;
+        const int len = s.nlen[x];
+        if (len > cap) {  // the first item cut from the run bounds the round too
+          const VP v = make_item(s, inv_t, x, s.nnext[x] + cap);
+          if (vp_before(s, v, th)) th = v;
+          s.nlen[x] = cap;
+        }
       }
       __syncthreads();
-      total = block_exscan(s.noff, nn, s_red_i);
+    }
+    const int F = block_exscan(s.nlen, s.noff, nn, s_red);
+    for (int x = tid; x < nn; x += kThreads) {
+      const int o = s.noff[x], r0 = s.nnext[x], len = s.nlen[x];
+      for (int i = 0; i < len; ++i) s.iown[o + i] = ((uint32_t)x << 8) | (uint32_t)(r0 + i);
+    }
+    __syncthreads();
+    // item scores; theta = the K-best first child of any item
+    for (int i = tid; i < F; i += kThreads) {
+      const uint32_t e = s.iown[i];
+      const int x = (int)(e >> 8), r = (int)(e & 0xFFu);
+      const int d = s.ndep[x];
+      const double sz = __dadd_rn(s.nsz[x], s.zt[d * k + r]);
+      s.isc[i] = score_of(s, inv_t, sz, d + 1);
+      if (d + 1 < L) {
+        VP c;
+        c.base = x;
+        c.r1 = r;
+        c.r2 = 0;
+        c.depth = d + 2;
+        c.sz = __dadd_rn(sz, s.zt[(d + 1) * k]);
+        c.sc = score_of(s, inv_t, c.sz, c.depth);
+        if (vp_before(s, c, th)) th = c;
+      }
+    }
+    th = block_best(s, th, s_vred);
+    // safe items: those that precede theta
+    for (int i = tid; i < F; i += kThreads) s.iflag[i] = vp_before(s, item_vp(s, i), th);
+    __syncthreads();
+    int T = block_exscan(s.iflag, s.ipos, F, s_red);
+    if (T == 0) {
+      // Only reachable when a candidate scores above its parent (an lse below
+      // some inv_t*z): take the K-best item so that the loop progresses.
+      VP best = no_vp();
+      for (int i = tid; i < F; i += kThreads) {
+        const VP v = item_vp(s, i);
+        if (vp_before(s, v, best)) best = v;
+      }
+      best = block_best(s, best, s_vred);
+      for (int i = tid; i < F; i += kThreads) {
+        const uint32_t e = s.iown[i];
+        s.iflag[i] = (int)(e >> 8) == best.base && (int)(e & 0xFFu) == best.r1;
+      }
+      __syncthreads();
+      T = block_exscan(s.iflag, s.ipos, F, s_red);
       if (tid == 0) raise_status(p.status, DDT_ERR_INVALID_ARG);
     }
-    if (total <= R) {
-      for (int x = tid; x < nn; x += kThreads) {
-        const int c = s.ncnt[x];
-        const int r0 = s.nnext[x];
-        for (int i = 0; i < c; ++i) {
-          const int id = nn + s.noff[x] + i;
-          const VP v = make_item(s, inv_t, x, r0 + i);
-          s.nsz[id] = v.sz;
-          s.nsc[id] = v.sc;
-          s.npar[id] = x;
-          s.ndep[id] = v.depth;
-          s.nrank[id] = r0 + i;
-          s.nnext[id] = 0;
-        }
-      }
-      __syncthreads();
-      for (int x = tid; x < nn; x += kThreads) s.nnext[x] += s.ncnt[x];
-      __syncthreads();
-      nn += total;
-      nsel += total;
-      continue;
+    const int R = Bb - nsel;
+    const bool last = T >= R;
+    if (T > R) {
+      keep_best(s, F, R, &s_cut, s_dred, s_red, s_vred);
+      T = block_exscan(s.iflag, s.ipos, F, s_red);
     }
-
-    // final round: keep the R K-best safe items
-    for (int x = tid; x < nn; x += kThreads) {
-      const int c = min(s.ncnt[x], R);
-      s.noff[x] = c;
-    }
-    __syncthreads();
-    const int m = block_exscan(s.noff, nn, s_red_i);
-    if (m <= kSafeCap) {
-      int npow = 1;
-      while (npow < m) npow <<= 1;
-      for (int x = tid; x < nn; x += kThreads) {
-        const int c = min(s.ncnt[x], R);
-        for (int i = 0; i < c; ++i) s.safe[s.noff[x] + i] = ((uint32_t)x << 8) | (uint32_t)(s.nnext[x] + i);
-      }
-      for (int i = m + tid; i < npow; i += kThreads) s.safe[i] = 0xFFFFFFFFu;
-      __syncthreads();
-      auto item = [&](uint32_t e) -> VP {
-        if (e == 0xFFFFFFFFu) return no_vp();
-        return make_item(s, inv_t, (int)(e >> 8), (int)(e & 0xFF));
-      };
-      for (int size = 2; size <= npow; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-          for (int i = tid; i < npow / 2; i += kThreads) {
-            const int lo = 2 * i - (i & (stride - 1));
-            const int hi = lo + stride;
-            const bool up = (lo & size) == 0;
-            const uint32_t ea = s.safe[lo], eb = s.safe[hi];
-            const VP va = item(ea), vb = item(eb);
-            const bool sw = up ? vp_before(s, vb, va) : vp_before(s, va, vb);
-            if (sw) {
-              s.safe[lo] = eb;
-              s.safe[hi] = ea;
-            }
-          }
-          __syncthreads();
-        }
-      }
-      for (int i = tid; i < R; i += kThreads) {
-        const uint32_t e = s.safe[i];
-        const int x = (int)(e >> 8), r = (int)(e & 0xFF);
-        const VP v = make_item(s, inv_t, x, r);
-        const int id = nn + i;
-        s.nsz[id] = v.sz;
-        s.nsc[id] = v.sc;
+    // create the selected items as nodes
+    for (int i = tid; i < F; i += kThreads)
+      if (s.iflag[i]) {
+        const uint32_t e = s.iown[i];
+        const int x = (int)(e >> 8), r = (int)(e & 0xFFu);
+        const int id = nn + s.ipos[i];
+        const int d = s.ndep[x];
+        s.nsz[id] = __dadd_rn(s.nsz[x], s.zt[d * k + r]);
+        s.nsc[id] = s.isc[i];
         s.npar[id] = x;
-        s.ndep[id] = v.depth;
+        s.ndep[id] = d + 1;
         s.nrank[id] = r;
         s.nnext[id] = 0;
+        atomicAdd(&s.nnext[x], 1);
       }
-      __syncthreads();
-      for (int i = tid; i < R; i += kThreads) {
-        const uint32_t e = s.safe[i];
-        atomicMax(&s.nnext[e >> 8], (int)(e & 0xFF) + 1);
-      }
-      __syncthreads();
-    } else {
-      // very large final round: take the K-best safe head, R times
-      for (int x = tid; x < nn; x += kThreads) s.noff[x] = 0;  // taken per run
-      __syncthreads();
-      for (int i = 0; i < R; ++i) {
-        VP best = no_vp();
-        for (int x = tid; x < nn; x += kThreads)
-          if (s.noff[x] < s.ncnt[x]) {
-            const VP v = make_item(s, inv_t, x, s.nnext[x]);
-            if (vp_before(s, v, best)) best = v;
-          }
-        best = block_best(s, best, s_red_vp);
-        if (tid == 0) {
-          const int id = nn + i;
-          s.nsz[id] = best.sz;
-          s.nsc[id] = best.sc;
-          s.npar[id] = best.base;
-          s.ndep[id] = best.depth;
-          s.nrank[id] = best.r1;
-          s.nnext[id] = 0;
-          s.nnext[best.base] += 1;
-          s.noff[best.base] += 1;
-        }
-        __syncthreads();
-      }
-    }
-    nn += R;
-    nsel += R;
-    break;
+    __syncthreads();
+    nn += T;
+    nsel += T;
+    if (last) break;
   }
 
   // ---------------- breadth-first numbering ----------------
+  // nlen[x] <- row of x, ninv[row] <- x, noff[x] <- row of x's first child
   if (tid < DDT_TREE_L_MAX + 2) s_lvl[tid] = 0;
   __syncthreads();
   int maxd = 0;
@@ -429,44 +603,39 @@ __global__ void __launch_bounds__(kThreads) build_tree_kernel(TreeParams p) {
     atomicAdd(&s_lvl[s.ndep[x]], 1);
     maxd = max(maxd, s.ndep[x]);
   }
+  maxd = __reduce_max_sync(kFull, maxd);
+  if (lane == 0) s_red[warp] = maxd;
   __syncthreads();
-  if (tid == 0) {  // s_lvl[t] <- number of nodes of depth < t
+  if (tid == 0) {  // s_lvl[t] <- number of nodes of depth < t (= first row of depth t)
     int acc = 0;
     for (int t = 0; t <= L + 1; ++t) {
       const int c = s_lvl[t];
       s_lvl[t] = acc;
       acc += c;
     }
-  }
-  maxd = __reduce_max_sync(0xFFFFFFFFu, maxd);
-  if ((tid & 31) == 0) s_red_i[tid >> 5] = maxd;
-  __syncthreads();
-  maxd = 0;
-  for (int w = 0; w < kThreads / 32; ++w) maxd = max(maxd, s_red_i[w]);
-  __syncthreads();
-  if (tid == 0) {
-    s.ncnt[0] = 0;   // BFS index of the root
-    s.noff[0] = 1;   // first child of the root
+    int md = 0;
+    for (int w = 0; w < kWarps; ++w) md = max(md, s_red[w]);
+    s_maxd = md;
+    s.nlen[0] = 0;
+    s.noff[0] = 1;
     s.ninv[0] = 0;
   }
   __syncthreads();
-  for (int t = 1; t <= maxd; ++t) {
+  const int md = s_maxd;
+  for (int t = 1; t <= md; ++t) {
     const int lstart = s_lvl[t], lend = s_lvl[t + 1];
-    // BFS index of level-t nodes; stage their child counts in BFS order
     for (int x = tid; x < nn; x += kThreads)
       if (s.ndep[x] == t) {
         const int j = s.noff[s.npar[x]] + s.nrank[x];
-        s.ncnt[x] = j;
+        s.nlen[x] = j;
         s.ninv[j] = x;
       }
     __syncthreads();
-    // first-child index of each level-t node: exclusive scan of child counts
-    int* tmp = (int*)s.safe;
-    for (int j = lstart + tid; j < lend; j += kThreads) tmp[j - lstart] = s.nnext[s.ninv[j]];
+    // first-child rows of level t: lend + exclusive scan of child counts
+    for (int j = lstart + tid; j < lend; j += kThreads) s.iflag[j - lstart] = s.nnext[s.ninv[j]];
     __syncthreads();
-    // levels can exceed 2*kThreads rows only when n_max > 1024 (not allowed)
-    block_exscan(tmp, lend - lstart, s_red_i);
-    for (int j = lstart + tid; j < lend; j += kThreads) s.noff[s.ninv[j]] = lend + tmp[j - lstart];
+    block_exscan(s.iflag, s.ipos, lend - lstart, s_red);
+    for (int j = lstart + tid; j < lend; j += kThreads) s.noff[s.ninv[j]] = lend + s.ipos[j - lstart];
     __syncthreads();
   }
 
@@ -481,7 +650,7 @@ __global__ void __launch_bounds__(kThreads) build_tree_kernel(TreeParams p) {
       const int x = s.ninv[j];
       const int d = s.ndep[x];
       o_tok[j] = x == 0 ? p.root_token[b] : s.tt[(d - 1) * k + s.nrank[x]];
-      o_par[j] = x == 0 ? -1 : s.ncnt[s.npar[x]];
+      o_par[j] = x == 0 ? -1 : s.nlen[s.npar[x]];
       o_dep[j] = d;
       o_pos[j] = ctx + d;
     } else {
@@ -491,39 +660,60 @@ __global__ void __launch_bounds__(kThreads) build_tree_kernel(TreeParams p) {
       o_pos[j] = -1;
     }
   }
+  // ancestor-or-self masks, level by level: row j = row(parent j) | bit j,
+  // staged in the (now free) item buffer when it holds them
   const int W = p.W;
   uint32_t* o_mask = p.mask + (int64_t)b * NM * W;
-  for (int i = tid; i < NM * W; i += kThreads) {
-    const int j = i / W, w = i - j * W;
-    uint32_t word = 0;
-    if (j < nn && w <= (j >> 5)) {
-      for (int x = s.ninv[j]; x >= 0; x = s.npar[x]) {
-        const int a = s.ncnt[x];
-        if (a < 32 * w) break;
-        if ((a >> 5) == w) word |= 1u << (a & 31);
-      }
+  const bool staged = (int64_t)nn * W <= 2 * (int64_t)icap;
+  uint32_t* m = staged ? (uint32_t*)s.isc : o_mask;
+  for (int i = tid; i < (staged ? nn * W : NM * W); i += kThreads) m[i] = (i == 0) ? 1u : 0u;
+  __syncthreads();
+  for (int t = 1; t <= md; ++t) {
+    const int lstart = s_lvl[t], lend = s_lvl[t + 1];
+    for (int i = tid; i < (lend - lstart) * W; i += kThreads) {
+      const int j = lstart + i / W, w = i % W;
+      uint32_t word = m[(int64_t)s.nlen[s.npar[s.ninv[j]]] * W + w];
+      if ((j >> 5) == w) word |= 1u << (j & 31);
+      m[(int64_t)j * W + w] = word;
     }
-    o_mask[i] = word;
+    __syncthreads();
   }
+  if (staged)
+    for (int i = tid; i < NM * W; i += kThreads) o_mask[i] = i < nn * W ? m[i] : 0u;
   // surrogate: sum of exp(score) over the draft nodes
   double acc = 0.0;
   for (int x = 1 + tid; x < nn; x += kThreads) acc += exp(s.nsc[x]);
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
-  if ((tid & 31) == 0) s_red_d[tid >> 5] = acc;
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
+  if (lane == 0) s_dred[warp] = acc;
   __syncthreads();
   if (tid == 0) {
     double t = 0.0;
-    for (int w = 0; w < kThreads / 32; ++w) t += s_red_d[w];
+    for (int w = 0; w < kWarps; ++w) t += s_dred[w];
     p.n_nodes[b] = nn;
     if (p.surrogate) p.surrogate[b] = t;
   }
 }
 
-size_t tree_smem_bytes(int L, int k, int n_max) {
+size_t tree_smem_bytes(int L, int k, int n_max, int icap) {
   auto a = [](size_t x) { return (x + 15) & ~(size_t)15; };
-  return a(sizeof(double) * (L + 1)) + 2 * a(sizeof(double) * n_max) + a(sizeof(float) * L * k) +
-         a(sizeof(int) * L * k) + 7 * a(sizeof(int) * n_max) + a(sizeof(uint32_t) * kSafeCap);
+  return a(sizeof(double) * (L + 1)) + a(sizeof(double) * L * k) + 2 * a(sizeof(double) * n_max) +
+         a(sizeof(double) * icap) + a(sizeof(int) * L * k) + 7 * a(sizeof(int) * n_max) +
+         3 * a(sizeof(int) * icap) + a(sizeof(int) * kBins);
+}
+
+// Item buffer: the biggest frontier (n_max*k items), within the shared
+// memory left by everything else; never fewer than n_max items (a truncated
+// round keeps at least one item per run).
+int item_cap(int L, int k, int n_max) {
+  int cap = n_max * k;
+  if (cap > kItemCapMax) cap = kItemCapMax;
+  if (cap < n_max) cap = n_max;
+  const size_t fixed = tree_smem_bytes(L, k, n_max, 0) + 4 * 16;
+  const size_t per_item = sizeof(double) + 3 * sizeof(int);
+  const int fit = (int)((kSmemMax - 4096 - fixed) / per_item);
+  if (cap > fit) cap = fit;
+  return cap;
 }
 
 }  // namespace
@@ -546,6 +736,7 @@ ddt_status launch_build_tree(const int32_t* ids, const float* zk, const float* l
   p.B_max = B_max;
   p.n_max = B_max + 1;
   p.W = (p.n_max + 31) / 32;
+  p.icap = item_cap(L, k, p.n_max);
   p.root_token = root_token;
   p.ctx_len = ctx_len;
   p.tok = tok;
@@ -557,7 +748,7 @@ ddt_status launch_build_tree(const int32_t* ids, const float* zk, const float* l
   p.surrogate = surrogate;
   p.status = dev_status;
   if (batch == 0) return DDT_OK;
-  const size_t smem = tree_smem_bytes(L, k, p.n_max);
+  const size_t smem = tree_smem_bytes(L, k, p.n_max, p.icap);
   if (ensure_smem_attr((const void*)build_tree_kernel, smem) != cudaSuccess) return DDT_ERR_CUDA;
   build_tree_kernel<<<batch, kThreads, smem, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? DDT_OK : DDT_ERR_CUDA;

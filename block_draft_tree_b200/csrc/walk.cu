@@ -14,7 +14,8 @@
 //     (value, then smaller id);
 //   * the last CTA of a row (atomic ticket) merges the chunk keys into the
 //     row's argmax; the last row of a sequence to finish (a second ticket)
-//     runs the walk with one warp, reading the argmaxes back from L2.
+//     stages the sequence's argmaxes and tree in shared memory with one
+//     coalesced pass and walks it with one warp.
 // No CTA ever waits on another, so there is no spin and nothing to time out.
 #include "common.cuh"
 #include "launch.h"
@@ -52,20 +53,20 @@ __device__ __forceinline__ uint64_t block_max_key(uint64_t v, uint64_t* sm) {
   return r;
 }
 
-__device__ void walk_sequence(const WalkParams& p, int b, int n) {
+// One warp walks sequence b with its argmaxes and tree staged in shared memory.
+__device__ void walk_sequence(const WalkParams& p, int b, int n, const int* s_amax, const int* s_tok,
+                              const int* s_par, const int* s_dep) {
   const int lane = threadIdx.x & 31;
-  const int32_t* tok = p.tok + (int64_t)b * p.n_max;
-  const int32_t* par = p.parent + (int64_t)b * p.n_max;
-  const int32_t* dep = p.depth + (int64_t)b * p.n_max;
   int x = 0, a = 0, bonus = 0;
 #pragma unroll 1
   for (;;) {
-    const int t = __ldcg(&p.amax[(int64_t)b * p.n_max + x]);
+    const int t = s_amax[x];
     int next = -1;
-    if (a < p.L && dep[x] < p.L) {
+    if (a < p.L && s_dep[x] < p.L) {
+      // children of x come after x (rows are breadth-first)
       for (int c0 = x + 1; c0 < n; c0 += 32) {
         const int c = c0 + lane;
-        const bool hit = c < n && par[c] == x && tok[c] == t;
+        const bool hit = c < n && s_par[c] == x && s_tok[c] == t;
         const unsigned bal = __ballot_sync(0xFFFFFFFFu, hit);
         if (bal) {
           next = c0 + __ffs(bal) - 1;
@@ -95,13 +96,52 @@ __device__ void walk_sequence(const WalkParams& p, int b, int n) {
 }
 
 template <bool BF16>
+struct Chunk {
+  static constexpr int EPV = BF16 ? 8 : 4;
+  static constexpr int VPT = kChunk / kThreads / EPV;
+  uint4 v[VPT];
+};
+
+// Issue the loads of one (row, chunk) item (full chunks only).
+template <bool BF16>
+__device__ __forceinline__ void load_chunk(Chunk<BF16>& c, const char* rowp, int64_t c0) {
+  constexpr int EPV = Chunk<BF16>::EPV, ES = BF16 ? 2 : 4;
+#pragma unroll
+  for (int q = 0; q < Chunk<BF16>::VPT; ++q)
+    c.v[q] = ld_stream_v4(rowp + (c0 + (int64_t)(q * kThreads + threadIdx.x) * EPV) * ES);
+}
+
+// Thread-local argmax of a loaded chunk; each thread sees its indices in
+// increasing order, so strict > keeps the smallest index among equal values.
+template <bool BF16>
+__device__ __forceinline__ void argmax_chunk(const Chunk<BF16>& c, int c0, float& bv, int& bi) {
+  constexpr int EPV = Chunk<BF16>::EPV;
+#pragma unroll
+  for (int q = 0; q < Chunk<BF16>::VPT; ++q) {
+    const int base = c0 + (q * kThreads + (int)threadIdx.x) * EPV;
+    const uint32_t w[4] = {c.v[q].x, c.v[q].y, c.v[q].z, c.v[q].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (BF16) {
+        const float lo = bf16_lo(w[e]), hi = bf16_hi(w[e]);
+        if (lo > bv || bi < 0) { bv = lo; bi = base + 2 * e; }
+        if (hi > bv) { bv = hi; bi = base + 2 * e + 1; }
+      } else {
+        const float f = __uint_as_float(w[e]);
+        if (f > bv || bi < 0) { bv = f; bi = base + e; }
+      }
+    }
+  }
+}
+
+template <bool BF16>
 __global__ void __launch_bounds__(kThreads) walk_kernel(WalkParams p) {
-  constexpr int EPV = BF16 ? 8 : 4;
-  constexpr int EPT = kChunk / kThreads;
-  constexpr int VPT = EPT / EPV;
+  constexpr int EPV = Chunk<BF16>::EPV;
   constexpr int ES = BF16 ? 2 : 4;
   __shared__ uint64_t s_red[kThreads / 32];
   __shared__ int s_flag;
+  __shared__ int s_amax[DDT_TREE_B_MAX + 1], s_tok[DDT_TREE_B_MAX + 1];
+  __shared__ int s_par[DDT_TREE_B_MAX + 1], s_dep[DDT_TREE_B_MAX + 1];
 
   const int chunk = blockIdx.x, j = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x;
@@ -113,48 +153,28 @@ __global__ void __launch_bounds__(kThreads) walk_kernel(WalkParams p) {
   if (j >= n) return;
   const int64_t row = (int64_t)b * p.n_max + j;
   const char* rowp = (const char*)p.logits + row * p.row_stride * ES;
-  const int64_t c0 = (int64_t)chunk * kChunk;
+  const int c0 = chunk * kChunk;
 
-  // thread-local argmax; each thread sees its indices in increasing order
   float bv = -INFINITY;
   int bi = -1;
   if (p.vec_ok && c0 + kChunk <= p.V) {
-    uint4 v[VPT];
-#pragma unroll
-    for (int q = 0; q < VPT; ++q)
-      v[q] = ld_stream_v4(rowp + (c0 + (int64_t)(q * kThreads + tid) * EPV) * ES);
-#pragma unroll
-    for (int q = 0; q < VPT; ++q) {
-      const int base = (int)(c0 + (q * kThreads + tid) * EPV);
-      const uint32_t w[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        if (BF16) {
-          const float lo = bf16_lo(w[e]), hi = bf16_hi(w[e]);
-          if (lo > bv || bi < 0) { bv = lo; bi = base + 2 * e; }
-          if (hi > bv) { bv = hi; bi = base + 2 * e + 1; }
-        } else {
-          const float f = __uint_as_float(w[e]);
-          if (f > bv || bi < 0) { bv = f; bi = base + e; }
-        }
-      }
-    }
+    Chunk<BF16> cur;
+    load_chunk<BF16>(cur, rowp, c0);
+    argmax_chunk<BF16>(cur, c0, bv, bi);
   } else {
-    for (int q = 0; q < VPT; ++q)
+    for (int q = 0; q < Chunk<BF16>::VPT; ++q)
       for (int e = 0; e < EPV; ++e) {
-        const int64_t idx = c0 + (int64_t)(q * kThreads + tid) * EPV + e;
+        const int idx = c0 + (q * kThreads + tid) * EPV + e;
         if (idx >= p.V) continue;
         const float f = BF16 ? bf16_to_f32(((const uint16_t*)rowp)[idx]) : ((const float*)rowp)[idx];
-        if (f > bv || bi < 0) { bv = f; bi = (int)idx; }
+        if (f > bv || bi < 0) { bv = f; bi = idx; }
       }
   }
   uint64_t key = bi < 0 ? 0ull : cand_key(bv, (uint32_t)bi);
   key = block_max_key(key, s_red);
 
-  bool row_done = false;
   if (p.S == 1) {
     if (tid == 0) p.amax[row] = (int32_t)key_id(key);
-    row_done = true;
   } else {
     if (tid == 0) {
       p.part[row * p.S + chunk] = key;
@@ -162,24 +182,21 @@ __global__ void __launch_bounds__(kThreads) walk_kernel(WalkParams p) {
       s_flag = (atomicAdd(&p.row_ticket[row], 1u) == (unsigned)(p.S - 1));
     }
     __syncthreads();
-    if (s_flag) {
-      __threadfence();
-      uint64_t m = 0;
-      for (int c = tid; c < p.S; c += kThreads) {
-        const uint64_t u = ld_cg_u64(&p.part[row * p.S + c]);
-        m = u > m ? u : m;
-      }
-      __syncthreads();
-      m = block_max_key(m, s_red);
-      for (int c = tid; c < p.S; c += kThreads) p.part[row * p.S + c] = 0ull;
-      if (tid == 0) {
-        p.amax[row] = (int32_t)key_id(m);
-        p.row_ticket[row] = 0u;
-      }
-      row_done = true;
+    if (!s_flag) return;
+    __threadfence();
+    uint64_t m = 0;
+    for (int c = tid; c < p.S; c += kThreads) {
+      const uint64_t u = ld_cg_u64(&p.part[row * p.S + c]);
+      m = u > m ? u : m;
+    }
+    __syncthreads();
+    m = block_max_key(m, s_red);
+    if (tid == 0) {
+      p.amax[row] = (int32_t)key_id(m);
+      p.row_ticket[row] = 0u;  // the counter region is left zero
     }
   }
-  if (!row_done) return;
+  // the row is done; the last row of the sequence walks it
   if (tid == 0) {
     __threadfence();
     s_flag = (atomicAdd(&p.seq_count[b], 1u) == (unsigned)(n - 1));
@@ -187,11 +204,15 @@ __global__ void __launch_bounds__(kThreads) walk_kernel(WalkParams p) {
   __syncthreads();
   if (!s_flag) return;
   __threadfence();
-  if (tid < 32) walk_sequence(p, b, n);
+  for (int r = tid; r < n; r += kThreads) {
+    s_amax[r] = __ldcg(&p.amax[(int64_t)b * p.n_max + r]);
+    s_tok[r] = p.tok[(int64_t)b * p.n_max + r];
+    s_par[r] = p.parent[(int64_t)b * p.n_max + r];
+    s_dep[r] = p.depth[(int64_t)b * p.n_max + r];
+  }
   __syncthreads();
-  // leave the workspace as it was found: all zero
-  for (int r = tid; r < n; r += kThreads) p.amax[(int64_t)b * p.n_max + r] = 0;
-  if (tid == 0) p.seq_count[b] = 0u;
+  if (tid < 32) walk_sequence(p, b, n, s_amax, s_tok, s_par, s_dep);
+  if (tid == 0) p.seq_count[b] = 0u;  // the counter region is left zero
 }
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -201,8 +222,8 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 size_t walk_workspace_size(int batch, int n_max, int V) {
   const int S = (V + kChunk - 1) / kChunk;
   const size_t rows = (size_t)batch * n_max;
-  return align256(sizeof(unsigned) * rows) + align256(sizeof(unsigned) * batch) +
-         align256(sizeof(int32_t) * rows) + align256(sizeof(uint64_t) * rows * S);
+  return (size_t)DDT_WS_COUNTER_BYTES + align256(sizeof(int32_t) * rows) +
+         align256(sizeof(uint64_t) * rows * S);
 }
 
 ddt_status launch_tree_walk(const void* logits, ddt_dtype dt, int batch, int n_max, int V,
@@ -231,10 +252,9 @@ ddt_status launch_tree_walk(const void* logits, ddt_dtype dt, int batch, int n_m
   p.status = dev_status;
   const size_t rows = (size_t)batch * n_max;
   char* w = (char*)ws;
-  p.row_ticket = (unsigned*)w;
-  w += align256(sizeof(unsigned) * rows);
-  p.seq_count = (unsigned*)w;
-  w += align256(sizeof(unsigned) * batch);
+  p.row_ticket = (unsigned*)w;  // counter region: rows tickets, then batch counters
+  p.seq_count = (unsigned*)w + rows;
+  w += DDT_WS_COUNTER_BYTES;
   p.amax = (int32_t*)w;
   w += align256(sizeof(int32_t) * rows);
   p.part = (uint64_t*)w;

@@ -19,10 +19,12 @@
  *   - Every tensor pointer is a DEVICE pointer owned by the caller.  The
  *     library allocates no device memory; scratch comes from a caller-owned
  *     workspace sized by the matching *_workspace_size() function.
- *   - A workspace must be zero-filled before its first use.  Every call that
- *     returns DDT_OK leaves it zero-filled again when its kernels finish, so
- *     it can be reused by the next call on the same stream.  Calls that
- *     share one workspace must not overlap on the GPU.
+ *   - Every workspace starts with a counter region of DDT_WS_COUNTER_BYTES
+ *     that must be zero-filled before the workspace's first use; every call
+ *     that returns DDT_OK leaves it zero again when its kernels finish.  The
+ *     rest of a workspace may hold anything.  One workspace can therefore
+ *     serve calls of any stage and shape one after another on one stream;
+ *     calls that share a workspace must not overlap on the GPU.
  *   - Calls are asynchronous on `stream` and perform no host synchronisation,
  *     so they can be captured into a CUDA graph.
  *   - Arguments are validated on the host before any launch: an invalid
@@ -57,6 +59,9 @@ typedef enum ddt_status {
 } ddt_status;
 
 typedef enum ddt_dtype { DDT_BF16 = 0, DDT_F32 = 1 } ddt_dtype;
+
+/* Size of the counter region at the start of every workspace. */
+#define DDT_WS_COUNTER_BYTES (256u << 10)
 
 /* Implementation limits. */
 #define DDT_TOPK_K_MAX 32     /* candidates per position */
@@ -186,6 +191,9 @@ ddt_status ddt_build_tree(const int32_t* ids, const float* zk, const float* lse,
  *           a ctx_len above it is clamped and flagged in dev_status.
  * Limits: d in {64, 128}; hq % hkv == 0; n_max <= 1024; all base pointers
  * 16-byte aligned; page_size a multiple of 16.
+ * Paths: d = 128 with (hq/hkv) dividing 128, at least 64 query rows per kv
+ * head and (paged) num_pages > 0 with page_size dividing 128 or a multiple of
+ * 128 runs on the tensor cores (tcgen05, TMA); everything else on CUDA cores.
  * ------------------------------------------------------------------------ */
 typedef struct ddt_attn_args {
   const void* q;
@@ -194,6 +202,7 @@ typedef struct ddt_attn_args {
   const int32_t* page_table; /* NULL: dense cache */
   int page_size;
   int max_pages;
+  int num_pages;             /* paged: pages in the pool (bounds the page loads); 0 = unknown */
   int64_t t_max;             /* dense: tokens per sequence in k_cache/v_cache */
   const int32_t* ctx_len;
   int max_ctx;
