@@ -61,7 +61,8 @@ struct Params {
   float* lse_out;
   int32_t* status;
   int nsplit, tiles_per_split, qtiles;
-  float* part_o;    // [grp][qtile][split][BM][D]
+  int cluster;      // the splits of a query tile form a cluster and merge on chip
+  float* part_o;    // [grp][qtile][split][BM][D] (split partials without a cluster)
   float2* part_ml;  // [grp][qtile][split][BM]
 };
 
@@ -188,6 +189,37 @@ __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// Distributed shared memory of the cluster (the KV splits of one query tile).
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ float2 ld_cluster_f2(uint32_t addr) {
+  float2 v;
+  asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)m) : "memory");
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version bits.
 __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
   uint64_t d = 0;
@@ -257,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int ntiles = t_hi - t_lo;
   const int64_t part_row0 = (((int64_t)grp * p.qtiles + qtile) * p.nsplit + split) * BM;
 
-  if (ntiles == 0) {  // nothing in this split: an empty partial (or zero rows)
+  if (ntiles == 0 && !p.cluster) {  // nothing in this split: an empty partial (or zero rows)
     if (tid >= 64) {
       const int row = tid - 64;
       const int qr = q0 + row;
@@ -275,7 +307,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
 
-  if (tid == 0) {
+  const bool work = ntiles > 0;
+  if (work && tid == 0) {
     mbar_init(&bars->q_full, 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars->kv_full[s], 1);
@@ -288,7 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bars->abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 0) {
+  if (work && warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(&bars->tmem_base)),
                  "r"(kTmemCols)
@@ -300,9 +333,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   fence_after();
   const uint32_t tmem = bars->tmem_base;
 
-  if (warp == 0) {
+  if (!work) {
+    // an empty split of a cluster: nothing to compute, an empty partial below
+  } else if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      prefetch_tmap(&tm_kt);
+      prefetch_tmap(&tm_vt);
       const int j0 = q0 / g;
       mbar_expect_tx(&bars->q_full, (uint32_t)kTile);
       tma_load_3d(sQ, &tm_q, 0, kvh * g, b * p.n_max + j0, &bars->q_full);
@@ -503,8 +543,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->pv_done, (uint32_t)(ntiles - 1) & 1u, bars));
     fence_after();
-    // epilogue: O row -> partial or final output
-    float* po = p.part_o + (part_row0 + row) * D;
+    // epilogue: O row -> final output, a cluster partial in shared memory,
+    // or a partial in the workspace
+    float* po = p.cluster ? (float*)(sK) + row * D : p.part_o + (part_row0 + row) * D;
     const bool final_out = p.nsplit == 1;
     const float inv = (l > 0.f) ? 1.f / l : 0.f;
     uint16_t* dst = nullptr;
@@ -539,7 +580,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     const bool has = ok && row_valid && l > 0.f;
-    if (!final_out) {
+    if (p.cluster) {
+      ((float2*)(sK + BM * D * 4))[row] = has ? make_float2(m_used, l) : make_float2(-INFINITY, 0.f);
+    } else if (!final_out) {
       p.part_ml[part_row0 + row] = has ? make_float2(m_used, l) : make_float2(-INFINITY, 0.f);
     } else if (dst && p.lse_out) {
       p.lse_out[((int64_t)b * p.n_max + j) * p.hq + (kvh * g + qr % g)] =
@@ -547,15 +590,72 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  if (!work && tid >= 64)  // empty split of a cluster
+    ((float2*)(sK + BM * D * 4))[tid - 64] = make_float2(-INFINITY, 0.f);
+
   fence_before();
   __syncthreads();
-  if (bars->abort && tid == 0) raise_status(p.status, DDT_ERR_TIMEOUT);
-  if (warp == 0) {
+  if (work && bars->abort && tid == 0) raise_status(p.status, DDT_ERR_TIMEOUT);
+  if (work && warp == 0) {
     __syncwarp();
     fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
                  : "memory");
   }
+  if (!p.cluster) return;
+
+  // ---------------- on-chip merge of the cluster's split partials ----------------
+  // CTA r of the cluster owns query rows [r*rpc, (r+1)*rpc) of the tile; each
+  // warp takes one row at a time, a lane 4 of its 128 dims, and loads every
+  // split's (m, l) and O slice from the peers' shared memory in one go.
+  cluster_sync();
+  {
+    const int S = p.nsplit;  // 2..8
+    const int rank = (int)cluster_rank();
+    const int rpc = (BM + S - 1) / S;
+    const uint32_t o_base = smem_u32(sK), ml_base = smem_u32(sK + BM * D * 4);
+    for (int r = rank * rpc + warp; r < min(BM, (rank + 1) * rpc); r += kThreads / 32) {
+      const int qr2 = q0 + r;
+      if (qr2 >= R) break;
+      const int j2 = qr2 / g, h2 = kvh * g + qr2 % g;
+      // every split's (m, l) and O slice, loaded together
+      float2 ml[8];
+      float4 v[8];
+#pragma unroll
+      for (int s2 = 0; s2 < 8; ++s2)
+        if (s2 < S) {
+          ml[s2] = ld_cluster_f2(map_to_rank(ml_base + r * 8, s2));
+          v[s2] = ld_cluster_f4(map_to_rank(o_base + (r * D + 4 * lane) * 4, s2));
+        }
+      float M = -INFINITY;
+#pragma unroll
+      for (int s2 = 0; s2 < 8; ++s2)
+        if (s2 < S) M = fmaxf(M, ml[s2].x);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      float Lsum = 0.f;
+      if (M != -INFINITY && j2 < n) {
+#pragma unroll
+        for (int s2 = 0; s2 < 8; ++s2)
+          if (s2 < S && ml[s2].x != -INFINITY) {
+            const float wgt = ex2(ml[s2].x - M);
+            Lsum += ml[s2].y * wgt;
+            acc.x = fmaf(wgt, v[s2].x, acc.x);
+            acc.y = fmaf(wgt, v[s2].y, acc.y);
+            acc.z = fmaf(wgt, v[s2].z, acc.z);
+            acc.w = fmaf(wgt, v[s2].w, acc.w);
+          }
+      }
+      const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+      __nv_bfloat162 h0 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+      __nv_bfloat162 h1 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+      uint2* dst2 = (uint2*)(p.out + (((int64_t)b * p.n_max + j2) * p.hq + h2) * D);
+      dst2[lane] = make_uint2(*(uint32_t*)&h0, *(uint32_t*)&h1);
+      if (lane == 0 && p.lse_out)
+        p.lse_out[((int64_t)b * p.n_max + j2) * p.hq + h2] =
+            Lsum > 0.f ? (M + __log2f(Lsum)) * 0.69314718055994531f : -INFINITY;
+    }
+  }
+  cluster_sync();  // peers' shared memory stays alive until every CTA has read it
 }
 
 // Merge the per-split partials: one warp per query row, 4 dims per lane.
@@ -574,21 +674,45 @@ __global__ void __launch_bounds__(256) attn_tc_combine(const Params p) {
   const int j = qr / g, h = kvh * g + qr % g;
   const int64_t base = (((int64_t)grp * p.qtiles + qtile) * p.nsplit) * BM + r;
   float M = -INFINITY;
-  for (int s = 0; s < p.nsplit; ++s) M = fmaxf(M, p.part_ml[base + (int64_t)s * BM].x);
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float L = 0.f;
-  if (M != -INFINITY && j < n) {
-    for (int s = 0; s < p.nsplit; ++s) {
-      const float2 ml = p.part_ml[base + (int64_t)s * BM];
-      if (ml.x == -INFINITY) continue;
-      const float w = ex2(ml.x - M);
-      L += ml.y * w;
-      const float4 v = ((const float4*)(p.part_o + (base + (int64_t)s * BM) * D))[lane];
-      acc.x = fmaf(w, v.x, acc.x);
-      acc.y = fmaf(w, v.y, acc.y);
-      acc.z = fmaf(w, v.z, acc.z);
-      acc.w = fmaf(w, v.w, acc.w);
-    }
+  // splits in groups of 8, each group's (m, l) and O slices loaded together
+  for (int s0 = 0; s0 < p.nsplit; s0 += 8) {
+    float2 ml[8];
+    float4 v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if (s0 + e < p.nsplit) {
+        ml[e] = p.part_ml[base + (int64_t)(s0 + e) * BM];
+        v[e] = ((const float4*)(p.part_o + (base + (int64_t)(s0 + e) * BM) * D))[lane];
+      } else {
+        ml[e] = make_float2(-INFINITY, 0.f);
+      }
+    float Mg = M;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) Mg = fmaxf(Mg, ml[e].x);
+    if (Mg == -INFINITY) continue;
+    const float rescale = M == -INFINITY ? 0.f : ex2(M - Mg);
+    L *= rescale;
+    acc.x *= rescale;
+    acc.y *= rescale;
+    acc.z *= rescale;
+    acc.w *= rescale;
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if (ml[e].x != -INFINITY) {
+        const float w = ex2(ml[e].x - Mg);
+        L += ml[e].y * w;
+        acc.x = fmaf(w, v[e].x, acc.x);
+        acc.y = fmaf(w, v[e].y, acc.y);
+        acc.z = fmaf(w, v[e].z, acc.z);
+        acc.w = fmaf(w, v[e].w, acc.w);
+      }
+    M = Mg;
+  }
+  if (j >= n) {
+    L = 0.f;
+    acc = make_float4(0.f, 0.f, 0.f, 0.f);
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
   __nv_bfloat162 h0 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
@@ -666,10 +790,44 @@ void attn_tc_plan(const ddt_attn_args* a, int sms, int* qtiles, int* nsplit, int
   *nsplit = (tiles + t - 1) / t;
 }
 
+// Can the KV splits of one query tile run as a thread-block cluster (and
+// merge on chip)?  Up to 8 splits (the portable cluster size), when the
+// device can co-schedule such a cluster of these CTAs.
+bool attn_tc_cluster(int nsplit, long clusters) {
+  if (nsplit < 2 || nsplit > 8) return false;
+  static std::mutex mu;
+  static int known[9] = {0};  // co-resident clusters of each size; -1: none
+  std::lock_guard<std::mutex> lock(mu);
+  if (known[nsplit] == 0) {
+    bool ok = ensure_smem_attr((const void*)tc::attn_tc_kernel, tc::smem_bytes()) == cudaSuccess;
+    if (ok) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(1, nsplit, 1);
+      cfg.blockDim = dim3(tc::kThreads, 1, 1);
+      cfg.dynamicSmemBytes = tc::smem_bytes();
+      cudaLaunchAttribute attr;
+      attr.id = cudaLaunchAttributeClusterDimension;
+      attr.val.clusterDim.x = 1;
+      attr.val.clusterDim.y = nsplit;
+      attr.val.clusterDim.z = 1;
+      cfg.attrs = &attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      ok = cudaOccupancyMaxActiveClusters(&n, (void*)tc::attn_tc_kernel, &cfg) == cudaSuccess && n > 0;
+      known[nsplit] = ok ? n : -1;
+    } else {
+      known[nsplit] = -1;
+    }
+    cudaGetLastError();  // a failed query must not leave a sticky error behind
+  }
+  // only when every cluster of the launch runs in the first wave
+  return known[nsplit] > 0 && clusters <= known[nsplit];
+}
+
 size_t attn_tc_workspace_size(const ddt_attn_args* a, int sms) {
   int qt, ns, tps;
   attn_tc_plan(a, sms, &qt, &ns, &tps);
-  if (ns <= 1) return 0;
+  if (ns <= 1 || attn_tc_cluster(ns, (long)qt * a->batch * a->hkv)) return 0;
   const size_t rows = (size_t)a->batch * a->hkv * qt * ns * tc::BM;
   return ((rows * tc::D * sizeof(float) + 255) & ~(size_t)255) + rows * sizeof(float2);
 }
@@ -699,7 +857,8 @@ ddt_status launch_attn_tc(const ddt_attn_args* a, void* ws, int sms, cudaStream_
   p.lse_out = a->lse_out;
   p.status = a->dev_status;
   attn_tc_plan(a, sms, &p.qtiles, &p.nsplit, &p.tiles_per_split);
-  if (p.nsplit > 1) {
+  p.cluster = attn_tc_cluster(p.nsplit, (long)p.qtiles * a->batch * a->hkv) ? 1 : 0;
+  if (p.nsplit > 1 && !p.cluster) {
     const size_t rows = (size_t)a->batch * a->hkv * p.qtiles * p.nsplit * BM;
     p.part_o = (float*)ws;
     p.part_ml = (float2*)((char*)ws + ((rows * D * sizeof(float) + 255) & ~(size_t)255));
@@ -742,6 +901,23 @@ ddt_status launch_attn_tc(const ddt_attn_args* a, void* ws, int sms, cudaStream_
   const size_t smem = smem_bytes();
   if (ensure_smem_attr((const void*)attn_tc_kernel, smem) != cudaSuccess) return DDT_ERR_CUDA;
   dim3 grid(p.qtiles, p.nsplit, a->batch * a->hkv);
+  if (p.cluster) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 1;
+    attr.val.clusterDim.y = p.nsplit;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, attn_tc_kernel, mq, mk, mv, mkt, mvt, p) != cudaSuccess)
+      return DDT_ERR_CUDA;
+    return DDT_OK;
+  }
   attn_tc_kernel<<<grid, kThreads, smem, stream>>>(mq, mk, mv, mkt, mvt, p);
   if (cudaGetLastError() != cudaSuccess) return DDT_ERR_CUDA;
   if (p.nsplit > 1) {
