@@ -7,31 +7,32 @@
 // which is prefix-closed), 理論基礎 Propositions 1-2, and step 3 (compile
 // the tree into target inputs with an ancestor-only mask).
 //
-// One CTA of 256 threads per sequence.  Selection proceeds in frontier
-// rounds instead of popping a heap one node at a time, and selects exactly
-// the same set:
-//   * every selected node x keeps n_next[x], the number of its children
-//     already selected; they are always ranks 0..n_next[x]-1 because
-//     siblings come in the candidate order, which is the total order K;
-//   * the unselected children of selected nodes (the frontier) are, per x,
-//     the run of ranks n_next[x]..k-1, sorted by K;
-//   * each round lays the frontier items out in shared memory, one thread
-//     per item: theta = the K-best child any of them could have; every item
-//     that precedes theta precedes everything not yet generated, so all of
-//     them are among the best remaining prefixes and are selected together;
-//   * when they would overshoot the budget, the last round keeps the R best
-//     of them: histograms of their fp64 scores narrow the cut to one bin,
-//     whose few items are ranked exactly under K.
-// Each round selects at least the K-best frontier item, so the loop ends.
-// A frontier too large for the item buffer is truncated per run, and the
-// first item cut from each run joins theta, so truncation never lets a
-// worse prefix in ahead of a better one.  The selected set is then numbered
-// breadth-first, level by level, and the ancestor masks are built level by
-// level (in shared memory when they fit).
-//
 // Order K (best first): equal depth -> larger fp64 sum of raw logits, then
 // reverse-lexicographic token ids; different depths -> larger fp64 score
-// inv_t*sum(z) - sum(lse), then the shallower prefix.
+// inv_t*sum(z) - sum(lse), then the shallower prefix.  At equal depth the
+// score is a monotone function of the sum, so K is the lexicographic order
+// on (score desc, depth asc, sum desc, reversed tokens); comparisons use the
+// score as a 64-bit integer key and fall back to the rest only on equal keys.
+//
+// One CTA of 256 threads per sequence; thread t owns nodes t, t+256, ...
+// Selection runs in frontier rounds and selects exactly the set a one-node-
+// at-a-time best-first search would:
+//   * every selected node x keeps nnext[x], its selected-children count; they
+//     are ranks 0..nnext[x]-1, since siblings come in candidate order, which
+//     is K (the candidates of a position are sorted by logit, then id);
+//   * the frontier is, per node, the run of ranks nnext[x]..k-1; the best
+//     prefix not in any run is the first child of some run head, so
+//     theta = the K-best run-head first child bounds everything ungenerated;
+//   * every run item that precedes theta is among the best remaining
+//     prefixes: each node counts its run's items before theta, one scan
+//     numbers them, and they are created together (three barriers a round);
+//   * when they overshoot the budget, the R best are kept by a radix select
+//     on their score keys (8 bits a pass), exact ties ranked under K.
+// Each round selects at least the best run head, so the loop ends.
+// Breadth-first rows are then the order of (depth, rank path): each node
+// carries its path of candidate ranks as a packed key and its row is its
+// rank by key within its depth, so no level-by-level pass is needed; the
+// ancestor masks follow the parent rows.
 #include "common.cuh"
 #include "launch.h"
 
@@ -40,10 +41,9 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kBins = 256;        // histogram bins of the final-round cut
-constexpr int kExactMax = 16;     // boundary items ranked exactly
-constexpr int kMaxPasses = 4;     // histogram passes before ranking what is left
-constexpr int kItemCapMax = 10240;
+constexpr int kBins = 256;           // radix-select digit
+constexpr int kTieList = 256;        // exact ties ranked by counting
+constexpr int kItemCapMax = 16384;
 constexpr size_t kSmemMax = 227 * 1024;
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
@@ -55,7 +55,7 @@ struct TreeParams {
   double inv_t;
   const int32_t* k_per_seq;
   const int32_t* budget;
-  int B_max, n_max, W, icap;
+  int B_max, n_max, W, icap, kw, rb;
   const int32_t* root_token;
   const int32_t* ctx_len;
   int32_t *tok, *parent, *depth, *pos;
@@ -66,27 +66,65 @@ struct TreeParams {
 };
 
 struct Smem {
-  double* zt;       // [L*k] raw logits of the candidates
-  int* tt;          // [L*k] candidate token ids
-  double* S;        // [L+1] prefix sums of lse
-  double* nsz;      // [n_max] node logit sums
-  double* nsc;      // [n_max] node scores
-  int* npar;        // [n_max] parent node (creation index)
-  int* ndep;        // [n_max]
-  int* nrank;       // [n_max] candidate rank at the node's own position
-  int* nnext;       // [n_max] selected-children count
-  int* nlen;        // [n_max] items of the run this round / BFS row
-  int* noff;        // [n_max] offset of the run's items / first-child row
-  int* ninv;        // [n_max] BFS row -> node
-  uint32_t* iown;   // [icap] item: node << 8 | rank
-  double* isc;      // [icap] item score
-  int* iflag;       // [icap] item selected this round
-  int* ipos;        // [icap] scan of iflag
-  int* hist;        // [kBins]
-  int k;
+  double* zt;      // [L*k] raw logits of the candidates
+  double* S;       // [L+1] prefix sums of lse
+  double* nsz;     // [n_max] node logit sums
+  double* nsc;     // [n_max] node scores
+  int* tt;         // [L*k] candidate token ids
+  int* npar;       // [n_max] parent node (creation index)
+  int* ndep;       // [n_max]
+  int* nrank;      // [n_max] candidate rank at the node's own position
+  int* nnext;      // [n_max] selected-children count
+  int* nrow;       // [n_max] breadth-first row of a node
+  int* ninv;       // [n_max] row -> node; also the depth buckets
+  int* prow;       // [n_max] row -> parent row
+  uint64_t* pkey;  // [n_max*kw] rank path, most significant word first
+  uint64_t* nrk;   // [n_max] reversed id-rank path (own position first), top 64 bits
+  int* idr;        // [L*k] rank of each candidate's token id within its position
+  uint64_t* ckey;  // [icap] cut candidates: score key
+  uint32_t* cid;   // [icap] cut candidates: node << 8 | rank, bit 31 = kept
+  int k, kw, rb;
 };
 
-// A prefix given as a selected node plus up to two appended ranks.
+// A prefix under the order K in integer form (see pk_before).
+struct PK {
+  uint64_t sk, rk;
+  double sz;
+  int dep;
+  uint32_t h;
+};
+
+// Shared scratch of the reductions, scans and the cut.
+struct Red {
+  uint64_t wkey[kWarps];
+  uint32_t wid[kWarps];
+  int wtie[kWarps];
+  int wsum[kWarps];
+  uint64_t wmn[kWarps], wmx[kWarps];
+  double wd[kWarps];
+  PK wpk[kWarps];
+  double csz[kTieList];
+  uint64_t crk[kTieList];
+  int cdep[kTieList];
+  uint32_t chd[kTieList];
+  int hist[2][kBins];
+  int digit, above, hcount, nlist;
+  int list[kTieList];
+  int lvl[DDT_TREE_L_MAX + 2];
+};
+
+// fp64 score as an integer key: larger score <-> larger key; -0 == +0.
+__device__ __forceinline__ uint64_t score_key(double sc) {
+  uint64_t u = (uint64_t)__double_as_longlong(sc);
+  if ((u << 1) == 0) u = 0;
+  return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
+}
+
+__device__ __forceinline__ double score_of(const Smem& s, double inv_t, double sz, int t) {
+  return __dsub_rn(__dmul_rn(inv_t, sz), s.S[t]);
+}
+
+// A prefix given as a selected node plus one or two appended ranks.
 struct VP {
   double sz, sc;
   int depth, base, r1, r2;
@@ -101,10 +139,8 @@ __device__ __forceinline__ int vp_token(const Smem& s, const VP& v, int t) {
   return s.tt[(t - 1) * s.k + s.nrank[x]];
 }
 
-// true iff a strictly precedes b under K.  depth < 0 marks "no prefix" (last).
+// true iff a strictly precedes b under K (full comparison).
 __device__ __forceinline__ bool vp_before(const Smem& s, const VP& a, const VP& b) {
-  if (b.depth < 0) return a.depth >= 0;
-  if (a.depth < 0) return false;
   if (a.depth == b.depth) {
     if (a.sz != b.sz) return a.sz > b.sz;
     for (int t = a.depth; t >= 1; --t) {
@@ -117,70 +153,195 @@ __device__ __forceinline__ bool vp_before(const Smem& s, const VP& a, const VP& 
   return a.depth < b.depth;
 }
 
-__device__ __forceinline__ double score_of(const Smem& s, double inv_t, double sz, int t) {
-  return __dsub_rn(__dmul_rn(inv_t, sz), s.S[t]);
+// Packed prefix handle: node << 16 | r1 << 8 | (r2 + 1); r2 = -1 is an item
+// (one appended rank), r2 = 0 a run head's first child.
+__device__ __forceinline__ uint32_t pack_vp(int x, int r1, int r2) {
+  return ((uint32_t)x << 16) | ((uint32_t)r1 << 8) | (uint32_t)(r2 + 1);
 }
 
-// Frontier item (x, r): the child of node x with candidate rank r.
-__device__ __forceinline__ VP make_item(const Smem& s, double inv_t, int x, int r) {
+__device__ __forceinline__ VP unpack_vp(const Smem& s, double inv_t, uint32_t h) {
   VP v;
-  v.base = x;
-  v.r1 = r;
-  v.r2 = -1;
-  const int d = s.ndep[x];
+  v.base = (int)(h >> 16);
+  v.r1 = (int)((h >> 8) & 0xFFu);
+  v.r2 = (int)(h & 0xFFu) - 1;
+  const int d = s.ndep[v.base];
+  v.sz = __dadd_rn(s.nsz[v.base], s.zt[d * s.k + v.r1]);
   v.depth = d + 1;
-  v.sz = __dadd_rn(s.nsz[x], s.zt[d * s.k + r]);
+  if (v.r2 >= 0) {
+    v.sz = __dadd_rn(v.sz, s.zt[(d + 1) * s.k + v.r2]);
+    v.depth = d + 2;
+  }
   v.sc = score_of(s, inv_t, v.sz, v.depth);
   return v;
 }
 
-// Item i of the item buffer (its score already computed).
-__device__ __forceinline__ VP item_vp(const Smem& s, int i) {
-  VP v;
-  const uint32_t e = s.iown[i];
-  v.base = (int)(e >> 8);
-  v.r1 = (int)(e & 0xFFu);
-  v.r2 = -1;
-  const int d = s.ndep[v.base];
-  v.depth = d + 1;
-  v.sz = __dadd_rn(s.nsz[v.base], s.zt[d * s.k + v.r1]);
-  v.sc = s.isc[i];
-  return v;
+// The CTA's shared-memory layout, published once for the out-of-line full
+// comparison, so that its call sites pass two handles and nothing else.
+__shared__ Smem g_layout;
+__shared__ double g_inv_t;
+
+// Full comparison of two prefix handles (only equal score keys get here).
+__device__ __noinline__ bool slow_before(uint32_t ha, uint32_t hb) {
+  const Smem s = g_layout;
+  const double inv_t = g_inv_t;
+  return vp_before(s, unpack_vp(s, inv_t, ha), unpack_vp(s, inv_t, hb));
 }
 
-__device__ __forceinline__ VP no_vp() {
-  VP v;
-  v.sz = v.sc = 0.0;
-  v.depth = -1;
-  v.base = 0;
-  v.r1 = v.r2 = -1;
-  return v;
+__device__ __forceinline__ bool handle_before(const Smem&, double, uint32_t ha, uint32_t hb) {
+  return slow_before(ha, hb);
 }
 
-__device__ __forceinline__ VP shfl_vp(const VP& v, int o) {
-  VP r;
-  r.sz = __shfl_xor_sync(kFull, v.sz, o);
-  r.sc = __shfl_xor_sync(kFull, v.sc, o);
-  r.depth = __shfl_xor_sync(kFull, v.depth, o);
-  r.base = __shfl_xor_sync(kFull, v.base, o);
-  r.r1 = __shfl_xor_sync(kFull, v.r1, o);
-  r.r2 = __shfl_xor_sync(kFull, v.r2, o);
-  return r;
+// (ka, ha) strictly before (kb, hb); key 0 means "none" (last).
+__device__ __forceinline__ bool key_before(const Smem& s, double inv_t, uint64_t ka, uint32_t ha,
+                                           uint64_t kb, uint32_t hb) {
+  if (ka != kb) return ka > kb;
+  if (ka == 0 || ha == hb) return false;
+  return handle_before(s, inv_t, ha, hb);
 }
 
-// K-best over the block; every thread gets the result.
-__device__ VP block_best(const Smem& s, VP v, VP* red) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const VP u = shfl_vp(v, o);
-    if (vp_before(s, u, v)) v = u;
+// The order K as integers: (score key desc, depth asc, logit sum desc,
+// reversed id-rank path asc).  Within a position, token order is id-rank
+// order, so the reversed path compares like the reversed token ids; it keeps
+// the deepest 64 bits, and only prefixes that agree on all of them go to the
+// out-of-line comparison.
+__device__ __forceinline__ uint64_t rev_key(const Smem& s, uint64_t parent_rk, int t, int r) {
+  return ((uint64_t)s.idr[t * s.k + r] << (64 - s.rb)) | (parent_rk >> s.rb);
+}
+
+__device__ __forceinline__ PK make_pk(const Smem& s, double inv_t, uint32_t h) {
+  PK v;
+  const int x = (int)(h >> 16), r1 = (int)((h >> 8) & 0xFFu), r2 = (int)(h & 0xFFu) - 1;
+  const int d = s.ndep[x];
+  v.sz = __dadd_rn(s.nsz[x], s.zt[d * s.k + r1]);
+  v.rk = rev_key(s, s.nrk[x], d, r1);
+  v.dep = d + 1;
+  if (r2 >= 0) {
+    v.sz = __dadd_rn(v.sz, s.zt[(d + 1) * s.k + r2]);
+    v.rk = rev_key(s, v.rk, d + 1, r2);
+    v.dep = d + 2;
   }
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  v.sk = score_key(score_of(s, inv_t, v.sz, v.dep));
+  v.h = h;
+  return v;
+}
+
+__device__ __forceinline__ PK no_pk() {
+  PK v;
+  v.sk = v.rk = 0ull;
+  v.sz = 0.0;
+  v.dep = 0;
+  v.h = 0u;
+  return v;
+}
+
+// a strictly before b under K; sk == 0 is "none" (last).
+__device__ __forceinline__ bool pk_before(const Smem& s, const PK& a, const PK& b) {
+  if (a.sk != b.sk) return a.sk > b.sk;
+  if (a.sk == 0) return false;
+  if (a.dep != b.dep) return a.dep < b.dep;
+  if (a.sz != b.sz) return a.sz > b.sz;
+  if (a.rk != b.rk) return a.rk < b.rk;
+  if (a.dep * s.rb <= 64 || a.h == b.h) return false;  // whole path compared: same prefix
+  return slow_before(a.h, b.h);
+}
+
+__device__ __forceinline__ uint64_t shfl_u64(uint64_t v, int o) {
+  const uint32_t lo = __shfl_xor_sync(kFull, (uint32_t)v, o);
+  const uint32_t hi = __shfl_xor_sync(kFull, (uint32_t)(v >> 32), o);
+  return ((uint64_t)hi << 32) | lo;
+}
+
+// Block-wide maximum of the score keys with the handle of one holder,
+// returned to every thread; `tie` is set when the maximum is held by more
+// than one candidate (or by a thread that flagged a tie of its own), so that
+// the caller resolves it under the full order; `flag` is ORed over the block.
+// One barrier; the caller must barrier before the next call.
+__device__ __forceinline__ void block_max_key(uint64_t& key, uint32_t& h, int& tie, int& flag,
+                                              Red* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t hi = (uint32_t)(key >> 32);
+  uint32_t mhi = __reduce_max_sync(kFull, hi);
+  uint32_t mlo = __reduce_max_sync(kFull, hi == mhi ? (uint32_t)key : 0u);
+  uint64_t wk = ((uint64_t)mhi << 32) | mlo;
+  unsigned bal = __ballot_sync(kFull, key == wk);
+  const uint32_t wh = __shfl_sync(kFull, h, __ffs(bal) - 1);
+  const int wt = (__popc(bal) > 1) | __any_sync(kFull, tie && key == wk);
+  if (lane == 0) {
+    red->wkey[warp] = wk;
+    red->wid[warp] = wh;
+    red->wtie[warp] = wt;
+  }
+  flag = __syncthreads_or(flag);
+  // every warp reduces the per-warp results the same way
+  const uint64_t k8 = lane < kWarps ? red->wkey[lane] : 0ull;
+  const uint32_t h8 = lane < kWarps ? red->wid[lane] : 0u;
+  const int t8 = lane < kWarps ? red->wtie[lane] : 0;
+  hi = (uint32_t)(k8 >> 32);
+  mhi = __reduce_max_sync(kFull, hi);
+  mlo = __reduce_max_sync(kFull, hi == mhi ? (uint32_t)k8 : 0u);
+  wk = ((uint64_t)mhi << 32) | mlo;
+  bal = __ballot_sync(kFull, lane < kWarps && k8 == wk);
+  h = __shfl_sync(kFull, h8, __ffs(bal) - 1);
+  tie = wk != 0 && ((__popc(bal) > 1) | __any_sync(kFull, t8 && k8 == wk));
+  key = wk;
+}
+
+struct KeyHandle {
+  uint64_t key;
+  uint32_t h;
+};
+
+// K-best (key, handle) over the block under the full order, returned to
+// every thread (the rare paths: exact ties and degenerate inputs).  One
+// barrier; the caller must barrier before the next reduction.
+__device__ __noinline__ KeyHandle block_best_slow(uint64_t key, uint32_t h, Red* red) {
+  const Smem s = g_layout;
+  const double inv_t = g_inv_t;
+  for (int o = 16; o > 0; o >>= 1) {
+    const uint64_t ok = shfl_u64(key, o);
+    const uint32_t oh = __shfl_xor_sync(kFull, h, o);
+    if (key_before(s, inv_t, ok, oh, key, h)) {
+      key = ok;
+      h = oh;
+    }
+  }
+  const int warp = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) {
+    red->wkey[warp] = key;
+    red->wid[warp] = h;
+  }
   __syncthreads();
-  VP b = red[0];
+  key = red->wkey[0];
+  h = red->wid[0];
+  for (int w = 1; w < kWarps; ++w) {
+    const uint64_t ok = red->wkey[w];
+    const uint32_t oh = red->wid[w];
+    if (key_before(s, inv_t, ok, oh, key, h)) {
+      key = ok;
+      h = oh;
+    }
+  }
+  return KeyHandle{key, h};
+}
+
+// K-best prefix over the block by pk_before, returned to every thread.  One
+// barrier; the caller must barrier before the next reduction.
+__device__ __forceinline__ PK block_best_pk(const Smem& s, PK v, Red* red) {
+  for (int o = 16; o > 0; o >>= 1) {
+    PK u;
+    u.sk = shfl_u64(v.sk, o);
+    u.rk = shfl_u64(v.rk, o);
+    u.sz = __shfl_xor_sync(kFull, v.sz, o);
+    u.dep = __shfl_xor_sync(kFull, v.dep, o);
+    u.h = __shfl_xor_sync(kFull, v.h, o);
+    if (pk_before(s, u, v)) v = u;
+  }
+  const int warp = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) red->wpk[warp] = v;
+  __syncthreads();
+  PK b = red->wpk[0];
   for (int w = 1; w < kWarps; ++w)
-    if (vp_before(s, red[w], b)) b = red[w];
-  __syncthreads();
+    if (pk_before(s, red->wpk[w], b)) b = red->wpk[w];
   return b;
 }
 
@@ -193,227 +354,300 @@ __device__ __forceinline__ int warp_incl_scan(int v, int lane) {
   return v;
 }
 
-// out[i] = in[0] + ... + in[i-1] for i < n (out may alias in); returns the
-// total.  Thread t scans the contiguous block [t*c, (t+1)*c).
-__device__ int block_exscan(const int* in, int* out, int n, int* red) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int c = (n + kThreads - 1) / kThreads;
-  const int lo = min(tid * c, n), hi = min(lo + c, n);
-  int sum = 0;
-  for (int i = lo; i < hi; ++i) sum += in[i];
-  const int inc = warp_incl_scan(sum, lane);
-  if (lane == 31) red[warp] = inc;
-  __syncthreads();
-  int before = 0, total = 0;
+// Exclusive scan of one value per thread in thread order; returns the
+// thread's offset, sets `total` and ORs `flag` over the block.  One barrier;
+// the caller must barrier before the next call.
+__device__ __forceinline__ int block_exscan1(int v, int& total, int& flag, Red* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int inc = warp_incl_scan(v, lane);
+  if (lane == 31) red->wsum[warp] = inc;
+  flag = __syncthreads_or(flag);
+  int before = 0, tot = 0;
+#pragma unroll
   for (int w = 0; w < kWarps; ++w) {
-    before += (w < warp) ? red[w] : 0;
-    total += red[w];
+    const int c = red->wsum[w];
+    before += (w < warp) ? c : 0;
+    tot += c;
   }
-  int run = before + inc - sum;
-  for (int i = lo; i < hi; ++i) {
-    const int v = in[i];
-    out[i] = run;
-    run += v;
-  }
-  __syncthreads();
-  return total;
+  total = tot;
+  return before + inc - v;
 }
 
-__device__ int block_sum(int v, int* red) {
-  v = __reduce_add_sync(kFull, v);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
-  __syncthreads();
-  int t = 0;
-  for (int w = 0; w < kWarps; ++w) t += red[w];
-  __syncthreads();
-  return t;
-}
-
-// One histogram pass of the final-round cut.
-struct Pass {
-  double lo, scale;
-  int bstar;
-};
-
-// Position of a score relative to the cut: 1 above it (kept), -1 below it
-// (dropped), 0 in the boundary bin of every pass so far.  Each pass bins
-// with the same arithmetic, so an item's state never depends on rounding
-// of a recomputed bin edge.
-__device__ __forceinline__ int cut_state(double sc, const Pass* ps, int np) {
-  for (int q = 0; q < np; ++q) {
-    int bin = (int)((sc - ps[q].lo) * ps[q].scale);
-    bin = min(max(bin, 0), kBins - 1);
-    if (bin > ps[q].bstar) return 1;
-    if (bin < ps[q].bstar) return -1;
+// Rank the nl candidates of red->list (all with the same score key) among
+// themselves under K and keep the `need` best (bit 30 of cid).  Each
+// candidate's (depth, sum, reversed path) is published once, so the ranking
+// compares shared-memory words.  nl <= kTieList.
+__device__ void rank_ties(const Smem& s, double inv_t, int nl, int need, Red* red) {
+  const int tid = threadIdx.x;
+  for (int q = tid; q < nl; q += kThreads) {
+    const PK v = make_pk(s, inv_t, (s.cid[red->list[q]] & 0x3FFFFFFFu) << 8);
+    red->csz[q] = v.sz;
+    red->crk[q] = v.rk;
+    red->cdep[q] = v.dep;
+    red->chd[q] = v.h;
   }
-  return 0;
-}
-
-struct CutShared {
-  Pass ps[kMaxPasses];
-  int np, above, in_cut, nb;
-  double lo, hi;
-  int list[kBins];
-};
-
-// Final round: among the F items with iflag set (more than R of them), keep
-// the R K-best (iflag cleared on the others).  The kept items of a run are a
-// prefix of it, since a run is K-ordered.
-__device__ void keep_best(const Smem& s, int F, int R, CutShared* cs, double* dred, int* red,
-                          VP* vred) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  double lo = INFINITY, hi = -INFINITY;
-  int in_cut = 0;
-  for (int i = tid; i < F; i += kThreads)
-    if (s.iflag[i]) {
-      lo = fmin(lo, s.isc[i]);
-      hi = fmax(hi, s.isc[i]);
-      ++in_cut;
+  __syncthreads();
+  for (int q = tid; q < nl; q += kThreads) {
+    const int dq = red->cdep[q];
+    const double zq = red->csz[q];
+    const uint64_t rq = red->crk[q];
+    const bool exact = dq * s.rb <= 64;
+    int rank = 0;
+    for (int u = 0; u < nl; ++u) {
+      const int du = red->cdep[u];
+      const double zu = red->csz[u];
+      const uint64_t ru = red->crk[u];
+      bool b;
+      if (du != dq) b = du < dq;
+      else if (zu != zq) b = zu > zq;
+      else if (ru != rq) b = ru < rq;
+      else b = !exact && u != q && slow_before(red->chd[u], red->chd[q]);
+      rank += b;
     }
+    if (rank < need) s.cid[red->list[q]] |= 0x40000000u;
+  }
+  __syncthreads();
+}
+
+// Final round with at most one candidate per thread: candidate t has `above`
+// candidates with larger score keys and `eq` with equal ones (itself
+// included); it is kept if above + eq <= R, dropped if above >= R, and only
+// the one group of equal keys that straddles R is ranked under the full order.
+__device__ void cut_small(const Smem& s, int T, int R, Red* red) {
+  const int tid = threadIdx.x;
+  int above = 0, eq = 0;
+  if (tid == 0) red->nlist = 0;
+  if (tid < T) {
+    const uint64_t ki = s.ckey[tid];
+    int u = 0;
+    for (; u + 8 <= T; u += 8) {  // eight keys a step (T is even here or the tail catches it)
+      ulonglong2 v[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) v[e] = *reinterpret_cast<const ulonglong2*>(s.ckey + u + 2 * e);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        above += (v[e].x > ki) + (v[e].y > ki);
+        eq += (v[e].x == ki) + (v[e].y == ki);
+      }
+    }
+    for (; u < T; ++u) {
+      above += s.ckey[u] > ki;
+      eq += s.ckey[u] == ki;
+    }
+  }
+  const bool bnd = tid < T && above < R && above + eq > R;
+  if (__syncthreads_or(bnd)) {
+    if (bnd) red->list[atomicAdd(&red->nlist, 1)] = tid;
+    __syncthreads();
+    const int need = R - above;
+    // every member of the straddling group has the same `above`
+    if (bnd && red->list[0] == tid) red->digit = need;
+    __syncthreads();
+    rank_ties(s, g_inv_t, red->nlist, red->digit, red);
+  }
+  if (tid < T && (above + eq <= R || (s.cid[tid] & 0x40000000u)))
+    s.cid[tid] = (s.cid[tid] & 0x3FFFFFFFu) | 0x80000000u;
+  __syncthreads();
+}
+
+// Final round: keep the R K-best of the T > R candidates in ckey/cid (bit 31
+// of cid set on the kept ones).  Radix select on the score keys, 8 bits a
+// pass below the bits all keys share; candidates whose keys equal the R-th
+// key are ranked under the full order K.
+__device__ void cut_best(const Smem& s, double inv_t, int T, int R, Red* red) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint64_t mn = ~0ull, mx = 0;
+  for (int i = tid; i < T; i += kThreads) {
+    const uint64_t kk = s.ckey[i];
+    mn = kk < mn ? kk : mn;
+    mx = kk > mx ? kk : mx;
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
-    lo = fmin(lo, __shfl_xor_sync(kFull, lo, o));
-    hi = fmax(hi, __shfl_xor_sync(kFull, hi, o));
+    const uint64_t a = shfl_u64(mn, o), b = shfl_u64(mx, o);
+    mn = a < mn ? a : mn;
+    mx = b > mx ? b : mx;
   }
   if (lane == 0) {
-    dred[warp] = lo;
-    dred[kWarps + warp] = hi;
+    red->wmn[warp] = mn;
+    red->wmx[warp] = mx;
   }
-  in_cut = block_sum(in_cut, red);  // its barriers also publish dred
-  if (tid == 0) {
-    double l = INFINITY, h = -INFINITY;
-    for (int w = 0; w < kWarps; ++w) {
-      l = fmin(l, dred[w]);
-      h = fmax(h, dred[kWarps + w]);
-    }
-    cs->lo = l;
-    cs->hi = h;
-    cs->np = 0;
-    cs->above = 0;
-    cs->in_cut = in_cut;
-  }
+  red->hist[0][tid] = 0;
   __syncthreads();
-  // narrow the cut with score histograms
-  for (;;) {
-    const int np = cs->np;
-    if (np >= kMaxPasses || cs->in_cut <= kExactMax || !(cs->hi > cs->lo)) break;
-    for (int bn = tid; bn < kBins; bn += kThreads) s.hist[bn] = 0;
-    __syncthreads();
-    Pass pass;
-    pass.lo = cs->lo;
-    pass.scale = (double)kBins / (cs->hi - cs->lo);
-    for (int i = tid; i < F; i += kThreads) {
-      if (!s.iflag[i]) continue;
-      const double sc = s.isc[i];
-      if (cut_state(sc, cs->ps, np) != 0) continue;
-      atomicAdd(&s.hist[min(max((int)((sc - pass.lo) * pass.scale), 0), kBins - 1)], 1);
-    }
-    __syncthreads();
-    if (warp == 0) {
-      // lane l holds bins [8l, 8l+8); find the bin holding the R-th best from the top
-      int h[8], lt = 0;
+  mn = red->wmn[0];
+  mx = red->wmx[0];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        h[e] = s.hist[8 * lane + e];
-        lt += h[e];
-      }
-      int suf = lt;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int u = __shfl_down_sync(kFull, suf, o);
-        if (lane + o < 32) suf += u;
-      }
-      const int above_lane = cs->above + suf - lt;
-      const bool mine = above_lane < R && above_lane + lt >= R;
-      const unsigned who = __ballot_sync(kFull, mine);
-      const int src = who ? __ffs(who) - 1 : 0;
-      if (lane == src) {
-        int acc = above_lane, bs = 0, cnt = 0;
-        for (int e = 7; e >= 0; --e) {
-          if (acc + h[e] >= R) {
-            bs = 8 * lane + e;
-            cnt = h[e];
-            break;
-          }
-          acc += h[e];
+  for (int w = 1; w < kWarps; ++w) {
+    mn = red->wmn[w] < mn ? red->wmn[w] : mn;
+    mx = red->wmx[w] > mx ? red->wmx[w] : mx;
+  }
+  int need = R;
+  uint64_t prefix = mx, pmask = ~0ull;
+  bool ties = true;  // all keys equal until shown otherwise
+  if (mn != mx) {
+    int hb = 63 - __clzll((long long)(mn ^ mx));
+    pmask = hb == 63 ? 0ull : (~0ull << (hb + 1));
+    prefix = mx & pmask;
+    int buf = 0;
+    for (;;) {
+      const int shift = hb >= 7 ? hb - 7 : 0;
+      const uint64_t dmask = (1ull << (hb - shift + 1)) - 1;
+      red->hist[buf ^ 1][tid] = 0;  // the next pass's histogram
+      // warp-aggregated: one atomic per distinct digit in a warp
+      for (int i0 = warp * 32; i0 < T; i0 += kThreads) {
+        const int i = i0 + lane;
+        int dg = -1;
+        if (i < T) {
+          const uint64_t kk = s.ckey[i];
+          if ((kk & pmask) == prefix) dg = (int)((kk >> shift) & dmask);
         }
-        pass.bstar = bs;
-        cs->ps[np] = pass;
-        cs->np = np + 1;
-        cs->above = acc;
-        cs->in_cut = cnt;
-        cs->lo = pass.lo + bs / pass.scale;
-        cs->hi = pass.lo + (bs + 1) / pass.scale;
+        const unsigned grp = __match_any_sync(kFull, dg);
+        if (dg >= 0 && lane == __ffs(grp) - 1) atomicAdd(&red->hist[buf][dg], __popc(grp));
       }
+      __syncthreads();
+      // thread t holds bin 255 - t: scan from the top bin down
+      const int hcnt = red->hist[buf][kBins - 1 - tid];
+      int tot, nof = 0;
+      const int excl = block_exscan1(hcnt, tot, nof, red);
+      if (excl < need && excl + hcnt >= need) {
+        red->digit = kBins - 1 - tid;
+        red->above = excl;
+        red->hcount = hcnt;
+      }
+      __syncthreads();
+      const int digit = red->digit, hc = red->hcount;
+      need -= red->above;
+      prefix |= (uint64_t)digit << shift;
+      pmask |= dmask << shift;
+      buf ^= 1;
+      if (hc == need) {
+        ties = false;
+        break;
+      }
+      if (shift == 0) break;
+      hb = shift - 1;
     }
-    __syncthreads();
   }
-  const int np = cs->np;
-  const int need = R - cs->above;
-  // gather the boundary items
-  if (tid == 0) cs->nb = 0;
-  __syncthreads();
-  for (int i = tid; i < F; i += kThreads)
-    if (s.iflag[i] && cut_state(s.isc[i], cs->ps, np) == 0) {
-      const int q = atomicAdd(&cs->nb, 1);
-      if (q < kBins) cs->list[q] = i;
-    }
-  __syncthreads();
-  const int nb = cs->nb;
-  if (nb <= kBins) {
-    // rank each boundary item among them; keep the `need` best
-    for (int t = tid; t < nb; t += kThreads) {
-      const int i = cs->list[t];
-      const VP vi = item_vp(s, i);
-      int rank = 0;
-      for (int u = 0; u < nb; ++u)
-        if (u != t) rank += vp_before(s, item_vp(s, cs->list[u]), vi);
-      s.ipos[i] = rank < need;  // verdict for boundary items
-    }
+  if (!ties) {
+    for (int i = tid; i < T; i += kThreads)
+      if ((s.ckey[i] & pmask) >= prefix) s.cid[i] |= 0x80000000u;
     __syncthreads();
-    for (int i = tid; i < F; i += kThreads)
-      if (s.iflag[i]) {
-        const int st = cut_state(s.isc[i], cs->ps, np);
-        s.iflag[i] = st == 1 || (st == 0 && s.ipos[i]);
-      }
-    __syncthreads();
+    return;
+  }
+  // keys above the R-th key are kept; `need` of those equal to it are ranked
+  if (tid == 0) red->nlist = 0;
+  __syncthreads();
+  for (int i = tid; i < T; i += kThreads) {
+    const uint64_t kk = s.ckey[i];
+    if (kk > prefix) s.cid[i] |= 0x80000000u;
+    if (kk == prefix) {
+      const int q = atomicAdd(&red->nlist, 1);
+      if (q < kTieList) red->list[q] = i;
+    }
+  }
+  __syncthreads();
+  const int nl = red->nlist;
+  if (nl <= kTieList) {
+    rank_ties(s, inv_t, nl, need, red);
   } else {
-    // many exact score ties: take the K-best undecided boundary item, need times
-    for (int i = tid; i < F; i += kThreads)
-      if (s.iflag[i]) {
-        const int st = cut_state(s.isc[i], cs->ps, np);
-        s.iflag[i] = st == 1 ? 1 : (st == 0 ? 2 : 0);  // 2: boundary, undecided
-      }
-    __syncthreads();
+    // a very large exact tie: take the K-best undecided tied candidate, need times
     for (int t = 0; t < need; ++t) {
-      VP best = no_vp();
-      int bi = -1;
-      for (int i = tid; i < F; i += kThreads)
-        if (s.iflag[i] == 2) {
-          const VP v = item_vp(s, i);
-          if (vp_before(s, v, best)) {
-            best = v;
-            bi = i;
-          }
+      uint64_t key = 0;
+      uint32_t h = 0;
+      for (int i = tid; i < T; i += kThreads) {
+        if (s.ckey[i] != prefix || (s.cid[i] & 0x40000000u)) continue;
+        const uint32_t hi = (s.cid[i] & 0x3FFFFFFFu) << 8;
+        if (key_before(s, inv_t, prefix, hi, key, h)) {
+          key = prefix;
+          h = hi;
         }
-      const VP bb = block_best(s, best, vred);
-      if (bi >= 0 && bb.base == best.base && bb.r1 == best.r1 && bb.depth == best.depth)
-        s.iflag[bi] = 3;  // taken
+      }
+      h = block_best_slow(key, h, red).h;
+      for (int i = tid; i < T; i += kThreads)
+        if (s.ckey[i] == prefix && ((s.cid[i] & 0x3FFFFFFFu) << 8) == h) s.cid[i] |= 0x40000000u;
       __syncthreads();
     }
-    for (int i = tid; i < F; i += kThreads) s.iflag[i] = (s.iflag[i] == 1 || s.iflag[i] == 3);
-    __syncthreads();
+  }
+  for (int i = tid; i < T; i += kThreads)
+    if (s.cid[i] & 0x40000000u) s.cid[i] = (s.cid[i] & 0x3FFFFFFFu) | 0x80000000u;
+  __syncthreads();
+}
+
+// Rank path key of a new node at depth d+1 with rank r: its parent's key with
+// r placed in field d (rb bits per field, fields from the most significant
+// bit of word 0 on; a field may straddle two words).
+__device__ __forceinline__ void make_path_key(const Smem& s, int parent, int id, int d, int r) {
+  const uint64_t* pk = s.pkey + (size_t)parent * s.kw;
+  uint64_t* ck = s.pkey + (size_t)id * s.kw;
+  for (int w = 0; w < s.kw; ++w) ck[w] = pk[w];
+  const int o = d * s.rb, w = o >> 6, sh = 64 - (o & 63) - s.rb;
+  if (sh >= 0) {
+    ck[w] |= (uint64_t)r << sh;
+  } else {
+    ck[w] |= (uint64_t)r >> (-sh);
+    ck[w + 1] |= (uint64_t)r << (64 + sh);
   }
 }
 
-__global__ void __launch_bounds__(kThreads) build_tree_kernel(TreeParams p) {
+__device__ __forceinline__ bool path_less(const Smem& s, int a, int b) {
+  const uint64_t* ka = s.pkey + (size_t)a * s.kw;
+  const uint64_t* kb = s.pkey + (size_t)b * s.kw;
+  for (int w = 0; w < s.kw; ++w)
+    if (ka[w] != kb[w]) return ka[w] < kb[w];
+  return false;
+}
+
+// Item (x, r): key of the child of node x (depth d) with candidate rank r.
+__device__ __forceinline__ uint64_t item_key(const Smem& s, double inv_t, double base_sz, int d, int r) {
+  return score_key(score_of(s, inv_t, __dadd_rn(base_sz, s.zt[d * s.k + r]), d + 1));
+}
+
+// Items of node x's run from rank r0 (below rend) whose keys exceed tk, up
+// to the first one that does not; `tie` is set when that one's key equals
+// tk, which only the full order can decide.  Four keys at a time, so that
+// their shared-memory loads overlap.
+__device__ __forceinline__ int count_fast(const Smem& s, double inv_t, int x, int d, int r0, int rend,
+                                          uint64_t tk, int& tie) {
+  const double base = s.nsz[x];
+  int c = 0;
+  for (int r = r0; r < rend; r += 4) {
+    uint64_t kk[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) kk[e] = r + e < rend ? item_key(s, inv_t, base, d, r + e) : 0ull;
+    bool go = true;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (go) {
+        if (r + e < rend && kk[e] > tk) {
+          ++c;
+        } else {
+          tie |= (r + e < rend && kk[e] == tk);
+          go = false;
+        }
+      }
+    }
+    if (!go) break;
+  }
+  return c;
+}
+
+// The same count under the full order (the rare paths).
+__device__ __noinline__ int count_slow(int x, int r0, int rend, uint64_t tk, uint32_t th) {
+  const Smem s = g_layout;
+  const double inv_t = g_inv_t;
+  const int d = s.ndep[x];
+  const double base = s.nsz[x];
+  int c = 0;
+  for (int r = r0; r < rend; ++r) {
+    if (!key_before(s, inv_t, item_key(s, inv_t, base, d, r), pack_vp(x, r, -1), tk, th)) break;
+    ++c;
+  }
+  return c;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) build_tree_kernel(TreeParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  __shared__ int s_lvl[DDT_TREE_L_MAX + 2];
-  __shared__ int s_red[kWarps + 1];
-  __shared__ double s_dred[2 * kWarps];
-  __shared__ VP s_vred[kWarps];
-  __shared__ CutShared s_cut;
-  __shared__ int s_maxd;
+  __shared__ Red red;
 
   const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int L = p.L, k = p.k, NM = p.n_max, icap = p.icap;
@@ -421,6 +655,8 @@ __global__ void __launch_bounds__(kThreads) build_tree_kernel(TreeParams p) {
 
   Smem s;
   s.k = k;
+  s.kw = p.kw;
+  s.rb = p.rb;
   {
     unsigned char* q = smem_raw;
     auto take = [&](size_t bytes) {
@@ -432,41 +668,34 @@ __global__ void __launch_bounds__(kThreads) build_tree_kernel(TreeParams p) {
     s.zt = (double*)take(sizeof(double) * L * k);
     s.nsz = (double*)take(sizeof(double) * NM);
     s.nsc = (double*)take(sizeof(double) * NM);
-    s.isc = (double*)take(sizeof(double) * icap);
+    s.pkey = (uint64_t*)take(sizeof(uint64_t) * NM * p.kw);
+    s.nrk = (uint64_t*)take(sizeof(uint64_t) * NM);
+    s.ckey = (uint64_t*)take(sizeof(uint64_t) * icap);  // ckey and cid adjacent: the
+    s.cid = (uint32_t*)take(sizeof(uint32_t) * icap);   // mask staging area
     s.tt = (int*)take(sizeof(int) * L * k);
     s.npar = (int*)take(sizeof(int) * NM);
     s.ndep = (int*)take(sizeof(int) * NM);
     s.nrank = (int*)take(sizeof(int) * NM);
     s.nnext = (int*)take(sizeof(int) * NM);
-    s.nlen = (int*)take(sizeof(int) * NM);
-    s.noff = (int*)take(sizeof(int) * NM);
+    s.nrow = (int*)take(sizeof(int) * NM);
     s.ninv = (int*)take(sizeof(int) * NM);
-    s.iown = (uint32_t*)take(sizeof(uint32_t) * icap);
-    s.iflag = (int*)take(sizeof(int) * icap);
-    s.ipos = (int*)take(sizeof(int) * icap);
-    s.hist = (int*)take(sizeof(int) * kBins);
+    s.prow = (int*)take(sizeof(int) * NM);
+    s.idr = (int*)take(sizeof(int) * L * k);
+  }
+  if (tid == 0) {
+    g_layout = s;
+    g_inv_t = inv_t;
   }
 
-  // per-sequence candidate count and budget (clamped, flagged)
-  int kb = p.k_per_seq ? p.k_per_seq[b] : k;
-  int Bb = p.budget ? p.budget[b] : p.B_max;
-  if (kb < 1 || kb > k || Bb < 0 || Bb > p.B_max) {
-    if (tid == 0) raise_status(p.status, DDT_ERR_INVALID_ARG);
-    kb = min(max(kb, 1), k);
-    Bb = min(max(Bb, 0), p.B_max);
-  }
+  // global loads first; the budget and candidate count are only needed later
   for (int i = tid; i < L * k; i += kThreads) {
     s.zt[i] = (double)p.zk[(int64_t)b * L * k + i];
     s.tt[i] = p.ids[(int64_t)b * L * k + i];
   }
-  if (tid == 32) {
-    double acc = 0.0;
-    s.S[0] = 0.0;
-    for (int t = 1; t <= L; ++t) {
-      acc = __dadd_rn(acc, (double)p.lse[(int64_t)b * L + t - 1]);
-      s.S[t] = acc;
-    }
-  }
+  for (int t = tid; t < L; t += kThreads) s.S[t + 1] = (double)p.lse[(int64_t)b * L + t];
+  int kb = p.k_per_seq ? p.k_per_seq[b] : k;
+  int Bb = p.budget ? p.budget[b] : p.B_max;
+  for (int w = tid; w < p.kw; w += kThreads) s.pkey[w] = 0ull;
   if (tid == 0) {
     s.nsz[0] = 0.0;
     s.nsc[0] = 0.0;
@@ -474,10 +703,44 @@ __global__ void __launch_bounds__(kThreads) build_tree_kernel(TreeParams p) {
     s.ndep[0] = 0;
     s.nrank[0] = 0;
     s.nnext[0] = 0;
+    s.nrk[0] = 0ull;
+  }
+  __syncthreads();
+  // id ranks: within a position, token order is id-rank order
+  for (int i = tid; i < L * k; i += kThreads) {
+    const int t = i / k, tok = s.tt[i];
+    int below = 0;
+#pragma unroll 8
+    for (int r = 0; r < k; ++r) below += s.tt[t * k + r] < tok;
+    s.idr[i] = below;
+  }
+  if (tid == 0) {  // S[t] = lse_1 + ... + lse_t, summed in position order
+    double acc = 0.0;
+    s.S[0] = 0.0;
+    for (int t0 = 1; t0 <= L; t0 += 8) {
+      double v[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = t0 + e <= L ? s.S[t0 + e] : 0.0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        if (t0 + e <= L) {
+          acc = __dadd_rn(acc, v[e]);
+          s.S[t0 + e] = acc;
+        }
+    }
+  }
+  // per-sequence candidate count and budget (clamped, flagged)
+  if (kb < 1 || kb > k || Bb < 0 || Bb > p.B_max) {
+    if (tid == 0) raise_status(p.status, DDT_ERR_INVALID_ARG);
+    kb = min(max(kb, 1), k);
+    Bb = min(max(Bb, 0), p.B_max);
   }
   __syncthreads();
 
   // ---------------- selection ----------------
+  // ncnt[x] (in nrow, free until numbering): the items of x's run taken
+  // this round
+  int* ncnt = s.nrow;
   int nn = 1, nsel = 0;
   if (kb == 1) {
     // one candidate per position: the tree is the chain of the first B positions
@@ -491,6 +754,8 @@ __global__ void __launch_bounds__(kThreads) build_tree_kernel(TreeParams p) {
       s.ndep[t] = t;
       s.nrank[t] = 0;
       s.nnext[t] = t < len ? 1 : 0;
+      for (int w = 0; w < p.kw; ++w) s.pkey[(size_t)t * p.kw + w] = 0ull;
+      s.nrk[t] = 0ull;  // one node per depth: never compared
     }
     if (tid == 0) s.nnext[0] = len > 0 ? 1 : 0;
     nn = 1 + len;
@@ -499,145 +764,265 @@ __global__ void __launch_bounds__(kThreads) build_tree_kernel(TreeParams p) {
   }
 #pragma unroll 1
   while (nsel < Bb) {
-    // runs of this round, truncated to fit the item buffer
-    int tot = 0;
+    // theta: the K-best first child of a run head
+    uint64_t tk = 0;
+    uint32_t th = 0;
+    int ttie = 0, front = 0;
     for (int x = tid; x < nn; x += kThreads) {
-      const int len = (s.ndep[x] < L) ? max(0, kb - s.nnext[x]) : 0;
-      s.nlen[x] = len;
-      tot += len;
-    }
-    tot = block_sum(tot, s_red);
-    if (tot == 0) break;
-    const int cap = tot <= icap ? DDT_TOPK_K_MAX : max(1, icap / nn);
-    VP th = no_vp();
-    if (tot > icap) {
-      for (int x = tid; x < nn; x += kThreads) {
-        const int len = s.nlen[x];
-        if (len > cap) {  // the first item cut from the run bounds the round too
-          const VP v = make_item(s, inv_t, x, s.nnext[x] + cap);
-          if (vp_before(s, v, th)) th = v;
-          s.nlen[x] = cap;
+      const int d = s.ndep[x], nx = s.nnext[x];
+      if (d < L && nx < kb) {
+        front = 1;
+        if (d + 1 < L) {
+          const double sz = __dadd_rn(__dadd_rn(s.nsz[x], s.zt[d * k + nx]), s.zt[(d + 1) * k]);
+          const uint64_t kk = score_key(score_of(s, inv_t, sz, d + 2));
+          if (kk > tk) {
+            tk = kk;
+            th = pack_vp(x, nx, 0);
+            ttie = 0;
+          } else if (kk == tk) {
+            ttie = 1;
+          }
         }
       }
+    }
+    block_max_key(tk, th, ttie, front, &red);
+    if (!front) break;
+    if (ttie) {
+      // several first children share the best score: the full order decides
       __syncthreads();
-    }
-    const int F = block_exscan(s.nlen, s.noff, nn, s_red);
-    for (int x = tid; x < nn; x += kThreads) {
-      const int o = s.noff[x], r0 = s.nnext[x], len = s.nlen[x];
-      for (int i = 0; i < len; ++i) s.iown[o + i] = ((uint32_t)x << 8) | (uint32_t)(r0 + i);
-    }
-    __syncthreads();
-    // item scores; theta = the K-best first child of any item
-    for (int i = tid; i < F; i += kThreads) {
-      const uint32_t e = s.iown[i];
-      const int x = (int)(e >> 8), r = (int)(e & 0xFFu);
-      const int d = s.ndep[x];
-      const double sz = __dadd_rn(s.nsz[x], s.zt[d * k + r]);
-      s.isc[i] = score_of(s, inv_t, sz, d + 1);
-      if (d + 1 < L) {
-        VP c;
-        c.base = x;
-        c.r1 = r;
-        c.r2 = 0;
-        c.depth = d + 2;
-        c.sz = __dadd_rn(sz, s.zt[(d + 1) * k]);
-        c.sc = score_of(s, inv_t, c.sz, c.depth);
-        if (vp_before(s, c, th)) th = c;
+      PK best = no_pk();
+      for (int x = tid; x < nn; x += kThreads) {
+        const int d = s.ndep[x], nx = s.nnext[x];
+        if (d < L - 1 && nx < kb) {
+          const PK c = make_pk(s, inv_t, pack_vp(x, nx, 0));
+          if (c.sk == tk && pk_before(s, c, best)) best = c;
+        }
       }
+      th = block_best_pk(s, best, &red).h;
     }
-    th = block_best(s, th, s_vred);
-    // safe items: those that precede theta
-    for (int i = tid; i < F; i += kThreads) s.iflag[i] = vp_before(s, item_vp(s, i), th);
-    __syncthreads();
-    int T = block_exscan(s.iflag, s.ipos, F, s_red);
+    // run items before theta (tk == 0: no first child exists, all are)
+    int sum = 0, ctie = 0;
+    for (int x = tid; x < nn; x += kThreads) {
+      const int d = s.ndep[x];
+      const int c = d < L ? count_fast(s, inv_t, x, d, s.nnext[x], kb, tk, ctie) : 0;
+      ncnt[x] = c;
+      sum += c;
+    }
+    int T;
+    int off = block_exscan1(sum, T, ctie, &red);
+    if (ctie) {
+      // an item scores exactly like theta: count again under the full order
+      __syncthreads();
+      const PK tp = make_pk(s, inv_t, th);
+      sum = 0;
+      for (int x = tid; x < nn; x += kThreads) {
+        int c = 0;
+        if (s.ndep[x] < L)
+          for (int r = s.nnext[x]; r < kb && pk_before(s, make_pk(s, inv_t, pack_vp(x, r, -1)), tp); ++r) ++c;
+        ncnt[x] = c;
+        sum += c;
+      }
+      int nof = 0;
+      off = block_exscan1(sum, T, nof, &red);
+    }
     if (T == 0) {
       // Only reachable when a candidate scores above its parent (an lse below
-      // some inv_t*z): take the K-best item so that the loop progresses.
-      VP best = no_vp();
-      for (int i = tid; i < F; i += kThreads) {
-        const VP v = item_vp(s, i);
-        if (vp_before(s, v, best)) best = v;
+      // some inv_t*z): take the K-best run head so that the loop progresses.
+      uint64_t bk = 0;
+      uint32_t bh = 0;
+      for (int x = tid; x < nn; x += kThreads) {
+        const int d = s.ndep[x], nx = s.nnext[x];
+        if (d < L && nx < kb) {
+          const uint64_t kk = item_key(s, inv_t, s.nsz[x], d, nx);
+          const uint32_t hh = pack_vp(x, nx, -1);
+          if (key_before(s, inv_t, kk, hh, bk, bh)) {
+            bk = kk;
+            bh = hh;
+          }
+        }
       }
-      best = block_best(s, best, s_vred);
-      for (int i = tid; i < F; i += kThreads) {
-        const uint32_t e = s.iown[i];
-        s.iflag[i] = (int)(e >> 8) == best.base && (int)(e & 0xFFu) == best.r1;
+      bh = block_best_slow(bk, bh, &red).h;
+      sum = 0;
+      for (int x = tid; x < nn; x += kThreads) {
+        ncnt[x] = x == (int)(bh >> 16) ? 1 : 0;
+        sum += ncnt[x];
       }
-      __syncthreads();
-      T = block_exscan(s.iflag, s.ipos, F, s_red);
+      int nof = 0;
+      off = block_exscan1(sum, T, nof, &red);
       if (tid == 0) raise_status(p.status, DDT_ERR_INVALID_ARG);
     }
     const int R = Bb - nsel;
-    const bool last = T >= R;
-    if (T > R) {
-      keep_best(s, F, R, &s_cut, s_dred, s_red, s_vred);
-      T = block_exscan(s.iflag, s.ipos, F, s_red);
-    }
-    // create the selected items as nodes
-    for (int i = tid; i < F; i += kThreads)
-      if (s.iflag[i]) {
-        const uint32_t e = s.iown[i];
-        const int x = (int)(e >> 8), r = (int)(e & 0xFFu);
-        const int id = nn + s.ipos[i];
-        const int d = s.ndep[x];
-        s.nsz[id] = __dadd_rn(s.nsz[x], s.zt[d * k + r]);
-        s.nsc[id] = s.isc[i];
-        s.npar[id] = x;
-        s.ndep[id] = d + 1;
-        s.nrank[id] = r;
-        s.nnext[id] = 0;
-        atomicAdd(&s.nnext[x], 1);
+    if (T > R && T > icap) {
+      // Too many to stage: keep at most m items per run.  The first item cut
+      // from a run bounds this round too, so theta becomes the K-best of
+      // theta and those items, and the count is redone within the first m.
+      const int m = max(1, icap / nn);
+      uint64_t k2 = tk;
+      uint32_t h2 = th;
+      for (int x = tid; x < nn; x += kThreads)
+        if (ncnt[x] > m) {
+          const int r = s.nnext[x] + m;
+          const uint64_t kk = item_key(s, inv_t, s.nsz[x], s.ndep[x], r);
+          const uint32_t hh = pack_vp(x, r, -1);
+          if (key_before(s, inv_t, kk, hh, k2, h2)) {
+            k2 = kk;
+            h2 = hh;
+          }
+        }
+      const KeyHandle b2 = block_best_slow(k2, h2, &red);
+      sum = 0;
+      for (int x = tid; x < nn; x += kThreads) {
+        int c = ncnt[x];
+        if (c > 0) {
+          const int nx = s.nnext[x];
+          c = count_slow(x, nx, nx + min(c, m), b2.key, b2.h);
+        }
+        ncnt[x] = c;
+        sum += c;
       }
+      int nof = 0;
+      off = block_exscan1(sum, T, nof, &red);
+    }
+    if (T > R) {
+      // final round: stage the T candidates and keep the R best
+      int o = off;
+      for (int x = tid; x < nn; x += kThreads) {
+        const int c = ncnt[x];
+        if (c > 0) {
+          const int d = s.ndep[x], nx = s.nnext[x];
+          const double base = s.nsz[x];
+          for (int i = 0; i < c; ++i) {
+            s.ckey[o + i] = item_key(s, inv_t, base, d, nx + i);
+            s.cid[o + i] = ((uint32_t)x << 8) | (uint32_t)(nx + i);
+          }
+          o += c;
+        }
+      }
+      __syncthreads();
+      if (T <= kThreads)
+        cut_small(s, T, R, &red);
+      else
+        cut_best(s, inv_t, T, R, &red);
+      o = off;
+      sum = 0;
+      for (int x = tid; x < nn; x += kThreads) {
+        const int c = ncnt[x];
+        int kept = 0;
+        for (int i = 0; i < c; ++i) kept += (int)(s.cid[o + i] >> 31);
+        o += c;
+        ncnt[x] = kept;
+        sum += kept;
+      }
+      int nof = 0;
+      off = block_exscan1(sum, T, nof, &red);
+    }
+    // create the selected items as nodes (loads of four at a time first)
+    int id = nn + off;
+    for (int x = tid; x < nn; x += kThreads) {
+      const int c = ncnt[x];
+      if (c > 0) {
+        const int d = s.ndep[x], nx = s.nnext[x];
+        const double base = s.nsz[x], Sd = s.S[d + 1];
+        const uint64_t pk0 = s.pkey[(size_t)x * s.kw], prk = s.nrk[x];
+        for (int i0 = 0; i0 < c; i0 += 4) {
+          double z[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) z[e] = i0 + e < c ? s.zt[d * k + nx + i0 + e] : 0.0;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            if (i0 + e < c) {
+              const int r = nx + i0 + e, idn = id + i0 + e;
+              const double sz = __dadd_rn(base, z[e]);
+              s.nsz[idn] = sz;
+              s.nsc[idn] = __dsub_rn(__dmul_rn(inv_t, sz), Sd);
+              s.npar[idn] = x;
+              s.ndep[idn] = d + 1;
+              s.nrank[idn] = r;
+              s.nnext[idn] = 0;
+              s.nrk[idn] = rev_key(s, prk, d, r);
+              if (s.kw == 1)
+                s.pkey[idn] = pk0 | ((uint64_t)r << (64 - (d + 1) * s.rb));
+              else
+                make_path_key(s, x, idn, d, r);
+            }
+          }
+        }
+        id += c;
+        s.nnext[x] = nx + c;
+      }
+    }
     __syncthreads();
     nn += T;
     nsel += T;
-    if (last) break;
   }
 
   // ---------------- breadth-first numbering ----------------
-  // nlen[x] <- row of x, ninv[row] <- x, noff[x] <- row of x's first child
-  if (tid < DDT_TREE_L_MAX + 2) s_lvl[tid] = 0;
+  // Rows are ordered by (depth, rank path): a node's row is the first row of
+  // its depth plus the number of same-depth nodes with a smaller path key.
+  if (tid < L + 2) red.lvl[tid] = 0;
   __syncthreads();
-  int maxd = 0;
-  for (int x = tid; x < nn; x += kThreads) {
-    atomicAdd(&s_lvl[s.ndep[x]], 1);
-    maxd = max(maxd, s.ndep[x]);
-  }
-  maxd = __reduce_max_sync(kFull, maxd);
-  if (lane == 0) s_red[warp] = maxd;
+  // a node's slot within its depth bucket (in ninv, free until the rows)
+  for (int x = tid; x < nn; x += kThreads) s.ninv[x] = atomicAdd(&red.lvl[s.ndep[x]], 1);
   __syncthreads();
-  if (tid == 0) {  // s_lvl[t] <- number of nodes of depth < t (= first row of depth t)
-    int acc = 0;
-    for (int t = 0; t <= L + 1; ++t) {
-      const int c = s_lvl[t];
-      s_lvl[t] = acc;
-      acc += c;
+  if (warp == 0) {  // lvl[t] <- first row of depth t, for t = 0..L+1
+    int v[3], sm = 0;
+#pragma unroll
+    for (int e = 0; e < 3; ++e) {
+      const int t = 3 * lane + e;
+      v[e] = t < L + 2 ? red.lvl[t] : 0;
+      sm += v[e];
     }
-    int md = 0;
-    for (int w = 0; w < kWarps; ++w) md = max(md, s_red[w]);
-    s_maxd = md;
-    s.nlen[0] = 0;
-    s.noff[0] = 1;
-    s.ninv[0] = 0;
+    int run = warp_incl_scan(sm, lane) - sm;
+#pragma unroll
+    for (int e = 0; e < 3; ++e) {
+      const int t = 3 * lane + e;
+      if (t < L + 2) red.lvl[t] = run;
+      run += v[e];
+    }
   }
   __syncthreads();
-  const int md = s_maxd;
-  for (int t = 1; t <= md; ++t) {
-    const int lstart = s_lvl[t], lend = s_lvl[t + 1];
-    for (int x = tid; x < nn; x += kThreads)
-      if (s.ndep[x] == t) {
-        const int j = s.noff[s.npar[x]] + s.nrank[x];
-        s.nlen[x] = j;
-        s.ninv[j] = x;
-      }
-    __syncthreads();
-    // first-child rows of level t: lend + exclusive scan of child counts
-    for (int j = lstart + tid; j < lend; j += kThreads) s.iflag[j - lstart] = s.nnext[s.ninv[j]];
-    __syncthreads();
-    block_exscan(s.iflag, s.ipos, lend - lstart, s_red);
-    for (int j = lstart + tid; j < lend; j += kThreads) s.noff[s.ninv[j]] = lend + s.ipos[j - lstart];
-    __syncthreads();
+  // depth buckets: node ids (in prow, free until the parent rows are
+  // written) and, when they fit, a copy of the path keys in bucket order (in
+  // the free cut buffer) so that the ranking reads them with broadcasts
+  int* bucket = s.prow;
+  const int kw = s.kw;
+  const bool copy_keys = (int64_t)nn * kw * 8 <= 12 * (int64_t)icap;
+  uint64_t* bkey = s.ckey;
+  for (int x = tid; x < nn; x += kThreads) {
+    const int q = red.lvl[s.ndep[x]] + s.ninv[x];
+    bucket[q] = x;
+    if (copy_keys)
+      for (int w = 0; w < kw; ++w) bkey[(size_t)q * kw + w] = s.pkey[(size_t)x * kw + w];
   }
+  __syncthreads();
+  // rank bucket position q among its depth: threads of a warp take
+  // consecutive positions, so they mostly scan the same bucket together
+  for (int q = tid; q < nn; q += kThreads) {
+    const int x = bucket[q];
+    const int d = s.ndep[x], lo = red.lvl[d], hi = red.lvl[d + 1];
+    int below = 0;
+    if (copy_keys && kw == 1) {
+      const uint64_t kx = bkey[q];
+      int u = lo;
+      if ((u & 1) && u < hi) below += bkey[u++] < kx;  // then 16-byte aligned pairs
+      for (; u + 1 < hi; u += 2) {
+        const ulonglong2 v = *reinterpret_cast<const ulonglong2*>(bkey + u);
+        below += (v.x < kx) + (v.y < kx);
+      }
+      if (u < hi) below += bkey[u] < kx;
+    } else if (copy_keys && kw == 2) {
+      const uint64_t k0 = bkey[2 * q], k1 = bkey[2 * q + 1];
+      for (int u = lo; u < hi; ++u) {
+        const ulonglong2 v = *reinterpret_cast<const ulonglong2*>(bkey + 2 * u);
+        below += (v.x < k0) || (v.x == k0 && v.y < k1);
+      }
+    } else {
+      for (int u = lo; u < hi; ++u) below += path_less(s, bucket[u], x);
+    }
+    s.nrow[x] = lo + below;
+    s.ninv[lo + below] = x;
+  }
+  __syncthreads();
 
   // ---------------- outputs ----------------
   const int32_t ctx = p.ctx_len ? p.ctx_len[b] : 0;
@@ -649,10 +1034,12 @@ __global__ void __launch_bounds__(kThreads) build_tree_kernel(TreeParams p) {
     if (j < nn) {
       const int x = s.ninv[j];
       const int d = s.ndep[x];
+      const int pr = x == 0 ? -1 : s.nrow[s.npar[x]];
       o_tok[j] = x == 0 ? p.root_token[b] : s.tt[(d - 1) * k + s.nrank[x]];
-      o_par[j] = x == 0 ? -1 : s.nlen[s.npar[x]];
+      o_par[j] = pr;
       o_dep[j] = d;
       o_pos[j] = ctx + d;
+      s.prow[j] = pr;
     } else {
       o_tok[j] = -1;
       o_par[j] = -1;
@@ -660,60 +1047,78 @@ __global__ void __launch_bounds__(kThreads) build_tree_kernel(TreeParams p) {
       o_pos[j] = -1;
     }
   }
-  // ancestor-or-self masks, level by level: row j = row(parent j) | bit j,
-  // staged in the (now free) item buffer when it holds them
+  __syncthreads();
+  // ancestor-or-self masks: row j walks its parent rows, which decrease, so
+  // each mask word is complete when the walk moves below it and is written
+  // once; staged in the (now free) cut buffer when it holds them
   const int W = p.W;
   uint32_t* o_mask = p.mask + (int64_t)b * NM * W;
-  const bool staged = (int64_t)nn * W <= 2 * (int64_t)icap;
-  uint32_t* m = staged ? (uint32_t*)s.isc : o_mask;
-  for (int i = tid; i < (staged ? nn * W : NM * W); i += kThreads) m[i] = (i == 0) ? 1u : 0u;
-  __syncthreads();
-  for (int t = 1; t <= md; ++t) {
-    const int lstart = s_lvl[t], lend = s_lvl[t + 1];
-    for (int i = tid; i < (lend - lstart) * W; i += kThreads) {
-      const int j = lstart + i / W, w = i % W;
-      uint32_t word = m[(int64_t)s.nlen[s.npar[s.ninv[j]]] * W + w];
-      if ((j >> 5) == w) word |= 1u << (j & 31);
-      m[(int64_t)j * W + w] = word;
+  const bool staged = (int64_t)nn * W <= 3 * (int64_t)icap;
+  uint32_t* m = staged ? (uint32_t*)s.ckey : o_mask;
+  for (int j = tid; j < nn; j += kThreads) {
+    uint32_t* row = m + (int64_t)j * W;
+    int wcur = j >> 5;
+    for (int w = wcur + 1; w < W; ++w) row[w] = 0u;
+    uint32_t acc = 0u;
+    for (int a = j;;) {
+      const int wa = a >> 5;
+      while (wa < wcur) {
+        row[wcur--] = acc;
+        acc = 0u;
+      }
+      acc |= 1u << (a & 31);
+      if (a == 0) break;
+      a = s.prow[a];
     }
-    __syncthreads();
+    row[wcur] = acc;  // wcur == 0 here: the root is row 0
   }
-  if (staged)
+  if (staged) {
+    __syncthreads();
     for (int i = tid; i < NM * W; i += kThreads) o_mask[i] = i < nn * W ? m[i] : 0u;
+  } else {
+    for (int i = nn * W + tid; i < NM * W; i += kThreads) o_mask[i] = 0u;
+  }
   // surrogate: sum of exp(score) over the draft nodes
   double acc = 0.0;
   for (int x = 1 + tid; x < nn; x += kThreads) acc += exp(s.nsc[x]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
-  if (lane == 0) s_dred[warp] = acc;
+  if (lane == 0) red.wd[warp] = acc;
   __syncthreads();
   if (tid == 0) {
     double t = 0.0;
-    for (int w = 0; w < kWarps; ++w) t += s_dred[w];
+    for (int w = 0; w < kWarps; ++w) t += red.wd[w];
     p.n_nodes[b] = nn;
     if (p.surrogate) p.surrogate[b] = t;
   }
 }
 
-size_t tree_smem_bytes(int L, int k, int n_max, int icap) {
+size_t tree_smem_bytes(int L, int k, int n_max, int kw, int icap) {
   auto a = [](size_t x) { return (x + 15) & ~(size_t)15; };
   return a(sizeof(double) * (L + 1)) + a(sizeof(double) * L * k) + 2 * a(sizeof(double) * n_max) +
-         a(sizeof(double) * icap) + a(sizeof(int) * L * k) + 7 * a(sizeof(int) * n_max) +
-         3 * a(sizeof(int) * icap) + a(sizeof(int) * kBins);
+         a(sizeof(uint64_t) * n_max * kw) + a(sizeof(uint64_t) * n_max) + a(sizeof(uint64_t) * icap) +
+         a(sizeof(uint32_t) * icap) + a(sizeof(int) * L * k) +
+         a(sizeof(int) * L * k) + 7 * a(sizeof(int) * n_max);
 }
 
-// Item buffer: the biggest frontier (n_max*k items), within the shared
-// memory left by everything else; never fewer than n_max items (a truncated
-// round keeps at least one item per run).
-int item_cap(int L, int k, int n_max) {
+// Cut buffer: the biggest frontier (n_max*k items), within the shared memory
+// left by everything else; never fewer than n_max items (a truncated round
+// keeps at least one item per run).
+int item_cap(int L, int k, int n_max, int kw) {
   int cap = n_max * k;
   if (cap > kItemCapMax) cap = kItemCapMax;
   if (cap < n_max) cap = n_max;
-  const size_t fixed = tree_smem_bytes(L, k, n_max, 0) + 4 * 16;
-  const size_t per_item = sizeof(double) + 3 * sizeof(int);
-  const int fit = (int)((kSmemMax - 4096 - fixed) / per_item);
+  const size_t fixed = tree_smem_bytes(L, k, n_max, kw, 0) + 2 * 16 + sizeof(Red);
+  const size_t per_item = sizeof(uint64_t) + sizeof(uint32_t);
+  const int fit = (int)((kSmemMax - 1024 - fixed) / per_item);
   if (cap > fit) cap = fit;
   return cap;
+}
+
+int rank_bits(int k) {
+  int rb = 1;
+  while ((1 << rb) < k) ++rb;
+  return rb;
 }
 
 }  // namespace
@@ -736,7 +1141,10 @@ ddt_status launch_build_tree(const int32_t* ids, const float* zk, const float* l
   p.B_max = B_max;
   p.n_max = B_max + 1;
   p.W = (p.n_max + 31) / 32;
-  p.icap = item_cap(L, k, p.n_max);
+  p.rb = rank_bits(k);
+  p.kw = (L * p.rb + 63) / 64;
+  if (p.kw < 1) p.kw = 1;
+  p.icap = item_cap(L, k, p.n_max, p.kw);
   p.root_token = root_token;
   p.ctx_len = ctx_len;
   p.tok = tok;
@@ -748,7 +1156,7 @@ ddt_status launch_build_tree(const int32_t* ids, const float* zk, const float* l
   p.surrogate = surrogate;
   p.status = dev_status;
   if (batch == 0) return DDT_OK;
-  const size_t smem = tree_smem_bytes(L, k, p.n_max, p.icap);
+  const size_t smem = tree_smem_bytes(L, k, p.n_max, p.kw, p.icap);
   if (ensure_smem_attr((const void*)build_tree_kernel, smem) != cudaSuccess) return DDT_ERR_CUDA;
   build_tree_kernel<<<batch, kThreads, smem, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? DDT_OK : DDT_ERR_CUDA;
