@@ -44,6 +44,7 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 256;           // radix-select digit
 constexpr int kTieList = 256;        // exact ties ranked by counting
 constexpr int kItemCapMax = 16384;
+constexpr int kWide = 64;            // wider levels are numbered from their parents' rows
 constexpr size_t kSmemMax = 227 * 1024;
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
@@ -110,6 +111,8 @@ struct Red {
   int hist[2][kBins];
   int digit, above, hcount, nlist;
   int list[kTieList];
+  int list2[kTieList];
+  __align__(16) uint64_t lkey[kTieList];
   int lvl[DDT_TREE_L_MAX + 2];
 };
 
@@ -373,14 +376,14 @@ __device__ __forceinline__ int block_exscan1(int v, int& total, int& flag, Red* 
   return before + inc - v;
 }
 
-// Rank the nl candidates of red->list (all with the same score key) among
-// themselves under K and keep the `need` best (bit 30 of cid).  Each
-// candidate's (depth, sum, reversed path) is published once, so the ranking
-// compares shared-memory words.  nl <= kTieList.
-__device__ void rank_ties(const Smem& s, double inv_t, int nl, int need, Red* red) {
+// Rank the nl candidates list[0..nl) (indices into ckey/cid, all with the
+// same score key) among themselves under K and keep the `need` best (bit 30
+// of cid).  Each candidate's (depth, sum, reversed path) is published once,
+// so the ranking compares shared-memory words.  nl <= kTieList.
+__device__ void rank_ties(const Smem& s, double inv_t, const int* list, int nl, int need, Red* red) {
   const int tid = threadIdx.x;
   for (int q = tid; q < nl; q += kThreads) {
-    const PK v = make_pk(s, inv_t, (s.cid[red->list[q]] & 0x3FFFFFFFu) << 8);
+    const PK v = make_pk(s, inv_t, (s.cid[list[q]] & 0x3FFFFFFFu) << 8);
     red->csz[q] = v.sz;
     red->crk[q] = v.rk;
     red->cdep[q] = v.dep;
@@ -404,73 +407,93 @@ __device__ void rank_ties(const Smem& s, double inv_t, int nl, int need, Red* re
       else b = !exact && u != q && slow_before(red->chd[u], red->chd[q]);
       rank += b;
     }
-    if (rank < need) s.cid[red->list[q]] |= 0x40000000u;
+    if (rank < need) s.cid[list[q]] |= 0x40000000u;
   }
   __syncthreads();
 }
 
-// Final round with at most one candidate per thread: candidate t has `above`
-// candidates with larger score keys and `eq` with equal ones (itself
-// included); it is kept if above + eq <= R, dropped if above >= R, and only
-// the one group of equal keys that straddles R is ranked under the full order.
-__device__ void cut_small(const Smem& s, int T, int R, Red* red) {
+// Among nl <= kThreads candidates (score keys keys[q], candidate index
+// idx[q], or q when idx is null) keep the `need` K-best (bit 30 of cid).
+// Candidate q has `above` candidates with larger keys and `eq` with equal
+// ones (itself included): kept if above + eq <= need, dropped if
+// above >= need; only the one group of equal keys that straddles `need` is
+// ranked under the full order.
+__device__ void keep_best_of(const Smem& s, const uint64_t* keys, const int* idx, int nl, int need,
+                             Red* red) {
   const int tid = threadIdx.x;
   int above = 0, eq = 0;
   if (tid == 0) red->nlist = 0;
-  if (tid < T) {
-    const uint64_t ki = s.ckey[tid];
+  if (tid < nl) {
+    const uint64_t ki = keys[tid];
     int u = 0;
-    for (; u + 8 <= T; u += 8) {  // eight keys a step (T is even here or the tail catches it)
+    for (; u + 8 <= nl; u += 8) {  // eight keys a step, loads first
       ulonglong2 v[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) v[e] = *reinterpret_cast<const ulonglong2*>(s.ckey + u + 2 * e);
+      for (int e = 0; e < 4; ++e) v[e] = *reinterpret_cast<const ulonglong2*>(keys + u + 2 * e);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         above += (v[e].x > ki) + (v[e].y > ki);
         eq += (v[e].x == ki) + (v[e].y == ki);
       }
     }
-    for (; u < T; ++u) {
-      above += s.ckey[u] > ki;
-      eq += s.ckey[u] == ki;
+    for (; u < nl; ++u) {
+      above += keys[u] > ki;
+      eq += keys[u] == ki;
     }
   }
-  const bool bnd = tid < T && above < R && above + eq > R;
+  const int me = tid < nl ? (idx ? idx[tid] : tid) : 0;
+  const bool bnd = tid < nl && above < need && above + eq > need;
   if (__syncthreads_or(bnd)) {
-    if (bnd) red->list[atomicAdd(&red->nlist, 1)] = tid;
+    if (bnd) {
+      red->list2[atomicAdd(&red->nlist, 1)] = me;
+      red->digit = need - above;  // the same in every member of the group
+    }
     __syncthreads();
-    const int need = R - above;
-    // every member of the straddling group has the same `above`
-    if (bnd && red->list[0] == tid) red->digit = need;
-    __syncthreads();
-    rank_ties(s, g_inv_t, red->nlist, red->digit, red);
+    rank_ties(s, g_inv_t, red->list2, red->nlist, red->digit, red);
   }
-  if (tid < T && (above + eq <= R || (s.cid[tid] & 0x40000000u)))
-    s.cid[tid] = (s.cid[tid] & 0x3FFFFFFFu) | 0x80000000u;
+  if (tid < nl && above + eq <= need) s.cid[me] |= 0x40000000u;
+  __syncthreads();
+}
+
+// Final round with at most one candidate per thread.
+__device__ void cut_small(const Smem& s, int T, int R, Red* red) {
+  keep_best_of(s, s.ckey, nullptr, T, R, red);
+  if (threadIdx.x < T) {
+    const uint32_t c = s.cid[threadIdx.x];
+    if (c & 0x40000000u) s.cid[threadIdx.x] = (c & 0x3FFFFFFFu) | 0x80000000u;
+  }
   __syncthreads();
 }
 
 // Final round: keep the R K-best of the T > R candidates in ckey/cid (bit 31
 // of cid set on the kept ones).  Radix select on the score keys, 8 bits a
-// pass below the bits all keys share; candidates whose keys equal the R-th
-// key are ranked under the full order K.
+// pass below the bits all keys share, until the bucket holding the R-th key
+// has at most kTieList candidates; those are gathered and ranked like a
+// small cut.
 __device__ void cut_best(const Smem& s, double inv_t, int T, int R, Red* red) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint64_t mn = ~0ull, mx = 0;
-  for (int i = tid; i < T; i += kThreads) {
-    const uint64_t kk = s.ckey[i];
-    mn = kk < mn ? kk : mn;
-    mx = kk > mx ? kk : mx;
-  }
+  for (int i0 = tid; i0 < T; i0 += 4 * kThreads) {
+    uint64_t kk[4];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const uint64_t a = shfl_u64(mn, o), b = shfl_u64(mx, o);
-    mn = a < mn ? a : mn;
-    mx = b > mx ? b : mx;
+    for (int e = 0; e < 4; ++e) kk[e] = i0 + e * kThreads < T ? s.ckey[i0 + e * kThreads] : s.ckey[i0];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      mn = kk[e] < mn ? kk[e] : mn;
+      mx = kk[e] > mx ? kk[e] : mx;
+    }
   }
-  if (lane == 0) {
-    red->wmn[warp] = mn;
-    red->wmx[warp] = mx;
+  {
+    uint32_t hi = (uint32_t)(mx >> 32);
+    const uint32_t mhi = __reduce_max_sync(kFull, hi);
+    const uint32_t mlo = __reduce_max_sync(kFull, hi == mhi ? (uint32_t)mx : 0u);
+    hi = (uint32_t)(mn >> 32);
+    const uint32_t nhi = __reduce_min_sync(kFull, hi);
+    const uint32_t nlo = __reduce_min_sync(kFull, hi == nhi ? (uint32_t)mn : ~0u);
+    if (lane == 0) {
+      red->wmx[warp] = ((uint64_t)mhi << 32) | mlo;
+      red->wmn[warp] = ((uint64_t)nhi << 32) | nlo;
+    }
   }
   red->hist[0][tid] = 0;
   __syncthreads();
@@ -481,9 +504,8 @@ __device__ void cut_best(const Smem& s, double inv_t, int T, int R, Red* red) {
     mn = red->wmn[w] < mn ? red->wmn[w] : mn;
     mx = red->wmx[w] > mx ? red->wmx[w] : mx;
   }
-  int need = R;
+  int need = R, bucket = T;
   uint64_t prefix = mx, pmask = ~0ull;
-  bool ties = true;  // all keys equal until shown otherwise
   if (mn != mx) {
     int hb = 63 - __clzll((long long)(mn ^ mx));
     pmask = hb == 63 ? 0ull : (~0ull << (hb + 1));
@@ -493,16 +515,22 @@ __device__ void cut_best(const Smem& s, double inv_t, int T, int R, Red* red) {
       const int shift = hb >= 7 ? hb - 7 : 0;
       const uint64_t dmask = (1ull << (hb - shift + 1)) - 1;
       red->hist[buf ^ 1][tid] = 0;  // the next pass's histogram
-      // warp-aggregated: one atomic per distinct digit in a warp
-      for (int i0 = warp * 32; i0 < T; i0 += kThreads) {
-        const int i = i0 + lane;
-        int dg = -1;
-        if (i < T) {
-          const uint64_t kk = s.ckey[i];
-          if ((kk & pmask) == prefix) dg = (int)((kk >> shift) & dmask);
+      // warp-aggregated: one atomic per distinct digit in a warp; four keys
+      // loaded per step
+      for (int i0 = warp * 32; i0 < T; i0 += 4 * kThreads) {
+        uint64_t kk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = i0 + e * kThreads + lane;
+          kk[e] = i < T ? s.ckey[i] : 0ull;
         }
-        const unsigned grp = __match_any_sync(kFull, dg);
-        if (dg >= 0 && lane == __ffs(grp) - 1) atomicAdd(&red->hist[buf][dg], __popc(grp));
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = i0 + e * kThreads + lane;
+          const int dg = (i < T && (kk[e] & pmask) == prefix) ? (int)((kk[e] >> shift) & dmask) : -1;
+          const unsigned grp = __match_any_sync(kFull, dg);
+          if (dg >= 0 && lane == __ffs(grp) - 1) atomicAdd(&red->hist[buf][dg], __popc(grp));
+        }
       }
       __syncthreads();
       // thread t holds bin 255 - t: scan from the top bin down
@@ -515,40 +543,34 @@ __device__ void cut_best(const Smem& s, double inv_t, int T, int R, Red* red) {
         red->hcount = hcnt;
       }
       __syncthreads();
-      const int digit = red->digit, hc = red->hcount;
       need -= red->above;
-      prefix |= (uint64_t)digit << shift;
+      bucket = red->hcount;
+      prefix |= (uint64_t)red->digit << shift;
       pmask |= dmask << shift;
       buf ^= 1;
-      if (hc == need) {
-        ties = false;
-        break;
-      }
-      if (shift == 0) break;
+      if (bucket <= kTieList || shift == 0) break;
       hb = shift - 1;
     }
   }
-  if (!ties) {
-    for (int i = tid; i < T; i += kThreads)
-      if ((s.ckey[i] & pmask) >= prefix) s.cid[i] |= 0x80000000u;
-    __syncthreads();
-    return;
-  }
-  // keys above the R-th key are kept; `need` of those equal to it are ranked
+  // above the bucket: kept; the bucket: gathered and ranked
   if (tid == 0) red->nlist = 0;
   __syncthreads();
   for (int i = tid; i < T; i += kThreads) {
-    const uint64_t kk = s.ckey[i];
-    if (kk > prefix) s.cid[i] |= 0x80000000u;
-    if (kk == prefix) {
+    const uint64_t km = s.ckey[i] & pmask;
+    if (km > prefix) s.cid[i] |= 0x80000000u;
+    if (km == prefix) {
       const int q = atomicAdd(&red->nlist, 1);
-      if (q < kTieList) red->list[q] = i;
+      if (q < kTieList) {
+        red->list[q] = i;
+        red->lkey[q] = s.ckey[i];
+      }
     }
   }
   __syncthreads();
   const int nl = red->nlist;
+  __syncthreads();  // every thread has read nlist before it is reused
   if (nl <= kTieList) {
-    rank_ties(s, inv_t, nl, need, red);
+    keep_best_of(s, red->lkey, red->list, nl, need, red);
   } else {
     // a very large exact tie: take the K-best undecided tied candidate, need times
     for (int t = 0; t < need; ++t) {
@@ -704,7 +726,9 @@ __global__ void __launch_bounds__(kThreads, 1) build_tree_kernel(TreeParams p) {
     s.nrank[0] = 0;
     s.nnext[0] = 0;
     s.nrk[0] = 0ull;
+    s.ninv[0] = 0;
   }
+  if (tid < L + 2) red.lvl[tid] = tid == 0 ? 1 : 0;
   __syncthreads();
   // id ranks: within a position, token order is id-rank order
   for (int i = tid; i < L * k; i += kThreads) {
@@ -756,6 +780,8 @@ __global__ void __launch_bounds__(kThreads, 1) build_tree_kernel(TreeParams p) {
       s.nnext[t] = t < len ? 1 : 0;
       for (int w = 0; w < p.kw; ++w) s.pkey[(size_t)t * p.kw + w] = 0ull;
       s.nrk[t] = 0ull;  // one node per depth: never compared
+      s.ninv[t] = 0;
+      red.lvl[t] = 1;
     }
     if (tid == 0) s.nnext[0] = len > 0 ? 1 : 0;
     nn = 1 + len;
@@ -802,11 +828,28 @@ __global__ void __launch_bounds__(kThreads, 1) build_tree_kernel(TreeParams p) {
     }
     // run items before theta (tk == 0: no first child exists, all are)
     int sum = 0, ctie = 0;
-    for (int x = tid; x < nn; x += kThreads) {
-      const int d = s.ndep[x];
-      const int c = d < L ? count_fast(s, inv_t, x, d, s.nnext[x], kb, tk, ctie) : 0;
-      ncnt[x] = c;
-      sum += c;
+    if (nn <= kWarps) {
+      // few nodes: a warp per node, a lane per rank of its run
+      if (warp < nn) {
+        const int x = warp, d = s.ndep[x], nx = s.nnext[x];
+        const int len = d < L ? kb - nx : 0;
+        const bool in = lane < len;
+        const uint64_t kk = in ? item_key(s, inv_t, s.nsz[x], d, nx + lane) : 0ull;
+        const unsigned gt = __ballot_sync(kFull, in && kk > tk);
+        const unsigned eqb = __ballot_sync(kFull, in && kk == tk);
+        const int c = gt == kFull ? 32 : __ffs(~gt) - 1;
+        if (c < len && ((eqb >> c) & 1u)) ctie = 1;
+        if (lane == 0) ncnt[x] = c;
+      }
+      ctie = __syncthreads_or(ctie);
+      sum = tid < nn ? ncnt[tid] : 0;
+    } else {
+      for (int x = tid; x < nn; x += kThreads) {
+        const int d = s.ndep[x];
+        const int c = d < L ? count_fast(s, inv_t, x, d, s.nnext[x], kb, tk, ctie) : 0;
+        ncnt[x] = c;
+        sum += c;
+      }
     }
     int T;
     int off = block_exscan1(sum, T, ctie, &red);
@@ -887,16 +930,16 @@ __global__ void __launch_bounds__(kThreads, 1) build_tree_kernel(TreeParams p) {
       // final round: stage the T candidates and keep the R best
       int o = off;
       for (int x = tid; x < nn; x += kThreads) {
-        const int c = ncnt[x];
-        if (c > 0) {
-          const int d = s.ndep[x], nx = s.nnext[x];
-          const double base = s.nsz[x];
-          for (int i = 0; i < c; ++i) {
-            s.ckey[o + i] = item_key(s, inv_t, base, d, nx + i);
-            s.cid[o + i] = ((uint32_t)x << 8) | (uint32_t)(nx + i);
-          }
-          o += c;
-        }
+        const int c = ncnt[x], nx = s.nnext[x];
+        for (int i = 0; i < c; ++i) s.cid[o + i] = ((uint32_t)x << 8) | (uint32_t)(nx + i);
+        o += c;
+      }
+      __syncthreads();
+#pragma unroll 4
+      for (int j = tid; j < T; j += kThreads) {
+        const uint32_t e = s.cid[j];
+        const int x = (int)(e >> 8);
+        s.ckey[j] = item_key(s, inv_t, s.nsz[x], s.ndep[x], (int)(e & 0xFFu));
       }
       __syncthreads();
       if (T <= kThreads)
@@ -916,54 +959,57 @@ __global__ void __launch_bounds__(kThreads, 1) build_tree_kernel(TreeParams p) {
       int nof = 0;
       off = block_exscan1(sum, T, nof, &red);
     }
-    // create the selected items as nodes (loads of four at a time first)
+    // create the selected items as nodes: the owners write parent and rank,
+    // then one thread per new node fills in the rest
     int id = nn + off;
     for (int x = tid; x < nn; x += kThreads) {
       const int c = ncnt[x];
       if (c > 0) {
-        const int d = s.ndep[x], nx = s.nnext[x];
-        const double base = s.nsz[x], Sd = s.S[d + 1];
-        const uint64_t pk0 = s.pkey[(size_t)x * s.kw], prk = s.nrk[x];
-        for (int i0 = 0; i0 < c; i0 += 4) {
-          double z[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) z[e] = i0 + e < c ? s.zt[d * k + nx + i0 + e] : 0.0;
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            if (i0 + e < c) {
-              const int r = nx + i0 + e, idn = id + i0 + e;
-              const double sz = __dadd_rn(base, z[e]);
-              s.nsz[idn] = sz;
-              s.nsc[idn] = __dsub_rn(__dmul_rn(inv_t, sz), Sd);
-              s.npar[idn] = x;
-              s.ndep[idn] = d + 1;
-              s.nrank[idn] = r;
-              s.nnext[idn] = 0;
-              s.nrk[idn] = rev_key(s, prk, d, r);
-              if (s.kw == 1)
-                s.pkey[idn] = pk0 | ((uint64_t)r << (64 - (d + 1) * s.rb));
-              else
-                make_path_key(s, x, idn, d, r);
-            }
-          }
+        const int nx = s.nnext[x];
+        for (int i = 0; i < c; ++i) {
+          s.npar[id + i] = x;
+          s.nrank[id + i] = nx + i;
         }
         id += c;
         s.nnext[x] = nx + c;
       }
     }
     __syncthreads();
+    for (int j = tid; j < T; j += kThreads) {
+      const int idn = nn + j, x = s.npar[idn], r = s.nrank[idn], d = s.ndep[x];
+      const double sz = __dadd_rn(s.nsz[x], s.zt[d * k + r]);
+      s.nsz[idn] = sz;
+      s.nsc[idn] = score_of(s, inv_t, sz, d + 1);
+      s.ndep[idn] = d + 1;
+      s.nnext[idn] = 0;
+      s.ninv[idn] = atomicAdd(&red.lvl[d + 1], 1);  // slot within its depth
+      s.nrk[idn] = rev_key(s, s.nrk[x], d, r);
+      if (s.kw == 1)
+        s.pkey[idn] = s.pkey[x] | ((uint64_t)r << (64 - (d + 1) * s.rb));
+      else
+        make_path_key(s, x, idn, d, r);
+    }
+    __syncthreads();
     nn += T;
     nsel += T;
   }
 
+  // surrogate: sum of exp(score) over the draft nodes (nsc is free after this)
+  {
+    double acc = 0.0;
+    for (int x = 1 + tid; x < nn; x += kThreads) acc += exp(s.nsc[x]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
+    if (lane == 0) red.wd[warp] = acc;
+  }
+
   // ---------------- breadth-first numbering ----------------
-  // Rows are ordered by (depth, rank path): a node's row is the first row of
-  // its depth plus the number of same-depth nodes with a smaller path key.
-  if (tid < L + 2) red.lvl[tid] = 0;
-  __syncthreads();
-  // a node's slot within its depth bucket (in ninv, free until the rows)
-  for (int x = tid; x < nn; x += kThreads) s.ninv[x] = atomicAdd(&red.lvl[s.ndep[x]], 1);
-  __syncthreads();
+  // Rows are ordered by (depth, rank path).  lvl[t] holds the node count of
+  // depth t and ninv[x] node x's slot among them, both kept since the node
+  // was created.  A level of at most kWide nodes is ranked by counting the
+  // same-depth nodes with smaller path keys (all such levels at once); a
+  // wider level takes its rows from its parents' rows: the children of the
+  // parent in row j follow those of rows < j, in rank order.
   if (warp == 0) {  // lvl[t] <- first row of depth t, for t = 0..L+1
     int v[3], sm = 0;
 #pragma unroll
@@ -989,32 +1035,37 @@ __global__ void __launch_bounds__(kThreads, 1) build_tree_kernel(TreeParams p) {
   const bool copy_keys = (int64_t)nn * kw * 8 <= 12 * (int64_t)icap;
   uint64_t* bkey = s.ckey;
   for (int x = tid; x < nn; x += kThreads) {
-    const int q = red.lvl[s.ndep[x]] + s.ninv[x];
+    const int d = s.ndep[x];
+    const int q = red.lvl[d] + s.ninv[x];
     bucket[q] = x;
-    if (copy_keys)
+    if (copy_keys && red.lvl[d + 1] - red.lvl[d] <= kWide)
       for (int w = 0; w < kw; ++w) bkey[(size_t)q * kw + w] = s.pkey[(size_t)x * kw + w];
   }
   __syncthreads();
-  // rank bucket position q among its depth: threads of a warp take
-  // consecutive positions, so they mostly scan the same bucket together
+  // narrow levels: rank bucket position q among its depth; threads of a warp
+  // take consecutive positions, so they mostly scan the same bucket together
   for (int q = tid; q < nn; q += kThreads) {
     const int x = bucket[q];
     const int d = s.ndep[x], lo = red.lvl[d], hi = red.lvl[d + 1];
+    if (hi - lo > kWide) continue;
     int below = 0;
     if (copy_keys && kw == 1) {
       const uint64_t kx = bkey[q];
       int u = lo;
-      if ((u & 1) && u < hi) below += bkey[u++] < kx;  // then 16-byte aligned pairs
-      for (; u + 1 < hi; u += 2) {
-        const ulonglong2 v = *reinterpret_cast<const ulonglong2*>(bkey + u);
-        below += (v.x < kx) + (v.y < kx);
+      if ((u & 1) && u < hi) below += bkey[u++] < kx;  // then 16-byte aligned
+      for (; u + 8 <= hi; u += 8) {                      // eight keys a step
+        ulonglong2 v[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[e] = *reinterpret_cast<const ulonglong2*>(bkey + u + 2 * e);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) below += (v[e].x < kx) + (v[e].y < kx);
       }
-      if (u < hi) below += bkey[u] < kx;
+      for (; u < hi; ++u) below += bkey[u] < kx;
     } else if (copy_keys && kw == 2) {
       const uint64_t k0 = bkey[2 * q], k1 = bkey[2 * q + 1];
       for (int u = lo; u < hi; ++u) {
         const ulonglong2 v = *reinterpret_cast<const ulonglong2*>(bkey + 2 * u);
-        below += (v.x < k0) || (v.x == k0 && v.y < k1);
+        below += (int)(v.x < k0) | ((int)(v.x == k0) & (int)(v.y < k1));
       }
     } else {
       for (int u = lo; u < hi; ++u) below += path_less(s, bucket[u], x);
@@ -1023,6 +1074,33 @@ __global__ void __launch_bounds__(kThreads, 1) build_tree_kernel(TreeParams p) {
     s.ninv[lo + below] = x;
   }
   __syncthreads();
+  // wide levels, in depth order: first-child rows of the level above by a
+  // scan of its child counts in row order, then each node's row
+  int* nfc = reinterpret_cast<int*>(s.nsc);
+  for (int d = 1; d <= L; ++d) {
+    const int lo = red.lvl[d], hi = red.lvl[d + 1];
+    if (hi - lo <= kWide) continue;
+    const int plo = red.lvl[d - 1], pw = lo - plo;
+    const int c = (pw + kThreads - 1) / kThreads;
+    const int r0 = plo + min(tid * c, pw), r1 = plo + min((tid + 1) * c, pw);
+    int sum = 0;
+    for (int j = r0; j < r1; ++j) sum += s.nnext[s.ninv[j]];
+    int tot, nof = 0;
+    int run = lo + block_exscan1(sum, tot, nof, &red);
+    for (int j = r0; j < r1; ++j) {
+      const int x = s.ninv[j];
+      nfc[x] = run;
+      run += s.nnext[x];
+    }
+    __syncthreads();
+    for (int q = lo + tid; q < hi; q += kThreads) {
+      const int x = bucket[q];
+      const int row = nfc[s.npar[x]] + s.nrank[x];
+      s.nrow[x] = row;
+      s.ninv[row] = x;
+    }
+    __syncthreads();
+  }
 
   // ---------------- outputs ----------------
   const int32_t ctx = p.ctx_len ? p.ctx_len[b] : 0;
@@ -1078,13 +1156,6 @@ __global__ void __launch_bounds__(kThreads, 1) build_tree_kernel(TreeParams p) {
   } else {
     for (int i = nn * W + tid; i < NM * W; i += kThreads) o_mask[i] = 0u;
   }
-  // surrogate: sum of exp(score) over the draft nodes
-  double acc = 0.0;
-  for (int x = 1 + tid; x < nn; x += kThreads) acc += exp(s.nsc[x]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
-  if (lane == 0) red.wd[warp] = acc;
-  __syncthreads();
   if (tid == 0) {
     double t = 0.0;
     for (int w = 0; w < kWarps; ++w) t += red.wd[w];
