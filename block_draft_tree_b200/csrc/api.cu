@@ -25,17 +25,19 @@ cudaError_t ensure_smem_attr(const void* func, size_t bytes) {
   return e;
 }
 
-namespace {
-
-size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
-bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
-
-int sm_count() {
+int device_sm_count() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) n = 148;
   return n > 0 ? n : 148;
 }
+
+namespace {
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+int sm_count() { return device_sm_count(); }
 
 bool ws_ok(const void* ws, size_t have, size_t need) {
   if (need == 0) return true;

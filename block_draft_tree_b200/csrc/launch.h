@@ -12,6 +12,9 @@ namespace ddt {
 // Raise a kernel's dynamic shared-memory limit once per (kernel, device).
 cudaError_t ensure_smem_attr(const void* func, size_t bytes);
 
+// Multiprocessors of the current device.
+int device_sm_count();
+
 size_t topk_workspace_size(int rows, int V, int k);
 ddt_status launch_topk(const void* logits, ddt_dtype dt, int rows, int V, int64_t row_stride,
                        int k, float inv_t, int32_t* ids, float* zk, float* logp, float* lse,
