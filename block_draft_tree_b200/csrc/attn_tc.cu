@@ -40,9 +40,10 @@ constexpr int BM = 128;                   // query rows per tile (MMA M)
 constexpr int BN = 128;                   // tokens per tile (MMA N of QK^T, K of PV)
 constexpr int D = 128;                    // head dim
 constexpr int kStages = 3;                // K/V ring depth
-constexpr int kThreads = 192;             // warp 0 TMA, warp 1 MMA, warps 2-5 softmax
+constexpr int kThreads = 320;             // warp 0 TMA, warp 1 MMA, warps 2-9 softmax
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP = 384;
+constexpr uint32_t kColX = 448;  // exchange columns of the softmax warp pairs
 constexpr int kHalf = BN * 128;           // one 64-wide d half: 128 rows x 128 B
 constexpr int kTile = 2 * kHalf;          // 32 KB
 constexpr long long kWaitCycles = 2000000000LL;
@@ -188,6 +189,28 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t tmem_ld1(uint32_t taddr) {
+  uint32_t v;
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(v) : "r"(taddr) : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+  return v;
+}
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+// AND of `pred` over a softmax warp pair (through a spare TMEM column).
+__device__ __forceinline__ bool __syncthreads_and_pair(bool pred, int bar_id, uint32_t taddr, int half) {
+  const bool w = __all_sync(0xFFFFFFFFu, pred);
+  tmem_st1(taddr + half, w ? 1u : 0u);
+  tmem_st_wait();
+  fence_before();
+  named_bar_sync(bar_id, 64);
+  fence_after();
+  return w && tmem_ld1(taddr + (half ^ 1)) != 0u;
+}
 
 // Distributed shared memory of the cluster (the KV splits of one query tile).
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -290,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t part_row0 = (((int64_t)grp * p.qtiles + qtile) * p.nsplit + split) * BM;
 
   if (ntiles == 0 && !p.cluster) {  // nothing in this split: an empty partial (or zero rows)
-    if (tid >= 64) {
+    if (tid >= 64 && tid < 64 + BM) {
       const int row = tid - 64;
       const int qr = q0 + row;
       if (p.nsplit > 1) {
@@ -316,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&bars->s_full[0], 1);
     mbar_init(&bars->s_full[1], 1);
-    mbar_init(&bars->p_full, 128);
+    mbar_init(&bars->p_full, 256);
     mbar_init(&bars->pv_done, 1);
     bars->abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -428,57 +451,74 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax warps
-    const int quarter = warp & 3;
+    // Two warps per TMEM lane quarter: warp w serves rows 32*(w%4)..+31 and
+    // the 64 score columns of half h = (w-2)/4.  The pair exchanges its row
+    // maxima (and, at the end, row sums) through spare TMEM columns and a
+    // 64-thread named barrier, every iteration, so the pair always meets the
+    // same barriers, also after a bounded wait gave up.
+    const int quarter = warp & 3, half = (warp - 2) >> 2;
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     const int qr = q0 + row;
     const int j = qr / g;
     const bool row_valid = qr < R && j < n;
     const uint32_t* mrow = p.mask + ((int64_t)b * p.n_max + (j < p.n_max ? j : 0)) * p.W;
+    const int bar_id = 1 + quarter;
+    const int c0 = half * (BN / 2);  // first score column of this half
     float m_used = -INFINITY, l = 0.f;
-    uint32_t r[BN];
+    uint32_t r[BN / 2];
     bool ok = true;
-    for (int i = 0; i < ntiles && ok; ++i) {
+    for (int i = 0; i < ntiles; ++i) {
       const TileInfo ti = tile_info(t_lo + i, nct, T, n);
-      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->s_full[i & 1], (uint32_t)(i >> 1) & 1u, bars));
-      if (!ok) break;
-      fence_after();
-      const uint32_t s_col = (i & 1) ? kColS1 : kColS0;
-#pragma unroll
-      for (int c = 0; c < BN / 32; ++c) tmem_ld32(lane_base + s_col + 32 * c, r + 32 * c);
-      tmem_ld_wait();
-      // Row maximum in the raw score domain (scale > 0 commutes with max).
-      // Full context tiles need no masking; partial and tree tiles mask with
-      // -inf, which the exp below turns into 0.
+      if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->s_full[i & 1], (uint32_t)(i >> 1) & 1u, bars));
+      float mx_raw = -INFINITY;
       const float c_log2 = p.scale_log2;
-      const bool full_tile = !ti.tree && ti.cnt == BN && row_valid;
-      if (!full_tile) {
-        uint32_t mw[4] = {0u, 0u, 0u, 0u};
-        if (ti.tree && row_valid) {
+      if (ok) {
+        fence_after();
+        const uint32_t s_col = ((i & 1) ? kColS1 : kColS0) + c0;
+        tmem_ld32(lane_base + s_col, r);
+        tmem_ld32(lane_base + s_col + 32, r + 32);
+        tmem_ld_wait();
+        // Full context tiles need no masking; partial and tree tiles mask
+        // with -inf, which the exp below turns into 0.
+        const bool full_tile = !ti.tree && ti.cnt == BN && row_valid;
+        if (!full_tile) {
+          uint32_t mw[2] = {0u, 0u};
+          if (ti.tree && row_valid) {
 #pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            const int word = (ti.base >> 5) + w;
-            mw[w] = word < p.W ? mrow[word] : 0u;
-          }
-        } else if (!ti.tree && row_valid) {
+            for (int w = 0; w < 2; ++w) {
+              const int word = ((ti.base + c0) >> 5) + w;
+              mw[w] = word < p.W ? mrow[word] : 0u;
+            }
+          } else if (!ti.tree && row_valid) {
 #pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            const int lo = 32 * w;
-            mw[w] = ti.cnt >= lo + 32 ? 0xFFFFFFFFu : (ti.cnt > lo ? ((1u << (ti.cnt - lo)) - 1u) : 0u);
+            for (int w = 0; w < 2; ++w) {
+              const int lo = c0 + 32 * w;
+              mw[w] = ti.cnt >= lo + 32 ? 0xFFFFFFFFu : (ti.cnt > lo ? ((1u << (ti.cnt - lo)) - 1u) : 0u);
+            }
           }
+#pragma unroll
+          for (int c = 0; c < BN / 2; ++c)
+            if (!((mw[c >> 5] >> (c & 31)) & 1u)) r[c] = 0xFF800000u;  // -inf
         }
+        float mx8[8];
 #pragma unroll
-        for (int c = 0; c < BN; ++c)
-          if (!((mw[c >> 5] >> (c & 31)) & 1u)) r[c] = 0xFF800000u;  // -inf
+        for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(r[e]);
+#pragma unroll
+        for (int c = 8; c < BN / 2; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(r[c]));
+        mx_raw = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       }
-      float mx8[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(r[e]);
-#pragma unroll
-      for (int c = 8; c < BN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(r[c]));
-      const float mx_raw = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      const float mx = mx_raw * c_log2;
+      // exchange the half-row maxima (raw score domain; scale > 0 commutes with max)
+      const uint32_t xcol = kColX + 2 * (i & 1);
+      tmem_st1(lane_base + xcol + half, __float_as_uint(mx_raw));
+      tmem_st_wait();
+      fence_before();
+      named_bar_sync(bar_id, 64);
+      fence_after();
+      const float other = __uint_as_float(tmem_ld1(lane_base + xcol + (half ^ 1)));
+      if (!ok) continue;
+      const float mx = fmaxf(mx_raw, other) * c_log2;
       const float m_new = fmaxf(m_used, mx);
       const bool move = m_new > m_used + kRescaleLog2 || (m_used == -INFINITY && m_new != -INFINITY);
       const float m_tgt = move ? m_new : m_used;
@@ -487,11 +527,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int e = 0; e < 8; ++e) rs8[e] = 0.f;
       if (m_tgt == -INFINITY) {
 #pragma unroll
-        for (int c = 0; c < BN / 2; ++c) r[c] = 0u;
+        for (int c = 0; c < BN / 4; ++c) r[c] = 0u;
       } else {
         // p = 2^(s*c - m): one FFMA and one MUFU per score; bf16 pairs packed in place
 #pragma unroll
-        for (int c = 0; c < BN; c += 2) {
+        for (int c = 0; c < BN / 2; c += 2) {
           const float a = ex2(fmaf(__uint_as_float(r[c]), c_log2, -m_tgt));
           const float bb = ex2(fmaf(__uint_as_float(r[c + 1]), c_log2, -m_tgt));
           rs8[(c >> 1) & 7] += a + bb;
@@ -503,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // PV of the previous tile must be done before P and O are touched
       if (i > 0) {
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->pv_done, (uint32_t)(i - 1) & 1u, bars));
-        if (!ok) break;
+        if (!ok) continue;
       }
       fence_after();
       if (move) {
@@ -511,30 +551,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float alpha = ex2(m_used - m_new);
           uint32_t o[32];
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            tmem_ld32(lane_base + kColO + 32 * c, o);
+          for (int c = 0; c < D / 64; ++c) {
+            const uint32_t oc = kColO + half * (D / 2) + 32 * c;
+            tmem_ld32(lane_base + oc, o);
             tmem_ld_wait();
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st32(lane_base + kColO + 32 * c, o);
+            tmem_st32(lane_base + oc, o);
           }
           l *= alpha;
         }
         m_used = m_new;
       }
       l += rs;
-      tmem_st32(lane_base + kColP, r);
-      tmem_st32(lane_base + kColP + 32, r + 32);
-      // token row `row` of a partial tile: zero its V row so that 0 * garbage cannot
-      // turn into NaN in the PV product
+      tmem_st32(lane_base + kColP + half * (BN / 4), r);
+      // token row `row` of a partial tile: zero its V row (this half's 64
+      // dims) so that 0 * garbage cannot turn into NaN in the PV product
       if (row >= ti.cnt) {
-        uint4* vrow0 = (uint4*)(sV + (i % kStages) * kTile + row * 128);
-        uint4* vrow1 = (uint4*)(sV + (i % kStages) * kTile + kHalf + row * 128);
+        uint4* vrow = (uint4*)(sV + (i % kStages) * kTile + half * kHalf + row * 128);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          vrow0[e] = make_uint4(0, 0, 0, 0);
-          vrow1[e] = make_uint4(0, 0, 0, 0);
-        }
+        for (int e = 0; e < 8; ++e) vrow[e] = make_uint4(0, 0, 0, 0);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       }
       tmem_st_wait();
@@ -542,25 +578,41 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&bars->p_full);
     }
     if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&bars->pv_done, (uint32_t)(ntiles - 1) & 1u, bars));
+    // the row sum over both halves
+    tmem_st1(lane_base + kColX + 4 + half, __float_as_uint(l));
+    tmem_st_wait();
+    fence_before();
+    named_bar_sync(bar_id, 64);
     fence_after();
-    // epilogue: O row -> final output, a cluster partial in shared memory,
-    // or a partial in the workspace
+    const float l_row = l + __uint_as_float(tmem_ld1(lane_base + kColX + 4 + (half ^ 1)));
+    const bool ok_row = __syncthreads_and_pair(ok, bar_id, lane_base + kColX + 6, half);
+    // epilogue: this half's 64 dims of the O row -> final output, a cluster
+    // partial in shared memory, or a partial in the workspace
     float* po = p.cluster ? (float*)(sK) + row * D : p.part_o + (part_row0 + row) * D;
     const bool final_out = p.nsplit == 1;
-    const float inv = (l > 0.f) ? 1.f / l : 0.f;
+    const float inv = (l_row > 0.f) ? 1.f / l_row : 0.f;
     uint16_t* dst = nullptr;
     if (final_out && qr < R)
       dst = p.out + (((int64_t)b * p.n_max + j) * p.hq + (kvh * g + qr % g)) * D;
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
+    for (int cc = 0; cc < D / 64; ++cc) {
+      const int c = half * (D / 64) + cc;  // 32-column block of O
       uint32_t o[32];
       tmem_ld32(lane_base + kColO + 32 * c, o);
       tmem_ld_wait();
-      if (!ok || !row_valid) {
+      if (!ok_row || !row_valid) {
 #pragma unroll
         for (int e = 0; e < 32; ++e) o[e] = 0u;
       }
-      if (!final_out) {
+      if (p.cluster) {
+        // 16-byte chunk k of the row goes to slot k ^ (row & 31), so that the
+        // 32 rows of a warp hit different banks
+        float4* q4 = (float4*)po;
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          q4[(8 * c + e) ^ (row & 31)] = make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
+                                                     __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]));
+      } else if (!final_out) {
         float4* q4 = (float4*)(po + 32 * c);
 #pragma unroll
         for (int e = 0; e < 8; ++e)
@@ -579,18 +631,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < 4; ++e) d4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
       }
     }
-    const bool has = ok && row_valid && l > 0.f;
-    if (p.cluster) {
-      ((float2*)(sK + BM * D * 4))[row] = has ? make_float2(m_used, l) : make_float2(-INFINITY, 0.f);
-    } else if (!final_out) {
-      p.part_ml[part_row0 + row] = has ? make_float2(m_used, l) : make_float2(-INFINITY, 0.f);
-    } else if (dst && p.lse_out) {
-      p.lse_out[((int64_t)b * p.n_max + j) * p.hq + (kvh * g + qr % g)] =
-          has ? (m_used + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+    const bool has = ok_row && row_valid && l_row > 0.f;
+    if (half == 0) {
+      if (p.cluster) {
+        ((float2*)(sK + BM * D * 4))[row] = has ? make_float2(m_used, l_row) : make_float2(-INFINITY, 0.f);
+      } else if (!final_out) {
+        p.part_ml[part_row0 + row] = has ? make_float2(m_used, l_row) : make_float2(-INFINITY, 0.f);
+      } else if (dst && p.lse_out) {
+        p.lse_out[((int64_t)b * p.n_max + j) * p.hq + (kvh * g + qr % g)] =
+            has ? (m_used + __log2f(l_row)) * 0.69314718055994531f : -INFINITY;
+      }
     }
   }
 
-  if (!work && tid >= 64)  // empty split of a cluster
+  if (!work && tid >= 64 && tid < 64 + BM)  // empty split of a cluster
     ((float2*)(sK + BM * D * 4))[tid - 64] = make_float2(-INFINITY, 0.f);
 
   fence_before();
@@ -606,53 +660,63 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---------------- on-chip merge of the cluster's split partials ----------------
   // CTA r of the cluster owns query rows [r*rpc, (r+1)*rpc) of the tile; each
-  // warp takes one row at a time, a lane 4 of its 128 dims, and loads every
-  // split's (m, l) and O slice from the peers' shared memory in one go.
+  // warp takes two rows at a time, a lane 4 of their 128 dims, and loads every
+  // split's (m, l) and O slice of both from the peers' shared memory in one go
+  // (O rows are stored with their 16-byte chunks XOR-swizzled by row).
   cluster_sync();
   {
     const int S = p.nsplit;  // 2..8
     const int rank = (int)cluster_rank();
     const int rpc = (BM + S - 1) / S;
     const uint32_t o_base = smem_u32(sK), ml_base = smem_u32(sK + BM * D * 4);
-    for (int r = rank * rpc + warp; r < min(BM, (rank + 1) * rpc); r += kThreads / 32) {
-      const int qr2 = q0 + r;
-      if (qr2 >= R) break;
-      const int j2 = qr2 / g, h2 = kvh * g + qr2 % g;
-      // every split's (m, l) and O slice, loaded together
-      float2 ml[8];
-      float4 v[8];
+    const int r_end = min(min(BM, (rank + 1) * rpc), R - q0);
+    for (int r0 = rank * rpc + 2 * warp; r0 < r_end; r0 += 2 * (kThreads / 32)) {
+      // two rows: every split's (m, l) and O slice of both, loaded together
+      float2 ml[2][8];
+      float4 v[2][8];
 #pragma unroll
-      for (int s2 = 0; s2 < 8; ++s2)
-        if (s2 < S) {
-          ml[s2] = ld_cluster_f2(map_to_rank(ml_base + r * 8, s2));
-          v[s2] = ld_cluster_f4(map_to_rank(o_base + (r * D + 4 * lane) * 4, s2));
-        }
-      float M = -INFINITY;
-#pragma unroll
-      for (int s2 = 0; s2 < 8; ++s2)
-        if (s2 < S) M = fmaxf(M, ml[s2].x);
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      float Lsum = 0.f;
-      if (M != -INFINITY && j2 < n) {
+      for (int q = 0; q < 2; ++q) {
+        const int r = min(r0 + q, r_end - 1);
 #pragma unroll
         for (int s2 = 0; s2 < 8; ++s2)
-          if (s2 < S && ml[s2].x != -INFINITY) {
-            const float wgt = ex2(ml[s2].x - M);
-            Lsum += ml[s2].y * wgt;
-            acc.x = fmaf(wgt, v[s2].x, acc.x);
-            acc.y = fmaf(wgt, v[s2].y, acc.y);
-            acc.z = fmaf(wgt, v[s2].z, acc.z);
-            acc.w = fmaf(wgt, v[s2].w, acc.w);
+          if (s2 < S) {
+            ml[q][s2] = ld_cluster_f2(map_to_rank(ml_base + r * 8, s2));
+            v[q][s2] = ld_cluster_f4(map_to_rank(o_base + (r * D + 4 * (lane ^ (r & 31))) * 4, s2));
           }
       }
-      const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-      __nv_bfloat162 h0 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-      __nv_bfloat162 h1 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-      uint2* dst2 = (uint2*)(p.out + (((int64_t)b * p.n_max + j2) * p.hq + h2) * D);
-      dst2[lane] = make_uint2(*(uint32_t*)&h0, *(uint32_t*)&h1);
-      if (lane == 0 && p.lse_out)
-        p.lse_out[((int64_t)b * p.n_max + j2) * p.hq + h2] =
-            Lsum > 0.f ? (M + __log2f(Lsum)) * 0.69314718055994531f : -INFINITY;
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int r = r0 + q;
+        if (r >= r_end) break;
+        const int qr2 = q0 + r;
+        const int j2 = qr2 / g, h2 = kvh * g + qr2 % g;
+        float M = -INFINITY;
+#pragma unroll
+        for (int s2 = 0; s2 < 8; ++s2)
+          if (s2 < S) M = fmaxf(M, ml[q][s2].x);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float Lsum = 0.f;
+        if (M != -INFINITY && j2 < n) {
+#pragma unroll
+          for (int s2 = 0; s2 < 8; ++s2)
+            if (s2 < S && ml[q][s2].x != -INFINITY) {
+              const float wgt = ex2(ml[q][s2].x - M);
+              Lsum += ml[q][s2].y * wgt;
+              acc.x = fmaf(wgt, v[q][s2].x, acc.x);
+              acc.y = fmaf(wgt, v[q][s2].y, acc.y);
+              acc.z = fmaf(wgt, v[q][s2].z, acc.z);
+              acc.w = fmaf(wgt, v[q][s2].w, acc.w);
+            }
+        }
+        const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+        __nv_bfloat162 h0 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+        __nv_bfloat162 h1 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+        uint2* dst2 = (uint2*)(p.out + (((int64_t)b * p.n_max + j2) * p.hq + h2) * D);
+        dst2[lane] = make_uint2(*(uint32_t*)&h0, *(uint32_t*)&h1);
+        if (lane == 0 && p.lse_out)
+          p.lse_out[((int64_t)b * p.n_max + j2) * p.hq + h2] =
+              Lsum > 0.f ? (M + __log2f(Lsum)) * 0.69314718055994531f : -INFINITY;
+      }
     }
   }
   cluster_sync();  // peers' shared memory stays alive until every CTA has read it
@@ -766,8 +830,13 @@ bool attn_tc_eligible(const ddt_attn_args* a) {
   return tc::encode_fn() != nullptr;
 }
 
-// KV-split plan of the tensor-core path: one CTA per SM, as few waves and
-// splits as possible.
+bool attn_tc_cluster(int nsplit, long clusters);
+
+// KV-split plan of the tensor-core path (one CTA per SM).  Splits that can
+// run as co-resident clusters merge on chip, so among those the plan takes
+// the one with the fewest tiles per split; it falls back to as few waves
+// and splits as possible (with partials and a combine kernel) only when no
+// cluster split fits or a plain split is clearly shorter.
 void attn_tc_plan(const ddt_attn_args* a, int sms, int* qtiles, int* nsplit, int* tps) {
   const int g = a->hq / a->hkv;
   const long R = (long)a->n_max * g;
@@ -786,10 +855,26 @@ void attn_tc_plan(const ddt_attn_args* a, int sms, int* qtiles, int* nsplit, int
     }
   }
   int t = (tiles + best - 1) / best;
+  const long plain_waves = (base * ((tiles + t - 1) / t) + sms - 1) / sms;
+  // the partials and their combine cost about as much as kMergeTiles tiles
+  constexpr int kMergeTiles = 3;
+  const long plain_cost = plain_waves * t + (best > 1 ? kMergeTiles : 0);
+  int cbest = 0, ct = 0;
+  for (int s = 2; s <= 8 && s <= tiles; ++s) {
+    const int ts = (tiles + s - 1) / s;
+    if (attn_tc_cluster(s, base) && (cbest == 0 || ts < ct)) {
+      cbest = s;
+      ct = ts;
+    }
+  }
+  if (cbest > 0 && ct <= plain_cost) {
+    *tps = ct;
+    *nsplit = (tiles + ct - 1) / ct;
+    return;
+  }
   *tps = t;
   *nsplit = (tiles + t - 1) / t;
 }
-
 // Can the KV splits of one query tile run as a thread-block cluster (and
 // merge on chip)?  Up to 8 splits (the portable cluster size), when the
 // device can co-schedule such a cluster of these CTAs.
