@@ -377,7 +377,7 @@ def run_ours(args):
                      "frac_hbm": round(gbs / hbm_peak, 4) if gbs else None}
     stages["attn"]["tflops"] = round(sb["attn_flops"] / (stage_us["attn"] * 1e-6) / 1e12, 2)
     dom = max(["topk", "attn", "walk"], key=lambda n: stage_us[n])
-    tags = {"topk": "topk_kernel", "attn": "attn_kernel", "walk": "walk_kernel"}
+    tags = {"topk": "topk", "attn": "attn", "walk": "walk"}  # keys of profiles/traffic.json
     roof = {"kernel": dom, "bound": "hbm", "achieved": stages[dom]["gbs"], "peak": hbm_peak,
             "unit": "GB/s", "frac": stages[dom]["frac_hbm"],
             "traffic": traffic_for(tags[dom]),
