@@ -49,6 +49,10 @@ def parse():
     ap.add_argument("--sets", type=int, default=5, help="rotating input sets")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="no timing: four rounds of one input set with an L2 flush before each, "
+                         "for an ncu capture filtered by kernel name (-k)")
+    ap.add_argument("--workload", default=None, help="workload for --profile (default: the bench's)")
     return ap.parse_args()
 
 
@@ -461,10 +465,37 @@ def run_ours(args):
     return 0
 
 
+def run_profile(args):
+    """Four rounds of one input set, each after an L2 flush (a target for ncu)."""
+    import torch
+    from block_draft_tree_b200 import synth
+    from block_draft_tree_b200.round import VerifyRound
+
+    w = synth.WORKLOADS[args.workload or WORKLOAD]
+    rnd = VerifyRound(batch=w.batch, L=w.L, V=w.V, k=w.k, B_max=w.B, hq=w.hq, hkv=w.hkv, d=w.d,
+                      max_ctx=w.ctx, draft_dtype=torch.bfloat16, target_dtype=torch.float32,
+                      inv_temperature=w.inv_temperature, paged=w.page_size > 0,
+                      page_size=w.page_size or 64,
+                      max_pages=(w.ctx + (w.page_size or 64) - 1) // (w.page_size or 64))
+    xh, seed = make_inputs(w, 0, 0)
+    xd = to_device(xh, w, torch)
+    xd["target"] = torch.randn((w.batch, w.n_max, w.V), dtype=torch.float32, device="cuda")
+    rnd.bind(xd)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    for i in range(4):
+        flush.fill_(i)
+        rnd.launch()
+    torch.cuda.synchronize()
+    print(json.dumps({"profile": w.name, "rounds": 4, "status": int(rnd.out["status"].item())}))
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.profile:
+        return run_profile(args)
     return run_ours(args)
 
 
