@@ -38,6 +38,7 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnParams p) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int rt = blockIdx.x, split = blockIdx.y;
   const int b = blockIdx.z / p.hkv, kvh = blockIdx.z % p.hkv;
+  pdl_wait();
   const int g = p.g;
   const int R = p.n_max * g;
   int n = p.n_nodes[b];
@@ -193,6 +194,7 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnParams p) {
     for (int i = 0; i < DV; ++i) po[lane + 32 * i] = o[r][i];
     if (lane == 0) p.part_ml[(grp * p.nsplit + split) * R + qr] = make_float2(m[r], l[r]);
   }
+  pdl_trigger();
   __threadfence();
   __syncthreads();
   if (tid == 0)
@@ -218,12 +220,14 @@ ddt_status launch_attn_simt(AttnParams& p, cudaStream_t stream) {
   dim3 grid(p.row_tiles, p.nsplit, p.batch * p.hkv);
   if (p.d == 128) {
     if (ensure_smem_attr((const void*)attn_simt_kernel<128>, smem) != cudaSuccess) return DDT_ERR_CUDA;
-    attn_simt_kernel<128><<<grid, kThreads, smem, stream>>>(p);
-  } else {
-    if (ensure_smem_attr((const void*)attn_simt_kernel<64>, smem) != cudaSuccess) return DDT_ERR_CUDA;
-    attn_simt_kernel<64><<<grid, kThreads, smem, stream>>>(p);
+    return launch_pdl(attn_simt_kernel<128>, grid, dim3(kThreads), smem, stream, 0, p) == cudaSuccess
+               ? DDT_OK
+               : DDT_ERR_CUDA;
   }
-  return cudaGetLastError() == cudaSuccess ? DDT_OK : DDT_ERR_CUDA;
+  if (ensure_smem_attr((const void*)attn_simt_kernel<64>, smem) != cudaSuccess) return DDT_ERR_CUDA;
+  return launch_pdl(attn_simt_kernel<64>, grid, dim3(kThreads), smem, stream, 0, p) == cudaSuccess
+             ? DDT_OK
+             : DDT_ERR_CUDA;
 }
 
 }  // namespace ddt

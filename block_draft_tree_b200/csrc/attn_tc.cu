@@ -295,6 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qtile = blockIdx.x, split = blockIdx.y, grp = blockIdx.z;
   const int b = grp / p.hkv, kvh = grp % p.hkv;
+  pdl_wait();
   const int g = p.g;
   const int R = p.n_max * g;
   const int q0 = qtile * BM;
@@ -644,6 +645,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  pdl_trigger();
   if (!work && tid >= 64 && tid < 64 + BM)  // empty split of a cluster
     ((float2*)(sK + BM * D * 4))[tid - 64] = make_float2(-INFINITY, 0.f);
 
@@ -725,6 +727,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Merge the per-split partials: one warp per query row, 4 dims per lane.
 __global__ void __launch_bounds__(256) attn_tc_combine(const Params p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_wait();
+  pdl_trigger();
   const int row = blockIdx.x * 8 + warp;          // row within the query tile
   const int qtile = row / BM, r = row % BM;
   const int grp = blockIdx.y;
@@ -986,28 +990,13 @@ ddt_status launch_attn_tc(const ddt_attn_args* a, void* ws, int sms, cudaStream_
   const size_t smem = smem_bytes();
   if (ensure_smem_attr((const void*)attn_tc_kernel, smem) != cudaSuccess) return DDT_ERR_CUDA;
   dim3 grid(p.qtiles, p.nsplit, a->batch * a->hkv);
-  if (p.cluster) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr;
-    attr.id = cudaLaunchAttributeClusterDimension;
-    attr.val.clusterDim.x = 1;
-    attr.val.clusterDim.y = p.nsplit;
-    attr.val.clusterDim.z = 1;
-    cfg.attrs = &attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, attn_tc_kernel, mq, mk, mv, mkt, mvt, p) != cudaSuccess)
+  if (launch_pdl(attn_tc_kernel, grid, dim3(kThreads), smem, stream, p.cluster ? p.nsplit : 0, mq, mk, mv, mkt,
+                 mvt, p) != cudaSuccess)
+    return DDT_ERR_CUDA;
+  if (p.nsplit > 1 && !p.cluster) {
+    if (launch_pdl(attn_tc_combine, dim3(p.qtiles * BM / 8, a->batch * a->hkv), dim3(256), 0, stream, 0, p) !=
+        cudaSuccess)
       return DDT_ERR_CUDA;
-    return DDT_OK;
-  }
-  attn_tc_kernel<<<grid, kThreads, smem, stream>>>(mq, mk, mv, mkt, mvt, p);
-  if (cudaGetLastError() != cudaSuccess) return DDT_ERR_CUDA;
-  if (p.nsplit > 1) {
-    attn_tc_combine<<<dim3(p.qtiles * BM / 8, a->batch * a->hkv), 256, 0, stream>>>(p);
-    if (cudaGetLastError() != cudaSuccess) return DDT_ERR_CUDA;
   }
   return DDT_OK;
 }

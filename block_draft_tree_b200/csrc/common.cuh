@@ -90,4 +90,12 @@ __device__ __forceinline__ void raise_status(int32_t* st, int code) {
 __device__ __forceinline__ uint64_t ld_cg_u64(const uint64_t* p) { return __ldcg((const unsigned long long*)p); }
 __device__ __forceinline__ float2 ld_cg_f2(const float2* p) { return __ldcg(p); }
 
+// Programmatic dependent launch: every kernel of the library is launched
+// with programmatic stream serialization, waits for the previous kernel's
+// results before its first read of any input, and lets the next kernel be
+// scheduled once its own main work is issued.  Without the launch attribute
+// both are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 }  // namespace ddt

@@ -130,6 +130,7 @@ __global__ void __launch_bounds__(kThreads, 3) topk_kernel(TopkParams p) {
   const int tid = threadIdx.x;
   const int chunk = blockIdx.x, row = blockIdx.y;
   const int64_t c0 = (int64_t)chunk * kChunk;
+  pdl_wait();
   const char* rowp = (const char*)p.logits + (int64_t)row * p.row_stride * ES;
 
   // word j of vector q of this thread holds elements starting at index
@@ -260,6 +261,7 @@ __global__ void __launch_bounds__(kThreads, 3) topk_kernel(TopkParams p) {
     return;
   }
 
+  pdl_trigger();
   // publish this chunk's partial, then take a ticket
   const int64_t pbase = (int64_t)row * p.S + chunk;
   for (int r = tid; r < p.k; r += kThreads) p.part_keys[pbase * p.k + r] = s_top[r];
@@ -352,11 +354,9 @@ ddt_status launch_topk(const void* logits, ddt_dtype dt, int rows, int V, int64_
   p.lse = lse;
   if (rows == 0) return DDT_OK;
   dim3 grid(p.S, rows);
-  if (dt == DDT_BF16)
-    topk_kernel<true><<<grid, kThreads, 0, stream>>>(p);
-  else
-    topk_kernel<false><<<grid, kThreads, 0, stream>>>(p);
-  return cudaGetLastError() == cudaSuccess ? DDT_OK : DDT_ERR_CUDA;
+  const cudaError_t e = dt == DDT_BF16 ? launch_pdl(topk_kernel<true>, grid, dim3(kThreads), 0, stream, 0, p)
+                                      : launch_pdl(topk_kernel<false>, grid, dim3(kThreads), 0, stream, 0, p);
+  return e == cudaSuccess ? DDT_OK : DDT_ERR_CUDA;
 }
 
 }  // namespace ddt

@@ -673,6 +673,8 @@ __global__ void __launch_bounds__(kThreads, 1) build_tree_kernel(TreeParams p) {
 
   const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int L = p.L, k = p.k, NM = p.n_max, icap = p.icap;
+  pdl_wait();
+  pdl_trigger();  // one CTA per sequence: the next kernel may take the other SMs
   const double inv_t = p.inv_t;
 
   Smem s;
@@ -1229,8 +1231,9 @@ ddt_status launch_build_tree(const int32_t* ids, const float* zk, const float* l
   if (batch == 0) return DDT_OK;
   const size_t smem = tree_smem_bytes(L, k, p.n_max, p.kw, p.icap);
   if (ensure_smem_attr((const void*)build_tree_kernel, smem) != cudaSuccess) return DDT_ERR_CUDA;
-  build_tree_kernel<<<batch, kThreads, smem, stream>>>(p);
-  return cudaGetLastError() == cudaSuccess ? DDT_OK : DDT_ERR_CUDA;
+  return launch_pdl(build_tree_kernel, dim3(batch), dim3(kThreads), smem, stream, 0, p) == cudaSuccess
+             ? DDT_OK
+             : DDT_ERR_CUDA;
 }
 
 }  // namespace ddt

@@ -145,6 +145,7 @@ __global__ void __launch_bounds__(kThreads) walk_kernel(WalkParams p) {
 
   const int chunk = blockIdx.x, j = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x;
+  pdl_wait();
   int n = p.n_nodes[b];
   if (n < 1 || n > p.n_max) {
     if (chunk == 0 && j == 0 && tid == 0) raise_status(p.status, DDT_ERR_INVALID_ARG);
@@ -170,6 +171,7 @@ __global__ void __launch_bounds__(kThreads) walk_kernel(WalkParams p) {
         if (f > bv || bi < 0) { bv = f; bi = idx; }
       }
   }
+  pdl_trigger();
   uint64_t key = bi < 0 ? 0ull : cand_key(bv, (uint32_t)bi);
   key = block_max_key(key, s_red);
 
@@ -260,11 +262,9 @@ ddt_status launch_tree_walk(const void* logits, ddt_dtype dt, int batch, int n_m
   p.part = (uint64_t*)w;
   if (batch == 0) return DDT_OK;
   dim3 grid(p.S, n_max, batch);
-  if (dt == DDT_BF16)
-    walk_kernel<true><<<grid, kThreads, 0, stream>>>(p);
-  else
-    walk_kernel<false><<<grid, kThreads, 0, stream>>>(p);
-  return cudaGetLastError() == cudaSuccess ? DDT_OK : DDT_ERR_CUDA;
+  const cudaError_t e = dt == DDT_BF16 ? launch_pdl(walk_kernel<true>, grid, dim3(kThreads), 0, stream, 0, p)
+                                      : launch_pdl(walk_kernel<false>, grid, dim3(kThreads), 0, stream, 0, p);
+  return e == cudaSuccess ? DDT_OK : DDT_ERR_CUDA;
 }
 
 }  // namespace ddt
