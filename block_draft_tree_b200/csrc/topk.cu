@@ -48,23 +48,28 @@ struct TopkParams {
   float* lse;
 };
 
+// Block merge of per-thread (max, sum of exp2((z-max)*c)): the block maximum
+// from a REDUX on the ordered keys, one rescale per thread, then a sum.  Two
+// barriers; every thread gets the result.
 __device__ __forceinline__ void block_ms_reduce(float& m, float& s, float c, float* sm_m,
                                                 float* sm_s) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    float m2 = __shfl_xor_sync(0xFFFFFFFFu, m, o);
-    float s2 = __shfl_xor_sync(0xFFFFFFFFu, s, o);
-    ms_merge(m, s, m2, s2, c);
-  }
-  if (lane == 0) {
-    sm_m[warp] = m;
-    sm_s[warp] = s;
-  }
+  const uint32_t wk = __reduce_max_sync(0xFFFFFFFFu, ord32(m));
+  if (lane == 0) sm_m[warp] = from_ord32(wk);
   __syncthreads();
-  m = -INFINITY;
-  s = 0.f;
-  for (int w = 0; w < kThreads / 32; ++w) ms_merge(m, s, sm_m[w], sm_s[w], c);
+  float M = sm_m[0];
+#pragma unroll
+  for (int w = 1; w < kThreads / 32; ++w) M = fmaxf(M, sm_m[w]);
+  float t = (m == -INFINITY || M == -INFINITY) ? 0.f : s * ex2((m - M) * c);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xFFFFFFFFu, t, o);
+  if (lane == 0) sm_s[warp] = t;
+  __syncthreads();
+  float S = 0.f;
+#pragma unroll
+  for (int w = 0; w < kThreads / 32; ++w) S += sm_s[w];
+  m = M;
+  s = S;
 }
 
 __device__ __forceinline__ uint64_t block_max_u64(uint64_t v, uint64_t* sm) {
@@ -273,44 +278,52 @@ __global__ void __launch_bounds__(kThreads, 3) topk_kernel(TopkParams p) {
   if (!s_last) return;
   __threadfence();
 
-  // last CTA of the row: merge the S partials
-  if (tid == 0) s_count = 0;
+  // last CTA of the row: every chunk's keys and (max, sum) in one round of
+  // loads, then the k best keys of the row ranked directly
+  const int tot = p.S * p.k;
   float M = -INFINITY, Ssum = 0.f;
   for (int cc = tid; cc < p.S; cc += kThreads) {
     const float2 ms = ld_cg_f2(&p.part_ms[(int64_t)row * p.S + cc]);
     ms_merge(M, Ssum, ms.x, ms.y, p.c);
   }
-  // threshold: the best k-th key of any single chunk (each chunk has k keys >= it)
-  uint64_t t = 0;
-  for (int cc = tid; cc < p.S; cc += kThreads) {
-    const uint64_t kk = ld_cg_u64(&p.part_keys[((int64_t)row * p.S + cc) * p.k + p.k - 1]);
-    t = kk > t ? kk : t;
-  }
-  t = block_max_u64(t, s_red);
-  if (t == 0) t = 1;
-  const int tot = p.S * p.k;
-  for (int i = tid; i < tot; i += kThreads) {
-    const uint64_t key = ld_cg_u64(&p.part_keys[(int64_t)row * tot + i]);
-    if (key >= t) {
-      const int pos = atomicAdd(&s_count, 1);
-      if (pos < kCandCap) s_cand[pos] = key;
-    }
-  }
-  block_ms_reduce(M, Ssum, p.c, s_wm, s_wsum);
-  const int n2 = s_count;
-  if (n2 <= kCandCap) {
-    rank_select(s_cand, n2, p.k, s_top);
+  if (tot <= kCandCap) {
+    for (int i = tid; i < tot; i += kThreads) s_cand[i] = ld_cg_u64(&p.part_keys[(int64_t)row * tot + i]);
+    block_ms_reduce(M, Ssum, p.c, s_wm, s_wsum);  // its barriers publish s_cand
+    rank_select(s_cand, tot, p.k, s_top);
   } else {
-    uint64_t prev = ~0ull;
-    for (int r = 0; r < p.k; ++r) {
-      uint64_t best = 0;
-      for (int i = tid; i < tot; i += kThreads) {
-        const uint64_t key = ld_cg_u64(&p.part_keys[(int64_t)row * tot + i]);
-        if (key < prev && key > best) best = key;
+    // many chunks: a threshold first (the best k-th key of any chunk: each
+    // chunk has k keys at or above it), then the keys that reach it
+    if (tid == 0) s_count = 0;
+    uint64_t t = 0;
+    for (int cc = tid; cc < p.S; cc += kThreads) {
+      const uint64_t kk = ld_cg_u64(&p.part_keys[((int64_t)row * p.S + cc) * p.k + p.k - 1]);
+      t = kk > t ? kk : t;
+    }
+    t = block_max_u64(t, s_red);
+    if (t == 0) t = 1;
+    for (int i = tid; i < tot; i += kThreads) {
+      const uint64_t key = ld_cg_u64(&p.part_keys[(int64_t)row * tot + i]);
+      if (key >= t) {
+        const int pos = atomicAdd(&s_count, 1);
+        if (pos < kCandCap) s_cand[pos] = key;
       }
-      best = block_max_u64(best, s_red);
-      if (tid == 0) s_top[r] = best;
-      prev = best;
+    }
+    block_ms_reduce(M, Ssum, p.c, s_wm, s_wsum);
+    const int n2 = s_count;
+    if (n2 <= kCandCap) {
+      rank_select(s_cand, n2, p.k, s_top);
+    } else {
+      uint64_t prev = ~0ull;
+      for (int r = 0; r < p.k; ++r) {
+        uint64_t best = 0;
+        for (int i = tid; i < tot; i += kThreads) {
+          const uint64_t key = ld_cg_u64(&p.part_keys[(int64_t)row * tot + i]);
+          if (key < prev && key > best) best = key;
+        }
+        best = block_max_u64(best, s_red);
+        if (tid == 0) s_top[r] = best;
+        prev = best;
+      }
     }
   }
   __syncthreads();
