@@ -243,6 +243,56 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)m) : "memory");
 }
 
+// Two fp32 values in one 64-bit register pair, and the sm_100 packed
+// two-wide fp32 arithmetic on such pairs (one instruction for both lanes).
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void unpack2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for a packed pair on the FMA pipe, to relieve the MUFU pipe in the
+// softmax.  Cody-Waite reduction: n = rint(x) from the 1.5*2^23 rounding
+// constant, f = x - n in [-1/2, 1/2]; 2^f from a cubic fitted here by least
+// squares to 2^f at 256 Chebyshev nodes of [-1/2, 1/2] with relative
+// weighting (largest relative error 7.8e-5 in fp32, far below the bf16
+// rounding of P); 2^n added to the exponent field.  x <= 8 here (the running
+// maximum lags the true one by at most 2^8); x below -126 is raised to -126:
+// masked scores give 2^-126, far below the output's precision.
+__device__ __forceinline__ void exp2_poly2(uint64_t x2, float& a, float& b) {
+  float xa, xb;
+  unpack2(x2, xa, xb);
+  const uint64_t xx = pack2(fmaxf(xa, -126.f), fmaxf(xb, -126.f));
+  const uint64_t t2 = fadd2(xx, pack2(12582912.f, 12582912.f));
+  const uint64_t f2 = ffma2(fadd2(t2, pack2(-12582912.f, -12582912.f)), pack2(-1.f, -1.f), xx);
+  uint64_t q2 = ffma2(pack2(5.508868396e-02f, 5.508868396e-02f), f2, pack2(2.426040471e-01f, 2.426040471e-01f));
+  q2 = ffma2(q2, f2, pack2(6.932762265e-01f, 6.932762265e-01f));
+  q2 = ffma2(q2, f2, pack2(9.999289513e-01f, 9.999289513e-01f));
+  float ta, tb, qa, qb;
+  unpack2(t2, ta, tb);
+  unpack2(q2, qa, qb);
+  a = __int_as_float(__float_as_int(qa) + ((__float_as_int(ta) - 0x4B400000) << 23));
+  b = __int_as_float(__float_as_int(qb) + ((__float_as_int(tb) - 0x4B400000) << 23));
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version bits.
 __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
   uint64_t d = 0;
@@ -506,9 +556,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(r[e]);
 #pragma unroll
-        for (int c = 8; c < BN / 2; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(r[c]));
-        mx_raw = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        for (int c = 8; c < BN / 2; c += 2)
+          mx8[(c >> 1) & 7] = fmax3(mx8[(c >> 1) & 7], __uint_as_float(r[c]), __uint_as_float(r[c + 1]));
+        mx_raw = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
       }
       // exchange the half-row maxima (raw score domain; scale > 0 commutes with max)
       const uint32_t xcol = kColX + 2 * (i & 1);
@@ -523,23 +573,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float m_new = fmaxf(m_used, mx);
       const bool move = m_new > m_used + kRescaleLog2 || (m_used == -INFINITY && m_new != -INFINITY);
       const float m_tgt = move ? m_new : m_used;
-      float rs8[8];
+      uint64_t rs2[4];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) rs8[e] = 0.f;
+      for (int e = 0; e < 4; ++e) rs2[e] = 0ull;  // (+0, +0)
       if (m_tgt == -INFINITY) {
 #pragma unroll
         for (int c = 0; c < BN / 4; ++c) r[c] = 0u;
       } else {
-        // p = 2^(s*c - m): one FFMA and one MUFU per score; bf16 pairs packed in place
+        // p = 2^(s*c - m), two scores at a time: a packed FFMA for the
+        // exponents, then MUFU ex2 -- or, for 3 pairs in 8, exp2_poly2 on the
+        // FMA pipe, so that neither pipe waits on the other; packed sums;
+        // bf16 pairs packed in place
+        const uint64_t c2 = pack2(c_log2, c_log2), nm2 = pack2(-m_tgt, -m_tgt);
 #pragma unroll
         for (int c = 0; c < BN / 2; c += 2) {
-          const float a = ex2(fmaf(__uint_as_float(r[c]), c_log2, -m_tgt));
-          const float bb = ex2(fmaf(__uint_as_float(r[c + 1]), c_log2, -m_tgt));
-          rs8[(c >> 1) & 7] += a + bb;
+          const uint64_t x2 = ffma2(pack2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), c2, nm2);
+          float a, bb;
+          if (((c >> 1) & 7) < 3) {
+            exp2_poly2(x2, a, bb);
+          } else {
+            float xa, xb;
+            unpack2(x2, xa, xb);
+            a = ex2(xa);
+            bb = ex2(xb);
+          }
+          rs2[(c >> 1) & 3] = fadd2(rs2[(c >> 1) & 3], pack2(a, bb));
           __nv_bfloat162 pk = __floats2bfloat162_rn(a, bb);
           r[c >> 1] = *(uint32_t*)&pk;
         }
       }
+      float rs8[8];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) unpack2(rs2[e], rs8[2 * e], rs8[2 * e + 1]);
       const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
       // PV of the previous tile must be done before P and O are touched
       if (i > 0) {
