@@ -130,6 +130,23 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------
+def max_over_ranks(value, world, device):
+    """The largest of every rank's value (a job's time is its slowest rank's)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, batch, steps, elapsed_ms):
+    """Rounds of all ranks per second: every rank runs `steps` rounds of its own
+    `batch` sequences (weak scaling), all within the slowest rank's time."""
+    return world * batch * steps / (elapsed_ms * 1e-3)
+
+
 def make_inputs(w, rank, s):
     """Host-side (numpy) inputs of one set: a different sequence per (rank, set)."""
     from block_draft_tree_b200 import synth
@@ -355,11 +372,8 @@ def run_ours(args):
     end.record()
     torch.cuda.synchronize()
     clk = clocks.stop() if clocks else None
-    elapsed_ms = start.elapsed_time(end)
+    elapsed_ms = max_over_ranks(start.elapsed_time(end), world, "cuda")
     if world > 1:
-        t = torch.tensor([elapsed_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
         dist.barrier()
 
     # per-stage durations: the instrumented replays that end the timed region
@@ -422,12 +436,8 @@ def run_ours(args):
             e2e_step(i)
         e2.record()
         torch.cuda.synchronize()
-        ms = s2.elapsed_time(e2)
-        if world > 1:
-            t = torch.tensor([ms], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
-        e2e = {"value": world * w.batch * args.e2e_steps / (ms * 1e-3), "unit": "rounds/s",
+        ms = max_over_ranks(s2.elapsed_time(e2), world, "cuda")
+        e2e = {"value": job_throughput(world, w.batch, args.e2e_steps, ms), "unit": "rounds/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
         # the graphs overwrote the target buffers with the same data: nothing to restore
 
@@ -450,7 +460,7 @@ def run_ours(args):
                          "single-threaded fp64 C oracle; %.1f s" % (time.perf_counter() - t0),
                "stage_s": {k: round(v, 4) for k, v in parts.items() if k.endswith("_s")}}
 
-    value = world * w.batch * args.steps / (elapsed_ms * 1e-3)
+    value = job_throughput(world, w.batch, args.steps, elapsed_ms)
     line = {"metric": METRIC, "value": value, "unit": "rounds/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
