@@ -24,9 +24,7 @@ namespace ddt {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kChunk = 8192;  // workspace sizing: partial slots per row never exceed V / kChunk + 1
-constexpr int kVReg = 8;      // 16-byte vectors per thread held in registers
-constexpr int kVSm = 2;       // and landed in shared memory by cp.async (no registers held)
+constexpr int kChunk = 8192;
 
 struct WalkParams {
   const void* logits;
@@ -97,48 +95,31 @@ __device__ void walk_sequence(const WalkParams& p, int b, int n, const int* s_am
   }
 }
 
-// One chunk: kVReg + kVSm 16-byte vectors per thread, all requested at once
-// (the extra kVSm through shared memory), so that one wave of CTAs has the
-// whole read in flight.
 template <bool BF16>
 struct Chunk {
   static constexpr int EPV = BF16 ? 8 : 4;
-  static constexpr int VPT = kVReg + kVSm;
-  static constexpr int ELEMS = kThreads * VPT * EPV;
-  uint4 v[kVReg];
+  static constexpr int VPT = kChunk / kThreads / EPV;
+  uint4 v[VPT];
 };
 
-// Issue the loads of one (row, chunk) item (full chunks only); vectors
-// kVReg.. land in ext[q - kVReg][threadIdx.x].
+// Issue the loads of one (row, chunk) item (full chunks only).
 template <bool BF16>
-__device__ __forceinline__ void load_chunk(Chunk<BF16>& c, uint4 (*ext)[kThreads], const char* rowp, int64_t c0) {
+__device__ __forceinline__ void load_chunk(Chunk<BF16>& c, const char* rowp, int64_t c0) {
   constexpr int EPV = Chunk<BF16>::EPV, ES = BF16 ? 2 : 4;
 #pragma unroll
-  for (int q = kVReg; q < Chunk<BF16>::VPT; ++q) {
-    const char* src = rowp + (c0 + (int64_t)(q * kThreads + threadIdx.x) * EPV) * ES;
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(
-                     &ext[q - kVReg][threadIdx.x])),
-                 "l"(src)
-                 : "memory");
-  }
-  asm volatile("cp.async.commit_group;" ::: "memory");
-#pragma unroll
-  for (int q = 0; q < kVReg; ++q)
+  for (int q = 0; q < Chunk<BF16>::VPT; ++q)
     c.v[q] = ld_stream_v4(rowp + (c0 + (int64_t)(q * kThreads + threadIdx.x) * EPV) * ES);
 }
 
 // Thread-local argmax of a loaded chunk; each thread sees its indices in
 // increasing order, so strict > keeps the smallest index among equal values.
 template <bool BF16>
-__device__ __forceinline__ void argmax_chunk(const Chunk<BF16>& c, const uint4 (*ext)[kThreads], int c0, float& bv,
-                                             int& bi) {
+__device__ __forceinline__ void argmax_chunk(const Chunk<BF16>& c, int c0, float& bv, int& bi) {
   constexpr int EPV = Chunk<BF16>::EPV;
-  asm volatile("cp.async.wait_all;" ::: "memory");  // this thread's own vectors only
 #pragma unroll
   for (int q = 0; q < Chunk<BF16>::VPT; ++q) {
     const int base = c0 + (q * kThreads + (int)threadIdx.x) * EPV;
-    const uint4 vq = q < kVReg ? c.v[q < kVReg ? q : 0] : ext[q >= kVReg ? q - kVReg : 0][threadIdx.x];
-    const uint32_t w[4] = {vq.x, vq.y, vq.z, vq.w};
+    const uint32_t w[4] = {c.v[q].x, c.v[q].y, c.v[q].z, c.v[q].w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       if (BF16) {
@@ -154,12 +135,11 @@ __device__ __forceinline__ void argmax_chunk(const Chunk<BF16>& c, const uint4 (
 }
 
 template <bool BF16>
-__global__ void __launch_bounds__(kThreads, 7) walk_kernel(WalkParams p) {
+__global__ void __launch_bounds__(kThreads) walk_kernel(WalkParams p) {
   constexpr int EPV = Chunk<BF16>::EPV;
   constexpr int ES = BF16 ? 2 : 4;
   __shared__ uint64_t s_red[kThreads / 32];
   __shared__ int s_flag;
-  __shared__ uint4 s_ext[kVSm][kThreads];
   __shared__ int s_amax[DDT_TREE_B_MAX + 1], s_tok[DDT_TREE_B_MAX + 1];
   __shared__ int s_par[DDT_TREE_B_MAX + 1], s_dep[DDT_TREE_B_MAX + 1];
 
@@ -174,15 +154,14 @@ __global__ void __launch_bounds__(kThreads, 7) walk_kernel(WalkParams p) {
   if (j >= n) return;
   const int64_t row = (int64_t)b * p.n_max + j;
   const char* rowp = (const char*)p.logits + row * p.row_stride * ES;
-  constexpr int CH = Chunk<BF16>::ELEMS;
-  const int c0 = chunk * CH;
+  const int c0 = chunk * kChunk;
 
   float bv = -INFINITY;
   int bi = -1;
-  if (p.vec_ok && c0 + CH <= p.V) {
+  if (p.vec_ok && c0 + kChunk <= p.V) {
     Chunk<BF16> cur;
-    load_chunk<BF16>(cur, s_ext, rowp, c0);
-    argmax_chunk<BF16>(cur, s_ext, c0, bv, bi);
+    load_chunk<BF16>(cur, rowp, c0);
+    argmax_chunk<BF16>(cur, c0, bv, bi);
   } else {
     for (int q = 0; q < Chunk<BF16>::VPT; ++q)
       for (int e = 0; e < EPV; ++e) {
@@ -259,8 +238,7 @@ ddt_status launch_tree_walk(const void* logits, ddt_dtype dt, int batch, int n_m
   p.batch = batch;
   p.n_max = n_max;
   p.V = V;
-  const int CH = kThreads * (kVReg + kVSm) * (dt == DDT_BF16 ? 8 : 4);
-  p.S = (V + CH - 1) / CH;
+  p.S = (V + kChunk - 1) / kChunk;
   p.L = L;
   p.row_stride = row_stride;
   const int es = dt == DDT_BF16 ? 2 : 4;
