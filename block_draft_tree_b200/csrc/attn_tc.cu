@@ -345,6 +345,36 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qtile = blockIdx.x, split = blockIdx.y, grp = blockIdx.z;
   const int b = grp / p.hkv, kvh = grp % p.hkv;
+
+  // set-up that reads no input runs before the wait for the previous kernel
+  if (tid == 0) {
+    mbar_init(&bars->q_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bars->kv_full[s], 1);
+      mbar_init(&bars->kv_empty[s], 1);
+    }
+    mbar_init(&bars->s_full[0], 1);
+    mbar_init(&bars->s_full[1], 1);
+    mbar_init(&bars->p_full, 256);
+    mbar_init(&bars->pv_done, 1);
+    bars->abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      prefetch_tmap(&tm_kt);
+      prefetch_tmap(&tm_vt);
+    }
+    __syncwarp();
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&bars->tmem_base)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
   pdl_wait();
   const int g = p.g;
   const int R = p.n_max * g;
@@ -363,6 +393,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int ntiles = t_hi - t_lo;
   const int64_t part_row0 = (((int64_t)grp * p.qtiles + qtile) * p.nsplit + split) * BM;
 
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
   if (ntiles == 0 && !p.cluster) {  // nothing in this split: an empty partial (or zero rows)
     if (tid >= 64 && tid < 64 + BM) {
       const int row = tid - 64;
@@ -378,45 +413,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (p.lse_out) p.lse_out[((int64_t)b * p.n_max + j) * p.hq + h] = -INFINITY;
       }
     }
+    if (warp == 0)
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                   : "memory");
     return;
   }
 
   const bool work = ntiles > 0;
-  if (work && tid == 0) {
-    mbar_init(&bars->q_full, 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bars->kv_full[s], 1);
-      mbar_init(&bars->kv_empty[s], 1);
-    }
-    mbar_init(&bars->s_full[0], 1);
-    mbar_init(&bars->s_full[1], 1);
-    mbar_init(&bars->p_full, 256);
-    mbar_init(&bars->pv_done, 1);
-    bars->abort = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  if (work && warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(&bars->tmem_base)),
-                 "r"(kTmemCols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
-  fence_before();
-  __syncthreads();
-  fence_after();
-  const uint32_t tmem = bars->tmem_base;
 
   if (!work) {
     // an empty split of a cluster: nothing to compute, an empty partial below
   } else if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      prefetch_tmap(&tm_q);
-      prefetch_tmap(&tm_k);
-      prefetch_tmap(&tm_v);
-      prefetch_tmap(&tm_kt);
-      prefetch_tmap(&tm_vt);
       const int j0 = q0 / g;
       mbar_expect_tx(&bars->q_full, (uint32_t)kTile);
       tma_load_3d(sQ, &tm_q, 0, kvh * g, b * p.n_max + j0, &bars->q_full);
@@ -717,7 +726,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   fence_before();
   __syncthreads();
   if (work && bars->abort && tid == 0) raise_status(p.status, DDT_ERR_TIMEOUT);
-  if (work && warp == 0) {
+  if (warp == 0) {
     __syncwarp();
     fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
