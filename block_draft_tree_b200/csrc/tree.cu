@@ -674,7 +674,6 @@ __global__ void __launch_bounds__(kThreads, 1) build_tree_kernel(TreeParams p) {
   const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int L = p.L, k = p.k, NM = p.n_max, icap = p.icap;
   pdl_wait();
-  pdl_trigger();  // one CTA per sequence: the next kernel may take the other SMs
   const double inv_t = p.inv_t;
 
   Smem s;
@@ -1158,6 +1157,7 @@ __global__ void __launch_bounds__(kThreads, 1) build_tree_kernel(TreeParams p) {
   } else {
     for (int i = nn * W + tid; i < NM * W; i += kThreads) o_mask[i] = 0u;
   }
+  pdl_trigger();  // the outputs are being written: the next kernel may be scheduled
   if (tid == 0) {
     double t = 0.0;
     for (int w = 0; w < kWarps; ++w) t += red.wd[w];
