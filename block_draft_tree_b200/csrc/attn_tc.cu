@@ -13,7 +13,8 @@
 //     columns = S double buffer 2x128, O 128, P 64; smem 224 KB: Q + a 3-deep K/V ring);
 //   * warp 0 issues TMA loads (Q once; K and V per token tile, 128B-swizzled,
 //     dense rows, 64-token pages, or the tree's own rows), warp 1 issues the
-//     MMAs from one thread, warps 2-5 own one TMEM lane (one query row) each;
+//     MMAs from one thread, warps 2-9 are the softmax: two warps per TMEM lane
+//     quarter (one query row per lane), 64 score columns each;
 //   * S = Q K^T lands in TMEM; the softmax warps read it, apply the
 //     context-length / ancestor-bitset mask, keep a base-2 running max that
 //     only moves (and rescales O) when it grows by more than 2^8, write
@@ -21,7 +22,8 @@
 //     O += P V with P as the TMEM-resident A operand and V as an MN-major
 //     shared-memory B operand;
 //   * with one split the CTA normalises and writes bf16 rows; with several
-//     it writes (O, m, l) partials and a second kernel merges them.
+//     the splits of a query tile merge on chip as one cluster, or write
+//     (O, m, l) partials that a second kernel merges.
 // Every mbarrier wait is bounded (about one second); a wait that gives up
 // raises DDT_ERR_TIMEOUT in the status word and the CTA stops issuing work.
 #include <cuda.h>
