@@ -27,6 +27,11 @@
  *     calls that share a workspace must not overlap on the GPU.
  *   - Calls are asynchronous on `stream` and perform no host synchronisation,
  *     so they can be captured into a CUDA graph.
+ *   - Kernels are launched with programmatic stream serialization: a call's
+ *     kernel may be scheduled while the previous kernel on the stream is
+ *     still running, but it waits for that kernel to complete (and its
+ *     writes to be visible) before it reads any input; no input is read
+ *     early.  Launched after a non-kernel operation, it runs as usual.
  *   - Arguments are validated on the host before any launch: an invalid
  *     argument returns DDT_ERR_INVALID_ARG / DDT_ERR_UNSUPPORTED /
  *     DDT_ERR_WORKSPACE and launches nothing.  Problems only visible on the
