@@ -17,7 +17,11 @@ curated summary of the authors' announcement), section "運作流程"
 * :func:`tree_attn`  -- step 3, ancestor-only masked attention of each
   tree row against the context KV cache and the tree's own KV;
 * :func:`tree_walk`  -- step 4, the greedy walk that accepts matching
-  children and returns the bonus token.
+  children and returns the bonus token;
+* :func:`tree_walk_sample` -- step 4 under a sampling decoding rule
+  (temperature > 0): each visited row draws its token from softmax(z / T)
+  by inversion with a Philox4x64-10 uniform (:func:`philox4x64_10`,
+  :func:`row_uniform`, :func:`sample_row`).
 
 Parity pins for every function live in ``tests/test_oracle_*.py``.
 """
@@ -73,7 +77,26 @@ def _load():
                                        ctypes.c_int, i32p, i32p, i32p, ctypes.c_int,
                                        ctypes.c_int, ctypes.POINTER(ctypes.c_int32),
                                        i32p, i32p, ctypes.POINTER(ctypes.c_int32)]
-        for f in (lib.ddto_topk, lib.ddto_build_tree, lib.ddto_tree_attn, lib.ddto_tree_walk):
+        u64p = np.ctypeslib.ndpointer(dtype=np.uint64, flags="C_CONTIGUOUS")
+        lib.ddto_philox4x64_10.argtypes = [u64p, u64p, u64p]
+        lib.ddto_philox4x64_10.restype = None
+        lib.ddto_word_to_uniform.argtypes = [ctypes.c_uint64]
+        lib.ddto_word_to_uniform.restype = ctypes.c_double
+        lib.ddto_row_uniform.argtypes = [ctypes.c_uint64, ctypes.c_uint64, ctypes.c_int,
+                                         ctypes.c_int]
+        lib.ddto_row_uniform.restype = ctypes.c_double
+        lib.ddto_sample_row.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64,
+                                        ctypes.c_int, ctypes.c_double, ctypes.c_double,
+                                        ctypes.POINTER(ctypes.c_double)]
+        lib.ddto_tree_walk_sample.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64,
+                                              ctypes.c_int, i32p, i32p, i32p, ctypes.c_int,
+                                              ctypes.c_int, ctypes.c_double, ctypes.c_uint64,
+                                              ctypes.c_uint64, ctypes.c_int,
+                                              ctypes.POINTER(ctypes.c_int32), i32p, i32p,
+                                              ctypes.POINTER(ctypes.c_int32),
+                                              ctypes.POINTER(ctypes.c_double)]
+        for f in (lib.ddto_topk, lib.ddto_build_tree, lib.ddto_tree_attn, lib.ddto_tree_walk,
+                  lib.ddto_sample_row, lib.ddto_tree_walk_sample):
             f.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -236,4 +259,67 @@ def tree_walk(logits, tok, parent, depth, n_nodes, L):
         res["acc_nodes"][b] = an[:L]
         res["acc_tok"][b] = at[:L]
         res["bonus"][b] = bo.value
+    return res
+
+
+def philox4x64_10(ctr, key) -> np.ndarray:
+    """Philox4x64-10 block at counter ``ctr`` (4 words) under ``key`` (2 words)."""
+    out = np.zeros(4, np.uint64)
+    _load().ddto_philox4x64_10(np.ascontiguousarray(ctr, np.uint64),
+                               np.ascontiguousarray(key, np.uint64), out)
+    return out
+
+
+def word_to_uniform(w: int) -> float:
+    """A 64-bit word to a uniform in (0, 1) (top 53 bits, centred)."""
+    return float(_load().ddto_word_to_uniform(int(w)))
+
+
+def row_uniform(seed: int, step: int, b: int, j: int) -> float:
+    """The uniform that tree row ``j`` of sequence ``b`` draws in round ``step``."""
+    return float(_load().ddto_row_uniform(int(seed), int(step), int(b), int(j)))
+
+
+def sample_row(row: np.ndarray, inv_temperature: float, u: float):
+    """One inverse-CDF draw from softmax(inv_temperature * row).  Returns
+    (token, margin), margin = distance of u*S from the chosen interval's
+    nearer end over S."""
+    row = np.ascontiguousarray(row)
+    p, is_bf16 = _raw(row)
+    mg = ctypes.c_double()
+    t = _load().ddto_sample_row(p, is_bf16, 0, row.shape[-1], float(inv_temperature), float(u),
+                                ctypes.byref(mg))
+    return int(t), float(mg.value)
+
+
+def tree_walk_sample(logits, tok, parent, depth, n_nodes, L, inv_temperature, seed, step):
+    """Step 4 under sampling for a batch.  Same outputs as :func:`tree_walk`
+    plus ``min_margin`` [batch], the smallest draw margin along each walk."""
+    logits = np.ascontiguousarray(logits)
+    bsz, n_max, V = logits.shape
+    res = {"acc_len": np.empty(bsz, np.int32), "acc_nodes": np.empty((bsz, L), np.int32),
+           "acc_tok": np.empty((bsz, L), np.int32), "bonus": np.empty(bsz, np.int32),
+           "min_margin": np.empty(bsz, np.float64)}
+    lib = _load()
+    for b in range(bsz):
+        row = np.ascontiguousarray(logits[b])
+        p, is_bf16 = _raw(row)
+        al = ctypes.c_int32()
+        bo = ctypes.c_int32()
+        mm = ctypes.c_double()
+        an = np.empty(max(L, 1), np.int32)
+        at = np.empty(max(L, 1), np.int32)
+        rc = lib.ddto_tree_walk_sample(p, is_bf16, V, V, np.ascontiguousarray(tok[b], np.int32),
+                                       np.ascontiguousarray(parent[b], np.int32),
+                                       np.ascontiguousarray(depth[b], np.int32), int(n_nodes[b]),
+                                       L, float(inv_temperature), int(seed), int(step), b,
+                                       ctypes.byref(al), an, at, ctypes.byref(bo),
+                                       ctypes.byref(mm))
+        if rc != 0:
+            raise ValueError("ddto_tree_walk_sample failed (%d)" % rc)
+        res["acc_len"][b] = al.value
+        res["acc_nodes"][b] = an[:L]
+        res["acc_tok"][b] = at[:L]
+        res["bonus"][b] = bo.value
+        res["min_margin"][b] = mm.value
     return res

@@ -515,3 +515,163 @@ int ddto_tree_walk(const void* logits, int is_bf16, int64_t row_stride, int V,
   *acc_len = a;
   return DDTO_OK;
 }
+
+/* ------------------------------------------------------------------ */
+/* Sampled walk (target temperature > 0)                               */
+/* ------------------------------------------------------------------ */
+/*
+ * Step 4 says the walk follows the target's decoding rule; the announcement
+ * reports results over several temperatures, so besides greedy decoding the
+ * rule may be sampling from softmax(z / T).  The walk stays lossless when
+ * each visited row draws its token from that distribution with a fresh
+ * uniform: every emitted token is then a draw from the target's conditional
+ * given the accepted prefix, exactly as if the target had decoded alone.
+ *
+ * Reading adopted (the page gives no sampler): inverse-CDF sampling over
+ * token ids in increasing order, one uniform u per (sequence, tree row),
+ * u taken from the counter-based generator Philox4x64-10 so that any
+ * implementation can reproduce the draw.
+ */
+
+/* 64 x 64 -> 128-bit product, split into high and low words. */
+static void mulhilo64(uint64_t a, uint64_t b, uint64_t* hi, uint64_t* lo) {
+  const unsigned __int128 p = (unsigned __int128)a * (unsigned __int128)b;
+  *hi = (uint64_t)(p >> 64);
+  *lo = (uint64_t)p;
+}
+
+/*
+ * Philox4x64-10 (Salmon, Moraes, Dror and Shaw, "Parallel Random Numbers:
+ * As Easy as 1, 2, 3", SC'11, section 4).  One round: words 0 and 2 of the
+ * counter are multiplied by the two round multipliers; the new word 0 is
+ * the high half of the second product xor word 1 xor key word 0, the new
+ * word 2 is the high half of the first product xor word 3 xor key word 1,
+ * and the low halves become words 1 and 3.  Between rounds the key words
+ * advance by the two Weyl increments (golden ratio and sqrt(3) - 1, as
+ * 64-bit fractions).  Ten rounds.
+ */
+void ddto_philox4x64_10(const uint64_t ctr[4], const uint64_t key[2], uint64_t out[4]) {
+  const uint64_t M0 = 0xD2E7470EE14C6C93ull, M1 = 0xCA5A826395121157ull;
+  const uint64_t W0 = 0x9E3779B97F4A7C15ull, W1 = 0xBB67AE8584CAA73Bull;
+  uint64_t x0 = ctr[0], x1 = ctr[1], x2 = ctr[2], x3 = ctr[3];
+  uint64_t k0 = key[0], k1 = key[1];
+  for (int round = 0; round < 10; ++round) {
+    if (round > 0) {
+      k0 += W0;
+      k1 += W1;
+    }
+    uint64_t hi0, lo0, hi1, lo1;
+    mulhilo64(M0, x0, &hi0, &lo0);
+    mulhilo64(M1, x2, &hi1, &lo1);
+    const uint64_t n0 = hi1 ^ x1 ^ k0, n2 = hi0 ^ x3 ^ k1;
+    x0 = n0;
+    x1 = lo1;
+    x2 = n2;
+    x3 = lo0;
+  }
+  out[0] = x0;
+  out[1] = x1;
+  out[2] = x2;
+  out[3] = x3;
+}
+
+/* A 64-bit word to a uniform in (0, 1): its top 52 bits, centred in their
+   interval of width 2^-52.  Every value is exact in binary64 and lies in
+   [2^-53, 1 - 2^-53], so it is never 0 and never 1. */
+double ddto_word_to_uniform(uint64_t w) {
+  return ((double)(w >> 12) + 0.5) * 0x1.0p-52;
+}
+
+/* The uniform of tree row j of sequence b in the round numbered `step`:
+   word 0 of Philox4x64-10 at counter (j, b, 0, 0) under key (seed, step). */
+double ddto_row_uniform(uint64_t seed, uint64_t step, int b, int j) {
+  const uint64_t ctr[4] = {(uint64_t)(uint32_t)j, (uint64_t)(uint32_t)b, 0, 0};
+  const uint64_t key[2] = {seed, step};
+  uint64_t out[4];
+  ddto_philox4x64_10(ctr, key, out);
+  return ddto_word_to_uniform(out[0]);
+}
+
+/*
+ * One draw from softmax(invT * z) over the V logits at row `base`, by
+ * inversion: with w_v = exp(invT*z_v - m), m = max_v invT*z_v, S = sum w_v
+ * and C_v = w_0 + ... + w_v (ids in increasing order), the token is the
+ * smallest v with C_v > u*S.  *margin receives the distance of u*S from the
+ * nearer end of the chosen interval [C_{v-1}, C_v), divided by S: a draw
+ * with a margin below a computation's relative rounding error may come out
+ * differently there.  Logits must be finite or -inf; a row with no finite
+ * logit yields token 0 (margin +inf).
+ */
+int ddto_sample_row(const void* logits, int is_bf16, int64_t base, int V, double invT, double u,
+                    double* margin) {
+  double m = -INFINITY;
+  for (int v = 0; v < V; ++v) {
+    const double y = invT * load_val(logits, is_bf16, base + v);
+    if (y > m) m = y;
+  }
+  if (m == -INFINITY) {
+    *margin = INFINITY;
+    return 0;
+  }
+  double S = 0.0;
+  for (int v = 0; v < V; ++v) S += exp(invT * load_val(logits, is_bf16, base + v) - m);
+  const double theta = u * S;
+  double C = 0.0;
+  int last_pos = 0;
+  for (int v = 0; v < V; ++v) {
+    const double w = exp(invT * load_val(logits, is_bf16, base + v) - m);
+    const double prev = C;
+    C += w;
+    if (w > 0.0) last_pos = v;
+    if (C > theta) {
+      const double d0 = theta - prev, d1 = C - theta;
+      *margin = (d0 < d1 ? d0 : d1) / S;
+      return v;
+    }
+  }
+  *margin = 0.0; /* u*S rounded onto the total: the last token of positive weight */
+  return last_pos;
+}
+
+/*
+ * Sampled walk of sequence b: as ddto_tree_walk, but the token taken at
+ * row x is ddto_sample_row(row x, invT, ddto_row_uniform(seed, step, b, x)).
+ * *min_margin receives the smallest draw margin along the walk.
+ */
+int ddto_tree_walk_sample(const void* logits, int is_bf16, int64_t row_stride, int V,
+                          const int32_t* tok, const int32_t* parent, const int32_t* depth,
+                          int n_nodes, int L, double invT, uint64_t seed, uint64_t step, int b,
+                          int32_t* acc_len, int32_t* acc_nodes, int32_t* acc_tok, int32_t* bonus,
+                          double* min_margin) {
+  if (!logits || V < 1 || n_nodes < 1 || L < 0 || !(invT > 0.0)) return DDTO_ERR_ARG;
+  for (int i = 0; i < L; ++i) {
+    acc_nodes[i] = -1;
+    acc_tok[i] = -1;
+  }
+  double mm = INFINITY;
+  int x = 0, a = 0;
+  for (;;) {
+    double mg;
+    const double u = ddto_row_uniform(seed, step, b, x);
+    const int t = ddto_sample_row(logits, is_bf16, (int64_t)x * row_stride, V, invT, u, &mg);
+    if (mg < mm) mm = mg;
+    int next = -1;
+    if (depth[x] < L)
+      for (int c = 0; c < n_nodes; ++c)
+        if (parent[c] == x && tok[c] == t) {
+          next = c;
+          break;
+        }
+    if (next < 0 || a >= L) {
+      *bonus = t;
+      break;
+    }
+    acc_nodes[a] = next;
+    acc_tok[a] = t;
+    ++a;
+    x = next;
+  }
+  *acc_len = a;
+  *min_margin = mm;
+  return DDTO_OK;
+}
