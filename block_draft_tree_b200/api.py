@@ -28,7 +28,7 @@ DDT_TREE_B_MAX = 1023
 
 EXPORTED = ("ddt_status_string", "ddt_mask_words", "ddt_topk_workspace_size", "ddt_topk",
             "ddt_build_tree", "ddt_tree_attn_workspace_size", "ddt_tree_attn",
-            "ddt_tree_walk_workspace_size", "ddt_tree_walk")
+            "ddt_tree_walk_workspace_size", "ddt_tree_walk", "ddt_tree_walk_sample")
 
 
 class DDTError(RuntimeError):
@@ -88,6 +88,10 @@ def load_library():
         lib.ddt_tree_walk.restype = i32
         lib.ddt_tree_walk.argtypes = [vp, i32, i32, i32, i32, i64, vp, vp, vp, vp, i32,
                                       vp, vp, vp, vp, vp, sz, vp, vp]
+        u64 = ctypes.c_uint64
+        lib.ddt_tree_walk_sample.restype = i32
+        lib.ddt_tree_walk_sample.argtypes = [vp, i32, i32, i32, i32, i64, vp, vp, vp, vp, i32,
+                                             f32, u64, u64, vp, vp, vp, vp, vp, sz, vp, vp]
         _lib = lib
         return lib
 
@@ -317,4 +321,35 @@ def tree_walk(logits: torch.Tensor, tok: torch.Tensor, parent: torch.Tensor,
                                _ptr(res["acc_len"]), _ptr(res["acc_nodes"]), _ptr(res["acc_tok"]),
                                _ptr(res["bonus"]), _ptr(ws), nb, _ptr(dev_status), _stream(dev))
     _check(rc, "ddt_tree_walk")
+    return res
+
+
+def tree_walk_sample(logits: torch.Tensor, tok: torch.Tensor, parent: torch.Tensor,
+                     depth: torch.Tensor, n_nodes: torch.Tensor, L: int, inv_temperature: float,
+                     seed: int, step: int, dev_status: Optional[torch.Tensor] = None):
+    """Stage 4 under temperature sampling (``ddt_tree_walk_sample``): row j of
+    sequence b draws its token from softmax(inv_temperature * z) with the
+    Philox4x64-10 uniform of counter (j, b, 0, 0) and key (seed, step).
+    Arguments and outputs otherwise as :func:`tree_walk`."""
+    lib = load_library()
+    dev = _need_cuda(logits, tok, parent, depth, n_nodes, dev_status)
+    if logits.dim() != 3 or logits.stride(2) != 1 or logits.stride(0) != logits.stride(1) * logits.shape[1]:
+        raise DDTError("logits must be [batch, n_max, V] with contiguous rows and a uniform row stride")
+    b, n_max, V = logits.shape
+    res = {"acc_len": torch.empty(b, dtype=torch.int32, device=dev),
+           "acc_nodes": torch.empty((b, L), dtype=torch.int32, device=dev),
+           "acc_tok": torch.empty((b, L), dtype=torch.int32, device=dev),
+           "bonus": torch.empty(b, dtype=torch.int32, device=dev)}
+    nb = int(lib.ddt_tree_walk_workspace_size(b, n_max, V))
+    ws = workspaces.get(dev, "walk", nb)
+    mask64 = (1 << 64) - 1
+    with torch.cuda.device(dev):
+        rc = lib.ddt_tree_walk_sample(_ptr(logits), _dtype_code(logits), b, n_max, V,
+                                      logits.stride(1), _ptr(tok), _ptr(parent), _ptr(depth),
+                                      _ptr(n_nodes), L, float(inv_temperature), int(seed) & mask64,
+                                      int(step) & mask64, _ptr(res["acc_len"]),
+                                      _ptr(res["acc_nodes"]), _ptr(res["acc_tok"]),
+                                      _ptr(res["bonus"]), _ptr(ws), nb, _ptr(dev_status),
+                                      _stream(dev))
+    _check(rc, "ddt_tree_walk_sample")
     return res

@@ -248,11 +248,13 @@ size_t ddt_tree_walk_workspace_size(int batch, int n_max, int V) {
   return walk_workspace_size(batch, n_max, V);
 }
 
-ddt_status ddt_tree_walk(const void* logits, ddt_dtype dtype, int batch, int n_max, int V,
-                         int64_t row_stride, const int32_t* tok, const int32_t* parent,
-                         const int32_t* depth, const int32_t* n_nodes, int L, int32_t* acc_len,
-                         int32_t* acc_nodes, int32_t* acc_tok, int32_t* bonus, void* workspace,
-                         size_t workspace_bytes, int32_t* dev_status, cudaStream_t stream) {
+namespace {
+ddt_status walk_common(const void* logits, ddt_dtype dtype, int batch, int n_max, int V,
+                       int64_t row_stride, const int32_t* tok, const int32_t* parent,
+                       const int32_t* depth, const int32_t* n_nodes, int L, int32_t* acc_len,
+                       int32_t* acc_nodes, int32_t* acc_tok, int32_t* bonus, void* workspace,
+                       size_t workspace_bytes, int32_t* dev_status, cudaStream_t stream,
+                       const WalkSampling* sampling) {
   if (batch < 0 || n_max < 1 || V < 1 || row_stride < V || L < 0) return DDT_ERR_INVALID_ARG;
   if (dtype != DDT_BF16 && dtype != DDT_F32) return DDT_ERR_UNSUPPORTED;
   if (n_max > DDT_TREE_B_MAX + 1 || batch > 65535 || L > DDT_TREE_L_MAX) return DDT_ERR_UNSUPPORTED;
@@ -263,7 +265,34 @@ ddt_status ddt_tree_walk(const void* logits, ddt_dtype dtype, int batch, int n_m
   if (!ws_ok(workspace, workspace_bytes, walk_workspace_size(batch, n_max, V)))
     return DDT_ERR_WORKSPACE;
   return launch_tree_walk(logits, dtype, batch, n_max, V, row_stride, tok, parent, depth, n_nodes,
-                          L, acc_len, acc_nodes, acc_tok, bonus, workspace, dev_status, stream);
+                          L, acc_len, acc_nodes, acc_tok, bonus, workspace, dev_status, stream,
+                          sampling);
+}
+}  // namespace
+
+ddt_status ddt_tree_walk(const void* logits, ddt_dtype dtype, int batch, int n_max, int V,
+                         int64_t row_stride, const int32_t* tok, const int32_t* parent,
+                         const int32_t* depth, const int32_t* n_nodes, int L, int32_t* acc_len,
+                         int32_t* acc_nodes, int32_t* acc_tok, int32_t* bonus, void* workspace,
+                         size_t workspace_bytes, int32_t* dev_status, cudaStream_t stream) {
+  return walk_common(logits, dtype, batch, n_max, V, row_stride, tok, parent, depth, n_nodes, L,
+                     acc_len, acc_nodes, acc_tok, bonus, workspace, workspace_bytes, dev_status,
+                     stream, nullptr);
+}
+
+ddt_status ddt_tree_walk_sample(const void* logits, ddt_dtype dtype, int batch, int n_max, int V,
+                                int64_t row_stride, const int32_t* tok, const int32_t* parent,
+                                const int32_t* depth, const int32_t* n_nodes, int L,
+                                float inv_temperature, uint64_t seed, uint64_t step,
+                                int32_t* acc_len, int32_t* acc_nodes, int32_t* acc_tok,
+                                int32_t* bonus, void* workspace, size_t workspace_bytes,
+                                int32_t* dev_status, cudaStream_t stream) {
+  if (!(inv_temperature > 0.f) || !(inv_temperature * kLog2e < INFINITY))
+    return DDT_ERR_INVALID_ARG;
+  const WalkSampling smp{inv_temperature, seed, step};
+  return walk_common(logits, dtype, batch, n_max, V, row_stride, tok, parent, depth, n_nodes, L,
+                     acc_len, acc_nodes, acc_tok, bonus, workspace, workspace_bytes, dev_status,
+                     stream, &smp);
 }
 
 }  // extern "C"

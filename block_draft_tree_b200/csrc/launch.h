@@ -56,11 +56,17 @@ ddt_status launch_build_tree(const int32_t* ids, const float* zk, const float* l
                              double* surrogate, int32_t* dev_status, cudaStream_t stream);
 
 size_t walk_workspace_size(int batch, int n_max, int V);
+// The sampling decoding rule of the walk (null: greedy).
+struct WalkSampling {
+  float inv_temperature;
+  uint64_t seed, step;
+};
 ddt_status launch_tree_walk(const void* logits, ddt_dtype dt, int batch, int n_max, int V,
                             int64_t row_stride, const int32_t* tok, const int32_t* parent,
                             const int32_t* depth, const int32_t* n_nodes, int L, int32_t* acc_len,
                             int32_t* acc_nodes, int32_t* acc_tok, int32_t* bonus, void* ws,
-                            int32_t* dev_status, cudaStream_t stream);
+                            int32_t* dev_status, cudaStream_t stream,
+                            const WalkSampling* sampling = nullptr);
 
 struct AttnParams;
 size_t attn_workspace_size(const ddt_attn_args* a);

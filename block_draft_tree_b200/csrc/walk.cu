@@ -17,6 +17,22 @@
 //     stages the sequence's argmaxes and tree in shared memory with one
 //     coalesced pass and walks it with one warp.
 // No CTA ever waits on another, so there is no spin and nothing to time out.
+//
+// Sampling rule (target temperature T > 0): the walk stays lossless when each
+// visited row draws its token from softmax(z / T) with a fresh uniform, so
+// the token of row j of sequence b is the inverse-CDF draw over token ids in
+// increasing order with u from Philox4x64-10 (Salmon, Moraes, Dror and Shaw,
+// "Parallel Random Numbers: As Easy as 1, 2, 3", SC'11) at counter
+// (j, b, 0, 0) under key (seed, step): u = (top 52 bits of word 0 + 1/2)
+// * 2^-52.  The scan then keeps, per chunk, the pair (m, s) = (max of
+// y = z*log2(e)/T, sum of 2^(y - m)) instead of an argmax key; the row's
+// last CTA merges the pairs, finds the chunk whose cumulative weight first
+// exceeds u times the total, and rescans that one chunk (from L2) with a
+// block prefix sum to find the token.  Weights and sums are fp64: the
+// draws land on tokens of probability ~1/V, so an fp32 cumulative sum
+// (relative error ~1e-7) would move a fair share of them to a neighbour.
+#include <cstring>
+
 #include "common.cuh"
 #include "launch.h"
 
@@ -37,6 +53,10 @@ struct WalkParams {
   unsigned* row_ticket;  // [batch*n_max]
   unsigned* seq_count;   // [batch]
   int32_t* status;
+  double a;              // sampling: log2(e) / T
+  uint64_t seed, step;   // sampling: Philox key
+  double exp2_tab[64];   // sampling: 2^(j/64)
+  double exp2_c[5];      // sampling: (ln 2)^i / i!, i = 1..5
 };
 
 __device__ __forceinline__ uint64_t block_max_key(uint64_t v, uint64_t* sm) {
@@ -134,11 +154,255 @@ __device__ __forceinline__ void argmax_chunk(const Chunk<BF16>& c, int c0, float
   }
 }
 
+// ---------------------------------------------------------------------------
+// Sampling rule
+// ---------------------------------------------------------------------------
+
+// Word 0 of the Philox4x64-10 block at counter (c0, c1, c2, c3) under key
+// (k0, k1).  A round multiplies counter words 0 and 2 by the round
+// multipliers; the new word 0 is hi(M1*x2) ^ x1 ^ k0, the new word 2 is
+// hi(M0*x0) ^ x3 ^ k1, the low halves become words 1 and 3, and the key
+// advances by the Weyl increments between rounds.
+__device__ __forceinline__ uint64_t philox4x64_10_w0(uint64_t x0, uint64_t x1, uint64_t x2,
+                                                     uint64_t x3, uint64_t k0, uint64_t k1) {
+  constexpr uint64_t M0 = 0xD2E7470EE14C6C93ull, M1 = 0xCA5A826395121157ull;
+  constexpr uint64_t W0 = 0x9E3779B97F4A7C15ull, W1 = 0xBB67AE8584CAA73Bull;
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint64_t hi0 = __umul64hi(M0, x0), lo0 = M0 * x0;
+    const uint64_t hi1 = __umul64hi(M1, x2), lo1 = M1 * x2;
+    x0 = hi1 ^ x1 ^ k0;
+    x1 = lo1;
+    x2 = hi0 ^ x3 ^ k1;
+    x3 = lo0;
+    k0 += W0;
+    k1 += W1;
+  }
+  return x0;
+}
+
+// The uniform in (0, 1) that tree row j of sequence b draws.
+__device__ __forceinline__ double row_uniform(const WalkParams& p, int b, int j) {
+  const uint64_t w = philox4x64_10_w0((uint32_t)j, (uint32_t)b, 0, 0, p.seed, p.step);
+  return ((double)(w >> 12) + 0.5) * 0x1.0p-52;
+}
+
+// 2^t in fp64 by Tang's table-driven method ("Table-driven implementation
+// of the exponential function in IEEE floating-point arithmetic", ACM TOMS
+// 15(2), 1989), for the non-positive arguments of the draw: t = n + j/64 + r
+// with |r| <= 1/128, 2^t = 2^n * 2^(j/64) * (1 + q(r)), q the Taylor series
+// of 2^r - 1 to degree 5 (truncation below 4e-17 relative).  The table
+// 2^(j/64) and the coefficients (ln 2)^i / i! come from the host.  Arguments
+// below -1000 (and -inf) give 0; the draw's weights are then negligible
+// against the largest weight, which is 1.
+__device__ __forceinline__ double tang_exp2(double t, const double* tab, const double* c) {
+  if (!(t >= -1000.0)) return 0.0;
+  const double shifter = 0x1.8p52;                    // round-to-integer by addition
+  const double sh = fma(t, 64.0, shifter);
+  const int k = __double2loint(sh);                   // round(64 t)
+  const double kd = sh - shifter;
+  const double r = fma(kd, -0.015625, t);             // exact
+  const double q = r * fma(fma(fma(fma(c[4], r, c[3]), r, c[2]), r, c[1]), r, c[0]);
+  const double tj = tab[k & 63];
+  const double y = fma(tj, q, tj);                    // in [1, 2)
+  const int n = k >> 6;                               // floor(k / 64)
+  return __hiloint2double(__double2hiint(y) + (n << 20), __double2loint(y));
+}
+
+struct Exp2Table {
+  double tab[64];
+  double c[5];
+};
+
+// Merge the pair (m2, s2) into (m, s); s is a sum of 2^(y - m).
+__device__ __forceinline__ void ms_add(double& m, double& s, double m2, double s2,
+                                       const Exp2Table& e) {
+  if (m2 == -INFINITY) return;
+  if (m2 > m) {
+    s = s * tang_exp2(m - m2, e.tab, e.c) + s2;
+    m = m2;
+  } else {
+    s += s2 * tang_exp2(m2 - m, e.tab, e.c);
+  }
+}
+
+// Thread pair (max y, sum 2^(y - max y)) over a loaded chunk, y = a*z in fp64.
 template <bool BF16>
+__device__ __forceinline__ void ms_chunk(const Chunk<BF16>& c, double a, const Exp2Table& e,
+                                         double& m, double& s) {
+  float zm = -INFINITY;
+#pragma unroll
+  for (int q = 0; q < Chunk<BF16>::VPT; ++q) {
+    const uint32_t w[4] = {c.v[q].x, c.v[q].y, c.v[q].z, c.v[q].w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (BF16) zm = fmaxf(zm, fmaxf(bf16_lo(w[i]), bf16_hi(w[i])));
+      else zm = fmaxf(zm, __uint_as_float(w[i]));
+    }
+  }
+  m = a * (double)zm;
+  s = 0.0;
+  if (zm == -INFINITY) return;
+#pragma unroll
+  for (int q = 0; q < Chunk<BF16>::VPT; ++q) {
+    const uint32_t w[4] = {c.v[q].x, c.v[q].y, c.v[q].z, c.v[q].w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (BF16) {
+        s += tang_exp2(fma(a, (double)bf16_lo(w[i]), -m), e.tab, e.c);
+        s += tang_exp2(fma(a, (double)bf16_hi(w[i]), -m), e.tab, e.c);
+      } else {
+        s += tang_exp2(fma(a, (double)__uint_as_float(w[i]), -m), e.tab, e.c);
+      }
+    }
+  }
+}
+
+// Block merge of the threads' pairs; the result is valid in thread 0.
+__device__ __forceinline__ double2 block_ms(double m, double s, double2* sm, const Exp2Table& e) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const double m2 = __shfl_xor_sync(0xFFFFFFFFu, m, o), s2 = __shfl_xor_sync(0xFFFFFFFFu, s, o);
+    ms_add(m, s, m2, s2, e);
+  }
+  if (lane == 0) sm[warp] = make_double2(m, s);
+  __syncthreads();
+  double2 r = sm[0];
+  for (int w = 1; w < kThreads / 32; ++w) ms_add(r.x, r.y, sm[w].x, sm[w].y, e);
+  return r;
+}
+
+// Inclusive prefix sum over the lanes of a warp.
+__device__ __forceinline__ double warp_incl_scan(double v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double u = __shfl_up_sync(0xFFFFFFFFu, v, o);
+    if (lane >= o) v += u;
+  }
+  return v;
+}
+
+struct SampleSmem {
+  double M, P, theta;
+  int cstar;
+  double wsum[kThreads / 32];
+  int hit, last;
+};
+
+__device__ __forceinline__ float load_logit(const char* rowp, int idx, bool bf16) {
+  return bf16 ? bf16_to_f32(((const uint16_t*)rowp)[idx]) : ((const float*)rowp)[idx];
+}
+
+// The token drawn for row (b, j) once every chunk pair of the row is in
+// `part`; called by the whole block, returns the token in every thread.
+template <bool BF16>
+__device__ int sample_row_token(const WalkParams& p, int b, int j, int64_t row, const char* rowp,
+                                const Exp2Table& e, SampleSmem& sm) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const double2* part = (const double2*)p.part + row * p.S;
+  if (warp == 0) {
+    double M = -INFINITY;
+    for (int c = lane; c < p.S; c += 32) M = fmax(M, __ldcg(&part[c]).x);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmax(M, __shfl_xor_sync(0xFFFFFFFFu, M, o));
+    // two identical passes of the chunk prefix sum: the total, then the
+    // first chunk whose inclusive prefix exceeds theta
+    double theta = 0.0, P = 0.0, Plast = 0.0;
+    int cstar = -1, clast = -1;
+    for (int pass = 0; pass < 2 && M != -INFINITY; ++pass) {
+      double carry = 0.0;
+      for (int g = 0; g < p.S; g += 32) {
+        const int c = g + lane;
+        double W = 0.0;
+        if (c < p.S) {
+          const double2 ms = __ldcg(&part[c]);
+          if (ms.x != -INFINITY) W = ms.y * tang_exp2(ms.x - M, e.tab, e.c);
+        }
+        const double incl = carry + warp_incl_scan(W);
+        double excl = __shfl_up_sync(0xFFFFFFFFu, incl, 1);
+        if (lane == 0) excl = carry;
+        if (pass == 1) {
+          const unsigned hit = __ballot_sync(0xFFFFFFFFu, c < p.S && incl > theta);
+          const unsigned pos = __ballot_sync(0xFFFFFFFFu, W > 0.0);
+          if (pos) {
+            const int l = 31 - __clz(pos);
+            clast = g + l;
+            Plast = __shfl_sync(0xFFFFFFFFu, excl, l);
+          }
+          if (hit) {
+            const int l = __ffs(hit) - 1;
+            cstar = g + l;
+            P = __shfl_sync(0xFFFFFFFFu, excl, l);
+            break;
+          }
+        }
+        carry = __shfl_sync(0xFFFFFFFFu, incl, 31);
+      }
+      if (pass == 0) theta = row_uniform(p, b, j) * carry;
+    }
+    if (cstar < 0) {  // theta rounded onto the total: the last chunk of positive weight
+      cstar = clast;
+      P = Plast;
+    }
+    if (lane == 0) {
+      sm.M = M;
+      sm.P = P;
+      sm.theta = theta;
+      sm.cstar = cstar;
+      sm.hit = INT_MAX;
+      sm.last = -1;
+    }
+  }
+  __syncthreads();
+  const int cstar = sm.cstar;
+  if (cstar < 0) return 0;  // no finite logit in the row
+  const double M = sm.M, theta = sm.theta, a = p.a;
+  // each thread owns kPer consecutive tokens of chunk cstar
+  constexpr int kPer = kChunk / kThreads;
+  const int e0 = cstar * kChunk + tid * kPer;
+  const int e1 = min(e0 + kPer, p.V);
+  double local = 0.0;
+  int last = -1;
+  for (int i = e0; i < e1; ++i) {
+    const double w = tang_exp2(fma(a, (double)load_logit(rowp, i, BF16), -M), e.tab, e.c);
+    local += w;
+    if (w > 0.0) last = i;
+  }
+  // block exclusive prefix of the threads' sums
+  const double incl = warp_incl_scan(local);
+  if (lane == 31) sm.wsum[warp] = incl;
+  __syncthreads();
+  double wbase = 0.0;
+  for (int v = 0; v < warp; ++v) wbase += sm.wsum[v];
+  double excl = __shfl_up_sync(0xFFFFFFFFu, incl, 1);
+  if (lane == 0) excl = 0.0;
+  const double base = sm.P + (wbase + excl);
+  if (base + local > theta) {
+    // the crossing may be in this thread's tokens: walk them in order
+    double cum = base;
+    int hit = last;
+    for (int i = e0; i < e1; ++i) {
+      cum += tang_exp2(fma(a, (double)load_logit(rowp, i, BF16), -M), e.tab, e.c);
+      if (cum > theta) {
+        hit = i;
+        break;
+      }
+    }
+    if (hit >= 0) atomicMin(&sm.hit, hit);
+  }
+  if (last >= 0) atomicMax(&sm.last, last);
+  __syncthreads();
+  return sm.hit != INT_MAX ? sm.hit : sm.last;
+}
+
+template <bool BF16, bool SAMPLE>
 __global__ void __launch_bounds__(kThreads) walk_kernel(WalkParams p) {
   constexpr int EPV = Chunk<BF16>::EPV;
   constexpr int ES = BF16 ? 2 : 4;
   __shared__ uint64_t s_red[kThreads / 32];
+  __shared__ __align__(16) uint64_t s_red2[2 * (kThreads / 32)];
   __shared__ int s_flag;
   __shared__ int s_amax[DDT_TREE_B_MAX + 1], s_tok[DDT_TREE_B_MAX + 1];
   __shared__ int s_par[DDT_TREE_B_MAX + 1], s_dep[DDT_TREE_B_MAX + 1];
@@ -156,46 +420,89 @@ __global__ void __launch_bounds__(kThreads) walk_kernel(WalkParams p) {
   const char* rowp = (const char*)p.logits + row * p.row_stride * ES;
   const int c0 = chunk * kChunk;
 
-  float bv = -INFINITY;
-  int bi = -1;
-  if (p.vec_ok && c0 + kChunk <= p.V) {
-    Chunk<BF16> cur;
-    load_chunk<BF16>(cur, rowp, c0);
-    argmax_chunk<BF16>(cur, c0, bv, bi);
-  } else {
-    for (int q = 0; q < Chunk<BF16>::VPT; ++q)
-      for (int e = 0; e < EPV; ++e) {
-        const int idx = c0 + (q * kThreads + tid) * EPV + e;
-        if (idx >= p.V) continue;
-        const float f = BF16 ? bf16_to_f32(((const uint16_t*)rowp)[idx]) : ((const float*)rowp)[idx];
-        if (f > bv || bi < 0) { bv = f; bi = idx; }
+  if constexpr (SAMPLE) {
+    __shared__ Exp2Table e;
+    __shared__ SampleSmem sm;
+    if (tid < 64) e.tab[tid] = p.exp2_tab[tid];
+    if (tid < 5) e.c[tid] = p.exp2_c[tid];
+    // chunk pair (max y, sum 2^(y - max y)), y = a*z
+    double m = -INFINITY, sum = 0.0;
+    if (p.vec_ok && c0 + kChunk <= p.V) {
+      Chunk<BF16> cur;
+      load_chunk<BF16>(cur, rowp, c0);
+      __syncthreads();
+      ms_chunk<BF16>(cur, p.a, e, m, sum);
+    } else {
+      __syncthreads();
+      for (int q = 0; q < Chunk<BF16>::VPT; ++q)
+        for (int i = 0; i < EPV; ++i) {
+          const int idx = c0 + (q * kThreads + tid) * EPV + i;
+          if (idx >= p.V) continue;
+          ms_add(m, sum, p.a * (double)load_logit(rowp, idx, BF16), 1.0, e);
+        }
+    }
+    pdl_trigger();
+    const double2 ms = block_ms(m, sum, (double2*)s_red2, e);
+    if (p.S > 1) {
+      if (tid == 0) {
+        ((double2*)p.part)[row * p.S + chunk] = ms;
+        __threadfence();
+        s_flag = (atomicAdd(&p.row_ticket[row], 1u) == (unsigned)(p.S - 1));
       }
-  }
-  pdl_trigger();
-  uint64_t key = bi < 0 ? 0ull : cand_key(bv, (uint32_t)bi);
-  key = block_max_key(key, s_red);
-
-  if (p.S == 1) {
-    if (tid == 0) p.amax[row] = (int32_t)key_id(key);
-  } else {
-    if (tid == 0) {
-      p.part[row * p.S + chunk] = key;
+      __syncthreads();
+      if (!s_flag) return;
       __threadfence();
-      s_flag = (atomicAdd(&p.row_ticket[row], 1u) == (unsigned)(p.S - 1));
+    } else {
+      if (tid == 0) ((double2*)p.part)[row] = ms;
+      __syncthreads();
     }
-    __syncthreads();
-    if (!s_flag) return;
-    __threadfence();
-    uint64_t m = 0;
-    for (int c = tid; c < p.S; c += kThreads) {
-      const uint64_t u = ld_cg_u64(&p.part[row * p.S + c]);
-      m = u > m ? u : m;
-    }
-    __syncthreads();
-    m = block_max_key(m, s_red);
+    const int t = sample_row_token<BF16>(p, b, j, row, rowp, e, sm);
     if (tid == 0) {
-      p.amax[row] = (int32_t)key_id(m);
-      p.row_ticket[row] = 0u;  // the counter region is left zero
+      p.amax[row] = t;
+      if (p.S > 1) p.row_ticket[row] = 0u;  // the counter region is left zero
+    }
+  } else {
+    float bv = -INFINITY;
+    int bi = -1;
+    if (p.vec_ok && c0 + kChunk <= p.V) {
+      Chunk<BF16> cur;
+      load_chunk<BF16>(cur, rowp, c0);
+      argmax_chunk<BF16>(cur, c0, bv, bi);
+    } else {
+      for (int q = 0; q < Chunk<BF16>::VPT; ++q)
+        for (int e = 0; e < EPV; ++e) {
+          const int idx = c0 + (q * kThreads + tid) * EPV + e;
+          if (idx >= p.V) continue;
+          const float f = BF16 ? bf16_to_f32(((const uint16_t*)rowp)[idx]) : ((const float*)rowp)[idx];
+          if (f > bv || bi < 0) { bv = f; bi = idx; }
+        }
+    }
+    pdl_trigger();
+    uint64_t key = bi < 0 ? 0ull : cand_key(bv, (uint32_t)bi);
+    key = block_max_key(key, s_red);
+
+    if (p.S == 1) {
+      if (tid == 0) p.amax[row] = (int32_t)key_id(key);
+    } else {
+      if (tid == 0) {
+        p.part[row * p.S + chunk] = key;
+        __threadfence();
+        s_flag = (atomicAdd(&p.row_ticket[row], 1u) == (unsigned)(p.S - 1));
+      }
+      __syncthreads();
+      if (!s_flag) return;
+      __threadfence();
+      uint64_t m = 0;
+      for (int c = tid; c < p.S; c += kThreads) {
+        const uint64_t u = ld_cg_u64(&p.part[row * p.S + c]);
+        m = u > m ? u : m;
+      }
+      __syncthreads();
+      m = block_max_key(m, s_red);
+      if (tid == 0) {
+        p.amax[row] = (int32_t)key_id(m);
+        p.row_ticket[row] = 0u;  // the counter region is left zero
+      }
     }
   }
   // the row is done; the last row of the sequence walks it
@@ -225,15 +532,32 @@ size_t walk_workspace_size(int batch, int n_max, int V) {
   const int S = (V + kChunk - 1) / kChunk;
   const size_t rows = (size_t)batch * n_max;
   return (size_t)DDT_WS_COUNTER_BYTES + align256(sizeof(int32_t) * rows) +
-         align256(sizeof(uint64_t) * rows * S);
+         align256(2 * sizeof(uint64_t) * rows * S);
 }
 
 ddt_status launch_tree_walk(const void* logits, ddt_dtype dt, int batch, int n_max, int V,
                             int64_t row_stride, const int32_t* tok, const int32_t* parent,
                             const int32_t* depth, const int32_t* n_nodes, int L, int32_t* acc_len,
                             int32_t* acc_nodes, int32_t* acc_tok, int32_t* bonus, void* ws,
-                            int32_t* dev_status, cudaStream_t stream) {
+                            int32_t* dev_status, cudaStream_t stream, const WalkSampling* sampling) {
   WalkParams p;
+  p.a = sampling ? (double)sampling->inv_temperature * 1.4426950408889634074 : 0.0;
+  if (sampling) {
+    static const Exp2Table host_tab = [] {
+      Exp2Table t;
+      for (int i = 0; i < 64; ++i) t.tab[i] = exp2((double)i / 64.0);
+      double c = 1.0;
+      for (int i = 1; i <= 5; ++i) {
+        c *= 0.69314718055994530942 / i;  // (ln 2)^i / i!
+        t.c[i - 1] = c;
+      }
+      return t;
+    }();
+    memcpy(p.exp2_tab, host_tab.tab, sizeof p.exp2_tab);
+    memcpy(p.exp2_c, host_tab.c, sizeof p.exp2_c);
+  }
+  p.seed = sampling ? sampling->seed : 0;
+  p.step = sampling ? sampling->step : 0;
   p.logits = logits;
   p.batch = batch;
   p.n_max = n_max;
@@ -262,8 +586,13 @@ ddt_status launch_tree_walk(const void* logits, ddt_dtype dt, int batch, int n_m
   p.part = (uint64_t*)w;
   if (batch == 0) return DDT_OK;
   dim3 grid(p.S, n_max, batch);
-  const cudaError_t e = dt == DDT_BF16 ? launch_pdl(walk_kernel<true>, grid, dim3(kThreads), 0, stream, 0, p)
-                                      : launch_pdl(walk_kernel<false>, grid, dim3(kThreads), 0, stream, 0, p);
+  cudaError_t e;
+  if (sampling)
+    e = dt == DDT_BF16 ? launch_pdl(walk_kernel<true, true>, grid, dim3(kThreads), 0, stream, 0, p)
+                       : launch_pdl(walk_kernel<false, true>, grid, dim3(kThreads), 0, stream, 0, p);
+  else
+    e = dt == DDT_BF16 ? launch_pdl(walk_kernel<true, false>, grid, dim3(kThreads), 0, stream, 0, p)
+                       : launch_pdl(walk_kernel<false, false>, grid, dim3(kThreads), 0, stream, 0, p);
   return e == cudaSuccess ? DDT_OK : DDT_ERR_CUDA;
 }
 

@@ -13,7 +13,8 @@
  *                      cache and its own ancestors (step 3; section 核心創新
  *                      "core innovation", ancestor-only attention mask);
  *   4. ddt_tree_walk   the greedy walk over the target's logits that accepts
- *                      matching children and returns the bonus token (step 4).
+ *                      matching children and returns the bonus token (step 4);
+ *      ddt_tree_walk_sample  the same walk under temperature sampling.
  *
  * Conventions shared by every entry point:
  *   - Every tensor pointer is a DEVICE pointer owned by the caller.  The
@@ -248,6 +249,38 @@ ddt_status ddt_tree_walk(const void* logits, ddt_dtype dtype, int batch, int n_m
                          const int32_t* depth, const int32_t* n_nodes, int L, int32_t* acc_len,
                          int32_t* acc_nodes, int32_t* acc_tok, int32_t* bonus, void* workspace,
                          size_t workspace_bytes, int32_t* dev_status, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Stage 4 under a sampling decoding rule (target temperature T > 0).
+ * DDTree page, 運作流程 step 4 (the walk follows the target's decoding
+ * rule) and 核心創新 (the target's output distribution is preserved): each
+ * visited row x draws its token from softmax(z_x / T), and the walk accepts
+ * and descends exactly as ddt_tree_walk does.  One fresh uniform per row
+ * keeps the walk lossless: every emitted token is a draw from the target's
+ * conditional given the accepted prefix.
+ *
+ * The draw of row j of sequence b is by inversion over token ids in
+ * increasing order: with w_v = exp(z_v/T - max), the token is the smallest
+ * v whose cumulative weight exceeds u * sum(w), where u = (w0 >> 12) + 1/2
+ * times 2^-52 and w0 is word 0 of Philox4x64-10 (Salmon, Moraes, Dror and
+ * Shaw, SC'11) at counter (j, b, 0, 0) under key (seed, step).  Weights
+ * and sums are fp64, so the draw agrees with exact arithmetic unless u*sum
+ * lies within about 1e-14 (relative) of an interval end.  Logits must be
+ * finite or -inf; a row with no finite logit draws token 0.
+ *
+ *   inv_temperature  1/T, finite and > 0 (larger -> closer to greedy)
+ *   seed, step       the Philox key: a stream per request (seed) and a
+ *                    fresh draw per round (step)
+ * Every other argument, the outputs and the workspace
+ * (ddt_tree_walk_workspace_size) are those of ddt_tree_walk.
+ * ------------------------------------------------------------------------ */
+ddt_status ddt_tree_walk_sample(const void* logits, ddt_dtype dtype, int batch, int n_max, int V,
+                                int64_t row_stride, const int32_t* tok, const int32_t* parent,
+                                const int32_t* depth, const int32_t* n_nodes, int L,
+                                float inv_temperature, uint64_t seed, uint64_t step,
+                                int32_t* acc_len, int32_t* acc_nodes, int32_t* acc_tok,
+                                int32_t* bonus, void* workspace, size_t workspace_bytes,
+                                int32_t* dev_status, cudaStream_t stream);
 
 #ifdef __cplusplus
 }

@@ -111,6 +111,21 @@ def test_walk_rejects_bad_arguments(lib):
     assert call(V=10 ** 6, stride=10 ** 6) == 3  # workspace required
 
 
+def test_walk_sample_rejects_bad_arguments(lib):
+    f = lib.ddt_tree_walk_sample
+    d = ctypes.c_void_p(16)
+
+    def call(b=1, n=9, V=64, stride=64, L=4, dt=1, it=1.0, logits=d):
+        return f(logits, dt, b, n, V, stride, d, d, d, d, L, it, 7, 0, d, d, d, d, None, 0,
+                 None, None)
+
+    assert call(it=0.0) == 1 and call(it=-0.5) == 1 and call(it=float("nan")) == 1
+    assert call(it=float("inf")) == 1 and call(it=3e38) == 1  # 1/T * log2(e) overflows
+    assert call(stride=3) == 1 and call(dt=5) == 2 and call(n=2000) == 2 and call(L=65) == 2
+    assert call(logits=None) == 1
+    assert call(V=10 ** 6, stride=10 ** 6) == 3  # workspace required
+
+
 def test_binding_refuses_cpu_tensors(lib):
     import torch
     with pytest.raises(api.DDTError):

@@ -1,0 +1,226 @@
+"""Parity of ddt_tree_walk_sample (CUDA, through the C ABI) with the oracle's
+sampled walk.
+
+Each visited row draws its token by inversion of softmax(z / T) with the
+Philox4x64-10 uniform of its (sequence, row).  Both sides compute the
+weights and their cumulative sums in fp64, in different orders, so a draw
+can only differ where u*S lies within rounding of an interval end.  The
+rule: when the oracle's smallest draw margin along a walk is at least
+SAMPLE_MARGIN (relative to S), the walk is bit-exact; otherwise every
+decision along the CUDA walk whose margin clears SAMPLE_MARGIN must equal
+the oracle's draw and the walk must be a valid walk of the tree.
+
+Error budget behind SAMPLE_MARGIN: each fp64 weight is within ~2 ulp of
+exp(y - m) (the exponent argument is formed with one rounding of a value
+below ~40 in magnitude, so ~1e-14 absolute, then a table-driven exp2);
+sums of <= 151936 non-negative terms add < 151936 * 2^-53 ~ 2e-11 relative
+in the worst case and far less in practice.  1e-10 stays clear of both.
+"""
+import numpy as np
+import pytest
+import torch
+from scipy import special, stats
+
+import oracle
+from block_draft_tree_b200 import api, synth
+
+from helpers import i32, logits_tensor, oracle_tree_inputs
+
+pytestmark = pytest.mark.gpu
+
+SAMPLE_MARGIN = 1e-10
+
+
+def _tree(w):
+    ids, zk, lse = oracle_tree_inputs(w, synth.draft_logits(w))
+    return oracle.build_tree(ids, zk, lse.astype(np.float64), w.budget_per_seq(),
+                             w.inv_temperature, root_token=synth.root_tokens(w),
+                             k_per_seq=w.k_per_seq(), n_max=w.n_max)
+
+
+def _sharpen(logits, tree, seed, boost):
+    """Give one seeded child of every inner row a logit of max + boost, so
+    that sampled walks descend with a fair probability."""
+    g = np.random.default_rng(seed)
+    out = logits.copy()
+    bf16 = out.dtype == np.uint16
+    for b in range(tree["tok"].shape[0]):
+        n = int(tree["n_nodes"][b])
+        par = tree["parent"][b][:n]
+        for x in range(n):
+            kids = np.nonzero(par == x)[0]
+            if len(kids) == 0:
+                continue
+            c = int(kids[g.integers(0, len(kids))])
+            t = int(tree["tok"][b][c])
+            if bf16:
+                row = (out[b, x].astype(np.uint32) << 16).view(np.float32)
+                out[b, x, t] = synth.to_bf16_bits(np.array([row.max() + boost], np.float32))[0]
+            else:
+                out[b, x, t] = out[b, x].max() + boost
+    return out
+
+
+def _row_draw(logits, b, x, invT, seed, step):
+    return oracle.sample_row(logits[b, x], invT, oracle.row_uniform(seed, step, b, x))
+
+
+def _compare(logits, tree, L, invT, seed, step, tensor=None):
+    ref = oracle.tree_walk_sample(logits, tree["tok"], tree["parent"], tree["depth"],
+                                  tree["n_nodes"], L, invT, seed, step)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    t = logits_tensor(logits) if tensor is None else tensor
+    got = api.tree_walk_sample(t, i32(tree["tok"]), i32(tree["parent"]), i32(tree["depth"]),
+                               i32(tree["n_nodes"]), L, invT, seed, step, dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    got = {k: v.cpu().numpy() for k, v in got.items()}
+    n_ambiguous = 0
+    for b in range(logits.shape[0]):
+        if ref["min_margin"][b] >= SAMPLE_MARGIN:
+            for key in ("acc_len", "acc_nodes", "acc_tok", "bonus"):
+                np.testing.assert_array_equal(got[key][b], ref[key][b], err_msg="%s[%d]" % (key, b))
+            continue
+        n_ambiguous += 1
+        # validity of the CUDA walk, decision by decision
+        a = int(got["acc_len"][b])
+        n = int(tree["n_nodes"][b])
+        x = 0
+        for i in range(a + 1):
+            t = int(got["acc_tok"][b][i]) if i < a else int(got["bonus"][b])
+            t_ref, mg = _row_draw(logits, b, x, invT, seed, step)
+            if mg >= SAMPLE_MARGIN:
+                assert t == t_ref, (b, x)
+            kids = [c for c in range(n) if tree["parent"][b][c] == x and tree["tok"][b][c] == t]
+            if i < a:
+                assert kids and int(got["acc_nodes"][b][i]) == kids[0]
+                x = kids[0]
+            else:
+                assert not kids or tree["depth"][b][x] >= L or a >= L
+    return ref, got, n_ambiguous
+
+
+@pytest.mark.parametrize("name,invT", [("tiny", 1.0), ("tiny", 1 / 0.7), ("b64", 1.0),
+                                       ("b64", 1 / 0.7), ("b256", 1.0), ("paged128", 1 / 0.7),
+                                       ("long512", 1.0)])
+def test_workload_sampled_walks(name, invT):
+    w = synth.WORKLOADS[name]
+    tree = _tree(w)
+    logits = synth.target_logits(w, tree["tok"], tree["parent"], tree["depth"], tree["n_nodes"])
+    boost = float(np.log(w.V)) + 2.0  # the boosted child holds most of the mass at T = 1
+    logits = _sharpen(logits, tree, w.index, boost)
+    ref, got, amb = _compare(logits, tree, w.L, invT, seed=1000 + w.index, step=3)
+    assert amb == 0  # no draw falls within 1e-10 of an interval end on these inputs
+    if w.batch * w.L >= 64:
+        assert ref["acc_len"].sum() > 0  # the walks do descend
+
+
+def test_bf16_logits_many_chunks():
+    w = synth.WORKLOADS["tiny"].scaled(batch=6, L=6, V=70000, k=4, B=40)
+    tree = _tree(w)
+    g = np.random.default_rng(3)
+    z = g.standard_normal((w.batch, w.n_max, w.V)).astype(np.float32) * 2
+    z = _sharpen(z, tree, 3, 9.0)
+    for step in range(3):
+        _compare(synth.to_bf16_bits(z), tree, w.L, 1.0, seed=55, step=step)
+        _compare(z, tree, w.L, 0.5, seed=55, step=step)
+
+
+@pytest.mark.parametrize("V", [1, 100, 8191, 8192, 8193, 50001])
+def test_ragged_vocab(V):
+    w = synth.WORKLOADS["tiny"].scaled(batch=3, L=4, V=max(V, 4), k=2, B=10)
+    tree = _tree(w)
+    tree = {k: v.copy() for k, v in tree.items()}
+    tree["tok"] = np.where(tree["tok"] >= 0, tree["tok"] % V, -1).astype(np.int32)
+    z = np.random.default_rng(V).standard_normal((3, w.n_max, V)).astype(np.float32)
+    z = _sharpen(z, tree, V, float(np.log(V)) + 1.0)
+    for step in range(4):
+        _compare(z, tree, w.L, 1.0, seed=V, step=step)
+
+
+def test_unaligned_rows_take_the_scalar_path():
+    w = synth.WORKLOADS["tiny"].scaled(batch=2, L=4, V=20001, k=3, B=12)
+    tree = _tree(w)
+    z = np.random.default_rng(8).standard_normal((2, w.n_max, w.V)).astype(np.float32)
+    z = _sharpen(z, tree, 8, 11.0)
+    big = torch.zeros((2, w.n_max, w.V + 3), dtype=torch.float32, device="cuda")
+    big[:, :, :w.V] = torch.from_numpy(z).cuda()
+    view = big.view(2 * w.n_max, w.V + 3)[:, :w.V].view(2, w.n_max, w.V)  # stride V+3
+    assert view.stride(1) == w.V + 3
+    for step in range(3):
+        _compare(z, tree, w.L, 1.0, seed=9, step=step, tensor=view)
+
+
+def test_masked_tokens_and_empty_rows():
+    w = synth.WORKLOADS["tiny"].scaled(batch=4, L=3, V=30000, k=2, B=6)
+    tree = _tree(w)
+    z = np.full((4, w.n_max, w.V), -np.inf, np.float32)
+    g = np.random.default_rng(12)
+    for b in range(3):  # a few finite logits per row, spread over chunks
+        for x in range(w.n_max):
+            idx = g.choice(w.V, 50, replace=False)
+            z[b, x, idx] = g.standard_normal(50) * 2
+    z = np.where(np.isfinite(z), z, np.float32(-np.inf)).astype(np.float32)
+    z[:3] = _sharpen(z[:3], {k: v[:3] for k, v in tree.items()}, 12, 4.0)
+    # sequence 3: every logit -inf -> token 0 at the root
+    ref, got, _ = _compare(z, tree, w.L, 1.0, seed=4, step=0)
+    for b in range(3):
+        a = int(got["acc_len"][b])
+        emitted = list(got["acc_tok"][b][:a]) + [int(got["bonus"][b])]
+        rows = [0] + list(got["acc_nodes"][b][:a])
+        for x, t in zip(rows, emitted):
+            assert np.isfinite(z[b, x, t])
+
+
+def test_zero_temperature_limit_matches_greedy_oracle():
+    w = synth.WORKLOADS["b64"]
+    tree = _tree(w)
+    logits = synth.target_logits(w, tree["tok"], tree["parent"], tree["depth"], tree["n_nodes"])
+    greedy = oracle.tree_walk(logits, tree["tok"], tree["parent"], tree["depth"], tree["n_nodes"], w.L)
+    got = api.tree_walk_sample(logits_tensor(logits), i32(tree["tok"]), i32(tree["parent"]),
+                               i32(tree["depth"]), i32(tree["n_nodes"]), w.L, 1e5, 1, 2)
+    torch.cuda.synchronize()
+    for key in ("acc_len", "acc_nodes", "acc_tok", "bonus"):
+        np.testing.assert_array_equal(got[key].cpu().numpy(), greedy[key], err_msg=key)
+
+
+def test_gpu_draws_follow_softmax():
+    """2048 one-row sequences over the same 40 logits: the root draws follow
+    softmax(z / T) (chi-square), and equal the oracle's draws."""
+    V, nb, T = 40, 2048, 0.8
+    z = np.random.default_rng(21).standard_normal(V).astype(np.float32)
+    logits = np.broadcast_to(z, (nb, 1, V)).copy()
+    tok = np.zeros((nb, 1), np.int32)
+    par = np.full((nb, 1), -1, np.int32)
+    dep = np.zeros((nb, 1), np.int32)
+    n = np.ones(nb, np.int32)
+    got = api.tree_walk_sample(logits_tensor(logits), i32(tok), i32(par), i32(dep), i32(n), 2,
+                               1 / T, 77, 0)
+    draws = got["bonus"].cpu().numpy()
+    ref = [oracle.sample_row(z, 1 / T, oracle.row_uniform(77, 0, b, 0)) for b in range(nb)]
+    for b in range(nb):
+        if ref[b][1] >= SAMPLE_MARGIN:
+            assert draws[b] == ref[b][0], b
+    counts = np.bincount(draws, minlength=V)
+    p = special.softmax(z.astype(np.float64) / T)
+    keep = p * nb >= 5
+    obs = np.append(counts[keep], counts[~keep].sum())
+    exp = np.append(p[keep] * nb, p[~keep].sum() * nb)
+    assert stats.chisquare(obs, exp).pvalue > 1e-4
+
+
+def test_repeated_calls_are_deterministic():
+    w = synth.WORKLOADS["b64"]
+    tree = _tree(w)
+    logits = _sharpen(synth.target_logits(w, tree["tok"], tree["parent"], tree["depth"],
+                                          tree["n_nodes"]), tree, 5, float(np.log(w.V)) + 2.0)
+    t = logits_tensor(logits)
+    args = (i32(tree["tok"]), i32(tree["parent"]), i32(tree["depth"]), i32(tree["n_nodes"]), w.L)
+    first = api.tree_walk_sample(t, *args, 1.0, 5, 9)
+    for _ in range(3):
+        again = api.tree_walk_sample(t, *args, 1.0, 5, 9)
+        for key in first:
+            assert torch.equal(first[key], again[key])
+    # the greedy walk still runs from the same workspace afterwards
+    api.tree_walk(t, *args)
+    torch.cuda.synchronize()
