@@ -593,42 +593,113 @@ double ddto_row_uniform(uint64_t seed, uint64_t step, int b, int j) {
 }
 
 /*
- * One draw from softmax(invT * z) over the V logits at row `base`, by
- * inversion: with w_v = exp(invT*z_v - m), m = max_v invT*z_v, S = sum w_v
- * and C_v = w_0 + ... + w_v (ids in increasing order), the token is the
+ * The draw's weights.  The token is an integer decided by floating point,
+ * so both sides take the decision in the kernel's precision: each weight
+ * is an fp32 evaluation of 2^(a*z), made exact in fp64 by construction,
+ * and only the cumulative sums are fp64.  Per token v:
+ *   a   = fl32(invT * log2(e))           (invT first rounded to fp32)
+ *   t_v = fl32(a * z_v)
+ *   k_v = t_v rounded to the nearest integer (ties to even), r_v = t_v - k_v
+ *   P_v = Horner evaluation in fp32, with fused multiply-adds, of the
+ *         degree-7 Taylor polynomial of 2^r (coefficients (ln 2)^i / i!
+ *         rounded to fp32), at r_v; P_v is within ~1e-7 of 2^(r_v)
+ *   w_v = P_v * 2^(k_v - K) exactly, K = k of the largest t; 0 when
+ *         k_v - K < -120 (so that every weight is a normal fp32 number)
+ *         or z_v = -inf.
+ * w_v / sum(w) differs from softmax(invT * z) by ~|t| * 6e-8 relative: the
+ * rounding of t, as in any fp32 softmax.
+ */
+static const float ddto_p2_coef[8] = {0x1.0p+0f,       0x1.62e43p-1f,  0x1.ebfbep-3f,
+                                      0x1.c6b08ep-5f,  0x1.3b2ab6p-7f, 0x1.5d87fep-10f,
+                                      0x1.430912p-13f, 0x1.ffcbfcp-17f};
+
+float ddto_sampler_exp2_poly(float r) {
+  float p = ddto_p2_coef[7];
+  for (int i = 6; i >= 0; --i) p = fmaf(p, r, ddto_p2_coef[i]);
+  return p;
+}
+
+float ddto_sampler_scale(double invT) {
+  return (float)((double)(float)invT * 1.4426950408889634074);
+}
+
+/* t -> (k, P_v) as above; returns 0 when t is -inf or NaN. */
+static int sampler_split(float t, int* k, float* P) {
+  if (!(t >= -4.0e6f)) return 0;
+  const float kf = nearbyintf(t); /* default rounding: to nearest, ties to even */
+  *k = (int)kf;
+  *P = ddto_sampler_exp2_poly(t - kf);
+  return 1;
+}
+
+/* The weights of one row (w[V]); returns their fp64 sum in index order. */
+static double sampler_weights(const void* logits, int is_bf16, int64_t base, int V, double invT,
+                              double* w) {
+  const float a = ddto_sampler_scale(invT);
+  float tmax = -INFINITY;
+  for (int v = 0; v < V; ++v) {
+    const float t = a * (float)load_val(logits, is_bf16, base + v);
+    if (t > tmax) tmax = t;
+  }
+  double S = 0.0;
+  int K = 0;
+  float Pm;
+  if (!sampler_split(tmax, &K, &Pm)) {
+    for (int v = 0; v < V; ++v) w[v] = 0.0;
+    return 0.0;
+  }
+  for (int v = 0; v < V; ++v) {
+    const float t = a * (float)load_val(logits, is_bf16, base + v);
+    int k;
+    float P;
+    w[v] = 0.0;
+    if (sampler_split(t, &k, &P) && k - K >= -120) w[v] = ldexp((double)P, k - K);
+    S += w[v];
+  }
+  return S;
+}
+
+/* The weights of a row, for the tests. */
+int ddto_sampler_row_weights(const void* logits, int is_bf16, int V, double invT, double* w) {
+  if (!logits || V < 1 || !(invT > 0.0)) return DDTO_ERR_ARG;
+  sampler_weights(logits, is_bf16, 0, V, invT, w);
+  return DDTO_OK;
+}
+
+/*
+ * One draw from the weights above by inversion: with S = sum w and
+ * C_v = w_0 + ... + w_v (ids in increasing order), the token is the
  * smallest v with C_v > u*S.  *margin receives the distance of u*S from the
  * nearer end of the chosen interval [C_{v-1}, C_v), divided by S: a draw
  * with a margin below a computation's relative rounding error may come out
- * differently there.  Logits must be finite or -inf; a row with no finite
- * logit yields token 0 (margin +inf).
+ * differently there.  A row with no finite logit yields token 0 (margin
+ * +inf).
  */
 int ddto_sample_row(const void* logits, int is_bf16, int64_t base, int V, double invT, double u,
                     double* margin) {
-  double m = -INFINITY;
-  for (int v = 0; v < V; ++v) {
-    const double y = invT * load_val(logits, is_bf16, base + v);
-    if (y > m) m = y;
-  }
-  if (m == -INFINITY) {
+  double* w = (double*)malloc(sizeof(double) * (size_t)V);
+  if (!w) return -1;
+  const double S = sampler_weights(logits, is_bf16, base, V, invT, w);
+  if (!(S > 0.0)) {
+    free(w);
     *margin = INFINITY;
     return 0;
   }
-  double S = 0.0;
-  for (int v = 0; v < V; ++v) S += exp(invT * load_val(logits, is_bf16, base + v) - m);
   const double theta = u * S;
   double C = 0.0;
   int last_pos = 0;
   for (int v = 0; v < V; ++v) {
-    const double w = exp(invT * load_val(logits, is_bf16, base + v) - m);
     const double prev = C;
-    C += w;
-    if (w > 0.0) last_pos = v;
+    C += w[v];
+    if (w[v] > 0.0) last_pos = v;
     if (C > theta) {
       const double d0 = theta - prev, d1 = C - theta;
       *margin = (d0 < d1 ? d0 : d1) / S;
+      free(w);
       return v;
     }
   }
+  free(w);
   *margin = 0.0; /* u*S rounded onto the total: the last token of positive weight */
   return last_pos;
 }
