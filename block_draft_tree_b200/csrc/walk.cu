@@ -24,15 +24,17 @@
 // increasing order with u from Philox4x64-10 (Salmon, Moraes, Dror and Shaw,
 // "Parallel Random Numbers: As Easy as 1, 2, 3", SC'11) at counter
 // (j, b, 0, 0) under key (seed, step): u = (top 52 bits of word 0 + 1/2)
-// * 2^-52.  The scan then keeps, per chunk, the pair (m, s) = (max of
-// y = z*log2(e)/T, sum of 2^(y - m)) instead of an argmax key; the row's
-// last CTA merges the pairs, finds the chunk whose cumulative weight first
-// exceeds u times the total, and rescans that one chunk (from L2) with a
-// block prefix sum to find the token.  Weights and sums are fp64: the
-// draws land on tokens of probability ~1/V, so an fp32 cumulative sum
-// (relative error ~1e-7) would move a fair share of them to a neighbour.
-#include <cstring>
-
+// * 2^-52.  The scan then keeps, per chunk, the pair (R, s): an integer
+// reference R (the largest exponent) and the fp64 sum s of the chunk's
+// weights against R, instead of an argmax key; the row's last CTA merges
+// the pairs, finds the chunk whose cumulative weight first exceeds u times
+// the total, and rescans that one chunk (from L2) with a block prefix sum
+// to find the token.  Each weight is an fp32 evaluation of 2^(t - R),
+// t = z*log2(e)/T, that is exact in fp64 by construction (see draw_weight),
+// so weights against different references differ by exact powers of two
+// and only the fp64 sums round: the draws land on tokens of probability
+// ~1/V, where an fp32 cumulative sum (~1e-7 relative error) would move a
+// fair share of them to a neighbour.
 #include "common.cuh"
 #include "launch.h"
 
@@ -53,10 +55,8 @@ struct WalkParams {
   unsigned* row_ticket;  // [batch*n_max]
   unsigned* seq_count;   // [batch]
   int32_t* status;
-  double a;              // sampling: log2(e) / T
+  float a;               // sampling: fl32(log2(e) / T)
   uint64_t seed, step;   // sampling: Philox key
-  double exp2_tab[64];   // sampling: 2^(j/64)
-  double exp2_c[5];      // sampling: (ln 2)^i / i!, i = 1..5
 };
 
 __device__ __forceinline__ uint64_t block_max_key(uint64_t v, uint64_t* sm) {
@@ -131,6 +131,32 @@ __device__ __forceinline__ void load_chunk(Chunk<BF16>& c, const char* rowp, int
     c.v[q] = ld_stream_v4(rowp + (c0 + (int64_t)(q * kThreads + threadIdx.x) * EPV) * ES);
 }
 
+// Loads of a chunk that may run past V: whole 16-byte vectors inside the
+// row, element loads for the one that straddles V, and -inf beyond it.
+template <bool BF16>
+__device__ __forceinline__ void load_chunk_tail(Chunk<BF16>& c, const char* rowp, int c0, int V) {
+  constexpr int EPV = Chunk<BF16>::EPV, ES = BF16 ? 2 : 4;
+#pragma unroll
+  for (int q = 0; q < Chunk<BF16>::VPT; ++q) {
+    const int idx = c0 + (q * kThreads + threadIdx.x) * EPV;
+    if (idx + EPV <= V) {
+      c.v[q] = ld_stream_v4(rowp + (int64_t)idx * ES);
+    } else {
+      uint32_t w[4];
+      for (int e = 0; e < 4; ++e) {
+        if (BF16) {
+          const uint32_t lo = idx + 2 * e < V ? ((const uint16_t*)rowp)[idx + 2 * e] : 0xFF80u;
+          const uint32_t hi = idx + 2 * e + 1 < V ? ((const uint16_t*)rowp)[idx + 2 * e + 1] : 0xFF80u;
+          w[e] = lo | (hi << 16);
+        } else {
+          w[e] = idx + e < V ? ((const uint32_t*)rowp)[idx + e] : 0xFF800000u;
+        }
+      }
+      c.v[q] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+}
+
 // Thread-local argmax of a loaded chunk; each thread sees its indices in
 // increasing order, so strict > keeps the smallest index among equal values.
 template <bool BF16>
@@ -187,90 +213,193 @@ __device__ __forceinline__ double row_uniform(const WalkParams& p, int b, int j)
   return ((double)(w >> 12) + 0.5) * 0x1.0p-52;
 }
 
-// 2^t in fp64 by Tang's table-driven method ("Table-driven implementation
-// of the exponential function in IEEE floating-point arithmetic", ACM TOMS
-// 15(2), 1989), for the non-positive arguments of the draw: t = n + j/64 + r
-// with |r| <= 1/128, 2^t = 2^n * 2^(j/64) * (1 + q(r)), q the Taylor series
-// of 2^r - 1 to degree 5 (truncation below 4e-17 relative).  The table
-// 2^(j/64) and the coefficients (ln 2)^i / i! come from the host.  Arguments
-// below -1000 (and -inf) give 0; the draw's weights are then negligible
-// against the largest weight, which is 1.
-__device__ __forceinline__ double tang_exp2(double t, const double* tab, const double* c) {
-  if (!(t >= -1000.0)) return 0.0;
-  const double shifter = 0x1.8p52;                    // round-to-integer by addition
-  const double sh = fma(t, 64.0, shifter);
-  const int k = __double2loint(sh);                   // round(64 t)
-  const double kd = sh - shifter;
-  const double r = fma(kd, -0.015625, t);             // exact
-  const double q = r * fma(fma(fma(fma(c[4], r, c[3]), r, c[2]), r, c[1]), r, c[0]);
-  const double tj = tab[k & 63];
-  const double y = fma(tj, q, tj);                    // in [1, 2)
-  const int n = k >> 6;                               // floor(k / 64)
-  return __hiloint2double(__double2hiint(y) + (n << 20), __double2loint(y));
+// The draw's weights.  The token is an integer decided by floating point,
+// so its arithmetic is fixed exactly: a = fl32(invT * log2 e),
+// t = fl32(a * z), k = nearest integer to t (ties to even), r = t - k,
+// P = fp32 Horner evaluation with fused multiply-adds of the degree-7
+// Taylor polynomial of 2^r (coefficients (ln 2)^i / i! rounded to fp32),
+// and w = P * 2^(k - R), an exact normal fp32 number, for an integer
+// reference R >= k (0 when k - R < -120 or z = -inf).  Weights taken
+// against different references differ by exact powers of two, so every
+// chunk and thread sums against its own maximum and the sums merge without
+// rounding the weights again.  A thread sums its 32 weights as two
+// double-float sums of 16 (an exact TwoSum per term; the low part, below
+// 2^-20 of the high part, rounds at 2^-24 of itself per term: relative
+// error below 2^-40), and everything after that is fp64.
+__device__ __forceinline__ float draw_poly(float r) {
+  float p = 0x1.ffcbfcp-17f;
+  p = fmaf(p, r, 0x1.430912p-13f);
+  p = fmaf(p, r, 0x1.5d87fep-10f);
+  p = fmaf(p, r, 0x1.3b2ab6p-7f);
+  p = fmaf(p, r, 0x1.c6b08ep-5f);
+  p = fmaf(p, r, 0x1.ebfbep-3f);
+  p = fmaf(p, r, 0x1.62e43p-1f);
+  return fmaf(p, r, 1.0f);
 }
 
-struct Exp2Table {
-  double tab[64];
-  double c[5];
-};
+constexpr float kRoundShift = 12582912.0f;  // 1.5 * 2^23: t + shift rounds t to an integer
+constexpr int kRoundShiftBits = 0x4B400000;
+constexpr int kNoRef = -(1 << 30);          // reference of a thread with no finite logit
 
-// Merge the pair (m2, s2) into (m, s); s is a sum of 2^(y - m).
-__device__ __forceinline__ void ms_add(double& m, double& s, double m2, double s2,
-                                       const Exp2Table& e) {
-  if (m2 == -INFINITY) return;
-  if (m2 > m) {
-    s = s * tang_exp2(m - m2, e.tab, e.c) + s2;
-    m = m2;
+// R = nearest integer to t (|t| < 2^22).
+__device__ __forceinline__ int draw_ref(float t) {
+  return t >= -4.0e6f ? __float_as_int(__fadd_rn(t, kRoundShift)) - kRoundShiftBits : kNoRef;
+}
+
+// w = P(t - k) * 2^(k - R), with t = a*z already rounded to fp32 and
+// R >= -4e6.  Branch free: for t below -2^22 (and -inf) the rounding trick
+// yields an exponent far below R - 120, so the final select discards it.
+__device__ __forceinline__ float draw_weight(float t, int R) {
+  const float sh = __fadd_rn(t, kRoundShift);
+  const int e = __float_as_int(sh) - (kRoundShiftBits + R);
+  const float r = __fsub_rn(t, __fsub_rn(sh, kRoundShift));
+  const float w = __int_as_float(__float_as_int(draw_poly(r)) + (e << 23));
+  return e >= -120 ? w : 0.f;
+}
+
+// Packed pairs of fp32 (lane 0 in the low word): every operation rounds
+// each lane exactly as its scalar form does.
+__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void upk2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+// b - a, rounded once (a*(-1) is exact).
+__device__ __forceinline__ uint64_t sub2(uint64_t b, uint64_t a) {
+  return fma2(a, pk2(-1.f, -1.f), b);
+}
+
+// The weights of a pair of arguments t (packed), as draw_weight.
+__device__ __forceinline__ uint64_t draw_weight2(uint64_t t2, int R) {
+  const uint64_t sh2 = add2(t2, pk2(kRoundShift, kRoundShift));
+  const uint64_t r2 = sub2(t2, add2(sh2, pk2(-kRoundShift, -kRoundShift)));
+  uint64_t p2 = fma2(pk2(0x1.ffcbfcp-17f, 0x1.ffcbfcp-17f), r2, pk2(0x1.430912p-13f, 0x1.430912p-13f));
+  p2 = fma2(p2, r2, pk2(0x1.5d87fep-10f, 0x1.5d87fep-10f));
+  p2 = fma2(p2, r2, pk2(0x1.3b2ab6p-7f, 0x1.3b2ab6p-7f));
+  p2 = fma2(p2, r2, pk2(0x1.c6b08ep-5f, 0x1.c6b08ep-5f));
+  p2 = fma2(p2, r2, pk2(0x1.ebfbep-3f, 0x1.ebfbep-3f));
+  p2 = fma2(p2, r2, pk2(0x1.62e43p-1f, 0x1.62e43p-1f));
+  p2 = fma2(p2, r2, pk2(1.f, 1.f));
+  float sa, sb, pa, pb;
+  upk2(sh2, sa, sb);
+  upk2(p2, pa, pb);
+  const int ea = __float_as_int(sa) - (kRoundShiftBits + R);
+  const int eb = __float_as_int(sb) - (kRoundShiftBits + R);
+  const float wa = ea >= -120 ? __int_as_float(__float_as_int(pa) + (ea << 23)) : 0.f;
+  const float wb = eb >= -120 ? __int_as_float(__float_as_int(pb) + (eb << 23)) : 0.f;
+  return pk2(wa, wb);
+}
+
+// hi + lo += w lane by lane, with hi + w split exactly (Knuth's TwoSum).
+__device__ __forceinline__ void two_sum_add2(uint64_t& hi, uint64_t& lo, uint64_t w) {
+  const uint64_t s = add2(hi, w);
+  const uint64_t bp = sub2(s, hi);
+  const uint64_t err = add2(sub2(hi, sub2(s, bp)), sub2(w, bp));
+  hi = s;
+  lo = add2(lo, err);
+}
+
+__device__ __forceinline__ float fmax3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+
+// s * 2^d for d <= 0, exact (0 below 2^-1000).
+__device__ __forceinline__ double scale2(double s, int d) {
+  return d < -1000 ? 0.0 : s * __hiloint2double((1023 + d) << 20, 0);
+}
+
+// Merge the pair (R2, s2) into (R, s); s is a sum of weights against R.
+__device__ __forceinline__ void rs_add(int& R, double& s, int R2, double s2) {
+  if (R2 == kNoRef) return;
+  if (R == kNoRef) {
+    R = R2;
+    s = s2;
+  } else if (R2 > R) {
+    s = scale2(s, R - R2) + s2;
+    R = R2;
   } else {
-    s += s2 * tang_exp2(m2 - m, e.tab, e.c);
+    s += scale2(s2, R2 - R);
   }
 }
 
-// Thread pair (max y, sum 2^(y - max y)) over a loaded chunk, y = a*z in fp64.
+// Thread pair (R, sum of weights against R) over a loaded chunk, two
+// tokens per packed instruction.  The thread's 32 weights are summed as two
+// interleaved double-float sums of 16.
 template <bool BF16>
-__device__ __forceinline__ void ms_chunk(const Chunk<BF16>& c, double a, const Exp2Table& e,
-                                         double& m, double& s) {
+__device__ __forceinline__ void rs_chunk(const Chunk<BF16>& c, float a, int& R, double& s) {
   float zm = -INFINITY;
 #pragma unroll
   for (int q = 0; q < Chunk<BF16>::VPT; ++q) {
     const uint32_t w[4] = {c.v[q].x, c.v[q].y, c.v[q].z, c.v[q].w};
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      if (BF16) zm = fmaxf(zm, fmaxf(bf16_lo(w[i]), bf16_hi(w[i])));
-      else zm = fmaxf(zm, __uint_as_float(w[i]));
-    }
-  }
-  m = a * (double)zm;
-  s = 0.0;
-  if (zm == -INFINITY) return;
-#pragma unroll
-  for (int q = 0; q < Chunk<BF16>::VPT; ++q) {
-    const uint32_t w[4] = {c.v[q].x, c.v[q].y, c.v[q].z, c.v[q].w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 4; i += 2) {
       if (BF16) {
-        s += tang_exp2(fma(a, (double)bf16_lo(w[i]), -m), e.tab, e.c);
-        s += tang_exp2(fma(a, (double)bf16_hi(w[i]), -m), e.tab, e.c);
+        zm = fmax3f(zm, bf16_lo(w[i]), bf16_hi(w[i]));
+        zm = fmax3f(zm, bf16_lo(w[i + 1]), bf16_hi(w[i + 1]));
       } else {
-        s += tang_exp2(fma(a, (double)__uint_as_float(w[i]), -m), e.tab, e.c);
+        zm = fmax3f(zm, __uint_as_float(w[i]), __uint_as_float(w[i + 1]));
       }
     }
   }
+  R = draw_ref(__fmul_rn(a, zm));  // fl32(a*z) is monotone in z
+  s = 0.0;
+  if (R == kNoRef) return;
+  const uint64_t a2 = pk2(a, a);
+  uint64_t hi = pk2(0.f, 0.f), lo = pk2(0.f, 0.f);
+#pragma unroll
+  for (int q = 0; q < Chunk<BF16>::VPT; ++q) {
+    const uint32_t w[4] = {c.v[q].x, c.v[q].y, c.v[q].z, c.v[q].w};
+    if (BF16) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        two_sum_add2(hi, lo, draw_weight2(mul2(a2, pk2(bf16_lo(w[i]), bf16_hi(w[i]))), R));
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; i += 2)
+        two_sum_add2(hi, lo, draw_weight2(mul2(a2, pk2(__uint_as_float(w[i]), __uint_as_float(w[i + 1]))), R));
+    }
+  }
+  float ha, hb, la, lb;
+  upk2(hi, ha, hb);
+  upk2(lo, la, lb);
+  s = ((double)ha + (double)la) + ((double)hb + (double)lb);
 }
 
 // Block merge of the threads' pairs; the result is valid in thread 0.
-__device__ __forceinline__ double2 block_ms(double m, double s, double2* sm, const Exp2Table& e) {
+__device__ __forceinline__ void block_rs(int& R, double& s, double2* sm) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
-    const double m2 = __shfl_xor_sync(0xFFFFFFFFu, m, o), s2 = __shfl_xor_sync(0xFFFFFFFFu, s, o);
-    ms_add(m, s, m2, s2, e);
+    const int R2 = __shfl_xor_sync(0xFFFFFFFFu, R, o);
+    const double s2 = __shfl_xor_sync(0xFFFFFFFFu, s, o);
+    rs_add(R, s, R2, s2);
   }
-  if (lane == 0) sm[warp] = make_double2(m, s);
+  if (lane == 0) sm[warp] = make_double2((double)R, s);
   __syncthreads();
-  double2 r = sm[0];
-  for (int w = 1; w < kThreads / 32; ++w) ms_add(r.x, r.y, sm[w].x, sm[w].y, e);
-  return r;
+  R = (int)sm[0].x;
+  s = sm[0].y;
+  for (int w = 1; w < kThreads / 32; ++w) rs_add(R, s, (int)sm[w].x, sm[w].y);
 }
 
 // Inclusive prefix sum over the lanes of a warp.
@@ -285,8 +414,8 @@ __device__ __forceinline__ double warp_incl_scan(double v) {
 }
 
 struct SampleSmem {
-  double M, P, theta;
-  int cstar;
+  double P, theta;
+  int R, cstar;
   double wsum[kThreads / 32];
   int hit, last;
 };
@@ -299,26 +428,26 @@ __device__ __forceinline__ float load_logit(const char* rowp, int idx, bool bf16
 // `part`; called by the whole block, returns the token in every thread.
 template <bool BF16>
 __device__ int sample_row_token(const WalkParams& p, int b, int j, int64_t row, const char* rowp,
-                                const Exp2Table& e, SampleSmem& sm) {
+                                SampleSmem& sm) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const double2* part = (const double2*)p.part + row * p.S;
   if (warp == 0) {
-    double M = -INFINITY;
-    for (int c = lane; c < p.S; c += 32) M = fmax(M, __ldcg(&part[c]).x);
+    int R = kNoRef;
+    for (int c = lane; c < p.S; c += 32) R = max(R, (int)__ldcg(&part[c]).x);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmax(M, __shfl_xor_sync(0xFFFFFFFFu, M, o));
+    for (int o = 16; o > 0; o >>= 1) R = max(R, __shfl_xor_sync(0xFFFFFFFFu, R, o));
     // two identical passes of the chunk prefix sum: the total, then the
     // first chunk whose inclusive prefix exceeds theta
     double theta = 0.0, P = 0.0, Plast = 0.0;
     int cstar = -1, clast = -1;
-    for (int pass = 0; pass < 2 && M != -INFINITY; ++pass) {
+    for (int pass = 0; pass < 2 && R != kNoRef; ++pass) {
       double carry = 0.0;
       for (int g = 0; g < p.S; g += 32) {
         const int c = g + lane;
         double W = 0.0;
         if (c < p.S) {
-          const double2 ms = __ldcg(&part[c]);
-          if (ms.x != -INFINITY) W = ms.y * tang_exp2(ms.x - M, e.tab, e.c);
+          const double2 rs = __ldcg(&part[c]);
+          if ((int)rs.x != kNoRef) W = scale2(rs.y, (int)rs.x - R);
         }
         const double incl = carry + warp_incl_scan(W);
         double excl = __shfl_up_sync(0xFFFFFFFFu, incl, 1);
@@ -347,7 +476,7 @@ __device__ int sample_row_token(const WalkParams& p, int b, int j, int64_t row, 
       P = Plast;
     }
     if (lane == 0) {
-      sm.M = M;
+      sm.R = R;
       sm.P = P;
       sm.theta = theta;
       sm.cstar = cstar;
@@ -358,7 +487,9 @@ __device__ int sample_row_token(const WalkParams& p, int b, int j, int64_t row, 
   __syncthreads();
   const int cstar = sm.cstar;
   if (cstar < 0) return 0;  // no finite logit in the row
-  const double M = sm.M, theta = sm.theta, a = p.a;
+  const int R = sm.R;
+  const double theta = sm.theta;
+  const float a = p.a;
   // each thread owns kPer consecutive tokens of chunk cstar
   constexpr int kPer = kChunk / kThreads;
   const int e0 = cstar * kChunk + tid * kPer;
@@ -366,7 +497,7 @@ __device__ int sample_row_token(const WalkParams& p, int b, int j, int64_t row, 
   double local = 0.0;
   int last = -1;
   for (int i = e0; i < e1; ++i) {
-    const double w = tang_exp2(fma(a, (double)load_logit(rowp, i, BF16), -M), e.tab, e.c);
+    const double w = (double)draw_weight(__fmul_rn(a, load_logit(rowp, i, BF16)), R);
     local += w;
     if (w > 0.0) last = i;
   }
@@ -384,7 +515,7 @@ __device__ int sample_row_token(const WalkParams& p, int b, int j, int64_t row, 
     double cum = base;
     int hit = last;
     for (int i = e0; i < e1; ++i) {
-      cum += tang_exp2(fma(a, (double)load_logit(rowp, i, BF16), -M), e.tab, e.c);
+      cum += (double)draw_weight(__fmul_rn(a, load_logit(rowp, i, BF16)), R);
       if (cum > theta) {
         hit = i;
         break;
@@ -421,31 +552,31 @@ __global__ void __launch_bounds__(kThreads) walk_kernel(WalkParams p) {
   const int c0 = chunk * kChunk;
 
   if constexpr (SAMPLE) {
-    __shared__ Exp2Table e;
     __shared__ SampleSmem sm;
-    if (tid < 64) e.tab[tid] = p.exp2_tab[tid];
-    if (tid < 5) e.c[tid] = p.exp2_c[tid];
-    // chunk pair (max y, sum 2^(y - max y)), y = a*z
-    double m = -INFINITY, sum = 0.0;
-    if (p.vec_ok && c0 + kChunk <= p.V) {
+    // chunk pair (reference R, sum of weights against R)
+    int R = kNoRef;
+    double sum = 0.0;
+    if (p.vec_ok) {
       Chunk<BF16> cur;
-      load_chunk<BF16>(cur, rowp, c0);
-      __syncthreads();
-      ms_chunk<BF16>(cur, p.a, e, m, sum);
+      if (c0 + kChunk <= p.V) load_chunk<BF16>(cur, rowp, c0);
+      else load_chunk_tail<BF16>(cur, rowp, c0, p.V);
+      rs_chunk<BF16>(cur, p.a, R, sum);
     } else {
-      __syncthreads();
       for (int q = 0; q < Chunk<BF16>::VPT; ++q)
         for (int i = 0; i < EPV; ++i) {
           const int idx = c0 + (q * kThreads + tid) * EPV + i;
           if (idx >= p.V) continue;
-          ms_add(m, sum, p.a * (double)load_logit(rowp, idx, BF16), 1.0, e);
+          const float t = __fmul_rn(p.a, load_logit(rowp, idx, BF16));
+          const int Rv = draw_ref(t);
+          rs_add(R, sum, Rv, Rv == kNoRef ? 0.0 : (double)draw_weight(t, Rv));
         }
     }
     pdl_trigger();
-    const double2 ms = block_ms(m, sum, (double2*)s_red2, e);
+    block_rs(R, sum, (double2*)s_red2);
+    const double2 rs = make_double2((double)R, sum);
     if (p.S > 1) {
       if (tid == 0) {
-        ((double2*)p.part)[row * p.S + chunk] = ms;
+        ((double2*)p.part)[row * p.S + chunk] = rs;
         __threadfence();
         s_flag = (atomicAdd(&p.row_ticket[row], 1u) == (unsigned)(p.S - 1));
       }
@@ -453,10 +584,10 @@ __global__ void __launch_bounds__(kThreads) walk_kernel(WalkParams p) {
       if (!s_flag) return;
       __threadfence();
     } else {
-      if (tid == 0) ((double2*)p.part)[row] = ms;
+      if (tid == 0) ((double2*)p.part)[row] = rs;
       __syncthreads();
     }
-    const int t = sample_row_token<BF16>(p, b, j, row, rowp, e, sm);
+    const int t = sample_row_token<BF16>(p, b, j, row, rowp, sm);
     if (tid == 0) {
       p.amax[row] = t;
       if (p.S > 1) p.row_ticket[row] = 0u;  // the counter region is left zero
@@ -541,21 +672,7 @@ ddt_status launch_tree_walk(const void* logits, ddt_dtype dt, int batch, int n_m
                             int32_t* acc_nodes, int32_t* acc_tok, int32_t* bonus, void* ws,
                             int32_t* dev_status, cudaStream_t stream, const WalkSampling* sampling) {
   WalkParams p;
-  p.a = sampling ? (double)sampling->inv_temperature * 1.4426950408889634074 : 0.0;
-  if (sampling) {
-    static const Exp2Table host_tab = [] {
-      Exp2Table t;
-      for (int i = 0; i < 64; ++i) t.tab[i] = exp2((double)i / 64.0);
-      double c = 1.0;
-      for (int i = 1; i <= 5; ++i) {
-        c *= 0.69314718055994530942 / i;  // (ln 2)^i / i!
-        t.c[i - 1] = c;
-      }
-      return t;
-    }();
-    memcpy(p.exp2_tab, host_tab.tab, sizeof p.exp2_tab);
-    memcpy(p.exp2_c, host_tab.c, sizeof p.exp2_c);
-  }
+  p.a = sampling ? (float)((double)sampling->inv_temperature * 1.4426950408889634074) : 0.f;
   p.seed = sampling ? sampling->seed : 0;
   p.step = sampling ? sampling->step : 0;
   p.logits = logits;

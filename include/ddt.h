@@ -260,13 +260,17 @@ ddt_status ddt_tree_walk(const void* logits, ddt_dtype dtype, int batch, int n_m
  * conditional given the accepted prefix.
  *
  * The draw of row j of sequence b is by inversion over token ids in
- * increasing order: with w_v = exp(z_v/T - max), the token is the smallest
- * v whose cumulative weight exceeds u * sum(w), where u = (w0 >> 12) + 1/2
- * times 2^-52 and w0 is word 0 of Philox4x64-10 (Salmon, Moraes, Dror and
- * Shaw, SC'11) at counter (j, b, 0, 0) under key (seed, step).  Weights
- * and sums are fp64, so the draw agrees with exact arithmetic unless u*sum
- * lies within about 1e-14 (relative) of an interval end.  Logits must be
- * finite or -inf; a row with no finite logit draws token 0.
+ * increasing order: the token is the smallest v whose cumulative weight
+ * exceeds u * sum(w), where u = (w0 >> 12) + 1/2 times 2^-52 and w0 is word
+ * 0 of Philox4x64-10 (Salmon, Moraes, Dror and Shaw, SC'11) at counter
+ * (j, b, 0, 0) under key (seed, step).  The weights are fp32 evaluations
+ * of exp(z/T - max) with a fixed arithmetic (a = fl32(log2(e)/T),
+ * t = fl32(a*z), k = round(t), w = P(t - k) * 2^(k - K) with P the fp32
+ * Horner form of the degree-7 Taylor polynomial of 2^r and K = round of
+ * the row's largest t; 0 below 2^-120), so they are reproducible exactly;
+ * their sums are at least double-float (~48-bit) accurate.  The distribution is softmax(z/T) up to the fp32 rounding of t
+ * (~|t| * 6e-8 relative).  Logits must be finite or -inf, with
+ * |z/T| < 2^21; a row with no finite logit draws token 0.
  *
  *   inv_temperature  1/T, finite and > 0 (larger -> closer to greedy)
  *   seed, step       the Philox key: a stream per request (seed) and a

@@ -1,20 +1,20 @@
 """Parity of ddt_tree_walk_sample (CUDA, through the C ABI) with the oracle's
 sampled walk.
 
-Each visited row draws its token by inversion of softmax(z / T) with the
-Philox4x64-10 uniform of its (sequence, row).  Both sides compute the
-weights and their cumulative sums in fp64, in different orders, so a draw
-can only differ where u*S lies within rounding of an interval end.  The
-rule: when the oracle's smallest draw margin along a walk is at least
+Each visited row draws its token by inversion with the Philox4x64-10
+uniform of its (sequence, row).  The weights follow one fixed fp32
+arithmetic on both sides and are exact fp64 numbers, so they agree bit for
+bit; only their fp64 cumulative sums differ, by summation order.  A draw can
+therefore only differ where u*S lies within rounding of an interval end.
+The rule: when the oracle's smallest draw margin along a walk is at least
 SAMPLE_MARGIN (relative to S), the walk is bit-exact; otherwise every
 decision along the CUDA walk whose margin clears SAMPLE_MARGIN must equal
 the oracle's draw and the walk must be a valid walk of the tree.
 
-Error budget behind SAMPLE_MARGIN: each fp64 weight is within ~2 ulp of
-exp(y - m) (the exponent argument is formed with one rounding of a value
-below ~40 in magnitude, so ~1e-14 absolute, then a table-driven exp2);
-sums of <= 151936 non-negative terms add < 151936 * 2^-53 ~ 2e-11 relative
-in the worst case and far less in practice.  1e-10 stays clear of both.
+Error budget behind SAMPLE_MARGIN: the kernel's per-thread double-float
+sums of 32 weights are within 2^-38 (~4e-12) of exact, and a sum of
+n <= 151936 non-negative fp64 terms in any order is within n * 2^-53
+(~2e-11) of the exact sum, relative to S; 1e-10 stays clear of both.
 """
 import numpy as np
 import pytest
