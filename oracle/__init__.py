@@ -18,6 +18,8 @@ curated summary of the authors' announcement), section "運作流程"
   tree row against the context KV cache and the tree's own KV;
 * :func:`tree_walk`  -- step 4, the greedy walk that accepts matching
   children and returns the bonus token;
+* :func:`kv_commit`  -- after step 4: the root and the accepted rows' K/V
+  appended to the committed context, which grows by acc_len + 1;
 * :func:`tree_walk_sample` -- step 4 under a sampling decoding rule
   (temperature > 0): each visited row draws its token from softmax(z / T)
   by inversion with a Philox4x64-10 uniform (:func:`philox4x64_10`,
@@ -102,6 +104,12 @@ def _load():
                                               ctypes.POINTER(ctypes.c_int32), i32p, i32p,
                                               ctypes.POINTER(ctypes.c_int32),
                                               ctypes.POINTER(ctypes.c_double)]
+        lib.ddto_kv_commit.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                                       ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                       ctypes.c_void_p, ctypes.POINTER(ctypes.c_int32),
+                                       ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                       ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+        lib.ddto_kv_commit.restype = ctypes.c_int
         for f in (lib.ddto_topk, lib.ddto_build_tree, lib.ddto_tree_attn, lib.ddto_tree_walk,
                   lib.ddto_sample_row, lib.ddto_tree_walk_sample):
             f.restype = ctypes.c_int
@@ -351,3 +359,45 @@ def tree_walk_sample(logits, tok, parent, depth, n_nodes, L, inv_temperature, se
         res["bonus"][b] = bo.value
         res["min_margin"][b] = mm.value
     return res
+
+
+def kv_commit(k_tree, v_tree, acc_len, acc_nodes, ctx_len, k_cache, v_cache, page_table=None,
+              page_size=64, num_pages=0):
+    """Append each sequence's root and accepted rows of the tree K/V to the
+    cache (in place on copies) and advance ctx_len by acc_len + 1.
+
+    ``k_tree``/``v_tree`` bf16 bits (uint16) [batch, n_max, hkv, d]; the
+    cache is dense [batch, t_max, hkv, d] (``page_table`` None) or a page pool
+    [pages, page_size, hkv, d].  Returns (k_cache, v_cache, ctx_len, ok) with
+    ok[b] False where a position fell outside the cache.
+    """
+    kt = np.ascontiguousarray(k_tree, np.uint16)
+    vt = np.ascontiguousarray(v_tree, np.uint16)
+    kc = np.array(k_cache, np.uint16, copy=True, order="C")
+    vc = np.array(v_cache, np.uint16, copy=True, order="C")
+    bsz, n_max, hkv, d = kt.shape
+    cl = np.array(ctx_len, np.int32, copy=True)
+    ok = np.ones(bsz, bool)
+    lib = _load()
+    for b in range(bsz):
+        a = int(acc_len[b])
+        nodes = np.ascontiguousarray(np.asarray(acc_nodes[b], np.int32)[:max(a, 1)])
+        c = ctypes.c_int32(int(cl[b]))
+        if page_table is None:
+            kb, vb = kc[b], vc[b]
+            t_max, pages, maxp = kb.shape[0], None, 0
+        else:
+            kb, vb = kc, vc
+            t_max = 0
+            pages = np.ascontiguousarray(page_table[b], np.int32)
+            maxp = pages.shape[0]
+        rc = lib.ddto_kv_commit(kt[b].ctypes.data_as(ctypes.c_void_p),
+                                vt[b].ctypes.data_as(ctypes.c_void_p), n_max, hkv, d, a,
+                                nodes.ctypes.data_as(ctypes.c_void_p), ctypes.byref(c),
+                                kb.ctypes.data_as(ctypes.c_void_p),
+                                vb.ctypes.data_as(ctypes.c_void_p), t_max,
+                                None if pages is None else pages.ctypes.data_as(ctypes.c_void_p),
+                                page_size, maxp, num_pages)
+        ok[b] = rc == 0
+        cl[b] = c.value
+    return kc, vc, cl, ok

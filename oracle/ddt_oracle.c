@@ -746,3 +746,63 @@ int ddto_tree_walk_sample(const void* logits, int is_bf16, int64_t row_stride, i
   *min_margin = mm;
   return DDTO_OK;
 }
+
+/* ------------------------------------------------------------------ */
+/* KV commit of the accepted path                                      */
+/* ------------------------------------------------------------------ */
+/*
+ * After the walk (step 4), the round has forwarded the root (the previous
+ * round's bonus token, which the target had produced but not yet run; page
+ * workflow, opening paragraph) and the accepted rows; the new bonus token
+ * has not been forwarded.  So the committed context of sequence b grows by
+ * acc_len + 1 positions: position ctx_len + i receives the K/V of the i-th
+ * row of the path root, acc_nodes[0], ..., acc_nodes[acc_len - 1] (the row
+ * at depth i, whose position id was ctx_len + i), and ctx_len advances by
+ * acc_len + 1.
+ *
+ * Layouts (bf16 as raw uint16): tree K/V [n_max][hkv][d] of this sequence;
+ * the cache either dense [t_max][hkv][d] of this sequence (page_table NULL)
+ * or a page pool [pages][page_size][hkv][d] with this sequence's page list.
+ * A position outside the cache (or a page id outside the pool) is not
+ * written; the function then returns DDTO_ERR_ARG after writing the rest.
+ */
+int ddto_kv_commit(const uint16_t* k_tree, const uint16_t* v_tree, int n_max, int hkv, int d,
+                   int acc_len, const int32_t* acc_nodes, int32_t* ctx_len, uint16_t* k_cache,
+                   uint16_t* v_cache, int64_t t_max, const int32_t* pages, int page_size,
+                   int max_pages, int num_pages) {
+  if (!k_tree || !v_tree || !ctx_len || !k_cache || !v_cache || acc_len < 0 || hkv < 1 || d < 1)
+    return DDTO_ERR_ARG;
+  const int64_t row = (int64_t)hkv * d;
+  const int c = *ctx_len;
+  int bad = 0;
+  for (int i = 0; i <= acc_len; ++i) {
+    const int r = i == 0 ? 0 : acc_nodes[i - 1];
+    if (r < 0 || r >= n_max) {
+      bad = 1;
+      continue;
+    }
+    const int64_t pos = (int64_t)c + i;
+    int64_t dst;
+    if (!pages) {
+      if (pos >= t_max) {
+        bad = 1;
+        continue;
+      }
+      dst = pos * row;
+    } else {
+      const int64_t pi = pos / page_size;
+      const int pg = pi < max_pages ? pages[pi] : -1;
+      if (pg < 0 || (num_pages > 0 && pg >= num_pages)) {
+        bad = 1;
+        continue;
+      }
+      dst = ((int64_t)pg * page_size + pos % page_size) * row;
+    }
+    for (int64_t e = 0; e < row; ++e) {
+      k_cache[dst + e] = k_tree[(int64_t)r * row + e];
+      v_cache[dst + e] = v_tree[(int64_t)r * row + e];
+    }
+  }
+  *ctx_len = c + acc_len + 1;
+  return bad ? DDTO_ERR_ARG : DDTO_OK;
+}
