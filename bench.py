@@ -276,6 +276,68 @@ def run_reference(args):
     return 0
 
 
+def measure_extensions(w, sets, graphs, hbm_peak, reps=30):
+    """Per-launch device time of the library's calls beyond the round proper
+    (the sampled walk), each launch after an L2 flush, on the round's own
+    target logits and trees.  Not part of the timed region."""
+    import torch
+
+    from block_draft_tree_b200 import api
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    inv_t = 1.0
+    times = []
+    n_rows = []
+    for rep in range(reps + 3):
+        j = rep % len(sets)
+        o = graphs[j][1].out
+        tgt = sets[j]["target"]
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        api.tree_walk_sample(tgt, o["tok"], o["parent"], o["depth"], o["n_nodes"], w.L, inv_t,
+                             seed=12345, step=rep)
+        b.record()
+        torch.cuda.synchronize()
+        if rep >= 3:
+            times.append(a.elapsed_time(b) * 1e3)
+            n_rows.append(int(o["n_nodes"].sum().item()))
+    us = statistics.median(times)
+    alg = statistics.mean(n_rows) * w.V * 4  # every tree row's fp32 target logits, read once
+    gbs = alg / (us * 1e-6) / 1e9
+    ext = {"walk_sample": {"us": round(us, 3), "alg_bytes": int(alg), "gbs": round(gbs, 1),
+                           "frac_hbm": round(gbs / hbm_peak, 4), "inv_temperature": inv_t,
+                           "launches": len(times), "l2": "flushed before each launch"}}
+
+    # KV commit of each round's accepted path, into copies of the cache (the
+    # timed rounds' own buffers stay as they were)
+    kc = sets[0]["k_cache"].clone()
+    vc = sets[0]["v_cache"].clone()
+    pt = sets[0].get("page_table")
+    cl = torch.empty_like(sets[0]["ctx_len"])
+    times, rows = [], []
+    for rep in range(reps + 3):
+        j = rep % len(sets)
+        o = graphs[j][1].out
+        cl.copy_(sets[j]["ctx_len"])
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        api.kv_commit(sets[j]["k_tree"], sets[j]["v_tree"], o["acc_len"], o["acc_nodes"], cl,
+                      kc, vc, page_table=pt, page_size=w.page_size or 64)
+        b.record()
+        torch.cuda.synchronize()
+        if rep >= 3:
+            times.append(a.elapsed_time(b) * 1e3)
+            rows.append(int(o["acc_len"].sum().item()) + w.batch)
+    us = statistics.median(times)
+    alg = statistics.mean(rows) * w.hkv * w.d * 2 * 2 * 2  # K and V rows, read and written
+    ext["kv_commit"] = {"us": round(us, 3), "alg_bytes": int(alg),
+                        "gbs": round(alg / (us * 1e-6) / 1e9, 2), "launches": len(times),
+                        "bound": "launch latency (a few KB per sequence)"}
+    return ext
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -402,6 +464,7 @@ def run_ours(args):
             "peak_kind": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind if peak_kind == "measured"
             else "fallback"}
     acc = [r.out["acc_len"].float().mean().item() for _, r in graphs]
+    ext = measure_extensions(w, sets, graphs, hbm_peak) if rank == 0 else None
 
     # end to end: pinned host inputs -> H2D -> round -> D2H of the result, every step
     e2e = None
@@ -467,7 +530,7 @@ def run_ours(args):
             "data": "synthetic", "config": workload_config(w, args.sets, set_bytes),
             "roofline": roof, "stages": stages, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps, "clocks": clk,
-            "mean_accepted": round(statistics.mean(acc), 3),
+            "mean_accepted": round(statistics.mean(acc), 3), "extensions": ext,
             "parallelism": "dp%d (independent sequences per GPU)" % world}
     print(json.dumps(line), flush=True)
     if world > 1:

@@ -28,7 +28,20 @@ DDT_TREE_B_MAX = 1023
 
 EXPORTED = ("ddt_status_string", "ddt_mask_words", "ddt_topk_workspace_size", "ddt_topk",
             "ddt_build_tree", "ddt_tree_attn_workspace_size", "ddt_tree_attn",
-            "ddt_tree_walk_workspace_size", "ddt_tree_walk", "ddt_tree_walk_sample")
+            "ddt_tree_walk_workspace_size", "ddt_tree_walk", "ddt_tree_walk_sample",
+            "ddt_kv_commit")
+
+
+class KVCommitArgs(ctypes.Structure):
+    """Mirror of ``ddt_kv_commit_args`` (field order and types as in ddt.h)."""
+    _fields_ = [("k_tree", ctypes.c_void_p), ("v_tree", ctypes.c_void_p),
+                ("acc_len", ctypes.c_void_p), ("acc_nodes", ctypes.c_void_p),
+                ("ctx_len", ctypes.c_void_p), ("k_cache", ctypes.c_void_p),
+                ("v_cache", ctypes.c_void_p), ("page_table", ctypes.c_void_p),
+                ("page_size", ctypes.c_int), ("max_pages", ctypes.c_int),
+                ("num_pages", ctypes.c_int), ("t_max", ctypes.c_int64),
+                ("batch", ctypes.c_int), ("n_max", ctypes.c_int), ("hkv", ctypes.c_int),
+                ("d", ctypes.c_int), ("L", ctypes.c_int), ("dev_status", ctypes.c_void_p)]
 
 
 class DDTError(RuntimeError):
@@ -88,6 +101,8 @@ def load_library():
         lib.ddt_tree_walk.restype = i32
         lib.ddt_tree_walk.argtypes = [vp, i32, i32, i32, i32, i64, vp, vp, vp, vp, i32,
                                       vp, vp, vp, vp, vp, sz, vp, vp]
+        lib.ddt_kv_commit.restype = i32
+        lib.ddt_kv_commit.argtypes = [ctypes.POINTER(KVCommitArgs), vp]
         u64 = ctypes.c_uint64
         lib.ddt_tree_walk_sample.restype = i32
         lib.ddt_tree_walk_sample.argtypes = [vp, i32, i32, i32, i32, i64, vp, vp, vp, vp, i32,
@@ -353,3 +368,44 @@ def tree_walk_sample(logits: torch.Tensor, tok: torch.Tensor, parent: torch.Tens
                                       _stream(dev))
     _check(rc, "ddt_tree_walk_sample")
     return res
+
+
+def kv_commit(k_tree: torch.Tensor, v_tree: torch.Tensor, acc_len: torch.Tensor,
+              acc_nodes: torch.Tensor, ctx_len: torch.Tensor, k_cache: torch.Tensor,
+              v_cache: torch.Tensor, page_table: Optional[torch.Tensor] = None,
+              page_size: int = 64, dev_status: Optional[torch.Tensor] = None):
+    """``ddt_kv_commit``: append each sequence's root and accepted rows of the
+    tree K/V ([batch, n_max, hkv, d] bf16) to the cache (dense [batch, t_max,
+    hkv, d] or a page pool [pages, page_size, hkv, d] with ``page_table``) and
+    advance ``ctx_len`` (int32, in place) by acc_len + 1."""
+    lib = load_library()
+    dev = _need_cuda(k_tree, v_tree, acc_len, acc_nodes, ctx_len, k_cache, v_cache, page_table,
+                     dev_status)
+    for t in (k_tree, v_tree, k_cache, v_cache):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise DDTError("kv_commit: tree K/V and caches must be contiguous bfloat16")
+    for t in (acc_len, acc_nodes, ctx_len, page_table):
+        if t is not None and (t.dtype != torch.int32 or not t.is_contiguous()):
+            raise DDTError("kv_commit: acc_len / acc_nodes / ctx_len / page_table must be "
+                           "contiguous int32")
+    b, n_max, hkv, d = k_tree.shape
+
+    def addr(t):
+        return None if t is None else t.data_ptr()
+
+    a = KVCommitArgs()
+    a.k_tree, a.v_tree = addr(k_tree), addr(v_tree)
+    a.acc_len, a.acc_nodes, a.ctx_len = addr(acc_len), addr(acc_nodes), addr(ctx_len)
+    a.k_cache, a.v_cache = addr(k_cache), addr(v_cache)
+    if page_table is None:
+        a.page_table, a.page_size, a.max_pages, a.num_pages = None, 0, 0, 0
+        a.t_max = k_cache.shape[1]
+    else:
+        a.page_table, a.page_size = addr(page_table), page_size
+        a.max_pages, a.num_pages, a.t_max = page_table.shape[1], k_cache.shape[0], 0
+    a.batch, a.n_max, a.hkv, a.d = b, n_max, hkv, d
+    a.L = acc_nodes.shape[1]
+    a.dev_status = addr(dev_status)
+    with torch.cuda.device(dev):
+        rc = lib.ddt_kv_commit(ctypes.byref(a), _stream(dev))
+    _check(rc, "ddt_kv_commit")

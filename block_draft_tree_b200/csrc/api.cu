@@ -295,4 +295,26 @@ ddt_status ddt_tree_walk_sample(const void* logits, ddt_dtype dtype, int batch, 
                      stream, &smp);
 }
 
+ddt_status ddt_kv_commit(const ddt_kv_commit_args* a, cudaStream_t stream) {
+  if (!a) return DDT_ERR_INVALID_ARG;
+  if (a->batch < 0 || a->n_max < 1 || a->hkv < 1 || a->d < 1 || a->L < 0)
+    return DDT_ERR_INVALID_ARG;
+  if (a->L > DDT_TREE_L_MAX || ((int64_t)a->hkv * a->d) % 8 != 0 ||
+      (int64_t)a->hkv * a->d > (1 << 20))
+    return DDT_ERR_UNSUPPORTED;
+  if (a->batch == 0) return DDT_OK;
+  if (!a->k_tree || !a->v_tree || !a->acc_len || !a->ctx_len || !a->k_cache || !a->v_cache ||
+      (a->L > 0 && !a->acc_nodes))
+    return DDT_ERR_INVALID_ARG;
+  if (!aligned16(a->k_tree) || !aligned16(a->v_tree) || !aligned16(a->k_cache) ||
+      !aligned16(a->v_cache))
+    return DDT_ERR_INVALID_ARG;
+  if (a->page_table) {
+    if (a->page_size < 1 || a->max_pages < 1 || a->num_pages < 0) return DDT_ERR_INVALID_ARG;
+  } else if (a->t_max < 1) {
+    return DDT_ERR_INVALID_ARG;
+  }
+  return launch_kv_commit(a, stream);
+}
+
 }  // extern "C"

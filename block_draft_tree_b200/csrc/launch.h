@@ -68,6 +68,8 @@ ddt_status launch_tree_walk(const void* logits, ddt_dtype dt, int batch, int n_m
                             int32_t* dev_status, cudaStream_t stream,
                             const WalkSampling* sampling = nullptr);
 
+ddt_status launch_kv_commit(const ddt_kv_commit_args* a, cudaStream_t stream);
+
 struct AttnParams;
 size_t attn_workspace_size(const ddt_attn_args* a);
 ddt_status launch_attn(const ddt_attn_args* a, void* ws, size_t ws_bytes, cudaStream_t stream);

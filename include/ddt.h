@@ -14,7 +14,9 @@
  *                      "core innovation", ancestor-only attention mask);
  *   4. ddt_tree_walk   the greedy walk over the target's logits that accepts
  *                      matching children and returns the bonus token (step 4);
- *      ddt_tree_walk_sample  the same walk under temperature sampling.
+ *      ddt_tree_walk_sample  the same walk under temperature sampling;
+ *   5. ddt_kv_commit   appends the root's and the accepted rows' K/V to the
+ *                      committed context for the next round.
  *
  * Conventions shared by every entry point:
  *   - Every tensor pointer is a DEVICE pointer owned by the caller.  The
@@ -249,6 +251,50 @@ ddt_status ddt_tree_walk(const void* logits, ddt_dtype dtype, int batch, int n_m
                          const int32_t* depth, const int32_t* n_nodes, int L, int32_t* acc_len,
                          int32_t* acc_nodes, int32_t* acc_tok, int32_t* bonus, void* workspace,
                          size_t workspace_bytes, int32_t* dev_status, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * After stage 4: commit the accepted path's K/V to the context.
+ * DDTree page, 運作流程 (workflow): a round starts from the bonus token the
+ * target produced but has not run yet, runs it as the tree's root with the
+ * draft rows, and the walk accepts a path.  The root and the accepted rows
+ * are therefore forwarded; their K/V join the committed context at the
+ * positions they were scored at, and the new bonus token (not forwarded)
+ * stays out.  For sequence b with a = acc_len[b] and c = ctx_len[b]:
+ * context position c + i receives the tree K/V of row 0 (i = 0) or of row
+ * acc_nodes[b][i-1] (i = 1..a), for every kv head; then ctx_len[b] = c + a + 1.
+ *
+ *   k_tree, v_tree  bf16 [batch][n_max][hkv][d] (as for ddt_tree_attn)
+ *   acc_len [batch], acc_nodes [batch][L]: the walk's outputs
+ *   ctx_len [batch]  read, then advanced in place
+ *   k_cache, v_cache dense (page_table == NULL): bf16 [batch][t_max][hkv][d];
+ *           paged: bf16 [pages][page_size][hkv][d] through
+ *           page_table [batch][max_pages] (as for ddt_tree_attn); pages the
+ *           new positions fall in must already be in the table.
+ * A position outside the cache (dense: >= t_max; paged: beyond max_pages, a
+ * negative page id or one >= num_pages when num_pages > 0), an acc_len
+ * outside [0, L] or an accepted row outside [0, n_max) is not written and
+ * raises DDT_ERR_INVALID_ARG in dev_status; ctx_len still advances by
+ * acc_len + 1.  Limits: hkv * d a multiple of 8; all base pointers 16-byte
+ * aligned.  No workspace.
+ * ------------------------------------------------------------------------ */
+typedef struct ddt_kv_commit_args {
+  const void* k_tree;
+  const void* v_tree;
+  const int32_t* acc_len;
+  const int32_t* acc_nodes;
+  int32_t* ctx_len;
+  void* k_cache;
+  void* v_cache;
+  const int32_t* page_table; /* NULL: dense cache */
+  int page_size;
+  int max_pages;
+  int num_pages;             /* paged: pages in the pool; 0 = unknown */
+  int64_t t_max;             /* dense: tokens per sequence */
+  int batch, n_max, hkv, d, L;
+  int32_t* dev_status;       /* may be NULL */
+} ddt_kv_commit_args;
+
+ddt_status ddt_kv_commit(const ddt_kv_commit_args* a, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
  * Stage 4 under a sampling decoding rule (target temperature T > 0).

@@ -126,6 +126,27 @@ def test_walk_sample_rejects_bad_arguments(lib):
     assert call(V=10 ** 6, stride=10 ** 6) == 3  # workspace required
 
 
+def test_kv_commit_rejects_bad_arguments(lib):
+    d = 4096  # any 16-byte aligned non-null address: nothing is launched
+
+    def call(**kw):
+        a = api.KVCommitArgs()
+        a.k_tree = a.v_tree = a.acc_len = a.acc_nodes = a.ctx_len = a.k_cache = a.v_cache = d
+        a.page_table, a.page_size, a.max_pages, a.num_pages, a.t_max = None, 0, 0, 0, 64
+        a.batch, a.n_max, a.hkv, a.d, a.L, a.dev_status = 1, 9, 8, 128, 4, None
+        for k, v in kw.items():
+            setattr(a, k, v)
+        return lib.ddt_kv_commit(ctypes.byref(a), None)
+
+    assert lib.ddt_kv_commit(None, None) == 1
+    assert call(n_max=0) == 1 and call(hkv=0) == 1 and call(L=-1) == 1
+    assert call(L=65) == 2 and call(hkv=1, d=3) == 2    # L above the limit; hkv*d % 8 != 0
+    assert call(k_tree=None) == 1 and call(k_cache=4100) == 1  # null; misaligned
+    assert call(t_max=0) == 1                           # dense cache without capacity
+    assert call(page_table=d, page_size=0, max_pages=4) == 1
+    assert call(batch=0, k_tree=None) == 0              # nothing to do
+
+
 def test_binding_refuses_cpu_tensors(lib):
     import torch
     with pytest.raises(api.DDTError):
