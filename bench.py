@@ -53,6 +53,9 @@ def parse():
                     help="no timing: four rounds of one input set with an L2 flush before each, "
                          "for an ncu capture filtered by kernel name (-k)")
     ap.add_argument("--workload", default=None, help="workload for --profile (default: the bench's)")
+    ap.add_argument("--extensions", action="store_true",
+                    help="with --profile: also run the sampled walk and the KV commit after "
+                         "each round")
     return ap.parse_args()
 
 
@@ -555,11 +558,21 @@ def run_profile(args):
     xd["target"] = torch.randn((w.batch, w.n_max, w.V), dtype=torch.float32, device="cuda")
     rnd.bind(xd)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    from block_draft_tree_b200 import api
+    o = rnd.out
     for i in range(4):
         flush.fill_(i)
         rnd.launch()
+        if args.extensions:  # the calls beyond the round, on the round's own outputs
+            api.tree_walk_sample(xd["target"], o["tok"], o["parent"], o["depth"], o["n_nodes"],
+                                 w.L, 1.0, seed=12345, step=i)
+            cl = xd["ctx_len"].clone()
+            api.kv_commit(xd["k_tree"], xd["v_tree"], o["acc_len"], o["acc_nodes"], cl,
+                          xd["k_cache"].clone(), xd["v_cache"].clone(),
+                          page_table=xd.get("page_table"), page_size=w.page_size or 64)
     torch.cuda.synchronize()
-    print(json.dumps({"profile": w.name, "rounds": 4, "status": int(rnd.out["status"].item())}))
+    print(json.dumps({"profile": w.name, "rounds": 4, "status": int(rnd.out["status"].item()),
+                      "extensions": bool(args.extensions)}))
     return 0
 
 
