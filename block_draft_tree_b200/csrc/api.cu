@@ -10,15 +10,26 @@
 
 namespace ddt {
 
+// Opt a kernel in to `bytes` of dynamic shared memory when its static plus
+// dynamic shared memory exceeds the 48 KB a launch gets by default.
 cudaError_t ensure_smem_attr(const void* func, size_t bytes) {
-  if (bytes <= 48 * 1024) return cudaSuccess;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   static std::mutex mu;
-  static std::map<std::pair<const void*, int>, size_t> done;
+  static std::map<std::pair<const void*, int>, size_t> done;      // dynamic bytes opted in
+  static std::map<std::pair<const void*, int>, size_t> static_of;  // static bytes of the kernel
   std::lock_guard<std::mutex> lock(mu);
-  size_t& have = done[std::make_pair(func, dev)];
+  const auto key = std::make_pair(func, dev);
+  auto st = static_of.find(key);
+  if (st == static_of.end()) {
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, func);
+    if (e != cudaSuccess) return e;
+    st = static_of.emplace(key, fa.sharedSizeBytes).first;
+  }
+  if (st->second + bytes <= 48 * 1024) return cudaSuccess;
+  size_t& have = done[key];
   if (have >= bytes) return cudaSuccess;
   e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   if (e == cudaSuccess) have = bytes;

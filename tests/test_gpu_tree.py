@@ -110,3 +110,12 @@ def test_device_values_out_of_range_are_flagged():
                    budget=i32([5, 99]), dev_status=st)
     torch.cuda.synchronize()
     assert st.item() == 1
+
+
+@pytest.mark.parametrize("L,k,B", [(16, 8, 256), (16, 8, 200), (16, 4, 384), (32, 8, 160),
+                                   (8, 16, 256)])
+def test_shared_memory_between_static_and_opt_in(L, k, B):
+    """Shapes whose dynamic shared memory fits in 48 KB only without the
+    builder's static scratch: the launch must still opt in."""
+    ids, zk, lse = _random_inputs(L * 100 + k + B, 2, L, 400, k)
+    _run(ids, zk, lse, B, 1.0)
