@@ -53,6 +53,14 @@ def parse():
                     help="no timing: four rounds of one input set with an L2 flush before each, "
                          "for an ncu capture filtered by kernel name (-k)")
     ap.add_argument("--workload", default=None, help="workload for --profile (default: the bench's)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="budget sweep: round time and acceptance for each B in --budgets")
+    ap.add_argument("--budgets", default="16,32,64,128,256,512")
+    ap.add_argument("--sweep-batch", type=int, default=8)
+    ap.add_argument("--sweep-draws", type=int, default=40)
+    ap.add_argument("--sweep-invt", type=float, default=3.0,
+                    help="inverse temperature of the drafter's marginals in the sweep (the b64 "
+                         "logits at 1.0 give the top token < 0.2%%; 3.0 gives ~0.8)")
     ap.add_argument("--extensions", action="store_true",
                     help="with --profile: also run the sampled walk and the KV commit after "
                          "each round")
@@ -576,12 +584,102 @@ def run_profile(args):
     return 0
 
 
+def plant_targets(target, probs, depth, n_nodes, L, gen):
+    """Synthetic target logits for the budget sweep: every tree row of depth
+    d < L gets, on top of ``target``'s N(0,1) noise, a logit of 100 at a token
+    drawn from the drafter's marginal q_{d+1} (``probs`` [batch, L, V]), one
+    independent draw per row; so a greedy walk accepts a path with exactly the
+    probability the factorised draft gives it, and the expected accepted
+    length is the tree's surrogate (DDTree page, 理論基礎, Proposition 1).
+    Returns the planted tokens [batch, n_max] (-1 where nothing is planted)."""
+    import torch
+    b, n_max, _ = target.shape
+    draws = torch.multinomial(probs.reshape(b * L, -1), n_max, replacement=True,
+                              generator=gen).reshape(b, L, n_max)
+    rows = torch.arange(n_max, device=target.device)
+    live = (rows[None, :] < n_nodes[:, None]) & (depth < L)
+    pos = depth.clamp(0, L - 1).long()
+    tok = torch.gather(draws, 1, pos[:, None, :]).squeeze(1)
+    tok = torch.where(live, tok, torch.full_like(tok, -1))
+    bi, xi = torch.nonzero(live, as_tuple=True)
+    target[bi, xi, tok[bi, xi]] = 100.0
+    return tok
+
+
+def run_sweep(args):
+    """Budget sweep (DDTree page, 實驗結果與權衡: acceptance grows with the node
+    budget B while the verifier's cost grows too).  For each B: device time of
+    one round (CUDA graph, median of launches after an L2 flush), and the mean
+    accepted length over target resamplings planted from the drafter's own
+    marginals, next to the tree's surrogate (their expectation)."""
+    import torch
+    from block_draft_tree_b200 import synth
+    from block_draft_tree_b200.round import VerifyRound
+
+    w0 = synth.WORKLOADS[args.workload or WORKLOAD]
+    budgets = [int(x) for x in args.budgets.split(",")]
+    batch = args.sweep_batch
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(2024)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    rows_out = []
+    for B in budgets:
+        w = w0.scaled(batch=batch, B=B, inv_temperature=args.sweep_invt)
+        rnd = VerifyRound(batch=w.batch, L=w.L, V=w.V, k=w.k, B_max=w.B, hq=w.hq, hkv=w.hkv,
+                          d=w.d, max_ctx=w.ctx, draft_dtype=torch.bfloat16,
+                          target_dtype=torch.float32, inv_temperature=w.inv_temperature)
+        xh, _ = make_inputs(w, 0, 0)
+        xd = to_device(xh, w, torch)
+        xd["target"] = torch.randn((w.batch, w.n_max, w.V), dtype=torch.float32, device="cuda",
+                                   generator=gen)
+        rnd.bind(xd)
+        rnd.launch()
+        torch.cuda.synchronize()
+        o = rnd.out
+        probs = torch.softmax(xd["draft"].float() * w.inv_temperature, dim=-1)
+        acc, surr = [], []
+        for r in range(args.sweep_draws):
+            xd["target"].normal_(generator=gen)
+            plant_targets(xd["target"], probs, o["depth"], o["n_nodes"], w.L, gen)
+            rnd.launch()
+            acc.append(o["acc_len"].double().mean().item())
+            surr.append(o["surrogate"].mean().item())
+        g = rnd.capture()
+        times = []
+        for rep in range(23):
+            flush.zero_()
+            a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            g.replay()
+            e.record()
+            torch.cuda.synchronize()
+            if rep >= 3:
+                times.append(a.elapsed_time(e) * 1e3)
+        us = statistics.median(times)
+        mean_acc = statistics.mean(acc)
+        rows_out.append({"B": B, "round_us": round(us, 2), "mean_accepted": round(mean_acc, 3),
+                         "surrogate": round(statistics.mean(surr), 3),
+                         "accepted_se": round(statistics.pstdev(acc) / max(1, len(acc)) ** 0.5, 3),
+                         "tokens_per_round": round(mean_acc + 1, 3),
+                         "tokens_per_s": round(w.batch * (mean_acc + 1) / (us * 1e-6), 1)})
+        print("# sweep row", json.dumps(rows_out[-1]), file=sys.stderr, flush=True)
+        del g, rnd, xd, probs
+        torch.cuda.empty_cache()
+    print(json.dumps({"sweep": w0.name, "batch": batch, "draws": args.sweep_draws,
+                      "draft_inv_temperature": args.sweep_invt,
+                      "target": "argmax planted from the drafter's marginals per row",
+                      "rows": rows_out}), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
     if args.profile:
         return run_profile(args)
+    if args.sweep:
+        return run_sweep(args)
     return run_ours(args)
 
 
