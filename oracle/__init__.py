@@ -18,6 +18,9 @@ curated summary of the authors' announcement), section "運作流程"
   tree row against the context KV cache and the tree's own KV;
 * :func:`tree_walk`  -- step 4, the greedy walk that accepts matching
   children and returns the bonus token;
+* :func:`lm_head_argmax`, :func:`walk_row_tokens` -- step 4 from the target's
+  hidden states and LM-head weights: each row's logits as an fp64 matmul,
+  its argmax (lowest id on ties), and the walk over those row tokens;
 * :func:`kv_commit`  -- after step 4: the root and the accepted rows' K/V
   appended to the committed context, which grows by acc_len + 1;
 * :func:`tree_walk_sample` -- step 4 under a sampling decoding rule
@@ -110,6 +113,10 @@ def _load():
                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                                        ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int]
         lib.ddto_kv_commit.restype = ctypes.c_int
+        lib.ddto_walk_row_tokens.argtypes = [i32p, i32p, i32p, i32p, ctypes.c_int, ctypes.c_int,
+                                             ctypes.POINTER(ctypes.c_int32), i32p, i32p,
+                                             ctypes.POINTER(ctypes.c_int32)]
+        lib.ddto_walk_row_tokens.restype = ctypes.c_int
         for f in (lib.ddto_topk, lib.ddto_build_tree, lib.ddto_tree_attn, lib.ddto_tree_walk,
                   lib.ddto_sample_row, lib.ddto_tree_walk_sample):
             f.restype = ctypes.c_int
@@ -401,3 +408,52 @@ def kv_commit(k_tree, v_tree, acc_len, acc_nodes, ctx_len, k_cache, v_cache, pag
         ok[b] = rc == 0
         cl[b] = c.value
     return kc, vc, cl, ok
+
+
+def _bf16_to_f64(bits):
+    return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def lm_head_argmax(hidden, weight):
+    """The target's decision at each row: logits = H W^T with every product
+    and sum in fp64 (the products of bf16 values are exact), argmax with the
+    lowest token id on ties.
+
+    ``hidden`` bf16 bits [rows, K], ``weight`` bf16 bits [V, K].  Returns
+    (token [rows] int32, top [rows] f64, gap [rows] f64): gap = top logit
+    minus the largest logit of any other token (0 on a tie)."""
+    h = _bf16_to_f64(hidden)
+    wt = _bf16_to_f64(weight)
+    logits = h @ wt.T
+    tok = np.argmax(logits, axis=1).astype(np.int32)  # first occurrence: lowest id
+    top = logits[np.arange(len(tok)), tok]
+    rest = logits.copy()
+    rest[np.arange(len(tok)), tok] = -np.inf
+    gap = top - rest.max(axis=1) if logits.shape[1] > 1 else np.full(len(tok), np.inf)
+    return tok, top, gap
+
+
+def walk_row_tokens(row_tok, tok, parent, depth, n_nodes, L):
+    """Step 4 over given row tokens [batch, n_max]; outputs as :func:`tree_walk`."""
+    row_tok = np.ascontiguousarray(row_tok, np.int32)
+    bsz = row_tok.shape[0]
+    res = {"acc_len": np.empty(bsz, np.int32), "acc_nodes": np.empty((bsz, L), np.int32),
+           "acc_tok": np.empty((bsz, L), np.int32), "bonus": np.empty(bsz, np.int32)}
+    lib = _load()
+    for b in range(bsz):
+        al = ctypes.c_int32()
+        bo = ctypes.c_int32()
+        an = np.empty(max(L, 1), np.int32)
+        at = np.empty(max(L, 1), np.int32)
+        rc = lib.ddto_walk_row_tokens(np.ascontiguousarray(row_tok[b]),
+                                      np.ascontiguousarray(tok[b], np.int32),
+                                      np.ascontiguousarray(parent[b], np.int32),
+                                      np.ascontiguousarray(depth[b], np.int32), int(n_nodes[b]), L,
+                                      ctypes.byref(al), an, at, ctypes.byref(bo))
+        if rc != 0:
+            raise ValueError("ddto_walk_row_tokens failed (%d)" % rc)
+        res["acc_len"][b] = al.value
+        res["acc_nodes"][b] = an[:L]
+        res["acc_tok"][b] = at[:L]
+        res["bonus"][b] = bo.value
+    return res

@@ -806,3 +806,45 @@ int ddto_kv_commit(const uint16_t* k_tree, const uint16_t* v_tree, int n_max, in
   *ctx_len = c + acc_len + 1;
   return bad ? DDTO_ERR_ARG : DDTO_OK;
 }
+
+/* ------------------------------------------------------------------ */
+/* Walk over given row tokens (the target's argmax of each tree row)   */
+/* ------------------------------------------------------------------ */
+/*
+ * Step 4 when the target's decision at each row is already known (for
+ * instance from an LM head whose logits are never stored): row_tok[j] is
+ * the token the target emits after row j.  From the root: if the current
+ * row has a child carrying that token (and depth < L), accept it and
+ * continue; otherwise that token is the bonus.  Same outputs as
+ * ddto_tree_walk.
+ */
+int ddto_walk_row_tokens(const int32_t* row_tok, const int32_t* tok, const int32_t* parent,
+                         const int32_t* depth, int n_nodes, int L, int32_t* acc_len,
+                         int32_t* acc_nodes, int32_t* acc_tok, int32_t* bonus) {
+  if (!row_tok || n_nodes < 1 || L < 0) return DDTO_ERR_ARG;
+  for (int i = 0; i < L; ++i) {
+    acc_nodes[i] = -1;
+    acc_tok[i] = -1;
+  }
+  int x = 0, a = 0;
+  for (;;) {
+    const int t = row_tok[x];
+    int next = -1;
+    if (depth[x] < L)
+      for (int c = 0; c < n_nodes; ++c)
+        if (parent[c] == x && tok[c] == t) {
+          next = c;
+          break;
+        }
+    if (next < 0 || a >= L) {
+      *bonus = t;
+      break;
+    }
+    acc_nodes[a] = next;
+    acc_tok[a] = t;
+    ++a;
+    x = next;
+  }
+  *acc_len = a;
+  return DDTO_OK;
+}
