@@ -414,22 +414,35 @@ def _bf16_to_f64(bits):
     return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
-def lm_head_argmax(hidden, weight):
+def lm_head_argmax(hidden, weight, block=None):
     """The target's decision at each row: logits = H W^T with every product
     and sum in fp64 (the products of bf16 values are exact), argmax with the
     lowest token id on ties.
 
     ``hidden`` bf16 bits [rows, K], ``weight`` bf16 bits [V, K].  Returns
     (token [rows] int32, top [rows] f64, gap [rows] f64): gap = top logit
-    minus the largest logit of any other token (0 on a tie)."""
+    minus the largest logit of any other token (0 on a tie).  ``block``
+    bounds the vocabulary rows widened to fp64 at a time (memory only: every
+    logit is its own dot product, and the running top two keep the first
+    occurrence)."""
     h = _bf16_to_f64(hidden)
-    wt = _bf16_to_f64(weight)
-    logits = h @ wt.T
-    tok = np.argmax(logits, axis=1).astype(np.int32)  # first occurrence: lowest id
-    top = logits[np.arange(len(tok)), tok]
-    rest = logits.copy()
-    rest[np.arange(len(tok)), tok] = -np.inf
-    gap = top - rest.max(axis=1) if logits.shape[1] > 1 else np.full(len(tok), np.inf)
+    rows, V = h.shape[0], weight.shape[0]
+    block = V if block is None else block
+    top = np.full(rows, -np.inf)
+    second = np.full(rows, -np.inf)
+    tok = np.zeros(rows, np.int32)
+    for v0 in range(0, V, block):
+        logits = h @ _bf16_to_f64(weight[v0:v0 + block]).T
+        bt = np.argmax(logits, axis=1)  # first occurrence: lowest id within the block
+        bv = logits[np.arange(rows), bt]
+        rest = logits.copy()
+        rest[np.arange(rows), bt] = -np.inf
+        b2 = rest.max(axis=1) if logits.shape[1] > 1 else np.full(rows, -np.inf)
+        new = bv > top  # strictly larger: an earlier block keeps its equal maximum
+        second = np.where(new, np.maximum(top, b2), np.maximum(second, bv))
+        top = np.where(new, bv, top)
+        tok = np.where(new, bt + v0, tok).astype(np.int32)
+    gap = top - second
     return tok, top, gap
 
 

@@ -61,3 +61,18 @@ def test_walk_over_row_tokens_equals_the_greedy_walk():
         b = oracle.tree_walk(logits, tok, parent, depth, n, L)
         for key in ("acc_len", "acc_nodes", "acc_tok", "bonus"):
             np.testing.assert_array_equal(a[key], b[key])
+
+
+def test_vocabulary_blocks_change_nothing():
+    """Blocking the vocabulary (for memory) gives the same tokens, tops and
+    gaps, ties across block boundaries included."""
+    rng = np.random.default_rng(2)
+    h = _bits(rng.standard_normal((9, 40)))
+    w = _bits(rng.standard_normal((700, 40)))
+    w[650] = w[13]  # an exact tie across blocks: the lower id must win
+    h[4] = _bits(np.ones(40))
+    whole = oracle.lm_head_argmax(h, w)
+    for block in (1, 64, 97, 700):
+        part = oracle.lm_head_argmax(h, w, block=block)
+        for x, y in zip(whole, part):
+            np.testing.assert_array_equal(x, y)
