@@ -29,7 +29,8 @@ DDT_TREE_B_MAX = 1023
 EXPORTED = ("ddt_status_string", "ddt_mask_words", "ddt_topk_workspace_size", "ddt_topk",
             "ddt_build_tree", "ddt_tree_attn_workspace_size", "ddt_tree_attn",
             "ddt_tree_walk_workspace_size", "ddt_tree_walk", "ddt_tree_walk_sample",
-            "ddt_kv_commit")
+            "ddt_kv_commit", "ddt_lm_head_max_rows", "ddt_lm_head_walk_workspace_size",
+            "ddt_lm_head_walk")
 
 
 class KVCommitArgs(ctypes.Structure):
@@ -42,6 +43,17 @@ class KVCommitArgs(ctypes.Structure):
                 ("num_pages", ctypes.c_int), ("t_max", ctypes.c_int64),
                 ("batch", ctypes.c_int), ("n_max", ctypes.c_int), ("hkv", ctypes.c_int),
                 ("d", ctypes.c_int), ("L", ctypes.c_int), ("dev_status", ctypes.c_void_p)]
+
+
+class LmHeadWalkArgs(ctypes.Structure):
+    """Mirror of ``ddt_lm_head_walk_args`` (field order and types as in ddt.h)."""
+    _fields_ = [("hidden", ctypes.c_void_p), ("weight", ctypes.c_void_p), ("K", ctypes.c_int),
+                ("V", ctypes.c_int), ("tok", ctypes.c_void_p), ("parent", ctypes.c_void_p),
+                ("depth", ctypes.c_void_p), ("n_nodes", ctypes.c_void_p), ("batch", ctypes.c_int),
+                ("n_max", ctypes.c_int), ("L", ctypes.c_int), ("acc_len", ctypes.c_void_p),
+                ("acc_nodes", ctypes.c_void_p), ("acc_tok", ctypes.c_void_p),
+                ("bonus", ctypes.c_void_p), ("row_token", ctypes.c_void_p),
+                ("dev_status", ctypes.c_void_p)]
 
 
 class DDTError(RuntimeError):
@@ -101,6 +113,12 @@ def load_library():
         lib.ddt_tree_walk.restype = i32
         lib.ddt_tree_walk.argtypes = [vp, i32, i32, i32, i32, i64, vp, vp, vp, vp, i32,
                                       vp, vp, vp, vp, vp, sz, vp, vp]
+        lib.ddt_lm_head_max_rows.restype = i32
+        lib.ddt_lm_head_max_rows.argtypes = []
+        lib.ddt_lm_head_walk_workspace_size.restype = sz
+        lib.ddt_lm_head_walk_workspace_size.argtypes = [ctypes.POINTER(LmHeadWalkArgs)]
+        lib.ddt_lm_head_walk.restype = i32
+        lib.ddt_lm_head_walk.argtypes = [ctypes.POINTER(LmHeadWalkArgs), vp, sz, vp]
         lib.ddt_kv_commit.restype = i32
         lib.ddt_kv_commit.argtypes = [ctypes.POINTER(KVCommitArgs), vp]
         u64 = ctypes.c_uint64
@@ -409,3 +427,45 @@ def kv_commit(k_tree: torch.Tensor, v_tree: torch.Tensor, acc_len: torch.Tensor,
     with torch.cuda.device(dev):
         rc = lib.ddt_kv_commit(ctypes.byref(a), _stream(dev))
     _check(rc, "ddt_kv_commit")
+
+
+def lm_head_walk(hidden: torch.Tensor, weight: torch.Tensor, tok: torch.Tensor,
+                 parent: torch.Tensor, depth: torch.Tensor, n_nodes: torch.Tensor, L: int,
+                 want_row_token: bool = False, dev_status: Optional[torch.Tensor] = None):
+    """``ddt_lm_head_walk``: the greedy walk straight from the target's hidden
+    states ([batch, n_max, K] bf16) and LM head ([V, K] bf16).  Returns the
+    walk outputs of :func:`tree_walk` (plus ``row_token`` [batch, n_max] when
+    asked)."""
+    lib = load_library()
+    dev = _need_cuda(hidden, weight, tok, parent, depth, n_nodes, dev_status)
+    for t in (hidden, weight):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise DDTError("lm_head_walk: hidden and weight must be contiguous bfloat16")
+    for t in (tok, parent, depth, n_nodes):
+        if t.dtype != torch.int32 or not t.is_contiguous():
+            raise DDTError("lm_head_walk: tree tensors must be contiguous int32")
+    b, n_max, K = hidden.shape
+    V = weight.shape[0]
+    if weight.shape[1] != K:
+        raise DDTError("lm_head_walk: weight must be [V, K] with the hidden size K")
+    res = {"acc_len": torch.empty(b, dtype=torch.int32, device=dev),
+           "acc_nodes": torch.empty((b, L), dtype=torch.int32, device=dev),
+           "acc_tok": torch.empty((b, L), dtype=torch.int32, device=dev),
+           "bonus": torch.empty(b, dtype=torch.int32, device=dev)}
+    if want_row_token:
+        res["row_token"] = torch.empty((b, n_max), dtype=torch.int32, device=dev)
+    a = LmHeadWalkArgs()
+    a.hidden, a.weight, a.K, a.V = hidden.data_ptr(), weight.data_ptr(), K, V
+    a.tok, a.parent, a.depth, a.n_nodes = (tok.data_ptr(), parent.data_ptr(), depth.data_ptr(),
+                                           n_nodes.data_ptr())
+    a.batch, a.n_max, a.L = b, n_max, L
+    a.acc_len, a.acc_nodes = res["acc_len"].data_ptr(), res["acc_nodes"].data_ptr()
+    a.acc_tok, a.bonus = res["acc_tok"].data_ptr(), res["bonus"].data_ptr()
+    a.row_token = res["row_token"].data_ptr() if want_row_token else None
+    a.dev_status = None if dev_status is None else dev_status.data_ptr()
+    nb = int(lib.ddt_lm_head_walk_workspace_size(ctypes.byref(a)))
+    ws = workspaces.get(dev, "lm_head", nb)
+    with torch.cuda.device(dev):
+        rc = lib.ddt_lm_head_walk(ctypes.byref(a), _ptr(ws), nb, _stream(dev))
+    _check(rc, "ddt_lm_head_walk")
+    return res

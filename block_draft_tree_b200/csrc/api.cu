@@ -306,6 +306,29 @@ ddt_status ddt_tree_walk_sample(const void* logits, ddt_dtype dtype, int batch, 
                      stream, &smp);
 }
 
+int ddt_lm_head_max_rows(void) { return lm_head_max_rows(); }
+
+size_t ddt_lm_head_walk_workspace_size(const ddt_lm_head_walk_args* a) {
+  (void)a;
+  return DDT_WS_COUNTER_BYTES;
+}
+
+ddt_status ddt_lm_head_walk(const ddt_lm_head_walk_args* a, void* workspace,
+                            size_t workspace_bytes, cudaStream_t stream) {
+  if (!a) return DDT_ERR_INVALID_ARG;
+  if (a->batch < 0 || a->n_max < 1 || a->L < 0 || a->K < 1 || a->V < 1) return DDT_ERR_INVALID_ARG;
+  if (a->K % 8 != 0 || a->n_max > DDT_TREE_B_MAX + 1 || a->L > DDT_TREE_L_MAX ||
+      (int64_t)a->batch * a->n_max > lm_head_max_rows())
+    return DDT_ERR_UNSUPPORTED;
+  if (a->batch == 0) return DDT_OK;
+  if (!a->hidden || !a->weight || !a->tok || !a->parent || !a->depth || !a->n_nodes ||
+      !a->acc_len || !a->bonus || (a->L > 0 && (!a->acc_nodes || !a->acc_tok)))
+    return DDT_ERR_INVALID_ARG;
+  if (!aligned16(a->hidden) || !aligned16(a->weight)) return DDT_ERR_INVALID_ARG;
+  if (!ws_ok(workspace, workspace_bytes, DDT_WS_COUNTER_BYTES)) return DDT_ERR_WORKSPACE;
+  return launch_lm_head_walk(a, workspace, stream);
+}
+
 ddt_status ddt_kv_commit(const ddt_kv_commit_args* a, cudaStream_t stream) {
   if (!a) return DDT_ERR_INVALID_ARG;
   if (a->batch < 0 || a->n_max < 1 || a->hkv < 1 || a->d < 1 || a->L < 0)

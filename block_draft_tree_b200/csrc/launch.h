@@ -69,6 +69,8 @@ ddt_status launch_tree_walk(const void* logits, ddt_dtype dt, int batch, int n_m
                             const WalkSampling* sampling = nullptr);
 
 ddt_status launch_kv_commit(const ddt_kv_commit_args* a, cudaStream_t stream);
+ddt_status launch_lm_head_walk(const ddt_lm_head_walk_args* a, void* ws, cudaStream_t stream);
+int lm_head_max_rows();
 
 struct AttnParams;
 size_t attn_workspace_size(const ddt_attn_args* a);

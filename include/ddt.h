@@ -15,6 +15,8 @@
  *   4. ddt_tree_walk   the greedy walk over the target's logits that accepts
  *                      matching children and returns the bonus token (step 4);
  *      ddt_tree_walk_sample  the same walk under temperature sampling;
+ *      ddt_lm_head_walk      the greedy walk straight from the target's
+ *                            hidden states (LM head on the tensor cores);
  *   5. ddt_kv_commit   appends the root's and the accepted rows' K/V to the
  *                      committed context for the next round.
  *
@@ -251,6 +253,46 @@ ddt_status ddt_tree_walk(const void* logits, ddt_dtype dtype, int batch, int n_m
                          const int32_t* depth, const int32_t* n_nodes, int L, int32_t* acc_len,
                          int32_t* acc_nodes, int32_t* acc_tok, int32_t* bonus, void* workspace,
                          size_t workspace_bytes, int32_t* dev_status, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Stage 4 from the target's hidden states (greedy): LM head, argmax, walk.
+ * DDTree page, 運作流程 step 4: the target's greedy token after tree row j
+ * is the argmax of its LM-head logits h_j W^T.  This call computes those
+ * logits on the tensor cores tile by tile (bf16 inputs, fp32 accumulation),
+ * keeps only each row's argmax (smaller token id on equal logits), and walks
+ * the trees as ddt_tree_walk does; the [rows x V] logits are never stored.
+ *
+ *   hidden  bf16 [batch][n_max][K]: the target's final hidden state of every
+ *           tree row (after its final norm), row-major
+ *   weight  bf16 [V][K]: the LM head (the nn.Linear [out][in] layout)
+ *   tok, parent, depth, n_nodes, L: the compiled tree (as ddt_tree_walk)
+ * Outputs: acc_len, acc_nodes, acc_tok, bonus as ddt_tree_walk; row_token
+ * (optional) int32 [batch][n_max]: every row's argmax.
+ * Limits: K a multiple of 8; batch*n_max <= ddt_lm_head_max_rows(); base
+ * pointers 16-byte aligned.  Rows beyond a sequence's n_nodes are computed
+ * but not used by the walk.  The workspace is the counter region only.
+ * ------------------------------------------------------------------------ */
+typedef struct ddt_lm_head_walk_args {
+  const void* hidden;
+  const void* weight;
+  int K, V;
+  const int32_t* tok;
+  const int32_t* parent;
+  const int32_t* depth;
+  const int32_t* n_nodes;
+  int batch, n_max, L;
+  int32_t* acc_len;
+  int32_t* acc_nodes;
+  int32_t* acc_tok;
+  int32_t* bonus;
+  int32_t* row_token;        /* may be NULL */
+  int32_t* dev_status;       /* may be NULL */
+} ddt_lm_head_walk_args;
+
+int ddt_lm_head_max_rows(void);
+size_t ddt_lm_head_walk_workspace_size(const ddt_lm_head_walk_args* a);
+ddt_status ddt_lm_head_walk(const ddt_lm_head_walk_args* a, void* workspace,
+                            size_t workspace_bytes, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
  * After stage 4: commit the accepted path's K/V to the context.

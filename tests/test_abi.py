@@ -147,6 +147,30 @@ def test_kv_commit_rejects_bad_arguments(lib):
     assert call(batch=0, k_tree=None) == 0              # nothing to do
 
 
+def test_lm_head_walk_rejects_bad_arguments(lib):
+    d = 4096  # any 16-byte aligned non-null address: nothing is launched
+    assert lib.ddt_lm_head_max_rows() >= 30000
+
+    def call(ws=None, nb=0, **kw):
+        a = api.LmHeadWalkArgs()
+        a.hidden = a.weight = a.tok = a.parent = a.depth = a.n_nodes = d
+        a.acc_len = a.acc_nodes = a.acc_tok = a.bonus = d
+        a.K, a.V, a.batch, a.n_max, a.L = 4096, 151936, 1, 65, 16
+        a.row_token = a.dev_status = None
+        for k, v in kw.items():
+            setattr(a, k, v)
+        return lib.ddt_lm_head_walk(ctypes.byref(a), ws, nb, None)
+
+    assert lib.ddt_lm_head_walk(None, None, 0, None) == 1
+    assert call(K=0) == 1 and call(V=0) == 1 and call(n_max=0) == 1 and call(L=-1) == 1
+    assert call(K=100) == 2                          # K not a multiple of 8
+    assert call(batch=1000, n_max=513) == 2          # more rows than the counter region holds
+    assert call(L=65) == 2 and call(n_max=1025) == 2
+    assert call(hidden=None) == 1 and call(weight=4100) == 1
+    assert call() == 3                               # workspace required
+    assert call(batch=0, hidden=None) == 0
+
+
 def test_binding_refuses_cpu_tensors(lib):
     import torch
     with pytest.raises(api.DDTError):
