@@ -287,6 +287,9 @@ def run_reference(args):
     return 0
 
 
+LM_HIDDEN = 4096  # synthetic target hidden size for the LM-head call
+
+
 def measure_extensions(w, sets, graphs, hbm_peak, reps=30):
     """Per-launch device time of the library's calls beyond the round proper
     (the sampled walk), each launch after an L2 flush, on the round's own
@@ -346,6 +349,34 @@ def measure_extensions(w, sets, graphs, hbm_peak, reps=30):
     ext["kv_commit"] = {"us": round(us, 3), "alg_bytes": int(alg),
                         "gbs": round(alg / (us * 1e-6) / 1e9, 2), "launches": len(times),
                         "bound": "launch latency (a few KB per sequence)"}
+
+    # the greedy walk straight from the target's hidden states: LM head on the
+    # tensor cores + argmax + walk (synthetic hidden size 4096, random head)
+    K = LM_HIDDEN
+    g = torch.Generator(device="cuda")
+    g.manual_seed(77)
+    hid = (torch.randn(w.batch, w.n_max, K, device="cuda", generator=g) * 0.5).bfloat16()
+    head = (torch.randn(w.V, K, device="cuda", generator=g) / K ** 0.5).bfloat16()
+    o = graphs[0][1].out
+    times = []
+    for rep in range(reps + 3):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        api.lm_head_walk(hid, head, o["tok"], o["parent"], o["depth"], o["n_nodes"], w.L)
+        b.record()
+        torch.cuda.synchronize()
+        if rep >= 3:
+            times.append(a.elapsed_time(b) * 1e3)
+    us = statistics.median(times)
+    alg = w.V * K * 2 + w.batch * w.n_max * K * 2  # the head and the hidden rows, read once
+    flops = 2.0 * w.batch * w.n_max * w.V * K
+    gbs = alg / (us * 1e-6) / 1e9
+    ext["lm_head_walk"] = {"us": round(us, 3), "alg_bytes": int(alg), "gbs": round(gbs, 1),
+                           "frac_hbm": round(gbs / hbm_peak, 4),
+                           "tflops": round(flops / (us * 1e-6) / 1e12, 1), "hidden": K,
+                           "launches": len(times),
+                           "l2": "the %.2f GB head exceeds L2" % (w.V * K * 2 / 1e9)}
+    del hid, head
     return ext
 
 
@@ -568,6 +599,11 @@ def run_profile(args):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
     from block_draft_tree_b200 import api
     o = rnd.out
+    if args.extensions:
+        g = torch.Generator(device="cuda")
+        g.manual_seed(77)
+        hid = (torch.randn(w.batch, w.n_max, LM_HIDDEN, device="cuda", generator=g) * 0.5).bfloat16()
+        head = (torch.randn(w.V, LM_HIDDEN, device="cuda", generator=g) / LM_HIDDEN ** 0.5).bfloat16()
     for i in range(4):
         flush.fill_(i)
         rnd.launch()
@@ -578,6 +614,7 @@ def run_profile(args):
             api.kv_commit(xd["k_tree"], xd["v_tree"], o["acc_len"], o["acc_nodes"], cl,
                           xd["k_cache"].clone(), xd["v_cache"].clone(),
                           page_table=xd.get("page_table"), page_size=w.page_size or 64)
+            api.lm_head_walk(hid, head, o["tok"], o["parent"], o["depth"], o["n_nodes"], w.L)
     torch.cuda.synchronize()
     print(json.dumps({"profile": w.name, "rounds": 4, "status": int(rnd.out["status"].item()),
                       "extensions": bool(args.extensions)}))
