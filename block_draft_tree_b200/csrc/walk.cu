@@ -257,71 +257,36 @@ __device__ __forceinline__ float draw_weight(float t, int R) {
   return e >= -120 ? w : 0.f;
 }
 
-// Packed pairs of fp32 (lane 0 in the low word): every operation rounds
-// each lane exactly as its scalar form does.
-__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ void upk2(uint64_t v, float& lo, float& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-// b - a, rounded once (a*(-1) is exact).
-__device__ __forceinline__ uint64_t sub2(uint64_t b, uint64_t a) {
-  return fma2(a, pk2(-1.f, -1.f), b);
-}
-
 // The weights of a pair of arguments t (packed), as draw_weight.
 __device__ __forceinline__ uint64_t draw_weight2(uint64_t t2, int R) {
-  const uint64_t sh2 = add2(t2, pk2(kRoundShift, kRoundShift));
-  const uint64_t r2 = sub2(t2, add2(sh2, pk2(-kRoundShift, -kRoundShift)));
-  uint64_t p2 = fma2(pk2(0x1.ffcbfcp-17f, 0x1.ffcbfcp-17f), r2, pk2(0x1.430912p-13f, 0x1.430912p-13f));
-  p2 = fma2(p2, r2, pk2(0x1.5d87fep-10f, 0x1.5d87fep-10f));
-  p2 = fma2(p2, r2, pk2(0x1.3b2ab6p-7f, 0x1.3b2ab6p-7f));
-  p2 = fma2(p2, r2, pk2(0x1.c6b08ep-5f, 0x1.c6b08ep-5f));
-  p2 = fma2(p2, r2, pk2(0x1.ebfbep-3f, 0x1.ebfbep-3f));
-  p2 = fma2(p2, r2, pk2(0x1.62e43p-1f, 0x1.62e43p-1f));
-  p2 = fma2(p2, r2, pk2(1.f, 1.f));
+  const uint64_t sh2 = fadd2(t2, pack2(kRoundShift, kRoundShift));
+  const uint64_t r2 = fsub2(t2, fadd2(sh2, pack2(-kRoundShift, -kRoundShift)));
+  uint64_t p2 = ffma2(pack2(0x1.ffcbfcp-17f, 0x1.ffcbfcp-17f), r2, pack2(0x1.430912p-13f, 0x1.430912p-13f));
+  p2 = ffma2(p2, r2, pack2(0x1.5d87fep-10f, 0x1.5d87fep-10f));
+  p2 = ffma2(p2, r2, pack2(0x1.3b2ab6p-7f, 0x1.3b2ab6p-7f));
+  p2 = ffma2(p2, r2, pack2(0x1.c6b08ep-5f, 0x1.c6b08ep-5f));
+  p2 = ffma2(p2, r2, pack2(0x1.ebfbep-3f, 0x1.ebfbep-3f));
+  p2 = ffma2(p2, r2, pack2(0x1.62e43p-1f, 0x1.62e43p-1f));
+  p2 = ffma2(p2, r2, pack2(1.f, 1.f));
   float sa, sb, pa, pb;
-  upk2(sh2, sa, sb);
-  upk2(p2, pa, pb);
+  unpack2(sh2, sa, sb);
+  unpack2(p2, pa, pb);
   const int ea = __float_as_int(sa) - (kRoundShiftBits + R);
   const int eb = __float_as_int(sb) - (kRoundShiftBits + R);
   const float wa = ea >= -120 ? __int_as_float(__float_as_int(pa) + (ea << 23)) : 0.f;
   const float wb = eb >= -120 ? __int_as_float(__float_as_int(pb) + (eb << 23)) : 0.f;
-  return pk2(wa, wb);
+  return pack2(wa, wb);
 }
 
 // hi + lo += w lane by lane, with hi + w split exactly (Knuth's TwoSum).
 __device__ __forceinline__ void two_sum_add2(uint64_t& hi, uint64_t& lo, uint64_t w) {
-  const uint64_t s = add2(hi, w);
-  const uint64_t bp = sub2(s, hi);
-  const uint64_t err = add2(sub2(hi, sub2(s, bp)), sub2(w, bp));
+  const uint64_t s = fadd2(hi, w);
+  const uint64_t bp = fsub2(s, hi);
+  const uint64_t err = fadd2(fsub2(hi, fsub2(s, bp)), fsub2(w, bp));
   hi = s;
-  lo = add2(lo, err);
+  lo = fadd2(lo, err);
 }
 
-__device__ __forceinline__ float fmax3f(float a, float b, float c) {
-  float d;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
-}
 
 
 // s * 2^d for d <= 0, exact (0 below 2^-1000).
@@ -355,34 +320,34 @@ __device__ __forceinline__ void rs_chunk(const Chunk<BF16>& c, float a, int& R, 
 #pragma unroll
     for (int i = 0; i < 4; i += 2) {
       if (BF16) {
-        zm = fmax3f(zm, bf16_lo(w[i]), bf16_hi(w[i]));
-        zm = fmax3f(zm, bf16_lo(w[i + 1]), bf16_hi(w[i + 1]));
+        zm = fmax3(zm, bf16_lo(w[i]), bf16_hi(w[i]));
+        zm = fmax3(zm, bf16_lo(w[i + 1]), bf16_hi(w[i + 1]));
       } else {
-        zm = fmax3f(zm, __uint_as_float(w[i]), __uint_as_float(w[i + 1]));
+        zm = fmax3(zm, __uint_as_float(w[i]), __uint_as_float(w[i + 1]));
       }
     }
   }
   R = draw_ref(__fmul_rn(a, zm));  // fl32(a*z) is monotone in z
   s = 0.0;
   if (R == kNoRef) return;
-  const uint64_t a2 = pk2(a, a);
-  uint64_t hi = pk2(0.f, 0.f), lo = pk2(0.f, 0.f);
+  const uint64_t a2 = pack2(a, a);
+  uint64_t hi = pack2(0.f, 0.f), lo = pack2(0.f, 0.f);
 #pragma unroll
   for (int q = 0; q < Chunk<BF16>::VPT; ++q) {
     const uint32_t w[4] = {c.v[q].x, c.v[q].y, c.v[q].z, c.v[q].w};
     if (BF16) {
 #pragma unroll
       for (int i = 0; i < 4; ++i)
-        two_sum_add2(hi, lo, draw_weight2(mul2(a2, pk2(bf16_lo(w[i]), bf16_hi(w[i]))), R));
+        two_sum_add2(hi, lo, draw_weight2(fmul2(a2, pack2(bf16_lo(w[i]), bf16_hi(w[i]))), R));
     } else {
 #pragma unroll
       for (int i = 0; i < 4; i += 2)
-        two_sum_add2(hi, lo, draw_weight2(mul2(a2, pk2(__uint_as_float(w[i]), __uint_as_float(w[i + 1]))), R));
+        two_sum_add2(hi, lo, draw_weight2(fmul2(a2, pack2(__uint_as_float(w[i]), __uint_as_float(w[i + 1]))), R));
     }
   }
   float ha, hb, la, lb;
-  upk2(hi, ha, hb);
-  upk2(lo, la, lb);
+  unpack2(hi, ha, hb);
+  unpack2(lo, la, lb);
   s = ((double)ha + (double)la) + ((double)hb + (double)lb);
 }
 
