@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--sets", type=int, default=5, help="rotating input sets")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extensions", action="store_true",
+                    help="skip the measurements beyond the round (e.g. for a launch list)")
     ap.add_argument("--profile", action="store_true",
                     help="no timing: four rounds of one input set with an L2 flush before each, "
                          "for an ncu capture filtered by kernel name (-k)")
@@ -506,7 +508,8 @@ def run_ours(args):
             "peak_kind": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind if peak_kind == "measured"
             else "fallback"}
     acc = [r.out["acc_len"].float().mean().item() for _, r in graphs]
-    ext = measure_extensions(w, sets, graphs, hbm_peak) if rank == 0 else None
+    ext = (measure_extensions(w, sets, graphs, hbm_peak)
+           if rank == 0 and not args.no_extensions else None)
 
     # end to end: pinned host inputs -> H2D -> round -> D2H of the result, every step
     e2e = None
