@@ -136,3 +136,41 @@ def test_repeated_calls_reuse_the_workspace():
             first = got
         for k in first:
             np.testing.assert_array_equal(got[k], first[k])
+
+
+def test_b256_rows_sampled_at_full_size():
+    """2056 rows (8 trees of 257) against the 151936 x 4096 head: the row
+    tokens of 64 sampled rows against the oracle's, row by row, and every
+    walk checked as a walk over the kernel's own row tokens."""
+    batch, n_max, L, K, V = 8, 257, 16, 4096, 151936
+    rng = np.random.default_rng(256)
+    w = _bits((rng.standard_normal((V, K)) / np.sqrt(K)).astype(np.float32))
+    hf = rng.standard_normal((batch, n_max, K)).astype(np.float32) * 0.5
+    toks, pars, deps = [], [], []
+    wf = (w.astype(np.uint32) << 16).view(np.float32)
+    for b in range(batch):
+        tok, par, dep = _tree(rng, n_max, L, V, n_max)
+        for x in range(n_max):  # plant every inner row on its first child
+            kids = np.nonzero(par[:n_max] == x)[0]
+            if len(kids):
+                t = int(tok[kids[0]])
+                hf[b, x] = 8.0 * wf[t] / float(wf[t] @ wf[t])
+        toks.append(tok)
+        pars.append(par)
+        deps.append(dep)
+    h = _bits(hf)
+    tok, par, dep = np.stack(toks), np.stack(pars), np.stack(deps)
+    n = np.full(batch, n_max, np.int32)
+    got = api.lm_head_walk(bf16_tensor(h), bf16_tensor(w), i32(tok), i32(par), i32(dep), i32(n), L,
+                           want_row_token=True)
+    torch.cuda.synchronize()
+    g = {k: v.cpu().numpy() for k, v in got.items()}
+    rows = rng.choice(batch * n_max, 64, replace=False)
+    rt, _, gap = oracle.lm_head_argmax(h.reshape(-1, K)[rows], w, block=16384)
+    clear = gap >= LOGIT_MARGIN
+    np.testing.assert_array_equal(g["row_token"].reshape(-1)[rows][clear], rt[clear])
+    assert clear.sum() >= 48
+    ref = oracle.walk_row_tokens(g["row_token"], tok, par, dep, n, L)
+    for key in ("acc_len", "acc_nodes", "acc_tok", "bonus"):
+        np.testing.assert_array_equal(g[key], ref[key])
+    assert ref["acc_len"].min() >= 1  # the planted first children are accepted
