@@ -124,7 +124,7 @@ def load_library():
         u64 = ctypes.c_uint64
         lib.ddt_tree_walk_sample.restype = i32
         lib.ddt_tree_walk_sample.argtypes = [vp, i32, i32, i32, i32, i64, vp, vp, vp, vp, i32,
-                                             f32, u64, u64, vp, vp, vp, vp, vp, sz, vp, vp]
+                                             f32, u64, u64, vp, vp, vp, vp, vp, vp, sz, vp, vp]
         _lib = lib
         return lib
 
@@ -359,13 +359,18 @@ def tree_walk(logits: torch.Tensor, tok: torch.Tensor, parent: torch.Tensor,
 
 def tree_walk_sample(logits: torch.Tensor, tok: torch.Tensor, parent: torch.Tensor,
                      depth: torch.Tensor, n_nodes: torch.Tensor, L: int, inv_temperature: float,
-                     seed: int, step: int, dev_status: Optional[torch.Tensor] = None):
+                     seed: int, step: int, dev_status: Optional[torch.Tensor] = None,
+                     step_counter: Optional[torch.Tensor] = None):
     """Stage 4 under temperature sampling (``ddt_tree_walk_sample``): row j of
     sequence b draws its token from softmax(inv_temperature * z) with the
     Philox4x64-10 uniform of counter (j, b, 0, 0) and key (seed, step).
+    ``step_counter`` (optional int64 [1] on the device) is added to ``step``
+    and advanced by one per call, for replays of a captured graph.
     Arguments and outputs otherwise as :func:`tree_walk`."""
     lib = load_library()
-    dev = _need_cuda(logits, tok, parent, depth, n_nodes, dev_status)
+    dev = _need_cuda(logits, tok, parent, depth, n_nodes, dev_status, step_counter)
+    if step_counter is not None and (step_counter.dtype != torch.int64 or step_counter.numel() != 1):
+        raise DDTError("step_counter must be a one-element int64 tensor")
     if logits.dim() != 3 or logits.stride(2) != 1 or logits.stride(0) != logits.stride(1) * logits.shape[1]:
         raise DDTError("logits must be [batch, n_max, V] with contiguous rows and a uniform row stride")
     b, n_max, V = logits.shape
@@ -380,7 +385,7 @@ def tree_walk_sample(logits: torch.Tensor, tok: torch.Tensor, parent: torch.Tens
         rc = lib.ddt_tree_walk_sample(_ptr(logits), _dtype_code(logits), b, n_max, V,
                                       logits.stride(1), _ptr(tok), _ptr(parent), _ptr(depth),
                                       _ptr(n_nodes), L, float(inv_temperature), int(seed) & mask64,
-                                      int(step) & mask64, _ptr(res["acc_len"]),
+                                      int(step) & mask64, _ptr(step_counter), _ptr(res["acc_len"]),
                                       _ptr(res["acc_nodes"]), _ptr(res["acc_tok"]),
                                       _ptr(res["bonus"]), _ptr(ws), nb, _ptr(dev_status),
                                       _stream(dev))

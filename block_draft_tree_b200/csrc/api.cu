@@ -269,7 +269,7 @@ ddt_status walk_common(const void* logits, ddt_dtype dtype, int batch, int n_max
   if (batch < 0 || n_max < 1 || V < 1 || row_stride < V || L < 0) return DDT_ERR_INVALID_ARG;
   if (dtype != DDT_BF16 && dtype != DDT_F32) return DDT_ERR_UNSUPPORTED;
   if (n_max > DDT_TREE_B_MAX + 1 || batch > 65535 || L > DDT_TREE_L_MAX) return DDT_ERR_UNSUPPORTED;
-  if ((size_t)batch * n_max + batch > kMaxCounters) return DDT_ERR_UNSUPPORTED;
+  if ((size_t)batch * n_max + batch + 1 > kMaxCounters) return DDT_ERR_UNSUPPORTED;
   if (batch > 0 && (!logits || !tok || !parent || !depth || !n_nodes || !acc_len || !bonus ||
                     (L > 0 && (!acc_nodes || !acc_tok))))
     return DDT_ERR_INVALID_ARG;
@@ -295,12 +295,13 @@ ddt_status ddt_tree_walk_sample(const void* logits, ddt_dtype dtype, int batch, 
                                 int64_t row_stride, const int32_t* tok, const int32_t* parent,
                                 const int32_t* depth, const int32_t* n_nodes, int L,
                                 float inv_temperature, uint64_t seed, uint64_t step,
-                                int32_t* acc_len, int32_t* acc_nodes, int32_t* acc_tok,
-                                int32_t* bonus, void* workspace, size_t workspace_bytes,
-                                int32_t* dev_status, cudaStream_t stream) {
+                                uint64_t* step_counter, int32_t* acc_len, int32_t* acc_nodes,
+                                int32_t* acc_tok, int32_t* bonus, void* workspace,
+                                size_t workspace_bytes, int32_t* dev_status, cudaStream_t stream) {
   if (!(inv_temperature > 0.f) || !(inv_temperature * kLog2e < INFINITY))
     return DDT_ERR_INVALID_ARG;
-  const WalkSampling smp{inv_temperature, seed, step};
+  if (step_counter && ((uintptr_t)step_counter & 7u)) return DDT_ERR_INVALID_ARG;
+  const WalkSampling smp{inv_temperature, seed, step, step_counter};
   return walk_common(logits, dtype, batch, n_max, V, row_stride, tok, parent, depth, n_nodes, L,
                      acc_len, acc_nodes, acc_tok, bonus, workspace, workspace_bytes, dev_status,
                      stream, &smp);

@@ -60,6 +60,7 @@ size_t walk_workspace_size(int batch, int n_max, int V);
 struct WalkSampling {
   float inv_temperature;
   uint64_t seed, step;
+  uint64_t* step_counter;  // optional device word added to step; advanced by one per call
 };
 ddt_status launch_tree_walk(const void* logits, ddt_dtype dt, int batch, int n_max, int V,
                             int64_t row_stride, const int32_t* tok, const int32_t* parent,

@@ -23,7 +23,7 @@
 // the token of row j of sequence b is the inverse-CDF draw over token ids in
 // increasing order with u from Philox4x64-10 (Salmon, Moraes, Dror and Shaw,
 // "Parallel Random Numbers: As Easy as 1, 2, 3", SC'11) at counter
-// (j, b, 0, 0) under key (seed, step): u = (top 52 bits of word 0 + 1/2)
+// (j, b, 0, 0) under key (seed, step [+ *step_counter]): u = (top 52 bits of word 0 + 1/2)
 // * 2^-52.  The scan then keeps, per chunk, the pair (R, s): an integer
 // reference R (the largest exponent) and the fp64 sum s of the chunk's
 // weights against R, instead of an argmax key; the row's last CTA merges
@@ -54,9 +54,11 @@ struct WalkParams {
   int32_t* amax;         // [batch*n_max]
   unsigned* row_ticket;  // [batch*n_max]
   unsigned* seq_count;   // [batch]
+  unsigned* draw_count;  // sampling with a step counter: rows drawn so far
   int32_t* status;
   float a;               // sampling: fl32(log2(e) / T)
   uint64_t seed, step;   // sampling: Philox key
+  uint64_t* step_counter;  // sampling: optional device word added to step, advanced per call
 };
 
 __device__ __forceinline__ uint64_t block_max_key(uint64_t v, uint64_t* sm) {
@@ -209,7 +211,8 @@ __device__ __forceinline__ uint64_t philox4x64_10_w0(uint64_t x0, uint64_t x1, u
 
 // The uniform in (0, 1) that tree row j of sequence b draws.
 __device__ __forceinline__ double row_uniform(const WalkParams& p, int b, int j) {
-  const uint64_t w = philox4x64_10_w0((uint32_t)j, (uint32_t)b, 0, 0, p.seed, p.step);
+  const uint64_t step = p.step + (p.step_counter ? __ldcg((const unsigned long long*)p.step_counter) : 0ull);
+  const uint64_t w = philox4x64_10_w0((uint32_t)j, (uint32_t)b, 0, 0, p.seed, step);
   return ((double)(w >> 12) + 0.5) * 0x1.0p-52;
 }
 
@@ -378,6 +381,18 @@ __device__ __forceinline__ double warp_incl_scan(double v) {
   return v;
 }
 
+// One more row of the call has drawn (or has nothing to draw); the last of
+// all batch * n_max rows advances the step counter, once every draw of the
+// call has read it, and leaves the draw count zero.
+__device__ __forceinline__ void count_draw(const WalkParams& p) {
+  __threadfence();
+  if (atomicAdd(p.draw_count, 1u) == (unsigned)(p.batch * p.n_max - 1)) {
+    __threadfence();
+    *p.step_counter += 1ull;
+    *p.draw_count = 0u;
+  }
+}
+
 struct SampleSmem {
   double P, theta;
   int R, cstar;
@@ -511,7 +526,10 @@ __global__ void __launch_bounds__(kThreads) walk_kernel(WalkParams p) {
     if (chunk == 0 && j == 0 && tid == 0) raise_status(p.status, DDT_ERR_INVALID_ARG);
     n = min(max(n, 1), p.n_max);
   }
-  if (j >= n) return;
+  if (j >= n) {
+    if (SAMPLE && p.step_counter && chunk == 0 && tid == 0) count_draw(p);  // a row without a draw
+    return;
+  }
   const int64_t row = (int64_t)b * p.n_max + j;
   const char* rowp = (const char*)p.logits + row * p.row_stride * ES;
   const int c0 = chunk * kChunk;
@@ -556,6 +574,7 @@ __global__ void __launch_bounds__(kThreads) walk_kernel(WalkParams p) {
     if (tid == 0) {
       p.amax[row] = t;
       if (p.S > 1) p.row_ticket[row] = 0u;  // the counter region is left zero
+      if (p.step_counter) count_draw(p);
     }
   } else {
     float bv = -INFINITY;
@@ -640,6 +659,7 @@ ddt_status launch_tree_walk(const void* logits, ddt_dtype dt, int batch, int n_m
   p.a = sampling ? (float)((double)sampling->inv_temperature * 1.4426950408889634074) : 0.f;
   p.seed = sampling ? sampling->seed : 0;
   p.step = sampling ? sampling->step : 0;
+  p.step_counter = sampling ? sampling->step_counter : nullptr;
   p.logits = logits;
   p.batch = batch;
   p.n_max = n_max;
@@ -662,6 +682,7 @@ ddt_status launch_tree_walk(const void* logits, ddt_dtype dt, int batch, int n_m
   char* w = (char*)ws;
   p.row_ticket = (unsigned*)w;  // counter region: rows tickets, then batch counters
   p.seq_count = (unsigned*)w + rows;
+  p.draw_count = p.seq_count + batch;
   w += DDT_WS_COUNTER_BYTES;
   p.amax = (int32_t*)w;
   w += align256(sizeof(int32_t) * rows);

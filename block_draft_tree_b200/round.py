@@ -17,11 +17,28 @@ from . import api
 
 
 class VerifyRound:
+    """One verification round on fixed shapes.
+
+    ``decode`` is the target's decoding rule in stage 4: ``"greedy"``
+    (``ddt_tree_walk`` over the bound target logits), ``"sample"``
+    (``ddt_tree_walk_sample`` at ``sample_inv_temperature`` with a device step
+    counter, so that every replay of a captured round draws fresh uniforms) or
+    ``"lm_head"`` (``ddt_lm_head_walk`` from the bound hidden states and LM
+    head; no logits are stored).  With ``commit`` the round ends with
+    ``ddt_kv_commit``: the root's and the accepted rows' K/V join the bound
+    cache and ``ctx_len`` advances in place.
+    """
+
     def __init__(self, *, batch: int, L: int, V: int, k: int, B_max: int, hq: int, hkv: int,
                  d: int, max_ctx: int, draft_dtype: torch.dtype = torch.bfloat16,
                  target_dtype: torch.dtype = torch.float32, inv_temperature: float = 1.0,
                  paged: bool = False, page_size: int = 64, max_pages: int = 0,
-                 device: str = "cuda"):
+                 decode: str = "greedy", sample_inv_temperature: float = 1.0, seed: int = 0,
+                 commit: bool = False, device: str = "cuda"):
+        if decode not in ("greedy", "sample", "lm_head"):
+            raise ValueError("decode must be 'greedy', 'sample' or 'lm_head'")
+        self.decode, self.commit = decode, commit
+        self.sample_inv_t, self.seed = float(sample_inv_temperature), int(seed)
         self.lib = api.load_library()
         self.dev = torch.device(device)
         self.batch, self.L, self.V, self.k, self.B_max = batch, L, V, k, B_max
@@ -52,6 +69,11 @@ class VerifyRound:
         self.ws_attn = None
         self.attn_args = None
         self.inputs = None
+        # stage 4 under sampling: the step that replays advance on the device
+        self.step_counter = torch.zeros(1, dtype=torch.int64, device=dev)
+        self.lm_args = None
+        self.ws_lm = None
+        self.commit_args = None
 
     # ------------------------------------------------------------------
     def bind(self, inputs: dict):
@@ -69,10 +91,44 @@ class VerifyRound:
         if self.ws_attn is None or self.ws_attn.numel() < n:
             self.ws_attn = torch.zeros(max(n, 256), dtype=torch.uint8, device=self.dev)
         self.ws_attn_n = n
+        if self.decode == "lm_head":
+            hid, head = inputs["hidden"], inputs["head"]
+            la = api.LmHeadWalkArgs()
+            la.hidden, la.weight = hid.data_ptr(), head.data_ptr()
+            la.K, la.V = hid.shape[-1], head.shape[0]
+            la.tok, la.parent = o["tok"].data_ptr(), o["parent"].data_ptr()
+            la.depth, la.n_nodes = o["depth"].data_ptr(), o["n_nodes"].data_ptr()
+            la.batch, la.n_max, la.L = self.batch, self.n_max, self.L
+            la.acc_len, la.acc_nodes = o["acc_len"].data_ptr(), o["acc_nodes"].data_ptr()
+            la.acc_tok, la.bonus = o["acc_tok"].data_ptr(), o["bonus"].data_ptr()
+            la.row_token, la.dev_status = None, o["status"].data_ptr()
+            self.lm_args = la
+            nl = int(self.lib.ddt_lm_head_walk_workspace_size(ctypes.byref(la)))
+            if self.ws_lm is None or self.ws_lm.numel() < nl:
+                self.ws_lm = torch.zeros(max(nl, 256), dtype=torch.uint8, device=self.dev)
+            self.ws_lm_n = nl
+        if self.commit:
+            ca = api.KVCommitArgs()
+            ca.k_tree, ca.v_tree = inputs["k_tree"].data_ptr(), inputs["v_tree"].data_ptr()
+            ca.acc_len, ca.acc_nodes = o["acc_len"].data_ptr(), o["acc_nodes"].data_ptr()
+            ca.ctx_len = inputs["ctx_len"].data_ptr()
+            ca.k_cache, ca.v_cache = inputs["k_cache"].data_ptr(), inputs["v_cache"].data_ptr()
+            pt = inputs.get("page_table")
+            if pt is None:
+                ca.page_table, ca.page_size, ca.max_pages, ca.num_pages = None, 0, 0, 0
+                ca.t_max = inputs["k_cache"].shape[1]
+            else:
+                ca.page_table, ca.page_size = pt.data_ptr(), self.page_size
+                ca.max_pages, ca.num_pages = pt.shape[1], inputs["k_cache"].shape[0]
+                ca.t_max = 0
+            ca.batch, ca.n_max, ca.hkv, ca.d, ca.L = self.batch, self.n_max, self.hkv, self.d, self.L
+            ca.dev_status = o["status"].data_ptr()
+            self.commit_args = ca
 
     def launch(self, stream: Optional[torch.cuda.Stream] = None, marks=None):
-        """Enqueue the four stages on ``stream``.  ``marks(i)`` is called
-        before stage i and after the last (i = 0..4), e.g. to record events."""
+        """Enqueue the four stages (and the commit) on ``stream``.  ``marks(i)``
+        is called before stage i and after the last (i = 0..4, and 5 after
+        the commit), e.g. to record events."""
         lib, o, x = self.lib, self.out, self.inputs
         s = ctypes.c_void_p((stream or torch.cuda.current_stream(self.dev)).cuda_stream)
         P = api._ptr
@@ -96,14 +152,32 @@ class VerifyRound:
         api._check(rc, "ddt_tree_attn")
         if marks:
             marks(3)
-        rc = lib.ddt_tree_walk(P(x["target"]), self.target_code, self.batch, self.n_max, self.V,
-                               x["target"].stride(1), P(o["tok"]), P(o["parent"]), P(o["depth"]),
-                               P(o["n_nodes"]), self.L, P(o["acc_len"]), P(o["acc_nodes"]),
-                               P(o["acc_tok"]), P(o["bonus"]), P(self.ws_walk), self.ws_walk_n,
-                               P(o["status"]), s)
-        api._check(rc, "ddt_tree_walk")
+        if self.decode == "greedy":
+            rc = lib.ddt_tree_walk(P(x["target"]), self.target_code, self.batch, self.n_max,
+                                   self.V, x["target"].stride(1), P(o["tok"]), P(o["parent"]),
+                                   P(o["depth"]), P(o["n_nodes"]), self.L, P(o["acc_len"]),
+                                   P(o["acc_nodes"]), P(o["acc_tok"]), P(o["bonus"]),
+                                   P(self.ws_walk), self.ws_walk_n, P(o["status"]), s)
+            api._check(rc, "ddt_tree_walk")
+        elif self.decode == "sample":
+            rc = lib.ddt_tree_walk_sample(P(x["target"]), self.target_code, self.batch, self.n_max,
+                                          self.V, x["target"].stride(1), P(o["tok"]),
+                                          P(o["parent"]), P(o["depth"]), P(o["n_nodes"]), self.L,
+                                          self.sample_inv_t, self.seed, 0, P(self.step_counter),
+                                          P(o["acc_len"]), P(o["acc_nodes"]), P(o["acc_tok"]),
+                                          P(o["bonus"]), P(self.ws_walk), self.ws_walk_n,
+                                          P(o["status"]), s)
+            api._check(rc, "ddt_tree_walk_sample")
+        else:
+            rc = lib.ddt_lm_head_walk(ctypes.byref(self.lm_args), P(self.ws_lm), self.ws_lm_n, s)
+            api._check(rc, "ddt_lm_head_walk")
         if marks:
             marks(4)
+        if self.commit:
+            rc = lib.ddt_kv_commit(ctypes.byref(self.commit_args), s)
+            api._check(rc, "ddt_kv_commit")
+            if marks:
+                marks(5)
 
     def capture(self, marks=None) -> torch.cuda.CUDAGraph:
         """Capture one round (with its current bindings) into a CUDA graph."""

@@ -363,6 +363,11 @@ ddt_status ddt_kv_commit(const ddt_kv_commit_args* a, cudaStream_t stream);
  *   inv_temperature  1/T, finite and > 0 (larger -> closer to greedy)
  *   seed, step       the Philox key: a stream per request (seed) and a
  *                    fresh draw per round (step)
+ *   step_counter     optional device uint64 (8-byte aligned), or NULL.  When
+ *                    given, the key's second word is step + *step_counter,
+ *                    and the call adds one to *step_counter after its last
+ *                    draw: a captured CUDA graph then draws fresh uniforms on
+ *                    every replay.  Calls sharing a counter must not overlap.
  * Every other argument, the outputs and the workspace
  * (ddt_tree_walk_workspace_size) are those of ddt_tree_walk.
  * ------------------------------------------------------------------------ */
@@ -370,9 +375,9 @@ ddt_status ddt_tree_walk_sample(const void* logits, ddt_dtype dtype, int batch, 
                                 int64_t row_stride, const int32_t* tok, const int32_t* parent,
                                 const int32_t* depth, const int32_t* n_nodes, int L,
                                 float inv_temperature, uint64_t seed, uint64_t step,
-                                int32_t* acc_len, int32_t* acc_nodes, int32_t* acc_tok,
-                                int32_t* bonus, void* workspace, size_t workspace_bytes,
-                                int32_t* dev_status, cudaStream_t stream);
+                                uint64_t* step_counter, int32_t* acc_len, int32_t* acc_nodes,
+                                int32_t* acc_tok, int32_t* bonus, void* workspace,
+                                size_t workspace_bytes, int32_t* dev_status, cudaStream_t stream);
 
 #ifdef __cplusplus
 }

@@ -116,7 +116,7 @@ def test_walk_sample_rejects_bad_arguments(lib):
     d = ctypes.c_void_p(16)
 
     def call(b=1, n=9, V=64, stride=64, L=4, dt=1, it=1.0, logits=d):
-        return f(logits, dt, b, n, V, stride, d, d, d, d, L, it, 7, 0, d, d, d, d, None, 0,
+        return f(logits, dt, b, n, V, stride, d, d, d, d, L, it, 7, 0, None, d, d, d, d, None, 0,
                  None, None)
 
     assert call(it=0.0) == 1 and call(it=-0.5) == 1 and call(it=float("nan")) == 1
@@ -124,6 +124,8 @@ def test_walk_sample_rejects_bad_arguments(lib):
     assert call(stride=3) == 1 and call(dt=5) == 2 and call(n=2000) == 2 and call(L=65) == 2
     assert call(logits=None) == 1
     assert call(V=10 ** 6, stride=10 ** 6) == 3  # workspace required
+    assert f(d, 1, 1, 9, 64, 64, d, d, d, d, 4, 1.0, 7, 0, ctypes.c_void_p(20), d, d, d, d, None,
+             0, None, None) == 1                 # a step counter must be 8-byte aligned
 
 
 def test_kv_commit_rejects_bad_arguments(lib):
