@@ -63,6 +63,9 @@ def parse():
     ap.add_argument("--sweep-invt", type=float, default=3.0,
                     help="inverse temperature of the drafter's marginals in the sweep (the b64 "
                          "logits at 1.0 give the top token < 0.2%%; 3.0 gives ~0.8)")
+    ap.add_argument("--stage-sweep", action="store_true",
+                    help="each stage kernel timed alone on every workload, with its roofline")
+    ap.add_argument("--stage-workloads", default="b64,b256,paged128,long512")
     ap.add_argument("--extensions", action="store_true",
                     help="with --profile: also run the sampled walk and the KV commit after "
                          "each round")
@@ -712,6 +715,79 @@ def run_sweep(args):
     return 0
 
 
+def run_stage_sweep(args):
+    """Each stage kernel timed alone on every workload (CUDA events, an L2
+    flush before each launch, median of 15), with its algorithmic bytes and
+    flops and the fraction of its binding roofline (measured peaks)."""
+    import torch
+    from block_draft_tree_b200 import synth
+    from block_draft_tree_b200.round import VerifyRound
+
+    hbm_peak, tf_peak, peak_kind = peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    out = []
+    for name in args.stage_workloads.split(","):
+        w = synth.WORKLOADS[name]
+        ps = w.page_size or 64
+        xh, _ = make_inputs(w, 0, 0)
+        max_ctx = int(xh["ctx_len"].max())  # the page table covers the longest context drawn
+        rnd = VerifyRound(batch=w.batch, L=w.L, V=w.V, k=w.k, B_max=w.B, hq=w.hq, hkv=w.hkv,
+                          d=w.d, max_ctx=max_ctx, draft_dtype=torch.bfloat16,
+                          target_dtype=torch.float32, inv_temperature=w.inv_temperature,
+                          paged=w.page_size > 0, page_size=ps, max_pages=(max_ctx + ps - 1) // ps)
+        xd = to_device(xh, w, torch)
+        xd["target"] = torch.randn((w.batch, w.n_max, w.V), dtype=torch.float32, device="cuda")
+        rnd.bind(xd)
+        rnd.launch()
+        torch.cuda.synchronize()
+        times = {}
+        for i, stage in enumerate(("topk", "tree", "attn", "walk")):
+            ts = []
+            for rep in range(18):
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                rnd.launch_stage(i)
+                b.record()
+                torch.cuda.synchronize()
+                if rep >= 3:
+                    ts.append(a.elapsed_time(b) * 1e3)
+            times[stage] = statistics.median(ts)
+        assert int(rnd.out["status"].item()) == 0, "device status raised"
+        n_nodes = rnd.out["n_nodes"].cpu().numpy().astype(np.int64)
+        ctx = xh["ctx_len"].astype(np.int64)
+        rows = w.batch * w.L
+        topk_b = rows * w.V * 2 + rows * w.k * 12 + rows * 4
+        kv_b = int(ctx.sum()) * w.hkv * w.d * 2 * 2
+        attn_b = kv_b + 2 * int(n_nodes.sum()) * w.hq * w.d * 2 + 2 * int(n_nodes.sum()) * w.hkv * w.d * 2
+        attn_f = 4.0 * w.d * w.hq * float((n_nodes * ctx).sum())
+        walk_b = int(n_nodes.sum()) * w.V * 4
+        row = {"workload": name}
+        for stage, byts in (("topk", topk_b), ("walk", walk_b)):
+            us = times[stage]
+            gbs = byts / (us * 1e-6) / 1e9
+            row[stage] = {"us": round(us, 2), "alg_bytes": byts, "gbs": round(gbs, 1),
+                          "frac_hbm": round(gbs / hbm_peak, 3)}
+        us = times["attn"]
+        gbs = attn_b / (us * 1e-6) / 1e9
+        tfl = attn_f / (us * 1e-6) / 1e12
+        t_hbm, t_tc = attn_b / (hbm_peak * 1e9), attn_f / (tf_peak * 1e12)
+        row["attn"] = {"us": round(us, 2), "alg_bytes": attn_b, "alg_flops": attn_f,
+                       "gbs": round(gbs, 1), "tflops": round(tfl, 1),
+                       "bound": "tensor" if t_tc > t_hbm else "hbm",
+                       "frac_binding": round(max(t_hbm, t_tc) / (us * 1e-6), 3)}
+        row["tree"] = {"us": round(times["tree"], 2), "bound": "latency (one CTA per sequence)"}
+        out.append(row)
+        print("# " + json.dumps(row), file=sys.stderr, flush=True)
+        del rnd, xd
+        torch.cuda.empty_cache()
+    print(json.dumps({"stage_sweep": out, "peaks": {"hbm_gbs": hbm_peak, "bf16_tflops": tf_peak,
+                                                    "kind": peak_kind},
+                      "timing": "each kernel alone, L2 flushed before each launch, median of 15"}),
+          flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -720,6 +796,8 @@ def main():
         return run_profile(args)
     if args.sweep:
         return run_sweep(args)
+    if args.stage_sweep:
+        return run_stage_sweep(args)
     return run_ours(args)
 
 

@@ -129,55 +129,60 @@ class VerifyRound:
         """Enqueue the four stages (and the commit) on ``stream``.  ``marks(i)``
         is called before stage i and after the last (i = 0..4, and 5 after
         the commit), e.g. to record events."""
+        n = 5 if self.commit else 4
+        for i in range(n):
+            if marks:
+                marks(i)
+            self.launch_stage(i, stream)
+        if marks:
+            marks(n)
+
+    def launch_stage(self, i: int, stream: Optional[torch.cuda.Stream] = None):
+        """Enqueue stage i alone: 0 top-k, 1 tree, 2 attention, 3 walk, 4 commit."""
         lib, o, x = self.lib, self.out, self.inputs
         s = ctypes.c_void_p((stream or torch.cuda.current_stream(self.dev)).cuda_stream)
         P = api._ptr
-        if marks:
-            marks(0)
-        rc = lib.ddt_topk(P(x["draft"]), self.draft_code, self.batch, self.L, self.V,
-                          x["draft"].stride(1), self.k, self.inv_t, P(o["ids"]), P(o["zk"]), None,
-                          P(o["lse"]), P(self.ws_topk), self.ws_topk_n, s)
-        api._check(rc, "ddt_topk")
-        if marks:
-            marks(1)
-        rc = lib.ddt_build_tree(P(o["ids"]), P(o["zk"]), P(o["lse"]), self.batch, self.L, self.k,
-                                self.inv_t, P(x.get("k_per_seq")), P(x.get("budget")),
-                                self.B_max, P(x["root"]), P(x["ctx_len"]), P(o["tok"]),
-                                P(o["parent"]), P(o["depth"]), P(o["pos"]), P(o["mask"]),
-                                P(o["n_nodes"]), P(o["surrogate"]), P(o["status"]), s)
-        api._check(rc, "ddt_build_tree")
-        if marks:
-            marks(2)
-        rc = lib.ddt_tree_attn(ctypes.byref(self.attn_args), P(self.ws_attn), self.ws_attn_n, s)
-        api._check(rc, "ddt_tree_attn")
-        if marks:
-            marks(3)
-        if self.decode == "greedy":
-            rc = lib.ddt_tree_walk(P(x["target"]), self.target_code, self.batch, self.n_max,
-                                   self.V, x["target"].stride(1), P(o["tok"]), P(o["parent"]),
-                                   P(o["depth"]), P(o["n_nodes"]), self.L, P(o["acc_len"]),
-                                   P(o["acc_nodes"]), P(o["acc_tok"]), P(o["bonus"]),
-                                   P(self.ws_walk), self.ws_walk_n, P(o["status"]), s)
-            api._check(rc, "ddt_tree_walk")
-        elif self.decode == "sample":
-            rc = lib.ddt_tree_walk_sample(P(x["target"]), self.target_code, self.batch, self.n_max,
-                                          self.V, x["target"].stride(1), P(o["tok"]),
-                                          P(o["parent"]), P(o["depth"]), P(o["n_nodes"]), self.L,
-                                          self.sample_inv_t, self.seed, 0, P(self.step_counter),
-                                          P(o["acc_len"]), P(o["acc_nodes"]), P(o["acc_tok"]),
-                                          P(o["bonus"]), P(self.ws_walk), self.ws_walk_n,
-                                          P(o["status"]), s)
-            api._check(rc, "ddt_tree_walk_sample")
-        else:
-            rc = lib.ddt_lm_head_walk(ctypes.byref(self.lm_args), P(self.ws_lm), self.ws_lm_n, s)
-            api._check(rc, "ddt_lm_head_walk")
-        if marks:
-            marks(4)
-        if self.commit:
+        if i == 0:
+            rc = lib.ddt_topk(P(x["draft"]), self.draft_code, self.batch, self.L, self.V,
+                              x["draft"].stride(1), self.k, self.inv_t, P(o["ids"]), P(o["zk"]),
+                              None, P(o["lse"]), P(self.ws_topk), self.ws_topk_n, s)
+            api._check(rc, "ddt_topk")
+        elif i == 1:
+            rc = lib.ddt_build_tree(P(o["ids"]), P(o["zk"]), P(o["lse"]), self.batch, self.L,
+                                    self.k, self.inv_t, P(x.get("k_per_seq")), P(x.get("budget")),
+                                    self.B_max, P(x["root"]), P(x["ctx_len"]), P(o["tok"]),
+                                    P(o["parent"]), P(o["depth"]), P(o["pos"]), P(o["mask"]),
+                                    P(o["n_nodes"]), P(o["surrogate"]), P(o["status"]), s)
+            api._check(rc, "ddt_build_tree")
+        elif i == 2:
+            rc = lib.ddt_tree_attn(ctypes.byref(self.attn_args), P(self.ws_attn), self.ws_attn_n, s)
+            api._check(rc, "ddt_tree_attn")
+        elif i == 3:
+            if self.decode == "greedy":
+                rc = lib.ddt_tree_walk(P(x["target"]), self.target_code, self.batch, self.n_max,
+                                       self.V, x["target"].stride(1), P(o["tok"]), P(o["parent"]),
+                                       P(o["depth"]), P(o["n_nodes"]), self.L, P(o["acc_len"]),
+                                       P(o["acc_nodes"]), P(o["acc_tok"]), P(o["bonus"]),
+                                       P(self.ws_walk), self.ws_walk_n, P(o["status"]), s)
+                api._check(rc, "ddt_tree_walk")
+            elif self.decode == "sample":
+                rc = lib.ddt_tree_walk_sample(P(x["target"]), self.target_code, self.batch,
+                                              self.n_max, self.V, x["target"].stride(1),
+                                              P(o["tok"]), P(o["parent"]), P(o["depth"]),
+                                              P(o["n_nodes"]), self.L, self.sample_inv_t,
+                                              self.seed, 0, P(self.step_counter), P(o["acc_len"]),
+                                              P(o["acc_nodes"]), P(o["acc_tok"]), P(o["bonus"]),
+                                              P(self.ws_walk), self.ws_walk_n, P(o["status"]), s)
+                api._check(rc, "ddt_tree_walk_sample")
+            else:
+                rc = lib.ddt_lm_head_walk(ctypes.byref(self.lm_args), P(self.ws_lm), self.ws_lm_n,
+                                          s)
+                api._check(rc, "ddt_lm_head_walk")
+        elif i == 4 and self.commit:
             rc = lib.ddt_kv_commit(ctypes.byref(self.commit_args), s)
             api._check(rc, "ddt_kv_commit")
-            if marks:
-                marks(5)
+        else:
+            raise ValueError("no stage %d in this round" % i)
 
     def capture(self, marks=None) -> torch.cuda.CUDAGraph:
         """Capture one round (with its current bindings) into a CUDA graph."""
