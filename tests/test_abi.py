@@ -177,3 +177,9 @@ def test_binding_refuses_cpu_tensors(lib):
     import torch
     with pytest.raises(api.DDTError):
         api.topk(torch.zeros(1, 2, 64), 4)
+
+
+def test_round_driver_rejects_an_unknown_decoding_rule():
+    from block_draft_tree_b200.round import VerifyRound
+    with pytest.raises(ValueError):
+        VerifyRound(batch=1, L=4, V=64, k=4, B_max=8, hq=4, hkv=1, d=64, max_ctx=128, decode="beam")
