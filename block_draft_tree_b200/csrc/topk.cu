@@ -118,8 +118,11 @@ __device__ void write_row(const TopkParams& p, int row, const uint64_t* s_top, f
   if (threadIdx.x == 0) p.lse[row] = row_lse;
 }
 
-template <bool BF16>
-__global__ void __launch_bounds__(kThreads, 3) topk_kernel(TopkParams p) {
+// MIN_CTAS: CTAs per SM the registers are budgeted for.  Three keep every
+// value in registers; four (64 registers, a few spilled) hide more of the
+// per-chunk compute behind other CTAs' loads when the grid spans many waves.
+template <bool BF16, int MIN_CTAS>
+__global__ void __launch_bounds__(kThreads, MIN_CTAS) topk_kernel(TopkParams p) {
   constexpr int EPV = BF16 ? 8 : 4;           // elements per 16-byte vector
   constexpr int EPT = kChunk / kThreads;      // 32 elements per thread
   constexpr int VPT = EPT / EPV;
@@ -367,8 +370,15 @@ ddt_status launch_topk(const void* logits, ddt_dtype dt, int rows, int V, int64_
   p.lse = lse;
   if (rows == 0) return DDT_OK;
   dim3 grid(p.S, rows);
-  const cudaError_t e = dt == DDT_BF16 ? launch_pdl(topk_kernel<true>, grid, dim3(kThreads), 0, stream, 0, p)
-                                      : launch_pdl(topk_kernel<false>, grid, dim3(kThreads), 0, stream, 0, p);
+  // many waves of chunks: the higher-occupancy build; a few: the spill-free one
+  const bool many = (long)p.S * rows > 4L * 3 * device_sm_count();
+  cudaError_t e;
+  if (dt == DDT_BF16)
+    e = many ? launch_pdl(topk_kernel<true, 4>, grid, dim3(kThreads), 0, stream, 0, p)
+             : launch_pdl(topk_kernel<true, 3>, grid, dim3(kThreads), 0, stream, 0, p);
+  else
+    e = many ? launch_pdl(topk_kernel<false, 4>, grid, dim3(kThreads), 0, stream, 0, p)
+             : launch_pdl(topk_kernel<false, 3>, grid, dim3(kThreads), 0, stream, 0, p);
   return e == cudaSuccess ? DDT_OK : DDT_ERR_CUDA;
 }
 
