@@ -20,7 +20,12 @@
  *     with an ancestor-only attention mask ("核心創新", third bullet);
  *   - step 4: the tree walk follows the target's decoding rule, accepts a
  *     child whose token matches, and carries the first mismatch forward as
- *     the next round's bonus token.
+ *     the next round's bonus token: greedily (ddto_tree_walk), by sampling
+ *     at a temperature (ddto_tree_walk_sample, with the Philox4x64-10
+ *     generator and the draw's fixed fp32 weights), or over row tokens
+ *     already decided (ddto_walk_row_tokens, e.g. an LM head's argmax);
+ *   - after step 4: the root's and the accepted rows' K/V join the committed
+ *     context (ddto_kv_commit).
  *
  * Readings where the page is silent (each restated in the design notes):
  *   - candidates at depth i are the top-k tokens of q_i by (logit desc,
