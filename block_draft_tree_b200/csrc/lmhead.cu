@@ -22,7 +22,9 @@
 //   * the last CTA to finish (grid ticket) turns the keys into row tokens and
 //     walks every sequence's tree with one warp, then clears the keys.
 // Every mbarrier wait is bounded (about one second); a wait that gives up
-// raises DDT_ERR_TIMEOUT in the status word and the CTA stops issuing work.
+// raises DDT_ERR_TIMEOUT in the status word and the CTA stops issuing work,
+// lets its loads and MMAs in flight complete (again with bounded waits),
+// frees its TMEM and returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -47,6 +49,7 @@ constexpr uint32_t kTmemCols = 512;     // two 256-column fp32 accumulators
 constexpr int kATile = BM * BK * 2;     // 16 KB
 constexpr int kBTile = BN * BK * 2;     // 32 KB
 constexpr long long kWaitCycles = 2000000000LL;
+constexpr long long kDrainCycles = 200000000LL;  // per wait while draining after an abort
 
 struct Params {
   int M, K, V, m_tiles, total_tiles, kblocks;
@@ -63,6 +66,7 @@ struct Params {
 struct __align__(8) Bars {
   uint64_t full[kStages], empty[kStages];
   uint64_t acc_full[2], acc_empty[2];
+  uint64_t drain;  // after a wait gave up: completion of every MMA issued
   uint32_t tmem_base;
   int abort;
   int last;
@@ -151,6 +155,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->acc_full[i], 1);
       mbar_init(&bars->acc_empty[i], 4 * 32);
     }
+    mbar_init(&bars->drain, 1);
     bars->abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -192,6 +197,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(sB + s * kBTile, &tm_w, kb * BK, nt * p.bn, &bars->full[s]);
         }
       }
+      if (*(volatile int*)&bars->abort) {
+        // a wait gave up: let the loads still in flight land before the CTA
+        // (and its shared memory) goes away; the last kStages issued loads
+        // are the only ones that can be outstanding
+        int keep_going = 0;
+        for (int q = it > kStages ? it - kStages : 0; q < it; ++q)
+          mbar_wait_bounded(&bars->full[q % kStages], (uint32_t)(q / kStages) & 1u, &keep_going,
+                            kDrainCycles);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -217,6 +231,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(&bars->empty[s]);
         }
         if (ok) mma_commit(&bars->acc_full[buf]);
+      }
+      if (*(volatile int*)&bars->abort) {
+        // a wait gave up: every MMA issued completes before TMEM is freed
+        int keep_going = 0;
+        mma_commit(&bars->drain);
+        mbar_wait_bounded(&bars->drain, 0u, &keep_going, kDrainCycles);
       }
     }
   } else {
