@@ -5,6 +5,7 @@
  * "Diffusion Draft Tree"; section 運作流程 "workflow", steps 1-4):
  *   1. ddt_topk        per-position softmax normaliser and top-k candidates of
  *                      the drafter's marginals q_i (step 1);
+ *      ddt_topk_noalloc  the same without a caller workspace;
  *   2. ddt_build_tree  the B most probable prefixes of the factorised draft
  *                      (step 2; section 理論基礎 "theory", Propositions 1-2),
  *                      compiled to token / parent / depth / position /
