@@ -93,10 +93,6 @@ def _load():
         lib.ddto_sample_row.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64,
                                         ctypes.c_int, ctypes.c_double, ctypes.c_double,
                                         ctypes.POINTER(ctypes.c_double)]
-        lib.ddto_sampler_exp2_poly.argtypes = [ctypes.c_float]
-        lib.ddto_sampler_exp2_poly.restype = ctypes.c_float
-        lib.ddto_sampler_scale.argtypes = [ctypes.c_double]
-        lib.ddto_sampler_scale.restype = ctypes.c_float
         lib.ddto_sampler_row_weights.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
                                                  ctypes.c_double, f64p]
         lib.ddto_sampler_row_weights.restype = ctypes.c_int
@@ -302,35 +298,31 @@ def row_uniform(seed: int, step: int, b: int, j: int) -> float:
     return float(_load().ddto_row_uniform(int(seed), int(step), int(b), int(j)))
 
 
-def sampler_exp2_poly(r: float) -> float:
-    """The draw's fp32 polynomial for 2^r on [-1/2, 1/2]."""
-    return float(_load().ddto_sampler_exp2_poly(float(r)))
-
-
-def sampler_scale(inv_temperature: float) -> float:
-    """a = fl32(fl32(inv_temperature) * log2(e)), the exponent scale of the draw."""
-    return float(_load().ddto_sampler_scale(float(inv_temperature)))
+def _f32(x: float) -> float:
+    """The fp32 value of a temperature argument (the C ABI takes a float)."""
+    return float(np.float32(x))
 
 
 def sampler_row_weights(row: np.ndarray, inv_temperature: float) -> np.ndarray:
-    """The draw's weights w_v = P(r_v) * 2^(k_v - K) of one row (fp64)."""
+    """The draw's weights of one row: w_v = exp(invT * z_v - max_u invT * z_u)
+    in fp64 (0 for -inf logits), invT being the fp32 value of the argument."""
     row = np.ascontiguousarray(row)
     p, is_bf16 = _raw(row)
     w = np.empty(row.shape[-1], np.float64)
-    rc = _load().ddto_sampler_row_weights(p, is_bf16, row.shape[-1], float(inv_temperature), w)
+    rc = _load().ddto_sampler_row_weights(p, is_bf16, row.shape[-1], _f32(inv_temperature), w)
     if rc != 0:
         raise ValueError("ddto_sampler_row_weights failed (%d)" % rc)
     return w
 
 
 def sample_row(row: np.ndarray, inv_temperature: float, u: float):
-    """One inverse-CDF draw over the weights of :func:`sampler_row_weights`
-    (softmax(inv_temperature * row) in fp32).  Returns (token, margin),
-    margin = distance of u*S from the chosen interval's nearer end over S."""
+    """One inverse-CDF draw from softmax(inv_temperature * row) (fp64 weights
+    of :func:`sampler_row_weights`).  Returns (token, margin), margin =
+    distance of u*S from the chosen interval's nearer end over S."""
     row = np.ascontiguousarray(row)
     p, is_bf16 = _raw(row)
     mg = ctypes.c_double()
-    t = _load().ddto_sample_row(p, is_bf16, 0, row.shape[-1], float(inv_temperature), float(u),
+    t = _load().ddto_sample_row(p, is_bf16, 0, row.shape[-1], _f32(inv_temperature), float(u),
                                 ctypes.byref(mg))
     return int(t), float(mg.value)
 
@@ -355,7 +347,7 @@ def tree_walk_sample(logits, tok, parent, depth, n_nodes, L, inv_temperature, se
         rc = lib.ddto_tree_walk_sample(p, is_bf16, V, V, np.ascontiguousarray(tok[b], np.int32),
                                        np.ascontiguousarray(parent[b], np.int32),
                                        np.ascontiguousarray(depth[b], np.int32), int(n_nodes[b]),
-                                       L, float(inv_temperature), int(seed), int(step), b,
+                                       L, _f32(inv_temperature), int(seed), int(step), b,
                                        ctypes.byref(al), an, at, ctypes.byref(bo),
                                        ctypes.byref(mm))
         if rc != 0:

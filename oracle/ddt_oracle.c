@@ -21,8 +21,8 @@
  *   - step 4: the tree walk follows the target's decoding rule, accepts a
  *     child whose token matches, and carries the first mismatch forward as
  *     the next round's bonus token: greedily (ddto_tree_walk), by sampling
- *     at a temperature (ddto_tree_walk_sample, with the Philox4x64-10
- *     generator and the draw's fixed fp32 weights), or over row tokens
+ *     at a temperature (ddto_tree_walk_sample: inversion of softmax(z/T)
+ *     in fp64 with a Philox4x64-10 uniform), or over row tokens
  *     already decided (ddto_walk_row_tokens, e.g. an LM head's argmax);
  *   - after step 4: the root's and the accepted rows' K/V join the committed
  *     context (ddto_kv_commit).
@@ -598,67 +598,25 @@ double ddto_row_uniform(uint64_t seed, uint64_t step, int b, int j) {
 }
 
 /*
- * The draw's weights.  The token is an integer decided by floating point,
- * so both sides take the decision in the kernel's precision: each weight
- * is an fp32 evaluation of 2^(a*z), made exact in fp64 by construction,
- * and only the cumulative sums are fp64.  Per token v:
- *   a   = fl32(invT * log2(e))           (invT first rounded to fp32)
- *   t_v = fl32(a * z_v)
- *   k_v = t_v rounded to the nearest integer (ties to even), r_v = t_v - k_v
- *   P_v = Horner evaluation in fp32, with fused multiply-adds, of the
- *         degree-7 Taylor polynomial of 2^r (coefficients (ln 2)^i / i!
- *         rounded to fp32), at r_v; P_v is within ~1e-7 of 2^(r_v)
- *   w_v = P_v * 2^(k_v - K) exactly, K = k of the largest t; 0 when
- *         k_v - K < -120 (so that every weight is a normal fp32 number)
- *         or z_v = -inf.
- * w_v / sum(w) differs from softmax(invT * z) by ~|t| * 6e-8 relative: the
- * rounding of t, as in any fp32 softmax.
+ * The draw's weights: the target's distribution softmax(invT * z) before
+ * normalisation, in fp64.  With m = max_v invT * z_v over the finite
+ * logits, w_v = exp(invT * z_v - m); a -inf logit weighs 0.  Returns
+ * S = sum_v w_v summed in index order, or 0 when no logit is finite.
  */
-static const float ddto_p2_coef[8] = {0x1.0p+0f,       0x1.62e43p-1f,  0x1.ebfbep-3f,
-                                      0x1.c6b08ep-5f,  0x1.3b2ab6p-7f, 0x1.5d87fep-10f,
-                                      0x1.430912p-13f, 0x1.ffcbfcp-17f};
-
-float ddto_sampler_exp2_poly(float r) {
-  float p = ddto_p2_coef[7];
-  for (int i = 6; i >= 0; --i) p = fmaf(p, r, ddto_p2_coef[i]);
-  return p;
-}
-
-float ddto_sampler_scale(double invT) {
-  return (float)((double)(float)invT * 1.4426950408889634074);
-}
-
-/* t -> (k, P_v) as above; returns 0 when t is -inf or NaN. */
-static int sampler_split(float t, int* k, float* P) {
-  if (!(t >= -4.0e6f)) return 0;
-  const float kf = nearbyintf(t); /* default rounding: to nearest, ties to even */
-  *k = (int)kf;
-  *P = ddto_sampler_exp2_poly(t - kf);
-  return 1;
-}
-
-/* The weights of one row (w[V]); returns their fp64 sum in index order. */
 static double sampler_weights(const void* logits, int is_bf16, int64_t base, int V, double invT,
                               double* w) {
-  const float a = ddto_sampler_scale(invT);
-  float tmax = -INFINITY;
+  double m = -INFINITY;
   for (int v = 0; v < V; ++v) {
-    const float t = a * (float)load_val(logits, is_bf16, base + v);
-    if (t > tmax) tmax = t;
+    const double y = invT * load_val(logits, is_bf16, base + v);
+    if (y > m) m = y;
   }
-  double S = 0.0;
-  int K = 0;
-  float Pm;
-  if (!sampler_split(tmax, &K, &Pm)) {
+  if (m == -INFINITY) {
     for (int v = 0; v < V; ++v) w[v] = 0.0;
     return 0.0;
   }
+  double S = 0.0;
   for (int v = 0; v < V; ++v) {
-    const float t = a * (float)load_val(logits, is_bf16, base + v);
-    int k;
-    float P;
-    w[v] = 0.0;
-    if (sampler_split(t, &k, &P) && k - K >= -120) w[v] = ldexp((double)P, k - K);
+    w[v] = exp(invT * load_val(logits, is_bf16, base + v) - m);
     S += w[v];
   }
   return S;

@@ -1,20 +1,18 @@
 """Parity of ddt_tree_walk_sample (CUDA, through the C ABI) with the oracle's
 sampled walk.
 
-Each visited row draws its token by inversion with the Philox4x64-10
-uniform of its (sequence, row).  The weights follow one fixed fp32
-arithmetic on both sides and are exact fp64 numbers, so they agree bit for
-bit; only their fp64 cumulative sums differ, by summation order.  A draw can
-therefore only differ where u*S lies within rounding of an interval end.
-The rule: when the oracle's smallest draw margin along a walk is at least
-SAMPLE_MARGIN (relative to S), the walk is bit-exact; otherwise every
-decision along the CUDA walk whose margin clears SAMPLE_MARGIN must equal
-the oracle's draw and the walk must be a valid walk of the tree.
+The oracle draws by inversion of softmax(z / T) with fp64 weights
+exp(invT*z - max) and the Philox4x64-10 uniform of the (sequence, row).  The
+kernel evaluates each weight in fp32, so its cumulative sums differ from the
+oracle's by a bounded amount, and a draw whose u*S falls within that bound of
+an interval end may land on the neighbouring token.  The tests derive the
+bound from the kernel's stated arithmetic and apply it draw by draw
+(:func:`allowed_tokens`): the kernel's token must lie in the set of tokens
+that some cumulative sums within the bound would select.  Where that set has
+one element (the large majority of draws) the draw is bit-exact with the
+oracle; the rest are counted and reported.
 
-Error budget behind SAMPLE_MARGIN: the kernel's per-thread double-float
-sums of 32 weights are within 2^-38 (~4e-12) of exact, and a sum of
-n <= 151936 non-negative fp64 terms in any order is within n * 2^-53
-(~2e-11) of the exact sum, relative to S; 1e-10 stays clear of both.
+The error model behind the bound is stated in ``helpers.allowed_tokens``.
 """
 import numpy as np
 import pytest
@@ -24,12 +22,10 @@ from scipy import special, stats
 import oracle
 from block_draft_tree_b200 import api, synth
 
-from helpers import i32, logits_tensor, oracle_tree_inputs
+from helpers import (DrawCount, allowed_tokens, check_sampled_walk, i32, logits_tensor,
+                     oracle_tree_inputs)
 
 pytestmark = pytest.mark.gpu
-
-SAMPLE_MARGIN = 1e-10
-
 
 def _tree(w):
     ids, zk, lse = oracle_tree_inputs(w, synth.draft_logits(w))
@@ -61,13 +57,8 @@ def _sharpen(logits, tree, seed, boost):
     return out
 
 
-def _row_draw(logits, b, x, invT, seed, step):
-    return oracle.sample_row(logits[b, x], invT, oracle.row_uniform(seed, step, b, x))
-
-
-def _compare(logits, tree, L, invT, seed, step, tensor=None):
-    ref = oracle.tree_walk_sample(logits, tree["tok"], tree["parent"], tree["depth"],
-                                  tree["n_nodes"], L, invT, seed, step)
+def _compare(logits, tree, L, invT, seed, step, tensor=None, count=None):
+    """Run the kernel and check its walk with :func:`helpers.check_sampled_walk`."""
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     t = logits_tensor(logits) if tensor is None else tensor
     got = api.tree_walk_sample(t, i32(tree["tok"]), i32(tree["parent"]), i32(tree["depth"]),
@@ -75,29 +66,9 @@ def _compare(logits, tree, L, invT, seed, step, tensor=None):
     torch.cuda.synchronize()
     assert st.item() == 0
     got = {k: v.cpu().numpy() for k, v in got.items()}
-    n_ambiguous = 0
-    for b in range(logits.shape[0]):
-        if ref["min_margin"][b] >= SAMPLE_MARGIN:
-            for key in ("acc_len", "acc_nodes", "acc_tok", "bonus"):
-                np.testing.assert_array_equal(got[key][b], ref[key][b], err_msg="%s[%d]" % (key, b))
-            continue
-        n_ambiguous += 1
-        # validity of the CUDA walk, decision by decision
-        a = int(got["acc_len"][b])
-        n = int(tree["n_nodes"][b])
-        x = 0
-        for i in range(a + 1):
-            t = int(got["acc_tok"][b][i]) if i < a else int(got["bonus"][b])
-            t_ref, mg = _row_draw(logits, b, x, invT, seed, step)
-            if mg >= SAMPLE_MARGIN:
-                assert t == t_ref, (b, x)
-            kids = [c for c in range(n) if tree["parent"][b][c] == x and tree["tok"][b][c] == t]
-            if i < a:
-                assert kids and int(got["acc_nodes"][b][i]) == kids[0]
-                x = kids[0]
-            else:
-                assert not kids or tree["depth"][b][x] >= L or a >= L
-    return ref, got, n_ambiguous
+    count = DrawCount() if count is None else count
+    ref = check_sampled_walk(logits, tree, L, invT, seed, step, got, count)
+    return ref, got, count
 
 
 @pytest.mark.parametrize("name,invT", [("tiny", 1.0), ("tiny", 1 / 0.7), ("b64", 1.0),
@@ -109,8 +80,10 @@ def test_workload_sampled_walks(name, invT):
     logits = synth.target_logits(w, tree["tok"], tree["parent"], tree["depth"], tree["n_nodes"])
     boost = float(np.log(w.V)) + 2.0  # the boosted child holds most of the mass at T = 1
     logits = _sharpen(logits, tree, w.index, boost)
-    ref, got, amb = _compare(logits, tree, w.L, invT, seed=1000 + w.index, step=3)
-    assert amb == 0  # no draw falls within 1e-10 of an interval end on these inputs
+    ref, got, count = _compare(logits, tree, w.L, invT, seed=1000 + w.index, step=3)
+    print("%s invT=%.4g: %d draws, %d within the error bound of an interval end"
+          % (name, invT, count.draws, count.ambiguous))
+    assert count.ambiguous <= max(2, 0.25 * count.draws)
     if w.batch * w.L >= 64:
         assert ref["acc_len"].sum() > 0  # the walks do descend
 
@@ -197,10 +170,15 @@ def test_gpu_draws_follow_softmax():
     got = api.tree_walk_sample(logits_tensor(logits), i32(tok), i32(par), i32(dep), i32(n), 2,
                                1 / T, 77, 0)
     draws = got["bonus"].cpu().numpy()
-    ref = [oracle.sample_row(z, 1 / T, oracle.row_uniform(77, 0, b, 0)) for b in range(nb)]
+    count = DrawCount()
     for b in range(nb):
-        if ref[b][1] >= SAMPLE_MARGIN:
-            assert draws[b] == ref[b][0], b
+        u = oracle.row_uniform(77, 0, b, 0)
+        allowed = allowed_tokens(z, 1 / T, u)
+        count.add(allowed)
+        assert draws[b] in allowed, (b, draws[b], allowed)
+        if len(allowed) == 1:
+            assert draws[b] == oracle.sample_row(z, 1 / T, u)[0], b
+    assert count.ambiguous <= 0.01 * nb
     counts = np.bincount(draws, minlength=V)
     p = special.softmax(z.astype(np.float64) / T)
     keep = p * nb >= 5
