@@ -30,7 +30,14 @@ EXPORTED = ("ddt_status_string", "ddt_mask_words", "ddt_topk_workspace_size", "d
             "ddt_build_tree", "ddt_tree_attn_workspace_size", "ddt_tree_attn",
             "ddt_tree_walk_workspace_size", "ddt_tree_walk", "ddt_tree_walk_sample",
             "ddt_kv_commit", "ddt_lm_head_max_rows", "ddt_lm_head_walk_workspace_size",
-            "ddt_lm_head_walk")
+            "ddt_lm_head_walk", "ddt_tree_attn_plan", "ddt_debug_set_wait_limit",
+            "ddt_topk_noalloc", "ddt_tree_walk_resolve_mode")
+
+# ddt_tree_walk's modes
+WALK_ALL_ROWS, WALK_LAZY, WALK_AUTO = 0, 1, 2
+
+# ddt_tree_attn_plan's paths
+ATTN_PATH_SIMT, ATTN_PATH_TC, ATTN_PATH_TC_CLUSTER, ATTN_PATH_TC_COMBINE = 0, 1, 2, 3
 
 
 class KVCommitArgs(ctypes.Structure):
@@ -108,11 +115,18 @@ def load_library():
         lib.ddt_tree_attn_workspace_size.argtypes = [ctypes.POINTER(AttnArgs)]
         lib.ddt_tree_attn.restype = i32
         lib.ddt_tree_attn.argtypes = [ctypes.POINTER(AttnArgs), vp, sz, vp]
+        lib.ddt_tree_attn_plan.restype = i32
+        lib.ddt_tree_attn_plan.argtypes = [ctypes.POINTER(AttnArgs), ctypes.POINTER(i32),
+                                           ctypes.POINTER(i32)]
+        lib.ddt_debug_set_wait_limit.restype = ctypes.c_longlong
+        lib.ddt_debug_set_wait_limit.argtypes = [ctypes.c_longlong]
         lib.ddt_tree_walk_workspace_size.restype = sz
         lib.ddt_tree_walk_workspace_size.argtypes = [i32, i32, i32]
         lib.ddt_tree_walk.restype = i32
-        lib.ddt_tree_walk.argtypes = [vp, i32, i32, i32, i32, i64, vp, vp, vp, vp, i32,
+        lib.ddt_tree_walk.argtypes = [vp, i32, i32, i32, i32, i64, vp, vp, vp, vp, i32, i32,
                                       vp, vp, vp, vp, vp, sz, vp, vp]
+        lib.ddt_tree_walk_resolve_mode.restype = i32
+        lib.ddt_tree_walk_resolve_mode.argtypes = [i32, i32, i32, i32, i32, i32]
         lib.ddt_lm_head_max_rows.restype = i32
         lib.ddt_lm_head_max_rows.argtypes = []
         lib.ddt_lm_head_walk_workspace_size.restype = sz
@@ -291,9 +305,33 @@ def tree_attn_workspace_size(q, k_cache, v_cache, k_tree, v_tree, mask, n_nodes,
                              max_ctx, scale=None, page_table=None) -> int:
     d = q.shape[-1]
     scale = 1.0 / math.sqrt(d) if scale is None else scale
+    # the output pointer only has to be valid for the argument check: q stands in
     a = _attn_args(q, k_cache, v_cache, k_tree, v_tree, mask, n_nodes, ctx_len, max_ctx, scale,
-                   page_table, None, None, None)
+                   page_table, q, None, None)
     return int(load_library().ddt_tree_attn_workspace_size(ctypes.byref(a)))
+
+
+def tree_attn_plan(q, k_cache, v_cache, k_tree, v_tree, mask, n_nodes, ctx_len, max_ctx,
+                   scale=None, page_table=None):
+    """``ddt_tree_attn_plan``: (path, kv_splits) that :func:`tree_attn` would
+    use for these arguments on the current device (one of the ATTN_PATH_*)."""
+    d = q.shape[-1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    a = _attn_args(q, k_cache, v_cache, k_tree, v_tree, mask, n_nodes, ctx_len, max_ctx, scale,
+                   page_table, q, None, None)
+    path, splits = ctypes.c_int(), ctypes.c_int()
+    with torch.cuda.device(q.device):
+        rc = load_library().ddt_tree_attn_plan(ctypes.byref(a), ctypes.byref(path),
+                                               ctypes.byref(splits))
+    _check(rc, "ddt_tree_attn_plan")
+    return path.value, splits.value
+
+
+def set_wait_limit(cycles: int) -> int:
+    """``ddt_debug_set_wait_limit``: bound (clock cycles) of the tensor-core
+    kernels' on-chip waits for later launches; <= 0 restores the default of
+    about one second.  Returns the previous setting.  A test hook."""
+    return int(load_library().ddt_debug_set_wait_limit(int(cycles)))
 
 
 def tree_attn(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
@@ -332,11 +370,20 @@ def tree_walk_workspace_size(batch: int, n_max: int, V: int) -> int:
     return int(load_library().ddt_tree_walk_workspace_size(batch, n_max, V))
 
 
+def tree_walk_resolve_mode(mode: int, dtype: torch.dtype, batch: int, n_max: int, V: int,
+                           L: int) -> int:
+    """``ddt_tree_walk_resolve_mode``: WALK_ALL_ROWS or WALK_LAZY, the walk that
+    ``mode`` runs for these sizes on the current device."""
+    code = _dtype_code(torch.empty(0, dtype=dtype))
+    return int(load_library().ddt_tree_walk_resolve_mode(mode, code, batch, n_max, V, L))
+
+
 def tree_walk(logits: torch.Tensor, tok: torch.Tensor, parent: torch.Tensor,
               depth: torch.Tensor, n_nodes: torch.Tensor, L: int,
-              dev_status: Optional[torch.Tensor] = None):
+              dev_status: Optional[torch.Tensor] = None, mode: int = WALK_AUTO):
     """Stage 4.  ``logits`` [batch, n_max, V] f32/bf16 (rows contiguous, uniform
-    stride).  Returns dict acc_len [batch], acc_nodes/acc_tok [batch, L], bonus [batch]."""
+    stride); ``mode`` one of WALK_ALL_ROWS, WALK_LAZY, WALK_AUTO.  Returns dict
+    acc_len [batch], acc_nodes/acc_tok [batch, L], bonus [batch]."""
     lib = load_library()
     dev = _need_cuda(logits, tok, parent, depth, n_nodes, dev_status)
     if logits.dim() != 3 or logits.stride(2) != 1 or logits.stride(0) != logits.stride(1) * logits.shape[1]:
@@ -350,7 +397,7 @@ def tree_walk(logits: torch.Tensor, tok: torch.Tensor, parent: torch.Tensor,
     ws = workspaces.get(dev, "walk", nb)
     with torch.cuda.device(dev):
         rc = lib.ddt_tree_walk(_ptr(logits), _dtype_code(logits), b, n_max, V, logits.stride(1),
-                               _ptr(tok), _ptr(parent), _ptr(depth), _ptr(n_nodes), L,
+                               _ptr(tok), _ptr(parent), _ptr(depth), _ptr(n_nodes), L, int(mode),
                                _ptr(res["acc_len"]), _ptr(res["acc_nodes"]), _ptr(res["acc_tok"]),
                                _ptr(res["bonus"]), _ptr(ws), nb, _ptr(dev_status), _stream(dev))
     _check(rc, "ddt_tree_walk")

@@ -1,8 +1,11 @@
 // api.cu -- the exported C ABI of libddt.so: host-side validation, workspace
 // layout and dispatch to the stage kernels.  See include/ddt.h.
+#include <atomic>
 #include <map>
 #include <mutex>
 #include <utility>
+
+#include <nvtx3/nvToolsExt.h>
 
 #include "attn_common.cuh"
 #include "ddt.h"
@@ -44,6 +47,16 @@ int device_sm_count() {
 }
 
 namespace {
+constexpr long long kDefaultWaitCycles = 2000000000LL;  // about one second at 1.9 GHz
+std::atomic<long long> g_wait_override{0};
+}  // namespace
+
+long long wait_limit_cycles() {
+  const long long v = g_wait_override.load(std::memory_order_relaxed);
+  return v > 0 ? v : kDefaultWaitCycles;
+}
+
+namespace {
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
@@ -60,6 +73,8 @@ bool ws_ok(const void* ws, size_t have, size_t need) {
 ddt_status launch_attn_simt(AttnParams& p, cudaStream_t stream);
 int attn_simt_rows_per_cta();
 bool attn_tc_eligible(const ddt_attn_args* a);
+void attn_tc_plan(const ddt_attn_args* a, int sms, int* qtiles, int* nsplit, int* tps);
+bool attn_tc_cluster(int nsplit, long clusters);
 size_t attn_tc_workspace_size(const ddt_attn_args* a, int sms);
 ddt_status launch_attn_tc(const ddt_attn_args* a, void* ws, int sms, cudaStream_t stream);
 
@@ -151,7 +166,35 @@ ddt_status launch_attn(const ddt_attn_args* a, void* ws, size_t ws_bytes, cudaSt
 
 }  // namespace ddt
 
+namespace ddt {
+// Every check of ddt_topk's arguments but the workspace's (shared with the
+// allocation-free entry point, so that both return the same codes).
+ddt_status topk_check(const void* logits, ddt_dtype dtype, int batch, int L, int V,
+                      int64_t row_stride, int k, float inv_temperature, const int32_t* ids,
+                      const float* zk, const float* lse) {
+  if (batch < 0 || L < 0 || V < 1 || k < 1 || row_stride < V) return DDT_ERR_INVALID_ARG;
+  if (dtype != DDT_BF16 && dtype != DDT_F32) return DDT_ERR_UNSUPPORTED;
+  if (k > DDT_TOPK_K_MAX) return DDT_ERR_UNSUPPORTED;
+  if (k > V) return DDT_ERR_INVALID_ARG;
+  if (!(inv_temperature > 0.f) || !(inv_temperature < INFINITY)) return DDT_ERR_INVALID_ARG;
+  const long rows = (long)batch * L;
+  if (rows > 65535) return DDT_ERR_UNSUPPORTED;
+  if (rows > 0 && (!logits || !ids || !zk || !lse)) return DDT_ERR_INVALID_ARG;
+  return DDT_OK;
+}
+}  // namespace ddt
+
 using namespace ddt;
+
+namespace {
+// An NVTX range around each launching entry point, so that a timeline
+// (Nsight Systems, ncu's range filters) shows the library's calls by name.
+// Without a tool attached the push and pop cost a few nanoseconds.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
+}  // namespace
 
 extern "C" {
 
@@ -169,6 +212,10 @@ const char* ddt_status_string(ddt_status s) {
 
 int ddt_mask_words(int n_max) { return n_max > 0 ? (n_max + 31) / 32 : 0; }
 
+long long ddt_debug_set_wait_limit(long long cycles) {
+  return g_wait_override.exchange(cycles > 0 ? cycles : 0);
+}
+
 size_t ddt_topk_workspace_size(int batch, int L, int V, int k) {
   if (batch < 0 || L < 0 || V < 1 || k < 1) return 0;
   return topk_workspace_size(batch * L, V, k);
@@ -178,14 +225,11 @@ ddt_status ddt_topk(const void* logits, ddt_dtype dtype, int batch, int L, int V
                     int64_t row_stride, int k, float inv_temperature, int32_t* ids, float* zk,
                     float* logp, float* lse, void* workspace, size_t workspace_bytes,
                     cudaStream_t stream) {
-  if (batch < 0 || L < 0 || V < 1 || k < 1 || row_stride < V) return DDT_ERR_INVALID_ARG;
-  if (dtype != DDT_BF16 && dtype != DDT_F32) return DDT_ERR_UNSUPPORTED;
-  if (k > DDT_TOPK_K_MAX) return DDT_ERR_UNSUPPORTED;
-  if (k > V) return DDT_ERR_INVALID_ARG;
-  if (!(inv_temperature > 0.f) || !(inv_temperature < INFINITY)) return DDT_ERR_INVALID_ARG;
+  const NvtxRange nvtx("ddt_topk");
+  const ddt_status st =
+      topk_check(logits, dtype, batch, L, V, row_stride, k, inv_temperature, ids, zk, lse);
+  if (st != DDT_OK) return st;
   const long rows = (long)batch * L;
-  if (rows > 65535) return DDT_ERR_UNSUPPORTED;
-  if (rows > 0 && (!logits || !ids || !zk || !lse)) return DDT_ERR_INVALID_ARG;
   if (!ws_ok(workspace, workspace_bytes, topk_workspace_size((int)rows, V, k)))
     return DDT_ERR_WORKSPACE;
   return launch_topk(logits, dtype, (int)rows, V, row_stride, k, inv_temperature, ids, zk, logp,
@@ -198,6 +242,7 @@ ddt_status ddt_build_tree(const int32_t* ids, const float* zk, const float* lse,
                           const int32_t* ctx_len, int32_t* tok, int32_t* parent, int32_t* depth,
                           int32_t* pos, uint32_t* mask, int32_t* n_nodes, double* surrogate,
                           int32_t* dev_status, cudaStream_t stream) {
+  const NvtxRange nvtx("ddt_build_tree");
   if (batch < 0 || L < 1 || k < 1 || B_max < 0) return DDT_ERR_INVALID_ARG;
   if (L > DDT_TREE_L_MAX || k > DDT_TOPK_K_MAX || B_max > DDT_TREE_B_MAX) return DDT_ERR_UNSUPPORTED;
   if (!(inv_temperature > 0.f) || !(inv_temperature < INFINITY)) return DDT_ERR_INVALID_ARG;
@@ -247,11 +292,32 @@ static const size_t kMaxCounters = DDT_WS_COUNTER_BYTES / sizeof(unsigned);
 
 ddt_status ddt_tree_attn(const ddt_attn_args* a, void* workspace, size_t workspace_bytes,
                          cudaStream_t stream) {
+  const NvtxRange nvtx("ddt_tree_attn");
   const ddt_status st = check_attn(a);
   if (st != DDT_OK) return st;
   if (!attn_tc_eligible(a) && attn_simt_counters(a) > kMaxCounters) return DDT_ERR_UNSUPPORTED;
   if (!ws_ok(workspace, workspace_bytes, attn_workspace_size(a))) return DDT_ERR_WORKSPACE;
   return launch_attn(a, workspace, workspace_bytes, stream);
+}
+
+ddt_status ddt_tree_attn_plan(const ddt_attn_args* a, int* path, int* kv_splits) {
+  const ddt_status st = check_attn(a);
+  if (st != DDT_OK) return st;
+  int pth, ns;
+  if (attn_tc_eligible(a)) {
+    int qt, tps;
+    attn_tc_plan(a, sm_count(), &qt, &ns, &tps);
+    if (ns <= 1) pth = DDT_ATTN_PATH_TC;
+    else if (attn_tc_cluster(ns, (long)qt * a->batch * a->hkv)) pth = DDT_ATTN_PATH_TC_CLUSTER;
+    else pth = DDT_ATTN_PATH_TC_COMBINE;
+  } else {
+    int rt, tps;
+    attn_plan(a, attn_simt_rows_per_cta(), &rt, &ns, &tps);
+    pth = DDT_ATTN_PATH_SIMT;
+  }
+  if (path) *path = pth;
+  if (kv_splits) *kv_splits = ns;
+  return DDT_OK;
 }
 
 size_t ddt_tree_walk_workspace_size(int batch, int n_max, int V) {
@@ -262,11 +328,13 @@ size_t ddt_tree_walk_workspace_size(int batch, int n_max, int V) {
 namespace {
 ddt_status walk_common(const void* logits, ddt_dtype dtype, int batch, int n_max, int V,
                        int64_t row_stride, const int32_t* tok, const int32_t* parent,
-                       const int32_t* depth, const int32_t* n_nodes, int L, int32_t* acc_len,
-                       int32_t* acc_nodes, int32_t* acc_tok, int32_t* bonus, void* workspace,
-                       size_t workspace_bytes, int32_t* dev_status, cudaStream_t stream,
-                       const WalkSampling* sampling) {
+                       const int32_t* depth, const int32_t* n_nodes, int L, int mode,
+                       int32_t* acc_len, int32_t* acc_nodes, int32_t* acc_tok, int32_t* bonus,
+                       void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                       cudaStream_t stream, const WalkSampling* sampling) {
   if (batch < 0 || n_max < 1 || V < 1 || row_stride < V || L < 0) return DDT_ERR_INVALID_ARG;
+  if (mode != DDT_WALK_ALL_ROWS && mode != DDT_WALK_LAZY && mode != DDT_WALK_AUTO)
+    return DDT_ERR_INVALID_ARG;
   if (dtype != DDT_BF16 && dtype != DDT_F32) return DDT_ERR_UNSUPPORTED;
   if (n_max > DDT_TREE_B_MAX + 1 || batch > 65535 || L > DDT_TREE_L_MAX) return DDT_ERR_UNSUPPORTED;
   if ((size_t)batch * n_max + batch + 1 > kMaxCounters) return DDT_ERR_UNSUPPORTED;
@@ -276,19 +344,27 @@ ddt_status walk_common(const void* logits, ddt_dtype dtype, int batch, int n_max
   if (!ws_ok(workspace, workspace_bytes, walk_workspace_size(batch, n_max, V)))
     return DDT_ERR_WORKSPACE;
   return launch_tree_walk(logits, dtype, batch, n_max, V, row_stride, tok, parent, depth, n_nodes,
-                          L, acc_len, acc_nodes, acc_tok, bonus, workspace, dev_status, stream,
-                          sampling);
+                          L, mode, acc_len, acc_nodes, acc_tok, bonus, workspace, dev_status,
+                          stream, sampling);
 }
 }  // namespace
 
 ddt_status ddt_tree_walk(const void* logits, ddt_dtype dtype, int batch, int n_max, int V,
                          int64_t row_stride, const int32_t* tok, const int32_t* parent,
-                         const int32_t* depth, const int32_t* n_nodes, int L, int32_t* acc_len,
-                         int32_t* acc_nodes, int32_t* acc_tok, int32_t* bonus, void* workspace,
-                         size_t workspace_bytes, int32_t* dev_status, cudaStream_t stream) {
+                         const int32_t* depth, const int32_t* n_nodes, int L, int mode,
+                         int32_t* acc_len, int32_t* acc_nodes, int32_t* acc_tok, int32_t* bonus,
+                         void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                         cudaStream_t stream) {
+  const NvtxRange nvtx("ddt_tree_walk");
   return walk_common(logits, dtype, batch, n_max, V, row_stride, tok, parent, depth, n_nodes, L,
-                     acc_len, acc_nodes, acc_tok, bonus, workspace, workspace_bytes, dev_status,
-                     stream, nullptr);
+                     mode, acc_len, acc_nodes, acc_tok, bonus, workspace, workspace_bytes,
+                     dev_status, stream, nullptr);
+}
+
+int ddt_tree_walk_resolve_mode(int mode, ddt_dtype dtype, int batch, int n_max, int V, int L) {
+  if (mode != DDT_WALK_ALL_ROWS && mode != DDT_WALK_LAZY && mode != DDT_WALK_AUTO) return -1;
+  if (batch < 0 || n_max < 1 || V < 1 || L < 0) return -1;
+  return walk_mode_for(mode, dtype, batch, n_max, V, L);
 }
 
 ddt_status ddt_tree_walk_sample(const void* logits, ddt_dtype dtype, int batch, int n_max, int V,
@@ -298,13 +374,14 @@ ddt_status ddt_tree_walk_sample(const void* logits, ddt_dtype dtype, int batch, 
                                 uint64_t* step_counter, int32_t* acc_len, int32_t* acc_nodes,
                                 int32_t* acc_tok, int32_t* bonus, void* workspace,
                                 size_t workspace_bytes, int32_t* dev_status, cudaStream_t stream) {
+  const NvtxRange nvtx("ddt_tree_walk_sample");
   if (!(inv_temperature > 0.f) || !(inv_temperature * kLog2e < INFINITY))
     return DDT_ERR_INVALID_ARG;
   if (step_counter && ((uintptr_t)step_counter & 7u)) return DDT_ERR_INVALID_ARG;
   const WalkSampling smp{inv_temperature, seed, step, step_counter};
   return walk_common(logits, dtype, batch, n_max, V, row_stride, tok, parent, depth, n_nodes, L,
-                     acc_len, acc_nodes, acc_tok, bonus, workspace, workspace_bytes, dev_status,
-                     stream, &smp);
+                     DDT_WALK_ALL_ROWS, acc_len, acc_nodes, acc_tok, bonus, workspace,
+                     workspace_bytes, dev_status, stream, &smp);
 }
 
 int ddt_lm_head_max_rows(void) { return lm_head_max_rows(); }
@@ -316,6 +393,7 @@ size_t ddt_lm_head_walk_workspace_size(const ddt_lm_head_walk_args* a) {
 
 ddt_status ddt_lm_head_walk(const ddt_lm_head_walk_args* a, void* workspace,
                             size_t workspace_bytes, cudaStream_t stream) {
+  const NvtxRange nvtx("ddt_lm_head_walk");
   if (!a) return DDT_ERR_INVALID_ARG;
   if (a->batch < 0 || a->n_max < 1 || a->L < 0 || a->K < 1 || a->V < 1) return DDT_ERR_INVALID_ARG;
   if (a->K % 8 != 0 || a->n_max > DDT_TREE_B_MAX + 1 || a->L > DDT_TREE_L_MAX ||
@@ -331,6 +409,7 @@ ddt_status ddt_lm_head_walk(const ddt_lm_head_walk_args* a, void* workspace,
 }
 
 ddt_status ddt_kv_commit(const ddt_kv_commit_args* a, cudaStream_t stream) {
+  const NvtxRange nvtx("ddt_kv_commit");
   if (!a) return DDT_ERR_INVALID_ARG;
   if (a->batch < 0 || a->n_max < 1 || a->hkv < 1 || a->d < 1 || a->L < 0)
     return DDT_ERR_INVALID_ARG;

@@ -25,7 +25,9 @@
 //     the splits of a query tile merge on chip as one cluster, or write
 //     (O, m, l) partials that a second kernel merges.
 // Every mbarrier wait is bounded (about one second); a wait that gives up
-// raises DDT_ERR_TIMEOUT in the status word and the CTA stops issuing work.
+// raises DDT_ERR_TIMEOUT in the status word and the CTA stops issuing work,
+// lets its loads and MMAs in flight complete (bounded too), frees TMEM and
+// returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -49,7 +51,6 @@ constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP = 384;
 constexpr uint32_t kColX = 448;  // exchange columns of the softmax warp pairs
 constexpr int kHalf = BN * 128;           // one 64-wide d half: 128 rows x 128 B
 constexpr int kTile = 2 * kHalf;          // 32 KB
-constexpr long long kWaitCycles = 2000000000LL;
 constexpr float kRescaleLog2 = 8.f;       // move the running max only when it grows by > 2^8
 
 struct Params {
@@ -68,6 +69,7 @@ struct Params {
   int cluster;      // the splits of a query tile form a cluster and merge on chip
   float* part_o;    // [grp][qtile][split][BM][D] (split partials without a cluster)
   float2* part_ml;  // [grp][qtile][split][BM]
+  long long wait_cycles;  // bound of every mbarrier wait
 };
 
 struct __align__(8) Bars {
@@ -77,6 +79,8 @@ struct __align__(8) Bars {
   uint64_t s_full[2];
   uint64_t p_full;
   uint64_t pv_done;
+  uint64_t drain;  // after a wait gave up: completion of every MMA issued
+  long long wait_cycles;
   uint32_t tmem_base;
   int abort;
 };
@@ -84,9 +88,9 @@ struct __align__(8) Bars {
 // ---------------------------------------------------------------- PTX helpers
 // (the shared tcgen05 / TMA / mbarrier wrappers are in tcgen05.cuh)
 // Bounded wait: false (and the CTA-wide abort flag set) if the phase does not
-// complete within kWaitCycles or another role already aborted.
+// complete within the launch's wait bound or another role already aborted.
 __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, Bars* bars) {
-  return mbar_wait_bounded(b, parity, &bars->abort, kWaitCycles);
+  return mbar_wait_bounded(b, parity, &bars->abort, bars->wait_cycles);
 }
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
@@ -209,6 +213,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars->s_full[1], 1);
     mbar_init(&bars->p_full, 256);
     mbar_init(&bars->pv_done, 1);
+    mbar_init(&bars->drain, 1);
+    bars->wait_cycles = p.wait_cycles;
     bars->abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -282,7 +288,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_expect_tx(&bars->q_full, (uint32_t)kTile);
       tma_load_3d(sQ, &tm_q, 0, kvh * g, b * p.n_max + j0, &bars->q_full);
       tma_load_3d(sQ + kHalf, &tm_q, 64, kvh * g, b * p.n_max + j0, &bars->q_full);
-      for (int i = 0; i < ntiles; ++i) {
+      int issued = 0;  // K/V tiles whose loads were issued
+      for (int i = 0; i < ntiles; ++i, issued = i) {
         const int s = i % kStages;
         const uint32_t ph = (uint32_t)(i / kStages) & 1u;
         if (!mbar_wait(&bars->kv_empty[s], ph ^ 1u, bars)) break;
@@ -323,6 +330,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      if (*(volatile int*)&bars->abort) {
+        // a wait gave up: let the loads still in flight land before the CTA
+        // (and its shared memory) goes away.  The Q tile and the last
+        // kStages K/V tiles issued are the only ones that can be outstanding;
+        // each of their stages has exactly one phase pending.
+        int keep_going = 0;
+        mbar_wait_bounded(&bars->q_full, 0u, &keep_going, kDrainCycles);
+        for (int q = issued > kStages ? issued - kStages : 0; q < issued; ++q)
+          mbar_wait_bounded(&bars->kv_full[q % kStages], (uint32_t)(q / kStages) & 1u, &keep_going,
+                            kDrainCycles);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -359,6 +377,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(&bars->pv_done);
           mma_commit(&bars->kv_empty[sp]);
         }
+      }
+      if (*(volatile int*)&bars->abort) {
+        // a wait gave up: every MMA issued completes before TMEM is freed
+        int keep_going = 0;
+        mma_commit(&bars->drain);
+        mbar_wait_bounded(&bars->drain, 0u, &keep_going, kDrainCycles);
       }
     }
   } else {
@@ -871,6 +895,7 @@ ddt_status launch_attn_tc(const ddt_attn_args* a, void* ws, int sms, cudaStream_
   p.out = (uint16_t*)a->out;
   p.lse_out = a->lse_out;
   p.status = a->dev_status;
+  p.wait_cycles = wait_limit_cycles();
   attn_tc_plan(a, sms, &p.qtiles, &p.nsplit, &p.tiles_per_split);
   p.cluster = attn_tc_cluster(p.nsplit, (long)p.qtiles * a->batch * a->hkv) ? 1 : 0;
   if (p.nsplit > 1 && !p.cluster) {

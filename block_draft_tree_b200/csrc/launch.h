@@ -17,6 +17,12 @@ cudaError_t ensure_smem_attr(const void* func, size_t bytes);
 // Multiprocessors of the current device.
 int device_sm_count();
 
+// Clock cycles after which a bounded mbarrier wait of the tensor-core kernels
+// gives up (about one second by default; see ddt_debug_set_wait_limit), and
+// the bound of each wait that drains loads and MMAs in flight after that.
+long long wait_limit_cycles();
+constexpr long long kDrainCycles = 200000000LL;
+
 // Launch with programmatic stream serialization (see pdl_wait/pdl_trigger),
 // optionally as clusters of cluster_y CTAs along y.
 template <typename... KArgs, typename... Args>
@@ -44,6 +50,9 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 }
 
 size_t topk_workspace_size(int rows, int V, int k);
+ddt_status topk_check(const void* logits, ddt_dtype dtype, int batch, int L, int V,
+                      int64_t row_stride, int k, float inv_temperature, const int32_t* ids,
+                      const float* zk, const float* lse);
 ddt_status launch_topk(const void* logits, ddt_dtype dt, int rows, int V, int64_t row_stride,
                        int k, float inv_t, int32_t* ids, float* zk, float* logp, float* lse,
                        void* ws, size_t ws_bytes, cudaStream_t stream);
@@ -64,10 +73,12 @@ struct WalkSampling {
 };
 ddt_status launch_tree_walk(const void* logits, ddt_dtype dt, int batch, int n_max, int V,
                             int64_t row_stride, const int32_t* tok, const int32_t* parent,
-                            const int32_t* depth, const int32_t* n_nodes, int L, int32_t* acc_len,
-                            int32_t* acc_nodes, int32_t* acc_tok, int32_t* bonus, void* ws,
-                            int32_t* dev_status, cudaStream_t stream,
+                            const int32_t* depth, const int32_t* n_nodes, int L, int mode,
+                            int32_t* acc_len, int32_t* acc_nodes, int32_t* acc_tok, int32_t* bonus,
+                            void* ws, int32_t* dev_status, cudaStream_t stream,
                             const WalkSampling* sampling = nullptr);
+// The walk DDT_WALK_AUTO resolves to for these sizes on the current device.
+int walk_mode_for(int mode, ddt_dtype dt, int batch, int n_max, int V, int L);
 
 ddt_status launch_kv_commit(const ddt_kv_commit_args* a, cudaStream_t stream);
 ddt_status launch_lm_head_walk(const ddt_lm_head_walk_args* a, void* ws, cudaStream_t stream);

@@ -48,8 +48,6 @@ constexpr int kThreads = 192;           // warp 0 TMA, warp 1 MMA, warps 2-5 epi
 constexpr uint32_t kTmemCols = 512;     // two 256-column fp32 accumulators
 constexpr int kATile = BM * BK * 2;     // 16 KB
 constexpr int kBTile = BN * BK * 2;     // 32 KB
-constexpr long long kWaitCycles = 2000000000LL;
-constexpr long long kDrainCycles = 200000000LL;  // per wait while draining after an abort
 
 struct Params {
   int M, K, V, m_tiles, total_tiles, kblocks;
@@ -61,12 +59,14 @@ struct Params {
   unsigned long long* keys;  // [M], in the workspace's counter region
   unsigned* ticket;
   int32_t* status;
+  long long wait_cycles;  // bound of every mbarrier wait
 };
 
 struct __align__(8) Bars {
   uint64_t full[kStages], empty[kStages];
   uint64_t acc_full[2], acc_empty[2];
   uint64_t drain;  // after a wait gave up: completion of every MMA issued
+  long long wait_cycles;
   uint32_t tmem_base;
   int abort;
   int last;
@@ -75,9 +75,9 @@ struct __align__(8) Bars {
 // ---------------------------------------------------------------- PTX helpers
 // (the shared tcgen05 / TMA / mbarrier wrappers are in tcgen05.cuh)
 // Bounded wait: false (and the CTA-wide abort flag set) if the phase does not
-// complete within kWaitCycles or another role already gave up.
+// complete within the launch's wait bound or another role already gave up.
 __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, Bars* bars) {
-  return mbar_wait_bounded(b, parity, &bars->abort, kWaitCycles);
+  return mbar_wait_bounded(b, parity, &bars->abort, bars->wait_cycles);
 }
 // K-major operand, 128-byte swizzle: 8-row groups 1024 bytes apart.
 __device__ __forceinline__ uint64_t sdesc_k(uint32_t saddr) { return sdesc(saddr, 16, 1024); }
@@ -156,6 +156,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->acc_empty[i], 4 * 32);
     }
     mbar_init(&bars->drain, 1);
+    bars->wait_cycles = p.wait_cycles;
     bars->abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -373,6 +374,7 @@ ddt_status launch_lm_head_walk(const ddt_lm_head_walk_args* a, void* ws, cudaStr
   p.keys = (unsigned long long*)ws;
   p.ticket = (unsigned*)((unsigned long long*)ws + kLmHeadMaxRows + 8);
   p.status = a->dev_status;
+  p.wait_cycles = wait_limit_cycles();
   const size_t smem = smem_bytes();
   if (ensure_smem_attr((const void*)lmhead_kernel, smem) != cudaSuccess) return DDT_ERR_CUDA;
   const int grid = p.total_tiles < sms ? p.total_tiles : sms;

@@ -5,21 +5,30 @@
 // per position; the tree's candidates at depth i are the k most likely
 // tokens of q_i (logit descending, smaller token id first on ties).
 //
-// Design (HBM-bound single pass over the logits):
-//   * grid = (chunks of 8192 logits, rows); 256 threads; each thread keeps
-//     32 logits in registers, loaded with 16-byte streaming loads.
-//   * from registers: thread max, thread sum of exp2((z-max)*c), and the
-//     thread maximum's order key;
-//   * the k-th largest thread maximum over the CTA (16 or 32 rounds of
-//     __syncthreads_count bisection) is a threshold that at least k logits
-//     of the chunk reach and that few others do (about k+1 on random rows);
-//     those candidates go to shared memory and are ranked exactly by the
-//     64-bit key (value, then smaller id);
-//   * per chunk partials (k keys, max, sum) go to the workspace; the last
-//     CTA of a row (atomic ticket, no waiting) merges them, writes the row's
-//     outputs and returns its ticket to zero.
-// Degenerate rows (many equal values beyond the candidate capacity) fall
-// back to k rounds of block-wide argmax: slower, same result.
+// Design (an HBM-bound stream over the logits):
+//   * the rows are cut into 16 KB chunks and the chunks, in row order, into
+//     one contiguous range per CTA, as many CTAs as fit on the device at
+//     once; every CTA streams its range through a 4-deep ring of shared
+//     memory filled by 16-byte asynchronous copies (each thread copies and
+//     later reads the same 64 bytes of a chunk, so no barrier guards the
+//     ring), so that 48 KB per CTA are always in flight;
+//   * per chunk, each thread folds its 32 (bf16) or 16 (f32) logits into a
+//     running (max, sum of 2^((z - max) * c)) and compares its chunk maximum
+//     with the CTA's current k-th best key: only a thread whose maximum beats
+//     it looks at its logits again and appends the ones that do to a
+//     candidate list, which is ranked exactly against the current k best.
+//     After the first chunk of a row almost no logit qualifies;
+//   * the first chunk of each row a CTA sees starts from a threshold that k
+//     logits are sure to reach: the k-th largest of the per-lane maxima of
+//     the warp that has the largest one (a sort of 32 keys inside the warp);
+//   * a CTA's part of a row ends in a partial (k best keys, max, sum) in the
+//     workspace; the last CTA of the row (atomic ticket, no waiting) merges
+//     the partials, writes the row's outputs and returns its ticket to zero.
+// The order key is 64 bits: the float's order-preserving bits, then the
+// complement of the token id, so ties go to the smaller id and every key is
+// distinct.  No CTA ever waits for another, so nothing can hang.
+#include <mutex>
+
 #include "common.cuh"
 #include "launch.h"
 
@@ -27,20 +36,25 @@ namespace ddt {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kChunk = 8192;
+constexpr int kChunkBytes = 16384;             // one chunk: 64 bytes per thread
+constexpr int kVecPerThread = kChunkBytes / 16 / kThreads;  // 4 vectors of 16 bytes
+constexpr int kStages = 4;                     // chunks of the ring
 constexpr int kCandCap = 1024;
 
 struct TopkParams {
   const void* logits;
-  int V;
+  int rows, V;
   int64_t row_stride;  // elements
   int k;
   float inv_t;
   float c;             // inv_t * log2(e)
   int S;               // chunks per row
+  int G;               // CTAs
+  int64_t T;           // chunks in all (rows * S)
+  int pmax;            // partial slots per row
   int vec_ok;          // 16-byte aligned rows
-  uint64_t* part_keys; // [rows][S][k]
-  float2* part_ms;     // [rows][S]
+  uint64_t* part_keys; // [rows][pmax][k]
+  float2* part_ms;     // [rows][pmax]
   unsigned* tickets;   // [rows]
   int32_t* ids;
   float* zk;
@@ -48,9 +62,28 @@ struct TopkParams {
   float* lse;
 };
 
-// Block merge of per-thread (max, sum of exp2((z-max)*c)): the block maximum
-// from a REDUX on the ordered keys, one rescale per thread, then a sum.  Two
-// barriers; every thread gets the result.
+// First chunk of CTA g's range, and the CTA whose range holds chunk ch.
+__host__ __device__ __forceinline__ int64_t range_lo(int64_t g, int64_t T, int64_t G) {
+  return g * T / G;
+}
+__host__ __device__ __forceinline__ int64_t owner_of(int64_t ch, int64_t T, int64_t G) {
+  return ((ch + 1) * G - 1) / T;
+}
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                   (uint32_t)__cvta_generic_to_shared(smem)),
+               "l"(gmem)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Block merge of per-thread (max, sum of exp2((z-max)*c)); every thread gets
+// the result.  Two barriers.
 __device__ __forceinline__ void block_ms_reduce(float& m, float& s, float c, float* sm_m,
                                                 float* sm_s) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -76,7 +109,7 @@ __device__ __forceinline__ uint64_t block_max_u64(uint64_t v, uint64_t* sm) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
-    uint64_t u = shfl_xor_u64(v, o);
+    const uint64_t u = shfl_xor_u64(v, o);
     v = u > v ? u : v;
   }
   __syncthreads();
@@ -87,15 +120,39 @@ __device__ __forceinline__ uint64_t block_max_u64(uint64_t v, uint64_t* sm) {
   return r;
 }
 
-// Exact rank selection of the k largest of n distinct keys in s_cand.
-__device__ void rank_select(const uint64_t* s_cand, int n, int k, uint64_t* s_top) {
+// The k largest of the distinct nonzero keys a[0..na) and b[0..nb) (either
+// may hold zeros: "no element"), in descending order, into out[0..k).
+__device__ void rank_select2(const uint64_t* a, int na, const uint64_t* b, int nb, int k,
+                             uint64_t* out) {
+  const int n = na + nb;
   for (int i = threadIdx.x; i < n; i += kThreads) {
-    const uint64_t key = s_cand[i];
+    const uint64_t key = i < na ? a[i] : b[i - na];
+    if (key == 0) continue;
     int r = 0;
-    for (int j = 0; j < n; ++j) r += (s_cand[j] > key);
-    if (r < k) s_top[r] = key;
+    for (int j = 0; j < na; ++j) r += (a[j] > key);
+    for (int j = 0; j < nb; ++j) r += (b[j] > key);
+    if (r < k) out[r] = key;
   }
-  for (int i = n + threadIdx.x; i < k; i += kThreads) s_top[i] = 0;
+}
+
+// The k-th largest key of the warp's lanes (0 when fewer than k lanes hold
+// one): a bitonic sort of the 32 keys, descending.
+__device__ __forceinline__ uint64_t warp_kth_key(uint64_t v, int k) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const uint64_t o = shfl_xor_u64(v, stride);
+      const bool up = (lane & stride) == 0;            // the lower lane of the pair
+      const bool desc = (lane & size) == 0;            // this block sorts descending
+      const bool keep_max = (up == desc);
+      v = keep_max ? (o > v ? o : v) : (o < v ? o : v);
+    }
+  }
+  const uint32_t lo = __shfl_sync(0xFFFFFFFFu, (uint32_t)v, k - 1);
+  const uint32_t hi = __shfl_sync(0xFFFFFFFFu, (uint32_t)(v >> 32), k - 1);
+  return ((uint64_t)hi << 32) | lo;
 }
 
 // Row log-sum-exp, rounded up to f32: inv_t*max + log(sum) in fp64, so that
@@ -118,267 +175,403 @@ __device__ void write_row(const TopkParams& p, int row, const uint64_t* s_top, f
   if (threadIdx.x == 0) p.lse[row] = row_lse;
 }
 
-// MIN_CTAS: CTAs per SM the registers are budgeted for.  Three keep every
-// value in registers; four (64 registers, a few spilled) hide more of the
-// per-chunk compute behind other CTAs' loads when the grid spans many waves.
-template <bool BF16, int MIN_CTAS>
-__global__ void __launch_bounds__(kThreads, MIN_CTAS) topk_kernel(TopkParams p) {
-  constexpr int EPV = BF16 ? 8 : 4;           // elements per 16-byte vector
-  constexpr int EPT = kChunk / kThreads;      // 32 elements per thread
-  constexpr int VPT = EPT / EPV;
-  constexpr int ES = BF16 ? 2 : 4;
-  constexpr int NW = EPT * ES / 4;            // 32-bit words held per thread
+struct Smem {
+  uint64_t cand[kCandCap];
+  uint64_t top[DDT_TOPK_K_MAX];
+  uint64_t top2[DDT_TOPK_K_MAX];
+  uint64_t red[kThreads / 32];
+  float wm[kThreads / 32], wsum[kThreads / 32];
+  int count, last;
+};
 
-  __shared__ uint64_t s_cand[kCandCap];
-  __shared__ uint64_t s_top[DDT_TOPK_K_MAX];
-  __shared__ uint64_t s_red[kThreads / 32];
-  __shared__ float s_wm[kThreads / 32], s_wsum[kThreads / 32];
-  __shared__ int s_count, s_last;
+// Issue this thread's copies of chunk ch into ring slot `slot` (vectors
+// entirely inside the row only; the one that straddles V is read from
+// global memory when the chunk is used).  Always commits one group.
+template <bool BF16>
+__device__ __forceinline__ void prefetch_chunk(const TopkParams& p, unsigned char* ring, int slot,
+                                               int64_t ch) {
+  constexpr int ES = BF16 ? 2 : 4, EPV = 16 / ES, EPC = kChunkBytes / ES;
+  if (p.vec_ok && ch < p.T) {
+    const int row = (int)(ch / p.S), cidx = (int)(ch % p.S);
+    const char* rowp = (const char*)p.logits + (int64_t)row * p.row_stride * ES;
+    const int e0 = cidx * EPC;
+#pragma unroll
+    for (int q = 0; q < kVecPerThread; ++q) {
+      const int v = q * kThreads + (int)threadIdx.x;
+      const int e = e0 + v * EPV;
+      if (e + EPV <= p.V) cp_async16(ring + slot * kChunkBytes + v * 16, rowp + (int64_t)e * ES);
+    }
+  }
+  cp_async_commit();
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkParams p) {
+  constexpr int ES = BF16 ? 2 : 4, EPV = 16 / ES, EPC = kChunkBytes / ES;
+  constexpr int NW = kVecPerThread * 4;  // 32-bit words of logits per thread per chunk
+  extern __shared__ __align__(16) unsigned char ring[];
+  __shared__ Smem sm;
 
   const int tid = threadIdx.x;
-  const int chunk = blockIdx.x, row = blockIdx.y;
-  const int64_t c0 = (int64_t)chunk * kChunk;
+  const int64_t c_lo = range_lo(blockIdx.x, p.T, p.G), c_hi = range_lo(blockIdx.x + 1, p.T, p.G);
   pdl_wait();
-  const char* rowp = (const char*)p.logits + (int64_t)row * p.row_stride * ES;
-
-  // word j of vector q of this thread holds elements starting at index
-  // c0 + (q*kThreads + tid)*EPV + j*(EPV/4); out-of-range elements read as -inf
-  uint32_t w[NW];
-  const bool full = p.vec_ok && (c0 + kChunk <= p.V);
-  if (full) {
-#pragma unroll
-    for (int q = 0; q < VPT; ++q) {
-      const uint4 v = ld_stream_v4(rowp + (c0 + (int64_t)(q * kThreads + tid) * EPV) * ES);
-      w[4 * q] = v.x;
-      w[4 * q + 1] = v.y;
-      w[4 * q + 2] = v.z;
-      w[4 * q + 3] = v.w;
-    }
-  } else {
-#pragma unroll
-    for (int q = 0; q < VPT; ++q)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int64_t e0 = c0 + (int64_t)(q * kThreads + tid) * EPV + j * (EPV / 4);
-        if (BF16) {
-          const uint32_t lo = e0 < p.V ? ((const uint16_t*)rowp)[e0] : 0xFF80u;
-          const uint32_t hi = e0 + 1 < p.V ? ((const uint16_t*)rowp)[e0 + 1] : 0xFF80u;
-          w[4 * q + j] = lo | (hi << 16);
-        } else {
-          w[4 * q + j] = e0 < p.V ? __float_as_uint(((const float*)rowp)[e0]) : 0xFF800000u;
-        }
-      }
-  }
-  const int ibase = (int)c0 + tid * EPV;
-  auto index_of = [&](int e) -> int {  // element e (0..EPT) of this thread
-    return ibase + (e / EPV) * kThreads * EPV + (e % EPV);
-  };
-  auto value_of = [&](int e) -> float {
-    if (BF16) return (e & 1) ? bf16_hi(w[e >> 1]) : bf16_lo(w[e >> 1]);
-    return __uint_as_float(w[e]);
-  };
-  int nvalid = EPT;
-  if (!full) {
-    nvalid = 0;
-#pragma unroll
-    for (int e = 0; e < EPT; ++e) nvalid += (index_of(e) < p.V);
-  }
-
-  // thread max (packed bf16 pairs where possible) and sum of exp2((z-max)*c)
-  float m;
-  if (BF16) {
-    __nv_bfloat162 m2 = *(const __nv_bfloat162*)&w[0];
-#pragma unroll
-    for (int j = 1; j < NW; ++j) m2 = __hmax2(m2, *(const __nv_bfloat162*)&w[j]);
-    m = fmaxf(__low2float(m2), __high2float(m2));
-  } else {
-    m = -INFINITY;
-#pragma unroll
-    for (int e = 0; e < EPT; ++e) m = fmaxf(m, value_of(e));
-  }
-  float s = 0.f;
-  if (m != -INFINITY) {
-    const float mc = m * p.c;
-    float s4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int e = 0; e < EPT; ++e) s4[e & 3] += ex2(fmaf(value_of(e), p.c, -mc));
-    s = (s4[0] + s4[1]) + (s4[2] + s4[3]);
-  }
-  // order key of the thread maximum (0: thread holds no element)
-  uint32_t tk = 0;
-  if (nvalid > 0) {
-    tk = BF16 ? ord16(__float_as_uint(m) >> 16) : ord32(m);
-    if (tk == 0) tk = 1;
-  }
-  if (tid == 0) s_count = 0;
-
-  // the k-th largest thread maximum over the CTA
-  constexpr int KB = BF16 ? 16 : 32;
-  uint32_t tau = 0;
-#pragma unroll 1
-  for (int bit = KB - 1; bit >= 0; --bit) {
-    const uint32_t cand = tau | (1u << bit);
-    if (__syncthreads_count(tk >= cand) >= p.k) tau = cand;
-  }
-  if (tau == 0) tau = 1;  // fewer than k threads hold elements: take them all
-
-  // candidates: elements whose order key reaches tau; with a float threshold
-  // this is one compare per element (ties included, -0 == +0 as in the keys)
-  {
-    const uint32_t tb = BF16 ? (tau & 0xFFFFu) : tau;
-    const uint32_t tbits = BF16 ? (((tb & 0x8000u) ? (tb & 0x7FFFu) : (~tb & 0xFFFFu)) << 16)
-                                : ((tb & 0x80000000u) ? (tb & 0x7FFFFFFFu) : ~tb);
-    // keys below the key of -inf only come from the take-everything sentinel
-    const float tf = tb < (BF16 ? 0x7Fu : 0x007FFFFFu) ? -INFINITY : __uint_as_float(tbits);
-#pragma unroll
-    for (int e = 0; e < EPT; ++e) {
-      const float v = value_of(e);
-      if (v >= tf) {
-        const int idx = index_of(e);
-        if (!full && idx >= p.V) continue;
-        const int pos = atomicAdd(&s_count, 1);
-        if (pos < kCandCap) s_cand[pos] = cand_key(v, (uint32_t)idx);
-      }
-    }
-  }
-  block_ms_reduce(m, s, p.c, s_wm, s_wsum);  // contains __syncthreads
-  const int n = s_count;
-  if (n <= kCandCap) {
-    rank_select(s_cand, n, p.k, s_top);
-  } else {
-    // degenerate chunk: k rounds of block-wide argmax below the previous pick
-    uint64_t prev = ~0ull;
-    for (int r = 0; r < p.k; ++r) {
-      uint64_t best = 0;
-#pragma unroll
-      for (int e = 0; e < EPT; ++e) {
-        const int idx = index_of(e);
-        if (!full && idx >= p.V) continue;
-        const uint64_t key = cand_key(value_of(e), (uint32_t)idx);
-        if (key < prev && key > best) best = key;
-      }
-      best = block_max_u64(best, s_red);
-      if (tid == 0) s_top[r] = best;
-      prev = best;
-    }
-  }
-  __syncthreads();
-
-  if (p.S == 1) {
-    write_row(p, row, s_top, row_lse_up(p.inv_t, m, s));
-    return;
-  }
-
+  for (int i = 0; i < kStages; ++i) prefetch_chunk<BF16>(p, ring, i, c_lo + i < c_hi ? c_lo + i : p.T);
   pdl_trigger();
-  // publish this chunk's partial, then take a ticket
-  const int64_t pbase = (int64_t)row * p.S + chunk;
-  for (int r = tid; r < p.k; r += kThreads) p.part_keys[pbase * p.k + r] = s_top[r];
-  if (tid == 0) p.part_ms[pbase] = make_float2(m, s);
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) s_last = (atomicAdd(&p.tickets[row], 1u) == (unsigned)(p.S - 1));
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
 
-  // last CTA of the row: every chunk's keys and (max, sum) in one round of
-  // loads, then the k best keys of the row ranked directly
-  const int tot = p.S * p.k;
-  float M = -INFINITY, Ssum = 0.f;
-  for (int cc = tid; cc < p.S; cc += kThreads) {
-    const float2 ms = ld_cg_f2(&p.part_ms[(int64_t)row * p.S + cc]);
-    ms_merge(M, Ssum, ms.x, ms.y, p.c);
-  }
-  if (tot <= kCandCap) {
-    for (int i = tid; i < tot; i += kThreads) s_cand[i] = ld_cg_u64(&p.part_keys[(int64_t)row * tot + i]);
-    block_ms_reduce(M, Ssum, p.c, s_wm, s_wsum);  // its barriers publish s_cand
-    rank_select(s_cand, tot, p.k, s_top);
-  } else {
-    // many chunks: a threshold first (the best k-th key of any chunk: each
-    // chunk has k keys at or above it), then the keys that reach it
-    if (tid == 0) s_count = 0;
-    uint64_t t = 0;
-    for (int cc = tid; cc < p.S; cc += kThreads) {
-      const uint64_t kk = ld_cg_u64(&p.part_keys[((int64_t)row * p.S + cc) * p.k + p.k - 1]);
-      t = kk > t ? kk : t;
-    }
-    t = block_max_u64(t, s_red);
-    if (t == 0) t = 1;
-    for (int i = tid; i < tot; i += kThreads) {
-      const uint64_t key = ld_cg_u64(&p.part_keys[(int64_t)row * tot + i]);
-      if (key >= t) {
-        const int pos = atomicAdd(&s_count, 1);
-        if (pos < kCandCap) s_cand[pos] = key;
-      }
-    }
-    block_ms_reduce(M, Ssum, p.c, s_wm, s_wsum);
-    const int n2 = s_count;
-    if (n2 <= kCandCap) {
-      rank_select(s_cand, n2, p.k, s_top);
-    } else {
-      uint64_t prev = ~0ull;
-      for (int r = 0; r < p.k; ++r) {
-        uint64_t best = 0;
-        for (int i = tid; i < tot; i += kThreads) {
-          const uint64_t key = ld_cg_u64(&p.part_keys[(int64_t)row * tot + i]);
-          if (key < prev && key > best) best = key;
+  float m = -INFINITY, s = 0.f;  // this thread's running (max, sum) for the current row
+  uint64_t tau = 0;              // the CTA's current k-th best key (0: fewer than k seen)
+  bool first = true;             // next chunk is the first of a row for this CTA
+  if (tid < DDT_TOPK_K_MAX) sm.top[tid] = 0;
+  for (int64_t ch = c_lo; ch < c_hi; ++ch) {
+    const int slot = (int)((ch - c_lo) % kStages);
+    const int row = (int)(ch / p.S), cidx = (int)(ch % p.S);
+    const int e0 = cidx * EPC;
+    const char* rowp = (const char*)p.logits + (int64_t)row * p.row_stride * ES;
+    cp_async_wait<kStages - 1>();
+    // this thread's logits: word j of vector q holds elements
+    // e0 + (q*kThreads + tid)*EPV + j*(EPV/4) ...; absent ones read as -inf
+    uint32_t w[NW];
+#pragma unroll
+    for (int q = 0; q < kVecPerThread; ++q) {
+      const int v = q * kThreads + tid;
+      const int e = e0 + v * EPV;
+      if (p.vec_ok && e + EPV <= p.V) {
+        const uint4 u = *(const uint4*)(ring + slot * kChunkBytes + v * 16);
+        w[4 * q] = u.x;
+        w[4 * q + 1] = u.y;
+        w[4 * q + 2] = u.z;
+        w[4 * q + 3] = u.w;
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int ej = e + j * (EPV / 4);
+          if (BF16) {
+            const uint32_t lo = ej < p.V ? ((const uint16_t*)rowp)[ej] : 0xFF80u;
+            const uint32_t hi = ej + 1 < p.V ? ((const uint16_t*)rowp)[ej + 1] : 0xFF80u;
+            w[4 * q + j] = lo | (hi << 16);
+          } else {
+            w[4 * q + j] = ej < p.V ? __float_as_uint(((const float*)rowp)[ej]) : 0xFF800000u;
+          }
         }
-        best = block_max_u64(best, s_red);
-        if (tid == 0) s_top[r] = best;
-        prev = best;
       }
     }
+    // the slot is free again: refill it with the chunk kStages ahead
+    prefetch_chunk<BF16>(p, ring, slot, ch + kStages < c_hi ? ch + kStages : p.T);
+
+    auto index_of = [&](int i) -> int {  // element i (0..NW*(EPV/4)) of this thread
+      const int per = EPV / 4;           // elements per word
+      const int q = i / (4 * per), r = i % (4 * per);
+      return e0 + (q * kThreads + tid) * EPV + r;
+    };
+    auto value_of = [&](int i) -> float {
+      if (BF16) return (i & 1) ? bf16_hi(w[i >> 1]) : bf16_lo(w[i >> 1]);
+      return __uint_as_float(w[i]);
+    };
+    constexpr int NE = BF16 ? 2 * NW : NW;  // elements per thread per chunk
+
+    // chunk maximum of this thread (-inf pads never exceed a real logit)
+    float mc;
+    if (BF16) {
+      __nv_bfloat162 m2 = *(const __nv_bfloat162*)&w[0];
+#pragma unroll
+      for (int j = 1; j < NW; ++j) m2 = __hmax2(m2, *(const __nv_bfloat162*)&w[j]);
+      mc = fmaxf(__low2float(m2), __high2float(m2));
+    } else {
+      mc = __uint_as_float(w[0]);
+#pragma unroll
+      for (int j = 1; j < NW; ++j) mc = fmaxf(mc, __uint_as_float(w[j]));
+    }
+    // running (max, sum of 2^((z - max) * c)), two logits per packed instruction
+    if (mc > m) {
+      if (m != -INFINITY) s *= ex2((m - mc) * p.c);
+      m = mc;
+    }
+    if (m != -INFINITY) {
+      const uint64_t c2 = pack2(p.c, p.c), nm2 = pack2(-m * p.c, -m * p.c);
+      uint64_t acc[2] = {pack2(0.f, 0.f), pack2(0.f, 0.f)};
+#pragma unroll
+      for (int i = 0; i < NE; i += 2) {
+        const uint64_t x2 = ffma2(pack2(value_of(i), value_of(i + 1)), c2, nm2);
+        float xa, xb;
+        unpack2(x2, xa, xb);
+        acc[(i >> 1) & 1] = fadd2(acc[(i >> 1) & 1], pack2(ex2(xa), ex2(xb)));
+      }
+      float a0, a1, b0, b1;
+      unpack2(acc[0], a0, a1);
+      unpack2(acc[1], b0, b1);
+      s += (a0 + a1) + (b0 + b1);
+    }
+
+    if (first) {
+      // a threshold k logits of this chunk reach: the k-th largest lane
+      // maximum of the best warp (exact 64-bit keys)
+      uint64_t kmax = 0;
+#pragma unroll
+      for (int i = 0; i < NE; ++i) {
+        const int idx = index_of(i);
+        if (idx < p.V) {
+          const uint64_t key = cand_key(value_of(i), (uint32_t)idx);
+          kmax = key > kmax ? key : kmax;
+        }
+      }
+      const uint64_t tw = warp_kth_key(kmax, p.k);
+      const uint64_t t0 = block_max_u64(tw, sm.red);  // barriers
+      if (tid == 0) sm.count = 0;
+      __syncthreads();
+      if (kmax >= t0 || t0 == 0) {
+#pragma unroll
+        for (int i = 0; i < NE; ++i) {
+          const int idx = index_of(i);
+          if (idx >= p.V) continue;
+          const uint64_t key = cand_key(value_of(i), (uint32_t)idx);
+          if (key >= t0) {
+            const int pos = atomicAdd(&sm.count, 1);
+            if (pos < kCandCap) sm.cand[pos] = key;
+          }
+        }
+      }
+      __syncthreads();
+      const int n = sm.count;
+      if (tid < DDT_TOPK_K_MAX) sm.top2[tid] = 0;
+      __syncthreads();
+      if (n <= kCandCap) {
+        rank_select2(sm.cand, n, nullptr, 0, p.k, sm.top2);
+      } else {
+        // degenerate chunk: k rounds of block-wide argmax below the previous pick
+        uint64_t prev = ~0ull;
+        for (int r = 0; r < p.k; ++r) {
+          uint64_t best = 0;
+#pragma unroll
+          for (int i = 0; i < NE; ++i) {
+            const int idx = index_of(i);
+            if (idx >= p.V) continue;
+            const uint64_t key = cand_key(value_of(i), (uint32_t)idx);
+            if (key < prev && key > best) best = key;
+          }
+          best = block_max_u64(best, sm.red);
+          if (tid == 0) sm.top2[r] = best;
+          prev = best;
+        }
+      }
+      __syncthreads();
+      if (tid < DDT_TOPK_K_MAX) sm.top[tid] = sm.top2[tid];
+      __syncthreads();
+      tau = sm.top[p.k - 1];
+      first = false;
+    } else {
+      // later chunks: only logits beating the current k-th best key (a
+      // logit equal to its value comes later, so it ranks below it)
+      const bool need = tau == 0 || mc > key_val(tau);
+      if (__syncthreads_or(need)) {
+        if (tid == 0) sm.count = 0;
+        __syncthreads();
+        if (need) {
+#pragma unroll
+          for (int i = 0; i < NE; ++i) {
+            const int idx = index_of(i);
+            if (idx >= p.V) continue;
+            const uint64_t key = cand_key(value_of(i), (uint32_t)idx);
+            if (key > tau) {
+              const int pos = atomicAdd(&sm.count, 1);
+              if (pos < kCandCap) sm.cand[pos] = key;
+            }
+          }
+        }
+        if (tid < DDT_TOPK_K_MAX) sm.top2[tid] = 0;
+        __syncthreads();
+        const int n = sm.count;
+        if (n <= kCandCap) {
+          rank_select2(sm.top, p.k, sm.cand, n, p.k, sm.top2);
+        } else {
+          // degenerate: the previous k best and this chunk, k rounds of argmax
+          uint64_t prev = ~0ull;
+          for (int r = 0; r < p.k; ++r) {
+            uint64_t best = 0;
+            for (int i = tid; i < p.k; i += kThreads) {
+              const uint64_t key = sm.top[i];
+              if (key < prev && key > best) best = key;
+            }
+#pragma unroll
+            for (int i = 0; i < NE; ++i) {
+              const int idx = index_of(i);
+              if (idx >= p.V) continue;
+              const uint64_t key = cand_key(value_of(i), (uint32_t)idx);
+              if (key < prev && key > best) best = key;
+            }
+            best = block_max_u64(best, sm.red);
+            if (tid == 0) sm.top2[r] = best;
+            prev = best;
+          }
+        }
+        __syncthreads();
+        if (tid < DDT_TOPK_K_MAX) sm.top[tid] = sm.top2[tid];
+        __syncthreads();
+        tau = sm.top[p.k - 1];
+      }
+    }
+
+    // end of this CTA's part of the row: publish it (or finish the row)
+    if (cidx == p.S - 1 || ch == c_hi - 1) {
+      float M = m, Ssum = s;
+      block_ms_reduce(M, Ssum, p.c, sm.wm, sm.wsum);
+      const int64_t g_first = owner_of((int64_t)row * p.S, p.T, p.G);
+      const int64_t g_last = owner_of((int64_t)row * p.S + p.S - 1, p.T, p.G);
+      if (g_first == g_last) {
+        write_row(p, row, sm.top, row_lse_up(p.inv_t, M, Ssum));
+      } else {
+        const int slot_p = (int)(blockIdx.x - g_first);
+        const int64_t pb = (int64_t)row * p.pmax + slot_p;
+        for (int r = tid; r < p.k; r += kThreads) p.part_keys[pb * p.k + r] = sm.top[r];
+        if (tid == 0) p.part_ms[pb] = make_float2(M, Ssum);
+        __threadfence();
+        __syncthreads();
+        const int np = (int)(g_last - g_first + 1);
+        if (tid == 0) sm.last = (atomicAdd(&p.tickets[row], 1u) == (unsigned)(np - 1));
+        __syncthreads();
+        if (sm.last) {
+          __threadfence();
+          // every partial's keys and (max, sum) in one round of loads, then
+          // the row's k best ranked directly
+          const int tot = np * p.k;
+          float Mr = -INFINITY, Sr = 0.f;
+          for (int cc = tid; cc < np; cc += kThreads) {
+            const float2 ms = ld_cg_f2(&p.part_ms[(int64_t)row * p.pmax + cc]);
+            ms_merge(Mr, Sr, ms.x, ms.y, p.c);
+          }
+          if (tid == 0) sm.count = 0;
+          if (tot <= kCandCap) {
+            for (int i = tid; i < tot; i += kThreads)
+              sm.cand[i] = ld_cg_u64(&p.part_keys[(int64_t)row * p.pmax * p.k + i]);
+          } else {
+            // many partials: each has k keys at or above its k-th, so the
+            // largest k-th key bounds the row's k-th from below
+            uint64_t t = 0;
+            for (int cc = tid; cc < np; cc += kThreads) {
+              const uint64_t kk = ld_cg_u64(&p.part_keys[((int64_t)row * p.pmax + cc) * p.k + p.k - 1]);
+              t = kk > t ? kk : t;
+            }
+            t = block_max_u64(t, sm.red);
+            for (int i = tid; i < tot; i += kThreads) {
+              const uint64_t key = ld_cg_u64(&p.part_keys[(int64_t)row * p.pmax * p.k + i]);
+              if (key != 0 && key >= t) {
+                const int pos = atomicAdd(&sm.count, 1);
+                if (pos < kCandCap) sm.cand[pos] = key;
+              }
+            }
+          }
+          if (tid < DDT_TOPK_K_MAX) sm.top2[tid] = 0;
+          block_ms_reduce(Mr, Sr, p.c, sm.wm, sm.wsum);  // its barriers publish cand / count
+          const int n = tot <= kCandCap ? tot : sm.count;
+          rank_select2(sm.cand, min(n, kCandCap), nullptr, 0, p.k, sm.top2);
+          __syncthreads();
+          write_row(p, row, sm.top2, row_lse_up(p.inv_t, Mr, Sr));
+          if (tid == 0) p.tickets[row] = 0u;  // the counter region is left zero
+        }
+      }
+      __syncthreads();
+      m = -INFINITY;
+      s = 0.f;
+      tau = 0;
+      first = true;
+      if (tid < DDT_TOPK_K_MAX) sm.top[tid] = 0;
+      __syncthreads();
+    }
   }
-  __syncthreads();
-  write_row(p, row, s_top, row_lse_up(p.inv_t, M, Ssum));
-  if (tid == 0) p.tickets[row] = 0u;  // the counter region is left zero
+  cp_async_wait<0>();
 }
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// CTAs the device runs at once (per SM, from the occupancy calculator).
+int ctas_per_sm(bool bf16) {
+  static std::mutex mu;
+  static int known[2] = {0, 0};
+  std::lock_guard<std::mutex> lock(mu);
+  int& n = known[bf16 ? 1 : 0];
+  if (n == 0) {
+    const void* fn = bf16 ? (const void*)topk_kernel<true> : (const void*)topk_kernel<false>;
+    const size_t smem = (size_t)kStages * kChunkBytes;
+    int v = 0;
+    if (ensure_smem_attr(fn, smem) == cudaSuccess &&
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, fn, kThreads, smem) == cudaSuccess && v > 0)
+      n = v;
+    else
+      n = 1;
+    cudaGetLastError();  // a failed query must not leave a sticky error behind
+  }
+  return n;
+}
+
+struct Plan {
+  int S, G, pmax;
+  int64_t T;
+};
+
+Plan plan_for(int rows, int V, int es, bool bf16) {
+  Plan pl;
+  const int epc = kChunkBytes / es;
+  pl.S = (V + epc - 1) / epc;
+  pl.T = (int64_t)rows * pl.S;
+  const int64_t slots = (int64_t)device_sm_count() * ctas_per_sm(bf16);
+  pl.G = (int)(pl.T < slots ? pl.T : slots);
+  if (pl.G < 1) pl.G = 1;
+  // the CTAs a row's chunks can span: CTAs hold floor or ceil of T/G chunks
+  // each, so those wholly inside a row number fewer than (S + 1) G / T
+  pl.pmax = (int)(((int64_t)pl.S + 1) * pl.G / (pl.T > 0 ? pl.T : 1)) + 3;
+  return pl;
+}
+
 }  // namespace
 
 size_t topk_workspace_size(int rows, int V, int k) {
-  const int S = (V + kChunk - 1) / kChunk;
-  if (S <= 1) return 0;
-  return (size_t)DDT_WS_COUNTER_BYTES + align256(sizeof(float2) * (size_t)rows * S) +
-         align256(sizeof(uint64_t) * (size_t)rows * S * k);
+  // bf16 rows have half as many chunks; size for the larger (f32) plan
+  const Plan pl = plan_for(rows, V, 4, false);
+  const Plan pb = plan_for(rows, V, 2, true);
+  const int pmax = pl.pmax > pb.pmax ? pl.pmax : pb.pmax;
+  if (pl.S <= 1 && pb.S <= 1) return 0;
+  return (size_t)DDT_WS_COUNTER_BYTES + align256(sizeof(float2) * (size_t)rows * pmax) +
+         align256(sizeof(uint64_t) * (size_t)rows * pmax * k);
 }
 
 ddt_status launch_topk(const void* logits, ddt_dtype dt, int rows, int V, int64_t row_stride,
                        int k, float inv_t, int32_t* ids, float* zk, float* logp, float* lse,
                        void* ws, size_t ws_bytes, cudaStream_t stream) {
+  (void)ws_bytes;
+  if (rows == 0) return DDT_OK;
+  const bool bf16 = dt == DDT_BF16;
+  const int es = bf16 ? 2 : 4;
+  const Plan pl = plan_for(rows, V, es, bf16);
+  // the workspace is sized for the larger of the two dtypes' plans
+  const Plan pf = plan_for(rows, V, 4, false), pb = plan_for(rows, V, 2, true);
   TopkParams p;
   p.logits = logits;
+  p.rows = rows;
   p.V = V;
   p.row_stride = row_stride;
   p.k = k;
   p.inv_t = inv_t;
   p.c = inv_t * kLog2e;
-  p.S = (V + kChunk - 1) / kChunk;
-  const int es = dt == DDT_BF16 ? 2 : 4;
+  p.S = pl.S;
+  p.G = pl.G;
+  p.T = pl.T;
+  p.pmax = pf.pmax > pb.pmax ? pf.pmax : pb.pmax;
   p.vec_ok = ((uintptr_t)logits % 16 == 0) && ((row_stride * es) % 16 == 0);
   char* w = (char*)ws;
   p.tickets = (unsigned*)w;  // counter region: one ticket per row
-  w += DDT_WS_COUNTER_BYTES;
+  if (w) w += DDT_WS_COUNTER_BYTES;
   p.part_ms = (float2*)w;
-  w += align256(sizeof(float2) * (size_t)rows * p.S);
+  if (w) w += align256(sizeof(float2) * (size_t)rows * p.pmax);
   p.part_keys = (uint64_t*)w;
   p.ids = ids;
   p.zk = zk;
   p.logp = logp;
   p.lse = lse;
-  if (rows == 0) return DDT_OK;
-  dim3 grid(p.S, rows);
-  // many waves of chunks: the higher-occupancy build; a few: the spill-free one
-  const bool many = (long)p.S * rows > 4L * 3 * device_sm_count();
-  cudaError_t e;
-  if (dt == DDT_BF16)
-    e = many ? launch_pdl(topk_kernel<true, 4>, grid, dim3(kThreads), 0, stream, 0, p)
-             : launch_pdl(topk_kernel<true, 3>, grid, dim3(kThreads), 0, stream, 0, p);
-  else
-    e = many ? launch_pdl(topk_kernel<false, 4>, grid, dim3(kThreads), 0, stream, 0, p)
-             : launch_pdl(topk_kernel<false, 3>, grid, dim3(kThreads), 0, stream, 0, p);
+  const size_t smem = (size_t)kStages * kChunkBytes;
+  const void* fn = bf16 ? (const void*)topk_kernel<true> : (const void*)topk_kernel<false>;
+  if (ensure_smem_attr(fn, smem) != cudaSuccess) return DDT_ERR_CUDA;
+  const cudaError_t e =
+      bf16 ? launch_pdl(topk_kernel<true>, dim3(pl.G), dim3(kThreads), smem, stream, 0, p)
+           : launch_pdl(topk_kernel<false>, dim3(pl.G), dim3(kThreads), smem, stream, 0, p);
   return e == cudaSuccess ? DDT_OK : DDT_ERR_CUDA;
 }
 

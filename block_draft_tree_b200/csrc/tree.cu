@@ -33,6 +33,8 @@
 // carries its path of candidate ranks as a packed key and its row is its
 // rank by key within its depth, so no level-by-level pass is needed; the
 // ancestor masks follow the parent rows.
+#include <climits>
+
 #include "common.cuh"
 #include "launch.h"
 
@@ -730,7 +732,34 @@ __global__ void __launch_bounds__(kThreads, 1) build_tree_kernel(TreeParams p) {
     s.ninv[0] = 0;
   }
   if (tid < L + 2) red.lvl[tid] = tid == 0 ? 1 : 0;
+  __shared__ int s_emax, s_emin;
+  if (tid == 0) {
+    s_emax = INT_MIN;
+    s_emin = INT_MAX;
+  }
   __syncthreads();
+  // Siblings are taken in candidate order, which is K only while every fp64
+  // sum of logits along a path is exact: then two children of one node
+  // compare as their own logits do.  With f32 logits that holds when the
+  // binary exponents of the nonzero finite candidates span at most
+  // 29 - ceil(log2 L) (24-bit significands inside a 53-bit sum of L terms).
+  {
+    int emax = INT_MIN, emin = INT_MAX;
+    for (int i = tid; i < L * k; i += kThreads) {
+      const uint32_t u = __float_as_uint(p.zk[(int64_t)b * L * k + i]);
+      const int ef = (int)((u >> 23) & 0xFFu);
+      if (ef == 0xFF || (u & 0x7FFFFFFFu) == 0) continue;  // inf, nan, +-0: exact in any sum
+      const int e = ef == 0 ? -126 : ef - 127;             // subnormals: lowest bit 2^-149
+      emax = max(emax, e);
+      emin = min(emin, e);
+    }
+    emax = __reduce_max_sync(kFull, emax);
+    emin = __reduce_min_sync(kFull, emin);
+    if ((tid & 31) == 0 && emax != INT_MIN) {
+      atomicMax(&s_emax, emax);
+      atomicMin(&s_emin, emin);
+    }
+  }
   // id ranks: within a position, token order is id-rank order
   for (int i = tid; i < L * k; i += kThreads) {
     const int t = i / k, tok = s.tt[i];
@@ -761,6 +790,8 @@ __global__ void __launch_bounds__(kThreads, 1) build_tree_kernel(TreeParams p) {
     Bb = min(max(Bb, 0), p.B_max);
   }
   __syncthreads();
+  if (tid == 0 && s_emax != INT_MIN && s_emax - s_emin > 29 - (32 - __clz(L - 1 > 0 ? L - 1 : 0)))
+    raise_status(p.status, DDT_ERR_UNSUPPORTED);  // path sums may round: the order may differ
 
   // ---------------- selection ----------------
   // ncnt[x] (in nrow, free until numbering): the items of x's run taken

@@ -30,11 +30,15 @@
 // the pairs, finds the chunk whose cumulative weight first exceeds u times
 // the total, and rescans that one chunk (from L2) with a block prefix sum
 // to find the token.  Each weight is an fp32 evaluation of 2^(t - R),
-// t = z*log2(e)/T, that is exact in fp64 by construction (see draw_weight),
+// t = z*log2(e)/T (with the rounding of t added back), that is exact in
+// fp64 by construction (see draw_weight),
 // so weights against different references differ by exact powers of two
 // and only the fp64 sums round: the draws land on tokens of probability
 // ~1/V, where an fp32 cumulative sum (~1e-7 relative error) would move a
 // fair share of them to a neighbour.
+#include <climits>
+#include <cmath>
+
 #include "common.cuh"
 #include "launch.h"
 
@@ -56,7 +60,7 @@ struct WalkParams {
   unsigned* seq_count;   // [batch]
   unsigned* draw_count;  // sampling with a step counter: rows drawn so far
   int32_t* status;
-  float a;               // sampling: fl32(log2(e) / T)
+  float a, a_lo;         // sampling: fl32(log2(e) / T) and fl32 of the rest
   uint64_t seed, step;   // sampling: Philox key
   uint64_t* step_counter;  // sampling: optional device word added to step, advanced per call
 };
@@ -217,18 +221,22 @@ __device__ __forceinline__ double row_uniform(const WalkParams& p, int b, int j)
 }
 
 // The draw's weights.  The token is an integer decided by floating point,
-// so its arithmetic is fixed exactly: a = fl32(invT * log2 e),
-// t = fl32(a * z), k = nearest integer to t (ties to even), r = t - k,
-// P = fp32 Horner evaluation with fused multiply-adds of the degree-7
-// Taylor polynomial of 2^r (coefficients (ln 2)^i / i! rounded to fp32),
-// and w = P * 2^(k - R), an exact normal fp32 number, for an integer
-// reference R >= k (0 when k - R < -120 or z = -inf).  Weights taken
-// against different references differ by exact powers of two, so every
-// chunk and thread sums against its own maximum and the sums merge without
-// rounding the weights again.  A thread sums its 32 weights as two
-// double-float sums of 16 (an exact TwoSum per term; the low part, below
-// 2^-20 of the high part, rounds at 2^-24 of itself per term: relative
-// error below 2^-40), and everything after that is fp64.
+// so its arithmetic is fixed exactly.  With A = log2(e)/T, a = fl32(A) and
+// a_lo = fl32(A - a): t = fl32(a*z), k = nearest integer to t (ties to
+// even), r = t - k (exact), P = fp32 Horner evaluation with fused
+// multiply-adds of the degree-7 Taylor polynomial of 2^r (coefficients
+// (ln 2)^i / i! rounded to fp32), then P += P * ln2 * e with
+// e = fma(a_lo, z, fma(a, z, -t)), the part of A*z that t lost (an exact
+// residual plus the rounding of A), and w = P * 2^(k - R), an exact normal
+// fp32 number, for an integer reference R >= k (0 when k - R < -120 or
+// z = -inf).  So a weight's error is the polynomial's (a few fp32 ulps) and
+// does not grow with |A*z|.  Weights taken against different references
+// differ by exact powers of two, so every chunk and thread sums against its
+// own maximum and the sums merge without rounding the weights again.  A
+// thread sums its 32 weights as two double-float sums of 16 (an exact
+// TwoSum per term; the low part, below 2^-20 of the high part, rounds at
+// 2^-24 of itself per term: relative error below 2^-40), and everything
+// after that is fp64.
 __device__ __forceinline__ float draw_poly(float r) {
   float p = 0x1.ffcbfcp-17f;
   p = fmaf(p, r, 0x1.430912p-13f);
@@ -243,25 +251,33 @@ __device__ __forceinline__ float draw_poly(float r) {
 constexpr float kRoundShift = 12582912.0f;  // 1.5 * 2^23: t + shift rounds t to an integer
 constexpr int kRoundShiftBits = 0x4B400000;
 constexpr int kNoRef = -(1 << 30);          // reference of a thread with no finite logit
+constexpr float kLn2f = 0.693147182f;       // ln 2 rounded to fp32
 
 // R = nearest integer to t (|t| < 2^22).
 __device__ __forceinline__ int draw_ref(float t) {
   return t >= -4.0e6f ? __float_as_int(__fadd_rn(t, kRoundShift)) - kRoundShiftBits : kNoRef;
 }
 
-// w = P(t - k) * 2^(k - R), with t = a*z already rounded to fp32 and
-// R >= -4e6.  Branch free: for t below -2^22 (and -inf) the rounding trick
-// yields an exponent far below R - 120, so the final select discards it.
-__device__ __forceinline__ float draw_weight(float t, int R) {
+// The weight of logit z against the reference R >= -4e6.  Branch free: for
+// t below -2^22 (and -inf) the rounding trick yields an exponent far below
+// R - 120, so the final select discards it (with whatever the correction
+// made of it).
+__device__ __forceinline__ float draw_weight(float z, float a, float a_lo, int R) {
+  const float t = __fmul_rn(a, z);
+  const float e_lo = __fmaf_rn(a_lo, z, __fmaf_rn(a, z, -t));
   const float sh = __fadd_rn(t, kRoundShift);
   const int e = __float_as_int(sh) - (kRoundShiftBits + R);
   const float r = __fsub_rn(t, __fsub_rn(sh, kRoundShift));
-  const float w = __int_as_float(__float_as_int(draw_poly(r)) + (e << 23));
+  float P = draw_poly(r);
+  P = __fmaf_rn(P, __fmul_rn(e_lo, kLn2f), P);
+  const float w = __int_as_float(__float_as_int(P) + (e << 23));
   return e >= -120 ? w : 0.f;
 }
 
-// The weights of a pair of arguments t (packed), as draw_weight.
-__device__ __forceinline__ uint64_t draw_weight2(uint64_t t2, int R) {
+// The weights of a pair of logits z (packed), as draw_weight.
+__device__ __forceinline__ uint64_t draw_weight2(uint64_t z2, uint64_t a2, uint64_t alo2, int R) {
+  const uint64_t t2 = fmul2(a2, z2);
+  const uint64_t e2 = ffma2(alo2, z2, ffma2(a2, z2, t2 ^ 0x8000000080000000ull));
   const uint64_t sh2 = fadd2(t2, pack2(kRoundShift, kRoundShift));
   const uint64_t r2 = fsub2(t2, fadd2(sh2, pack2(-kRoundShift, -kRoundShift)));
   uint64_t p2 = ffma2(pack2(0x1.ffcbfcp-17f, 0x1.ffcbfcp-17f), r2, pack2(0x1.430912p-13f, 0x1.430912p-13f));
@@ -271,6 +287,7 @@ __device__ __forceinline__ uint64_t draw_weight2(uint64_t t2, int R) {
   p2 = ffma2(p2, r2, pack2(0x1.ebfbep-3f, 0x1.ebfbep-3f));
   p2 = ffma2(p2, r2, pack2(0x1.62e43p-1f, 0x1.62e43p-1f));
   p2 = ffma2(p2, r2, pack2(1.f, 1.f));
+  p2 = ffma2(p2, fmul2(e2, pack2(kLn2f, kLn2f)), p2);
   float sa, sb, pa, pb;
   unpack2(sh2, sa, sb);
   unpack2(p2, pa, pb);
@@ -315,7 +332,7 @@ __device__ __forceinline__ void rs_add(int& R, double& s, int R2, double s2) {
 // tokens per packed instruction.  The thread's 32 weights are summed as two
 // interleaved double-float sums of 16.
 template <bool BF16>
-__device__ __forceinline__ void rs_chunk(const Chunk<BF16>& c, float a, int& R, double& s) {
+__device__ __forceinline__ void rs_chunk(const Chunk<BF16>& c, float a, float a_lo, int& R, double& s) {
   float zm = -INFINITY;
 #pragma unroll
   for (int q = 0; q < Chunk<BF16>::VPT; ++q) {
@@ -333,7 +350,7 @@ __device__ __forceinline__ void rs_chunk(const Chunk<BF16>& c, float a, int& R, 
   R = draw_ref(__fmul_rn(a, zm));  // fl32(a*z) is monotone in z
   s = 0.0;
   if (R == kNoRef) return;
-  const uint64_t a2 = pack2(a, a);
+  const uint64_t a2 = pack2(a, a), alo2 = pack2(a_lo, a_lo);
   uint64_t hi = pack2(0.f, 0.f), lo = pack2(0.f, 0.f);
 #pragma unroll
   for (int q = 0; q < Chunk<BF16>::VPT; ++q) {
@@ -341,11 +358,11 @@ __device__ __forceinline__ void rs_chunk(const Chunk<BF16>& c, float a, int& R, 
     if (BF16) {
 #pragma unroll
       for (int i = 0; i < 4; ++i)
-        two_sum_add2(hi, lo, draw_weight2(fmul2(a2, pack2(bf16_lo(w[i]), bf16_hi(w[i]))), R));
+        two_sum_add2(hi, lo, draw_weight2(pack2(bf16_lo(w[i]), bf16_hi(w[i])), a2, alo2, R));
     } else {
 #pragma unroll
       for (int i = 0; i < 4; i += 2)
-        two_sum_add2(hi, lo, draw_weight2(fmul2(a2, pack2(__uint_as_float(w[i]), __uint_as_float(w[i + 1]))), R));
+        two_sum_add2(hi, lo, draw_weight2(pack2(__uint_as_float(w[i]), __uint_as_float(w[i + 1])), a2, alo2, R));
     }
   }
   float ha, hb, la, lb;
@@ -469,7 +486,7 @@ __device__ int sample_row_token(const WalkParams& p, int b, int j, int64_t row, 
   if (cstar < 0) return 0;  // no finite logit in the row
   const int R = sm.R;
   const double theta = sm.theta;
-  const float a = p.a;
+  const float a = p.a, a_lo = p.a_lo;
   // each thread owns kPer consecutive tokens of chunk cstar
   constexpr int kPer = kChunk / kThreads;
   const int e0 = cstar * kChunk + tid * kPer;
@@ -477,7 +494,7 @@ __device__ int sample_row_token(const WalkParams& p, int b, int j, int64_t row, 
   double local = 0.0;
   int last = -1;
   for (int i = e0; i < e1; ++i) {
-    const double w = (double)draw_weight(__fmul_rn(a, load_logit(rowp, i, BF16)), R);
+    const double w = (double)draw_weight(load_logit(rowp, i, BF16), a, a_lo, R);
     local += w;
     if (w > 0.0) last = i;
   }
@@ -495,7 +512,7 @@ __device__ int sample_row_token(const WalkParams& p, int b, int j, int64_t row, 
     double cum = base;
     int hit = last;
     for (int i = e0; i < e1; ++i) {
-      cum += (double)draw_weight(__fmul_rn(a, load_logit(rowp, i, BF16)), R);
+      cum += (double)draw_weight(load_logit(rowp, i, BF16), a, a_lo, R);
       if (cum > theta) {
         hit = i;
         break;
@@ -543,15 +560,15 @@ __global__ void __launch_bounds__(kThreads) walk_kernel(WalkParams p) {
       Chunk<BF16> cur;
       if (c0 + kChunk <= p.V) load_chunk<BF16>(cur, rowp, c0);
       else load_chunk_tail<BF16>(cur, rowp, c0, p.V);
-      rs_chunk<BF16>(cur, p.a, R, sum);
+      rs_chunk<BF16>(cur, p.a, p.a_lo, R, sum);
     } else {
       for (int q = 0; q < Chunk<BF16>::VPT; ++q)
         for (int i = 0; i < EPV; ++i) {
           const int idx = c0 + (q * kThreads + tid) * EPV + i;
           if (idx >= p.V) continue;
-          const float t = __fmul_rn(p.a, load_logit(rowp, idx, BF16));
-          const int Rv = draw_ref(t);
-          rs_add(R, sum, Rv, Rv == kNoRef ? 0.0 : (double)draw_weight(t, Rv));
+          const float z = load_logit(rowp, idx, BF16);
+          const int Rv = draw_ref(__fmul_rn(p.a, z));
+          rs_add(R, sum, Rv, Rv == kNoRef ? 0.0 : (double)draw_weight(z, p.a, p.a_lo, Rv));
         }
     }
     pdl_trigger();
@@ -639,6 +656,229 @@ __global__ void __launch_bounds__(kThreads) walk_kernel(WalkParams p) {
   if (tid == 0) p.seq_count[b] = 0u;  // the counter region is left zero
 }
 
+// ---------------------------------------------------------------------------
+// Path-only walk
+// ---------------------------------------------------------------------------
+// The walk only ever needs the argmax of the rows it visits: the root and
+// the accepted rows, acc_len + 1 <= L + 1 of them, against every row of the
+// tree for the all-rows scan.  The path-only walk reads just those rows, at
+// the price of one dependent row after another.  One thread-block cluster
+// walks one sequence: every step, each CTA of the cluster takes the argmax
+// of its slice of the current row (16-byte streaming loads, all issued
+// before any is used), the CTAs exchange their 64-bit (value, smaller id)
+// keys through distributed shared memory with one cluster barrier, and
+// every CTA then finds the same child to descend to in its own copy of the
+// tree.  The CTAs take the same decisions on the same data, so every one of
+// them meets the same number of barriers.
+constexpr int kLazyThreads = 512;
+constexpr int kLazyBatch = 8;  // 16-byte vectors in flight per thread per pass
+constexpr int kLazyMaxCluster = 16;
+
+__device__ __forceinline__ uint32_t lz_cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void lz_cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Store a 64-bit key into the shared memory of CTA `rank` of the cluster.
+__device__ __forceinline__ void st_cluster_u64(uint64_t* local, uint32_t rank, uint64_t v) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
+               : "=r"(remote)
+               : "r"((uint32_t)__cvta_generic_to_shared(local)), "r"(rank));
+  asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(remote), "l"(v) : "memory");
+}
+
+// Argmax key of elements [e0, e1) of a row (e0 a multiple of the vector
+// width); each thread visits its indices in increasing order, so a strict >
+// keeps the smallest index among equal values.
+template <bool BF16>
+__device__ __forceinline__ uint64_t lazy_slice_key(const char* rowp, int e0, int e1, int V,
+                                                   bool vec_ok) {
+  constexpr int EPV = BF16 ? 8 : 4, ES = BF16 ? 2 : 4;
+  float bv = -INFINITY;
+  int bi = -1;
+  if (vec_ok) {
+    const int nvec = (e1 - e0 + EPV - 1) / EPV;
+    for (int v0 = 0; v0 < nvec; v0 += kLazyBatch * kLazyThreads) {
+      uint4 buf[kLazyBatch];
+#pragma unroll
+      for (int q = 0; q < kLazyBatch; ++q) {
+        const int v = v0 + q * kLazyThreads + (int)threadIdx.x;
+        const int idx = e0 + v * EPV;
+        if (v < nvec && idx + EPV <= V) buf[q] = ld_stream_v4(rowp + (int64_t)idx * ES);
+      }
+#pragma unroll
+      for (int q = 0; q < kLazyBatch; ++q) {
+        const int v = v0 + q * kLazyThreads + (int)threadIdx.x;
+        const int idx = e0 + v * EPV;
+        if (v >= nvec) continue;
+        if (idx + EPV <= V) {
+          const uint32_t w[4] = {buf[q].x, buf[q].y, buf[q].z, buf[q].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            if (BF16) {
+              const float lo = bf16_lo(w[e]), hi = bf16_hi(w[e]);
+              if (lo > bv || bi < 0) { bv = lo; bi = idx + 2 * e; }
+              if (hi > bv) { bv = hi; bi = idx + 2 * e + 1; }
+            } else {
+              const float f = __uint_as_float(w[e]);
+              if (f > bv || bi < 0) { bv = f; bi = idx + e; }
+            }
+          }
+        } else {  // the vector that straddles V: element loads inside the row only
+          for (int i = idx; i < min(idx + EPV, e1); ++i) {
+            const float f = BF16 ? bf16_to_f32(((const uint16_t*)rowp)[i]) : ((const float*)rowp)[i];
+            if (f > bv || bi < 0) { bv = f; bi = i; }
+          }
+        }
+      }
+    }
+  } else {
+    for (int i = e0 + (int)threadIdx.x; i < e1; i += kLazyThreads) {
+      const float f = BF16 ? bf16_to_f32(((const uint16_t*)rowp)[i]) : ((const float*)rowp)[i];
+      if (f > bv || bi < 0) { bv = f; bi = i; }
+    }
+  }
+  return bi < 0 ? 0ull : cand_key(bv, (uint32_t)bi);
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(kLazyThreads) walk_lazy_kernel(WalkParams p, int slice) {
+  constexpr int ES = BF16 ? 2 : 4;
+  __shared__ uint64_t s_keys[2][kLazyMaxCluster];
+  __shared__ uint64_t s_red[kLazyThreads / 32];
+  __shared__ int s_tok[DDT_TREE_B_MAX + 1], s_first[DDT_TREE_B_MAX + 1], s_cnt[DDT_TREE_B_MAX + 1];
+  __shared__ int s_dep[DDT_TREE_B_MAX + 1];
+  __shared__ int s_next, s_t;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int b = blockIdx.y;
+  const uint32_t rank = lz_cluster_rank();
+  const int csize = (int)gridDim.x;
+  pdl_wait();
+  pdl_trigger();
+  int n = p.n_nodes[b];
+  if (n < 1 || n > p.n_max) {
+    if (rank == 0 && tid == 0) raise_status(p.status, DDT_ERR_INVALID_ARG);
+    n = min(max(n, 1), p.n_max);
+  }
+  // the tree, with each row's first child and child count (rows are
+  // breadth-first, so a row's children are consecutive)
+  for (int r = tid; r < n; r += kLazyThreads) {
+    s_tok[r] = p.tok[(int64_t)b * p.n_max + r];
+    s_dep[r] = p.depth[(int64_t)b * p.n_max + r];
+    s_first[r] = INT_MAX;
+    s_cnt[r] = 0;
+  }
+  __syncthreads();
+  for (int r = 1 + tid; r < n; r += kLazyThreads) {
+    const int par = p.parent[(int64_t)b * p.n_max + r];
+    if (par >= 0 && par < r) {
+      atomicMin(&s_first[par], r);
+      atomicAdd(&s_cnt[par], 1);
+    }
+  }
+  __syncthreads();
+  const int e0 = (int)rank * slice, e1 = min(p.V, e0 + slice);
+  int x = 0, a = 0, t = 0;
+#pragma unroll 1
+  for (int step = 0;; ++step) {
+    const char* rowp = (const char*)p.logits + ((int64_t)b * p.n_max + x) * p.row_stride * ES;
+    uint64_t key = e0 < e1 ? lazy_slice_key<BF16>(rowp, e0, e1, p.V, p.vec_ok) : 0ull;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const uint64_t u = shfl_xor_u64(key, o);
+      key = u > key ? u : key;
+    }
+    if (lane == 0) s_red[warp] = key;
+    __syncthreads();
+    if (warp == 0) {
+      uint64_t k2 = lane < kLazyThreads / 32 ? s_red[lane] : 0ull;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const uint64_t u = shfl_xor_u64(k2, o);
+        k2 = u > k2 ? u : k2;
+      }
+      if (lane < csize) st_cluster_u64(&s_keys[step & 1][rank], (uint32_t)lane, k2);
+    }
+    lz_cluster_sync();
+    if (warp == 0) {
+      uint64_t k2 = lane < csize ? s_keys[step & 1][lane] : 0ull;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const uint64_t u = shfl_xor_u64(k2, o);
+        k2 = u > k2 ? u : k2;
+      }
+      const int tt = (int)key_id(k2);
+      int next = -1;
+      if (a < p.L && s_dep[x] < p.L && s_cnt[x] > 0) {
+        for (int c0 = s_first[x]; c0 < s_first[x] + s_cnt[x]; c0 += 32) {
+          const int c = c0 + lane;
+          const bool hit = c < s_first[x] + s_cnt[x] && s_tok[c] == tt;
+          const unsigned bal = __ballot_sync(0xFFFFFFFFu, hit);
+          if (bal) {
+            next = c0 + __ffs(bal) - 1;
+            break;
+          }
+        }
+      }
+      if (lane == 0) {
+        s_next = next;
+        s_t = tt;
+        if (rank == 0 && next >= 0) {
+          p.acc_nodes[(int64_t)b * p.L + a] = next;
+          p.acc_tok[(int64_t)b * p.L + a] = tt;
+        }
+      }
+    }
+    __syncthreads();
+    const int next = s_next;
+    t = s_t;
+    if (next < 0) break;
+    x = next;
+    ++a;
+  }
+  if (rank == 0) {
+    for (int i = a + tid; i < p.L; i += kLazyThreads) {
+      p.acc_nodes[(int64_t)b * p.L + i] = -1;
+      p.acc_tok[(int64_t)b * p.L + i] = -1;
+    }
+    if (tid == 0) {
+      p.acc_len[b] = a;
+      p.bonus[b] = t;
+    }
+  }
+}
+
+// Largest cluster (16, else 8) of path-only walk CTAs the device can run.
+int lazy_cluster_size() {
+  static int cached = 0;
+  if (cached) return cached;
+  int best = 8;
+  auto* fn = (const void*)walk_lazy_kernel<false>;
+  auto* fn2 = (const void*)walk_lazy_kernel<true>;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess &&
+      cudaFuncSetAttribute(fn2, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(16, 1, 1);
+    cfg.blockDim = dim3(kLazyThreads, 1, 1);
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 16;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int nc = 0;
+    if (cudaOccupancyMaxActiveClusters(&nc, fn, &cfg) == cudaSuccess && nc > 0) best = 16;
+  }
+  cudaGetLastError();  // a refused query must not leave a sticky error behind
+  cached = best;
+  return best;
+}
+
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 }  // namespace
@@ -650,13 +890,35 @@ size_t walk_workspace_size(int batch, int n_max, int V) {
          align256(2 * sizeof(uint64_t) * rows * S);
 }
 
+// Path-only or all-rows for DDT_WALK_AUTO.  The all-rows scan costs its
+// bytes at the rate it reaches on B200 plus its fixed part (tickets, the
+// merge, the walk); the path-only walk costs up to L + 1 dependent steps
+// (measured per step on B200, per wave of clusters).  AUTO takes the
+// path-only walk when even its worst case (every row down to depth L
+// accepted) is the cheaper.
+constexpr double kAllRowsGBs = 6000.0, kAllRowsFixedUs = 9.0;
+constexpr double kLazyStepUs = 2.0;
+
+int walk_mode_for(int mode, ddt_dtype dt, int batch, int n_max, int V, int L) {
+  if (mode != DDT_WALK_AUTO) return mode;
+  const double bytes = (double)batch * n_max * V * (dt == DDT_BF16 ? 2 : 4);
+  const double all_us = bytes / (kAllRowsGBs * 1e3) + kAllRowsFixedUs;
+  const int csize = lazy_cluster_size();
+  const double waves = std::ceil((double)batch * csize / (2.0 * device_sm_count()));
+  const double lazy_us = (L + 1) * kLazyStepUs * waves;
+  return lazy_us < all_us ? DDT_WALK_LAZY : DDT_WALK_ALL_ROWS;
+}
+
 ddt_status launch_tree_walk(const void* logits, ddt_dtype dt, int batch, int n_max, int V,
                             int64_t row_stride, const int32_t* tok, const int32_t* parent,
-                            const int32_t* depth, const int32_t* n_nodes, int L, int32_t* acc_len,
-                            int32_t* acc_nodes, int32_t* acc_tok, int32_t* bonus, void* ws,
-                            int32_t* dev_status, cudaStream_t stream, const WalkSampling* sampling) {
+                            const int32_t* depth, const int32_t* n_nodes, int L, int mode,
+                            int32_t* acc_len, int32_t* acc_nodes, int32_t* acc_tok, int32_t* bonus,
+                            void* ws, int32_t* dev_status, cudaStream_t stream,
+                            const WalkSampling* sampling) {
   WalkParams p;
-  p.a = sampling ? (float)((double)sampling->inv_temperature * 1.4426950408889634074) : 0.f;
+  const double A = sampling ? (double)sampling->inv_temperature * 1.4426950408889634074 : 0.0;
+  p.a = (float)A;
+  p.a_lo = (float)(A - (double)p.a);
   p.seed = sampling ? sampling->seed : 0;
   p.step = sampling ? sampling->step : 0;
   p.step_counter = sampling ? sampling->step_counter : nullptr;
@@ -688,8 +950,29 @@ ddt_status launch_tree_walk(const void* logits, ddt_dtype dt, int batch, int n_m
   w += align256(sizeof(int32_t) * rows);
   p.part = (uint64_t*)w;
   if (batch == 0) return DDT_OK;
-  dim3 grid(p.S, n_max, batch);
   cudaError_t e;
+  if (!sampling && walk_mode_for(mode, dt, batch, n_max, V, L) == DDT_WALK_LAZY) {
+    const int csize = lazy_cluster_size();
+    // each CTA's slice: a multiple of 8 elements (whole 16-byte vectors)
+    const int slice = ((V + csize - 1) / csize + 7) / 8 * 8;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(csize, batch, 1);
+    cfg.blockDim = dim3(kLazyThreads, 1, 1);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = (unsigned)csize;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    e = dt == DDT_BF16 ? cudaLaunchKernelEx(&cfg, walk_lazy_kernel<true>, p, slice)
+                       : cudaLaunchKernelEx(&cfg, walk_lazy_kernel<false>, p, slice);
+    return e == cudaSuccess ? DDT_OK : DDT_ERR_CUDA;
+  }
+  dim3 grid(p.S, n_max, batch);
   if (sampling)
     e = dt == DDT_BF16 ? launch_pdl(walk_kernel<true, true>, grid, dim3(kThreads), 0, stream, 0, p)
                        : launch_pdl(walk_kernel<false, true>, grid, dim3(kThreads), 0, stream, 0, p);

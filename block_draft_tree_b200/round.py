@@ -20,7 +20,7 @@ class VerifyRound:
     """One verification round on fixed shapes.
 
     ``decode`` is the target's decoding rule in stage 4: ``"greedy"``
-    (``ddt_tree_walk`` over the bound target logits), ``"sample"``
+    (``ddt_tree_walk`` over the bound target logits, in ``walk_mode``), ``"sample"``
     (``ddt_tree_walk_sample`` at ``sample_inv_temperature`` with a device step
     counter, so that every replay of a captured round draws fresh uniforms) or
     ``"lm_head"`` (``ddt_lm_head_walk`` from the bound hidden states and LM
@@ -34,10 +34,10 @@ class VerifyRound:
                  target_dtype: torch.dtype = torch.float32, inv_temperature: float = 1.0,
                  paged: bool = False, page_size: int = 64, max_pages: int = 0,
                  decode: str = "greedy", sample_inv_temperature: float = 1.0, seed: int = 0,
-                 commit: bool = False, device: str = "cuda"):
+                 commit: bool = False, walk_mode: int = api.WALK_AUTO, device: str = "cuda"):
         if decode not in ("greedy", "sample", "lm_head"):
             raise ValueError("decode must be 'greedy', 'sample' or 'lm_head'")
-        self.decode, self.commit = decode, commit
+        self.decode, self.commit, self.walk_mode = decode, commit, int(walk_mode)
         self.sample_inv_t, self.seed = float(sample_inv_temperature), int(seed)
         self.lib = api.load_library()
         self.dev = torch.device(device)
@@ -161,7 +161,8 @@ class VerifyRound:
             if self.decode == "greedy":
                 rc = lib.ddt_tree_walk(P(x["target"]), self.target_code, self.batch, self.n_max,
                                        self.V, x["target"].stride(1), P(o["tok"]), P(o["parent"]),
-                                       P(o["depth"]), P(o["n_nodes"]), self.L, P(o["acc_len"]),
+                                       P(o["depth"]), P(o["n_nodes"]), self.L, self.walk_mode,
+                                       P(o["acc_len"]),
                                        P(o["acc_nodes"]), P(o["acc_tok"]), P(o["bonus"]),
                                        P(self.ws_walk), self.ws_walk_n, P(o["status"]), s)
                 api._check(rc, "ddt_tree_walk")

@@ -85,6 +85,18 @@ const char* ddt_status_string(ddt_status s);
 /* Number of 32-bit mask words per tree row: ceil(n_max / 32). */
 int ddt_mask_words(int n_max);
 
+/* Test hook for the timeout path.  The tensor-core kernels (ddt_tree_attn on
+ * its tensor-core paths, ddt_lm_head_walk) bound every wait on an on-chip
+ * barrier; a wait that runs out raises DDT_ERR_TIMEOUT in dev_status, after
+ * which the kernel lets its copies and MMAs in flight complete, frees its
+ * tensor memory and returns, leaving the context usable.  By default a wait
+ * gives up after about one second (2e9 clock cycles).  This call sets the
+ * bound, in clock cycles, for every later launch in the process (cycles <= 0
+ * restores the default) and returns the previous setting (0 = default).
+ * A bound of a few cycles makes the waits run out on purpose.  It is not
+ * synchronised with launches on other host threads. */
+long long ddt_debug_set_wait_limit(long long cycles);
+
 /* ------------------------------------------------------------------------
  * Stage 1: per-position softmax normaliser and top-k.
  * DDTree page, 運作流程 step 1: the drafter returns one marginal q_i per
@@ -120,13 +132,17 @@ ddt_status ddt_topk(const void* logits, ddt_dtype dtype, int batch, int L, int V
  * plan, a plug-in whose host forbids cudaMalloc), so that it cannot supply
  * the workspace ddt_topk needs.
  *
- * Same arguments, outputs and results as ddt_topk, minus the workspace.
+ * Same arguments, outputs, results and status codes as ddt_topk, minus the
+ * workspace; arguments are checked before anything is enqueued.
  * Its scratch is a fixed array in device global memory owned by libddt.so:
  * DDT_TOPK_NOALLOC_SCRATCH_BYTES on every GPU that loads the library, held
  * until the process exits.  Shapes whose ddt_topk_workspace_size exceeds it
  * are rejected with DDT_ERR_WORKSPACE before anything is launched.
- * The first call on a device (with that device current) looks up the array's
- * device address once; make that first call before any stream capture.
+ * A call made outside stream capture (with its device current) looks up the
+ * array's device address and remembers it for that device; a call made
+ * during capture uses the remembered address, so make the first call on a
+ * device before any stream capture (and capture again after a device reset,
+ * which moves the array).
  * Every call on a device shares the array; each call clears the part it uses
  * (an asynchronous memset on `stream`), so consecutive calls on one stream
  * are independent, while calls that overlap on the GPU race on the array.
@@ -168,7 +184,13 @@ ddt_status ddt_topk_noalloc(const void* logits, ddt_dtype dtype, int batch, int 
  *   surrogate double [batch] (may be NULL): sum of exp(score) over the
  *        draft nodes, the expected acceptance length under the draft.
  * ctx_len may be NULL (treated as 0).  Limits: L <= DDT_TREE_L_MAX,
- * k <= DDT_TOPK_K_MAX, B_max <= DDT_TREE_B_MAX.
+ * k <= DDT_TOPK_K_MAX, B_max <= DDT_TREE_B_MAX.  The builder relies on the
+ * fp64 sums of logits along every path being exact (children of a node then
+ * come in candidate order); it checks that the binary exponents of the
+ * nonzero finite candidate logits of a sequence span at most
+ * 29 - ceil(log2 L) and raises DDT_ERR_UNSUPPORTED in dev_status when they
+ * do not (e.g. 1e-30 or subnormal logits beside 3.0): the tree it then
+ * writes may differ from the exact order at the budget's cut.
  * ------------------------------------------------------------------------ */
 ddt_status ddt_build_tree(const int32_t* ids, const float* zk, const float* lse, int batch, int L,
                           int k, float inv_temperature, const int32_t* k_per_seq,
@@ -232,6 +254,18 @@ size_t ddt_tree_attn_workspace_size(const ddt_attn_args* a);
 ddt_status ddt_tree_attn(const ddt_attn_args* a, void* workspace, size_t workspace_bytes,
                          cudaStream_t stream);
 
+/* How ddt_tree_attn would run this call on the current device (a query: it
+ * launches nothing).  *path: DDT_ATTN_PATH_SIMT (CUDA cores), _TC (tensor
+ * cores, one pass over the KV range per query tile), _TC_CLUSTER (KV splits
+ * of a query tile run as one thread-block cluster and merge through
+ * distributed shared memory) or _TC_COMBINE (KV splits write partials to the
+ * workspace and a second kernel merges them); *kv_splits: the number of KV
+ * splits per query tile (either pointer may be NULL).  Returns the status
+ * ddt_tree_attn's argument check would return. */
+enum { DDT_ATTN_PATH_SIMT = 0, DDT_ATTN_PATH_TC = 1, DDT_ATTN_PATH_TC_CLUSTER = 2,
+       DDT_ATTN_PATH_TC_COMBINE = 3 };
+ddt_status ddt_tree_attn_plan(const ddt_attn_args* a, int* path, int* kv_splits);
+
 /* ------------------------------------------------------------------------
  * Stage 4: greedy tree walk.
  * DDTree page, 運作流程 step 4: starting at the root, take the target's
@@ -244,16 +278,33 @@ ddt_status ddt_tree_attn(const ddt_attn_args* a, void* workspace, size_t workspa
  *           logits + (b*n_max + j)*row_stride elements; DDT_F32 or DDT_BF16.
  *   tok, parent, depth, n_nodes: the compiled tree of ddt_build_tree.
  *   L       the draft length (the deepest a row can be).
+ *   mode    how the rows' argmaxes are taken (same outputs for every mode):
+ *           DDT_WALK_ALL_ROWS  every tree row's argmax in one scan of all
+ *                              batch*n_max rows, then the walk: one pass at
+ *                              full bandwidth, reading rows the walk never
+ *                              visits;
+ *           DDT_WALK_LAZY      only the rows the walk visits (at most L + 1
+ *                              per sequence), one after another: one
+ *                              thread-block cluster per sequence;
+ *           DDT_WALK_AUTO      the library picks, from the sizes, the one
+ *                              that is faster on this device even when the
+ *                              walk goes down to depth L
+ *                              (ddt_tree_walk_resolve_mode tells which).
  * Outputs: acc_len int32 [batch] (0..L), acc_nodes / acc_tok int32
  * [batch][L] (accepted rows and their tokens in walk order; unused -1),
  * bonus int32 [batch].  Tokens emitted this round = acc_len + 1.
  * ------------------------------------------------------------------------ */
+enum { DDT_WALK_ALL_ROWS = 0, DDT_WALK_LAZY = 1, DDT_WALK_AUTO = 2 };
 size_t ddt_tree_walk_workspace_size(int batch, int n_max, int V);
 ddt_status ddt_tree_walk(const void* logits, ddt_dtype dtype, int batch, int n_max, int V,
                          int64_t row_stride, const int32_t* tok, const int32_t* parent,
-                         const int32_t* depth, const int32_t* n_nodes, int L, int32_t* acc_len,
-                         int32_t* acc_nodes, int32_t* acc_tok, int32_t* bonus, void* workspace,
-                         size_t workspace_bytes, int32_t* dev_status, cudaStream_t stream);
+                         const int32_t* depth, const int32_t* n_nodes, int L, int mode,
+                         int32_t* acc_len, int32_t* acc_nodes, int32_t* acc_tok, int32_t* bonus,
+                         void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                         cudaStream_t stream);
+/* The mode (DDT_WALK_ALL_ROWS or DDT_WALK_LAZY) that ddt_tree_walk runs for
+ * `mode` and these sizes on the current device; -1 for invalid arguments. */
+int ddt_tree_walk_resolve_mode(int mode, ddt_dtype dtype, int batch, int n_max, int V, int L);
 
 /* ------------------------------------------------------------------------
  * Stage 4 from the target's hidden states (greedy): LM head, argmax, walk.
@@ -354,12 +405,14 @@ ddt_status ddt_kv_commit(const ddt_kv_commit_args* a, cudaStream_t stream);
  * 0 of Philox4x64-10 (Salmon, Moraes, Dror and Shaw, SC'11) at counter
  * (j, b, 0, 0) under key (seed, step).  The weights are fp32 evaluations
  * of exp(z/T - max) with a fixed arithmetic (a = fl32(log2(e)/T),
- * t = fl32(a*z), k = round(t), w = P(t - k) * 2^(k - K) with P the fp32
- * Horner form of the degree-7 Taylor polynomial of 2^r and K = round of
- * the row's largest t; 0 below 2^-120), so they are reproducible exactly;
- * their sums are at least double-float (~48-bit) accurate.  The distribution is softmax(z/T) up to the fp32 rounding of t
- * (~|t| * 6e-8 relative).  Logits must be finite or -inf, with
- * |z/T| < 2^21; a row with no finite logit draws token 0.
+ * t = fl32(a*z), k = round(t), w = P(t - k) * (1 + ln2 * e) * 2^(k - K)
+ * with P the fp32 Horner form of the degree-7 Taylor polynomial of 2^r,
+ * e the part of z*log2(e)/T that t lost, K = round of the row's largest
+ * t; 0 below 2^-120), so they are reproducible exactly and each is within
+ * about 3e-7 (relative) of the exact weight whatever the size of z/T;
+ * their sums are at least double-float (~48-bit) accurate.  Logits must
+ * be finite or -inf, with |z/T| < 2^21; a row with no finite logit draws
+ * token 0.
  *
  *   inv_temperature  1/T, finite and > 0 (larger -> closer to greedy)
  *   seed, step       the Philox key: a stream per request (seed) and a
@@ -370,7 +423,8 @@ ddt_status ddt_kv_commit(const ddt_kv_commit_args* a, cudaStream_t stream);
  *                    draw: a captured CUDA graph then draws fresh uniforms on
  *                    every replay.  Calls sharing a counter must not overlap.
  * Every other argument, the outputs and the workspace
- * (ddt_tree_walk_workspace_size) are those of ddt_tree_walk.
+ * (ddt_tree_walk_workspace_size) are those of ddt_tree_walk; the draws scan
+ * every row (as DDT_WALK_ALL_ROWS).
  * ------------------------------------------------------------------------ */
 ddt_status ddt_tree_walk_sample(const void* logits, ddt_dtype dtype, int batch, int n_max, int V,
                                 int64_t row_stride, const int32_t* tok, const int32_t* parent,

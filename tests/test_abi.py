@@ -103,10 +103,11 @@ def test_walk_rejects_bad_arguments(lib):
     f = lib.ddt_tree_walk
     d = ctypes.c_void_p(16)
 
-    def call(b=1, n=9, V=64, stride=64, L=4, dt=1, logits=d):
-        return f(logits, dt, b, n, V, stride, d, d, d, d, L, d, d, d, d, None, 0, None, None)
+    def call(b=1, n=9, V=64, stride=64, L=4, dt=1, logits=d, mode=0):
+        return f(logits, dt, b, n, V, stride, d, d, d, d, L, mode, d, d, d, d, None, 0, None, None)
 
     assert call(stride=3) == 1 and call(dt=5) == 2 and call(n=2000) == 2 and call(L=65) == 2
+    assert call(mode=-1) == 1 and call(mode=3) == 1
     assert call(logits=None) == 1
     assert call(V=10 ** 6, stride=10 ** 6) == 3  # workspace required
 
@@ -183,3 +184,32 @@ def test_round_driver_rejects_an_unknown_decoding_rule():
     from block_draft_tree_b200.round import VerifyRound
     with pytest.raises(ValueError):
         VerifyRound(batch=1, L=4, V=64, k=4, B_max=8, hq=4, hkv=1, d=64, max_ctx=128, decode="beam")
+
+
+def test_noalloc_topk_rejects_like_topk(lib):
+    """ddt_topk_noalloc checks its arguments exactly as ddt_topk does, and
+    before it touches its scratch array (no CUDA call is made here)."""
+    f = lib.ddt_topk_noalloc
+    f.restype = ctypes.c_int
+    vp = ctypes.c_void_p
+    f.argtypes = [vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64,
+                  ctypes.c_int, ctypes.c_float, vp, vp, vp, vp, vp]
+    dummy = ctypes.c_void_p(16)
+    base = dict(logits=dummy, dt=0, b=1, L=4, V=64, stride=64, k=4, it=1.0)
+    cases = [dict(k=33), dict(k=65), dict(stride=10), dict(it=0.0), dict(it=float("inf")),
+             dict(dt=7), dict(b=-1), dict(logits=None), dict(b=4096, L=17)]
+    for kw in cases:
+        a = dict(base, **kw)
+        ref = lib.ddt_topk(a["logits"], a["dt"], a["b"], a["L"], a["V"], a["stride"], a["k"],
+                           a["it"], dummy, dummy, dummy, dummy, None, 0, None)
+        got = f(a["logits"], a["dt"], a["b"], a["L"], a["V"], a["stride"], a["k"], a["it"],
+                dummy, dummy, dummy, dummy, None)
+        assert ref != 0 and got == ref, (kw, ref, got)
+
+
+def test_walk_rejects_an_unknown_mode(lib):
+    dummy = ctypes.c_void_p(256)
+    rc = lib.ddt_tree_walk(dummy, 1, 1, 9, 100, 100, dummy, dummy, dummy, dummy, 4, 7,
+                           dummy, dummy, dummy, dummy, None, 0, None, None)
+    assert rc == 1
+    assert lib.ddt_tree_walk_resolve_mode(7, 1, 1, 9, 100, 4) == -1

@@ -119,3 +119,52 @@ def test_shared_memory_between_static_and_opt_in(L, k, B):
     builder's static scratch: the launch must still opt in."""
     ids, zk, lse = _random_inputs(L * 100 + k + B, 2, L, 400, k)
     _run(ids, zk, lse, B, 1.0)
+
+
+def _extreme_inputs(seed, b, L, V, k, small):
+    """f32 drafts whose candidates mix magnitudes: 3.0 and 2.5 beside 0, -0
+    and +-`small` (the eight largest logits of every row)."""
+    g = np.random.default_rng(seed)
+    z = np.full((b, L, V), -50.0, np.float32)
+    for bb in range(b):
+        for i in range(L):
+            picks = g.choice(V, 8, replace=False)
+            vals = np.array([3.0, small, 0.0, -0.0, small / 2, -small / 2, -small, 2.5], np.float32)
+            z[bb, i, picks] = vals
+    ids, zk, logp, lse = oracle.topk(z, k, 1.0)
+    return ids, zk, f32_up(lse)
+
+
+def _run_or_flag(ids, zk, lse, B_max):
+    """The GPU tree equals the oracle's, or the builder flags the input as
+    outside what it supports (DDT_ERR_UNSUPPORTED in the status word)."""
+    b = ids.shape[0]
+    root = np.arange(b, dtype=np.int32) + 3
+    ctx = np.full(b, 100, np.int32)
+    ref = oracle.build_tree(ids, zk, lse.astype(np.float64), B_max, 1.0, root_token=root,
+                            ctx_len=ctx, n_max=B_max + 1)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    got = api.build_tree(i32(ids), torch.from_numpy(zk.astype(np.float32)).cuda(),
+                         torch.from_numpy(lse.astype(np.float32)).cuda(), B_max, i32(root), 1.0,
+                         ctx_len=i32(ctx), dev_status=st)
+    torch.cuda.synchronize()
+    if st.item() == 2:
+        return "flagged"
+    assert st.item() == 0
+    for key in ("tok", "parent", "depth", "pos", "n_nodes"):
+        np.testing.assert_array_equal(got[key].cpu().numpy(), ref[key], err_msg=key)
+    np.testing.assert_array_equal(got["mask"].cpu().numpy().view(np.uint32), ref["mask"])
+    return "exact"
+
+
+def test_candidates_of_mixed_magnitude():
+    """The builder takes siblings in candidate order, which is the order K as
+    long as path sums of logits are exact in fp64.  Zeros (of either sign)
+    keep them exact and must give the oracle's tree; candidates 2^-20 beside
+    3.0 (sums that still fit) must too; subnormals or 1e-30 beside 3.0 can
+    round a path sum, and the builder must then flag the input."""
+    L, V, k, B = 6, 64, 8, 40
+    assert _run_or_flag(*_extreme_inputs(1, 4, L, V, k, small=0.0), B) == "exact"
+    assert _run_or_flag(*_extreme_inputs(2, 4, L, V, k, small=2.0 ** -20), B) == "exact"
+    assert _run_or_flag(*_extreme_inputs(3, 4, L, V, k, small=1e-30), B) == "flagged"
+    assert _run_or_flag(*_extreme_inputs(4, 4, L, V, k, small=2e-42), B) == "flagged"  # subnormal

@@ -70,7 +70,7 @@ def test_matches_workspace_entry_point_on_two_calls():
 
 def test_rejects_shapes_beyond_the_scratch():
     lib = api.load_library()
-    b, L, V, k = 64, 16, 151936, 32
+    b, L, V, k = 4095, 16, 151936, 32  # 65520 rows of partials
     assert lib.ddt_topk_workspace_size(b, L, V, k) > SCRATCH_BYTES
     dummy = ctypes.c_void_p(256)
     rc = _entry()(dummy, 0, b, L, V, V, k, 1.0, dummy, dummy, dummy, dummy, None)
