@@ -69,6 +69,16 @@ def parse():
     ap.add_argument("--extensions", action="store_true",
                     help="with --profile: also run the sampled walk and the KV commit after "
                          "each round")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="skip the rounds of the other workloads (b256, paged128, long512)")
+    ap.add_argument("--per-workload", default="b256,paged128,long512")
+    ap.add_argument("--clock-window-s", type=float, default=0.5,
+                    help="untimed replays before and after the timed region, so that the clock "
+                         "sampler sees the GPU under load around it")
+    ap.add_argument("--cpu-threads", type=int, default=0,
+                    help="threads of the threaded oracle baseline (0: every core of the host)")
+    ap.add_argument("--selftest-ranks", action="store_true",
+                    help="no GPU: each rank only exercises the multi-rank host logic on gloo")
     return ap.parse_args()
 
 
@@ -79,6 +89,15 @@ def peaks():
         return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
     except Exception:
         return 6650.0, 1590.0, "fallback"
+
+
+def input_set_bytes(w):
+    """Bytes of one input set of a round: draft logits, root tokens and
+    context lengths, queries, the context K/V, the tree K/V, target logits."""
+    es_draft = 4 if w.draft_dtype == "f32" else 2
+    return (w.batch * w.L * w.V * es_draft + 8 * w.batch + w.batch * w.n_max * w.hq * w.d * 2 +
+            2 * w.batch * w.ctx * w.hkv * w.d * 2 + 2 * w.batch * w.n_max * w.hkv * w.d * 2 +
+            w.batch * w.n_max * w.V * 4)
 
 
 def workload_config(w, sets, set_bytes):
@@ -157,6 +176,53 @@ def max_over_ranks(value, world, device):
     return float(t.item())
 
 
+def host_cores():
+    """Cores this process may run on, and the host's core count."""
+    try:
+        usable = len(os.sched_getaffinity(0))
+    except Exception:
+        usable = os.cpu_count() or 1
+    return usable, os.cpu_count() or usable
+
+
+def relaunch_command(argv, n, port):
+    """The torchrun command that runs this script as n ranks on this node."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            "--nproc-per-node", str(n), "--master-addr", "127.0.0.1",
+            "--master-port", str(port), os.path.abspath(__file__)] + list(argv)
+
+
+def relaunch_as_ranks(n):
+    """`bench.py --gpus N` started without a launcher: run it again under
+    torchrun as N ranks (one per GPU) and return their exit status."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    return subprocess.call(relaunch_command(sys.argv[1:], n, port))
+
+
+def run_selftest_ranks(args):
+    """Each rank: a gloo process group, the max-over-ranks time and the job
+    throughput of the real path, on the CPU; rank 0 prints one JSON line."""
+    import datetime
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if world > 1:
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    local_ms = 2.0 + rank
+    ms = max_over_ranks(local_ms, world, "cpu")
+    line = {"selftest": True, "n_gpus": world, "rank_ms": local_ms, "job_ms": ms,
+            "value": job_throughput(world, 1, args.steps, ms)}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def job_throughput(world, batch, steps, elapsed_ms):
     """Rounds of all ranks per second: every rank runs `steps` rounds of its own
     `batch` sequences (weak scaling), all within the slowest rank's time."""
@@ -225,31 +291,65 @@ def traffic_for(kernel_tag):
         return None
 
 
-def cpu_baseline(w, x_host, tree_from_gpu=None, attn_fraction=1.0):
-    """Time the CPU oracle on one round of the workload (bounded sample)."""
+def _chunks(n, parts):
+    step = max(1, -(-n // max(1, parts)))
+    return [(i, min(n, i + step)) for i in range(0, n, step)]
+
+
+def cpu_baseline(w, x_host, attn_fraction=1.0, threads=1):
+    """Time the CPU oracle on one round of the workload (attention on a
+    bounded sample of its (sequence, row, head) items, scaled to the round).
+    With threads > 1 the oracle's calls run on that many host threads over
+    independent pieces (rows of the top-k, sequences of the tree and the
+    walk, items of the attention); the oracle's arithmetic is unchanged and
+    its C calls release the interpreter lock."""
+    from concurrent.futures import ThreadPoolExecutor
+
     import oracle
     from block_draft_tree_b200 import synth
+    ex = ThreadPoolExecutor(max_workers=threads) if threads > 1 else None
+
+    def pmap(fn, pieces):
+        return list(ex.map(fn, pieces)) if ex else [fn(p) for p in pieces]
+
+    z = x_host["draft"]
     t0 = time.perf_counter()
-    ids, zk, logp, lse = oracle.topk(x_host["draft"], w.k, w.inv_temperature)
+    rows = z.reshape(-1, z.shape[-1])
+    parts = pmap(lambda r: oracle.topk(rows[r[0]:r[1]], w.k, w.inv_temperature),
+                 _chunks(rows.shape[0], threads))
+    ids = np.concatenate([p[0] for p in parts]).reshape(w.batch, w.L, w.k)
+    zk = np.concatenate([p[1] for p in parts]).reshape(w.batch, w.L, w.k)
+    lse = np.concatenate([p[3] for p in parts]).reshape(w.batch, w.L)
     t1 = time.perf_counter()
-    tree = oracle.build_tree(ids, zk, lse, w.budget_per_seq(), w.inv_temperature,
-                             root_token=x_host["root"], ctx_len=x_host["ctx_len"],
-                             k_per_seq=w.k_per_seq(), n_max=w.n_max)
+    bud, kps = w.budget_per_seq(), w.k_per_seq()
+    seq_parts = _chunks(w.batch, threads)
+    trees = pmap(lambda r: oracle.build_tree(ids[r[0]:r[1]], zk[r[0]:r[1]], lse[r[0]:r[1]],
+                                             bud[r[0]:r[1]], w.inv_temperature,
+                                             root_token=x_host["root"][r[0]:r[1]],
+                                             ctx_len=x_host["ctx_len"][r[0]:r[1]],
+                                             k_per_seq=kps[r[0]:r[1]], n_max=w.n_max), seq_parts)
+    tree = {k: np.concatenate([t[k] for t in trees]) for k in trees[0]}
     t2 = time.perf_counter()
     items = [(b, j, h) for b in range(w.batch) for j in range(int(tree["n_nodes"][b]))
              for h in range(w.hq)]
     n_all = len(items)
     n_s = max(1, int(round(n_all * attn_fraction)))
     items = np.array(items[:n_s], np.int32)
-    oracle.tree_attn(items, x_host["q"], x_host["k_cache"], x_host["v_cache"], x_host["ctx_len"],
-                     x_host["k_tree"], x_host["v_tree"], tree["mask"], tree["n_nodes"],
-                     1.0 / np.sqrt(w.d), page_table=x_host.get("page_table"),
-                     page_size=x_host.get("page_size", 64))
+    pmap(lambda r: oracle.tree_attn(items[r[0]:r[1]], x_host["q"], x_host["k_cache"],
+                                    x_host["v_cache"], x_host["ctx_len"], x_host["k_tree"],
+                                    x_host["v_tree"], tree["mask"], tree["n_nodes"],
+                                    1.0 / np.sqrt(w.d), page_table=x_host.get("page_table"),
+                                    page_size=x_host.get("page_size", 64)),
+         _chunks(n_s, 4 * threads))
     t3 = time.perf_counter()
     tgt = synth.target_logits(w, tree["tok"], tree["parent"], tree["depth"], tree["n_nodes"])
     t4 = time.perf_counter()
-    oracle.tree_walk(tgt, tree["tok"], tree["parent"], tree["depth"], tree["n_nodes"], w.L)
+    pmap(lambda r: oracle.tree_walk(tgt[r[0]:r[1]], tree["tok"][r[0]:r[1]],
+                                    tree["parent"][r[0]:r[1]], tree["depth"][r[0]:r[1]],
+                                    tree["n_nodes"][r[0]:r[1]], w.L), seq_parts)
     t5 = time.perf_counter()
+    if ex:
+        ex.shutdown()
     round_s = (t1 - t0) + (t2 - t1) + (t3 - t2) * n_all / n_s + (t5 - t4)
     return round_s, {"topk_s": t1 - t0, "tree_s": t2 - t1, "attn_s": (t3 - t2) * n_all / n_s,
                      "walk_s": t5 - t4, "attn_rows_timed": n_s, "attn_rows": n_all}
@@ -263,29 +363,32 @@ def run_reference(args):
     from block_draft_tree_b200 import synth
     w = synth.WORKLOADS[WORKLOAD]
     x, _ = make_inputs(w, 0, 0)
+    usable, total = host_cores()
+    threads = args.cpu_threads or usable
     # size the attention sample so that the whole run stays within a few minutes
-    probe_s, parts = cpu_baseline(w, x, attn_fraction=0.02)
+    probe_s, parts = cpu_baseline(w, x, attn_fraction=0.02, threads=threads)
     per_step_budget = 150.0 / max(1, args.steps + args.warmup)
     fixed = parts["topk_s"] + parts["tree_s"] + parts["walk_s"]
     per_row = parts["attn_s"] / parts["attn_rows"]
     frac = min(1.0, max(1.0 / parts["attn_rows"], (per_step_budget - fixed) / max(per_row * parts["attn_rows"], 1e-9)))
     for _ in range(args.warmup):
-        cpu_baseline(w, x, attn_fraction=frac)
+        cpu_baseline(w, x, attn_fraction=frac, threads=threads)
     times = []
     for _ in range(args.steps):
-        s, parts = cpu_baseline(w, x, attn_fraction=frac)
-        times.append(s)
+        s_, parts = cpu_baseline(w, x, attn_fraction=frac, threads=threads)
+        times.append(s_)
     round_s = statistics.mean(times)
     value = w.batch / round_s
     sample = ("full top-k, tree and walk; attention on %d of %d (row, head) items per step, "
-              "scaled to the full round" % (parts["attn_rows_timed"], parts["attn_rows"]))
+              "scaled to the full round; %d threads on a host of %d cores"
+              % (parts["attn_rows_timed"], parts["attn_rows"], threads, total))
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "rounds/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round_s * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": workload_config(w, 1, 0),
-            "cpu_baseline": {"value": value, "unit": "rounds/s", "cores": 1, "kind": "oracle",
-                             "sample": sample},
+            "config": workload_config(w, args.sets, input_set_bytes(w)),
+            "cpu_baseline": {"value": value, "unit": "rounds/s", "cores": threads,
+                             "host_cores": total, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "rounds/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -385,6 +488,187 @@ def measure_extensions(w, sets, graphs, hbm_peak, reps=30):
     return ext
 
 
+def device_inputs(w, seed):
+    """One input set of a workload generated on the GPU (seeded torch
+    generator): the same distributions as the seeded host generator
+    (block_draft_tree_b200.synth) -- N(0,1) drafts with +6/+4/+3 spikes at
+    distinct tokens, or Zipf(1.1) drafts over a fresh permutation per row;
+    N(0,1) bf16 queries and K/V; ragged contexts and a random page placement
+    for the paged workload -- drawn where the large workloads live, so that
+    building them takes milliseconds.  Target logits are N(0,1) here and
+    planted from the GPU's own tree (plant_greedy) once the tree exists."""
+    import torch
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    dev = "cuda"
+    rows = w.batch * w.L
+    if w.draft == "spikes":
+        z = torch.randn(rows, w.V, device=dev, generator=g)
+        t0 = torch.randint(0, w.V, (rows,), device=dev, generator=g)
+        r = torch.arange(rows, device=dev)
+        for i, sp in enumerate(w.spikes):  # distinct tokens: fixed offsets from a random start
+            z[r, (t0 + 7919 * i) % w.V] += sp
+    else:
+        ranks = torch.arange(1, w.V + 1, device=dev, dtype=torch.float64)
+        zipf = (-1.1 * torch.log(ranks)).float()
+        perm = torch.argsort(torch.rand(rows, w.V, device=dev, generator=g), dim=1)
+        z = torch.empty(rows, w.V, device=dev)
+        z.scatter_(1, perm, zipf.expand(rows, w.V).contiguous())
+    x = {"draft": z.reshape(w.batch, w.L, w.V).to(torch.bfloat16)}
+    del z
+    x["root"] = torch.randint(0, w.V, (w.batch,), device=dev, generator=g, dtype=torch.int32)
+    if w.ctx_min is None:
+        ctx = torch.full((w.batch,), w.ctx, device=dev, dtype=torch.int32)
+    else:
+        ctx = torch.randint(w.ctx_min, w.ctx + 1, (w.batch,), device=dev, generator=g,
+                            dtype=torch.int32)
+    x["ctx_len"] = ctx
+    bf = lambda *shape: torch.randn(*shape, device=dev, generator=g).to(torch.bfloat16)
+    x["q"] = bf(w.batch, w.n_max, w.hq, w.d)
+    x["k_tree"] = bf(w.batch, w.n_max, w.hkv, w.d)
+    x["v_tree"] = bf(w.batch, w.n_max, w.hkv, w.d)
+    if w.page_size:
+        ps = w.page_size
+        npg = (ctx.long() + ps - 1) // ps
+        total = int(npg.sum().item())
+        max_pages = int(npg.max().item())
+        perm = torch.randperm(total, device=dev, generator=g).to(torch.int32)
+        pt = torch.full((w.batch, max_pages), -1, device=dev, dtype=torch.int32)
+        off = 0
+        for b, n in enumerate(npg.tolist()):
+            pt[b, :n] = perm[off:off + n]
+            off += n
+        x["page_table"] = pt
+        shape = (total, ps, w.hkv, w.d)
+    else:
+        shape = (w.batch, w.ctx, w.hkv, w.d)
+    x["k_cache"] = bf(*shape)
+    x["v_cache"] = bf(*shape)
+    x["target"] = torch.randn(w.batch, w.n_max, w.V, device=dev, generator=g)
+    return x, g
+
+
+def plant_greedy(w, target, tok, parent, depth, n_nodes, g):
+    """Planted agreement on the GPU, as synth.target_logits plants it on the
+    host: every tree row with children, with probability max(0, p0 - decay *
+    depth), gets logit (row max + 2) at the token of one of its children
+    picked uniformly."""
+    import torch
+    b, n_max, V = target.shape
+    rows = torch.arange(n_max, device=target.device)
+    live = (rows[None, :] < n_nodes[:, None]) & (rows[None, :] > 0)
+    par = parent.long().clamp(min=0)
+    key = torch.rand(b, n_max, device=target.device, generator=g)
+    key = torch.where(live, key, torch.full_like(key, -1.0))
+    best = torch.full((b, n_max), -1.0, device=target.device)
+    best.scatter_reduce_(1, par, key, reduce="amax")  # per parent: the largest child key
+    chosen = live & (key == best.gather(1, par))
+    p = (w.plant_p0 - w.plant_decay * depth.float()).clamp(min=0.0)
+    u = torch.rand(b, n_max, device=target.device, generator=g)
+    plant_row = (u < p) & (rows[None, :] < n_nodes[:, None])  # per parent row
+    bi, ci = torch.nonzero(chosen, as_tuple=True)
+    xi = par[bi, ci]
+    keep = plant_row[bi, xi]
+    bi, ci, xi = bi[keep], ci[keep], xi[keep]
+    rowmax = target.amax(dim=2)
+    target[bi, xi, tok[bi, ci].long()] = rowmax[bi, xi] + 2.0
+
+
+def measure_per_workload(names, hbm_peak, tf_peak, steps, seed=5):
+    """One full round of each named workload (one CUDA graph per workload,
+    its inputs far larger than L2), timed like the headline: `steps` graph
+    replays between CUDA events; then the same round with event nodes
+    between the kernels, replayed a few times, for each stage's time and its
+    fraction of the binding roofline."""
+    import torch
+    from cuda.bindings import runtime as cudart
+
+    from block_draft_tree_b200 import api, synth
+    from block_draft_tree_b200.round import VerifyRound
+
+    out = {}
+    for name in names:
+        w = synth.WORKLOADS[name]
+        x, g = device_inputs(w, seed + w.index)
+        max_ctx = int(x["ctx_len"].max().item())
+        ps = w.page_size or 64
+        rnd = VerifyRound(batch=w.batch, L=w.L, V=w.V, k=w.k, B_max=w.B, hq=w.hq, hkv=w.hkv,
+                          d=w.d, max_ctx=max_ctx, draft_dtype=torch.bfloat16,
+                          target_dtype=torch.float32, inv_temperature=w.inv_temperature,
+                          paged=w.page_size > 0, page_size=ps,
+                          max_pages=(max_ctx + ps - 1) // ps)
+        if w.chain_seq0:
+            x["k_per_seq"] = torch.from_numpy(w.k_per_seq()).cuda()
+            x["budget"] = torch.from_numpy(w.budget_per_seq()).cuda()
+        rnd.bind(x)
+        rnd.launch()
+        torch.cuda.synchronize()
+        o = rnd.out
+        plant_greedy(w, x["target"], o["tok"], o["parent"], o["depth"], o["n_nodes"], g)
+        graph = rnd.capture()
+        evs = [cudart.cudaEventCreate()[1] for _ in range(5)]
+
+        def marks(i, evs=evs):
+            st = torch.cuda.current_stream().cuda_stream
+            cudart.cudaEventRecordWithFlags(evs[i], st, cudart.cudaEventRecordExternal)
+
+        timed = rnd.capture(marks)
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
+        assert int(o["status"].item()) == 0, "device status raised (%s)" % name
+        a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(steps):
+            graph.replay()
+        e.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(e) / steps
+        per = {n: [] for n in ("topk", "tree", "attn", "walk")}
+        for _ in range(5):
+            timed.replay()
+            torch.cuda.synchronize()
+            for i, n in enumerate(per):
+                per[n].append(cudart.cudaEventElapsedTime(evs[i], evs[i + 1])[1] * 1e3)
+        us = {n: statistics.median(v) for n, v in per.items()}
+        n_nodes = o["n_nodes"].long().cpu().numpy()
+        ctx = x["ctx_len"].long().cpu().numpy()
+        rows = w.batch * w.L
+        topk_b = rows * w.V * 2 + rows * w.k * 12 + rows * 4
+        attn_b = (int(ctx.sum()) * w.hkv * w.d * 2 * 2 + 2 * int(n_nodes.sum()) * w.hq * w.d * 2 +
+                  2 * int(n_nodes.sum()) * w.hkv * w.d * 2)
+        attn_f = 4.0 * w.d * w.hq * float((n_nodes * (ctx + n_nodes)).sum())
+        acc = o["acc_len"].long().cpu().numpy()
+        walk_mode = api.tree_walk_resolve_mode(rnd.walk_mode, torch.float32, w.batch, w.n_max,
+                                               w.V, w.L)
+        walk_rows = int(n_nodes.sum()) if walk_mode == api.WALK_ALL_ROWS else int((acc + 1).sum())
+        walk_b = walk_rows * w.V * 4
+        t_hbm, t_tc = attn_b / (hbm_peak * 1e9), attn_f / (tf_peak * 1e12)
+        st = {"topk": {"us": round(us["topk"], 2), "alg_bytes": topk_b,
+                       "gbs": round(topk_b / us["topk"] / 1e3, 1),
+                       "frac_hbm": round(topk_b / us["topk"] / 1e3 / hbm_peak, 4)},
+              "tree": {"us": round(us["tree"], 2), "bound": "latency"},
+              "attn": {"us": round(us["attn"], 2), "alg_bytes": attn_b, "alg_flops": attn_f,
+                       "gbs": round(attn_b / us["attn"] / 1e3, 1),
+                       "tflops": round(attn_f / us["attn"] / 1e6, 1),
+                       "bound": "tensor" if t_tc > t_hbm else "hbm",
+                       "frac_binding": round(max(t_hbm, t_tc) / (us["attn"] * 1e-6), 4)},
+              "walk": {"us": round(us["walk"], 2), "mode": "all rows" if walk_mode == 0 else
+                       "path only", "alg_bytes": walk_b,
+                       "gbs": round(walk_b / us["walk"] / 1e3, 1),
+                       "rows_read": walk_rows}}
+        out[name] = {"rounds_per_s": round(w.batch / (ms * 1e-3), 1), "ms_per_round": round(ms, 4),
+                     "steps": steps, "batch": w.batch, "mean_accepted": round(float(acc.mean()), 3),
+                     "stages": st,
+                     "inputs": "generated on the GPU; %.2f GB per set, above L2"
+                               % (sum(t.numel() * t.element_size() for t in x.values()) / 1e9)}
+        for ev in evs:
+            cudart.cudaEventDestroy(ev)
+        del graph, timed, rnd, x
+        torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -422,7 +706,7 @@ def run_ours(args):
         xd["target"].copy_(torch.from_numpy(tgt))
         sets.append(xd)
         hosts.append((xh, tgt))
-    set_bytes = sum(t.numel() * t.element_size() for t in sets[0].values())
+    set_bytes = input_set_bytes(w)
 
     # one graph per input set, with event nodes around the stages
     def make_events(n):
@@ -461,17 +745,30 @@ def run_ours(args):
     for g, r in graphs:
         assert int(r.out["status"].item()) == 0, "device status raised"
 
-    for i in range(args.warmup):
-        graphs[i % len(graphs)][0].replay()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    n_sets = len(graphs)
+
+    def load_for(seconds):
+        """Untimed replays for `seconds`, so that the clock sampler sees the
+        GPU under the same load just before and just after the timed region."""
+        t_end = time.perf_counter() + seconds
+        i = 0
+        while time.perf_counter() < t_end:
+            graphs[i % n_sets][0].replay()
+            i += 1
+            if i % 64 == 0:
+                torch.cuda.synchronize()
+        torch.cuda.synchronize()
+
     clocks = ClockSampler(local) if rank == 0 else None
     if clocks:
         clocks.start()
+    for i in range(args.warmup):
+        graphs[i % n_sets][0].replay()
+    load_for(args.clock_window_s)
+    if world > 1:
+        dist.barrier()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
-    n_sets = len(graphs)
     n_plain = max(0, args.steps - n_sets)
     start.record()
     for i in range(n_plain):
@@ -480,7 +777,11 @@ def run_ours(args):
         timed_graphs[i % n_sets].replay()
     end.record()
     torch.cuda.synchronize()
+    load_for(args.clock_window_s)
     clk = clocks.stop() if clocks else None
+    if clk is not None:
+        clk["window"] = ("nvidia-smi every 100 ms from %.1f s of untimed replays before the timed "
+                         "region to %.1f s after it" % (args.clock_window_s, args.clock_window_s))
     elapsed_ms = max_over_ranks(start.elapsed_time(end), world, "cuda")
     if world > 1:
         dist.barrier()
@@ -513,6 +814,9 @@ def run_ours(args):
     acc = [r.out["acc_len"].float().mean().item() for _, r in graphs]
     ext = (measure_extensions(w, sets, graphs, hbm_peak)
            if rank == 0 and not args.no_extensions else None)
+    per_wl = (measure_per_workload(args.per_workload.split(","), hbm_peak, tf_peak,
+                                   max(10, args.steps))
+              if rank == 0 and not args.no_per_workload else None)
 
     # end to end: pinned host inputs -> H2D -> round -> D2H of the result, every step
     e2e = None
@@ -564,12 +868,22 @@ def run_ours(args):
     cpu = None
     if not args.no_cpu_baseline and world == 1:
         xh, _ = hosts[0]
+        usable, total = host_cores()
+        threads = args.cpu_threads or usable
         t0 = time.perf_counter()
-        round_s, parts = cpu_baseline(w, xh, attn_fraction=1.0)
-        cpu = {"value": w.batch / round_s, "unit": "rounds/s", "cores": 1, "kind": "oracle",
-               "sample": "one full b64 round (all 2080 attention rows) of input set 0; "
-                         "single-threaded fp64 C oracle; %.1f s" % (time.perf_counter() - t0),
-               "stage_s": {k: round(v, 4) for k, v in parts.items() if k.endswith("_s")}}
+        round_mt, parts_mt = cpu_baseline(w, xh, attn_fraction=1.0, threads=threads)
+        t1 = time.perf_counter()
+        round_st, parts_st = cpu_baseline(w, xh, attn_fraction=1.0, threads=1)
+        t2 = time.perf_counter()
+        cpu = {"value": w.batch / round_mt, "unit": "rounds/s", "cores": threads,
+               "host_cores": total, "kind": "oracle",
+               "sample": "one full b64 round (all %d attention items) of input set 0, fp64 C "
+                         "oracle on %d threads (%.1f s), and again on one thread (%.1f s)"
+                         % (parts_mt["attn_rows"], threads, t1 - t0, t2 - t1),
+               "stage_s": {k: round(v, 4) for k, v in parts_mt.items() if k.endswith("_s")},
+               "single_thread": {"value": w.batch / round_st, "unit": "rounds/s", "cores": 1,
+                                 "stage_s": {k: round(v, 4) for k, v in parts_st.items()
+                                             if k.endswith("_s")}}}
 
     value = job_throughput(world, w.batch, args.steps, elapsed_ms)
     line = {"metric": METRIC, "value": value, "unit": "rounds/s", "n_gpus": world,
@@ -579,6 +893,7 @@ def run_ours(args):
             "roofline": roof, "stages": stages, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps, "clocks": clk,
             "mean_accepted": round(statistics.mean(acc), 3), "extensions": ext,
+            "per_workload": per_wl,
             "parallelism": "dp%d (independent sequences per GPU)" % world}
     print(json.dumps(line), flush=True)
     if world > 1:
@@ -790,6 +1105,10 @@ def run_stage_sweep(args):
 
 def main():
     args = parse()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return relaunch_as_ranks(args.gpus)
+    if args.selftest_ranks:
+        return run_selftest_ranks(args)
     if args.impl == "reference":
         return run_reference(args)
     if args.profile:

@@ -65,3 +65,31 @@ def test_job_throughput_counts_every_rank():
     # 2 ranks x batch 4 x 10 rounds in 5 ms = 16000 rounds/s
     assert bench.job_throughput(2, 4, 10, 5.0) == pytest.approx(16000.0)
     assert bench.max_over_ranks(3.25, 1, "cpu") == 3.25
+
+
+def test_bench_spawns_its_own_ranks():
+    """`bench.py --gpus 2` started without a launcher runs itself again as two
+    torchrun ranks; here the ranks only exercise the host logic on gloo (no
+    GPU): the job time is the slower rank's and rank 0 prints one line."""
+    import json
+    import subprocess
+    env = dict(os.environ)
+    for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT"):
+        env.pop(k, None)
+    res = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2",
+                          "--selftest-ranks", "--steps", "10"], env=env, capture_output=True,
+                         text=True, timeout=240)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [l for l in res.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, res.stdout
+    line = json.loads(lines[0])
+    assert line["n_gpus"] == 2 and line["job_ms"] == 3.0  # ranks took 2 ms and 3 ms
+    assert line["value"] == pytest.approx(2 * 10 / 3e-3)
+
+
+def test_relaunch_command():
+    cmd = bench.relaunch_command(["--gpus", "8", "--steps", "5"], 8, 29555)
+    assert cmd[1:4] == ["-m", "torch.distributed.run", "--nnodes=1"]
+    assert cmd[cmd.index("--nproc-per-node") + 1] == "8"
+    assert cmd[cmd.index("--master-addr") + 1] == "127.0.0.1"
+    assert cmd[-4:] == ["--gpus", "8", "--steps", "5"]
