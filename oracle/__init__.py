@@ -23,6 +23,10 @@ curated summary of the authors' announcement), section "運作流程"
   its argmax (lowest id on ties), and the walk over those row tokens;
 * :func:`kv_commit`  -- after step 4: the root and the accepted rows' K/V
   appended to the committed context, which grows by acc_len + 1;
+* :func:`plan_budget` -- after step 2: the node budget of every sequence of
+  a batch that maximises the round's expected emitted tokens per unit of
+  cost ("實驗結果與權衡": acceptance grows with B, so does the verifier's
+  cost; Proposition 1);
 * :func:`tree_walk_sample` -- step 4 under a sampling decoding rule
   (temperature > 0): each visited row draws its token from softmax(z / T)
   by inversion with a Philox4x64-10 uniform (:func:`philox4x64_10`,
@@ -113,6 +117,11 @@ def _load():
                                              ctypes.POINTER(ctypes.c_int32), i32p, i32p,
                                              ctypes.POINTER(ctypes.c_int32)]
         lib.ddto_walk_row_tokens.restype = ctypes.c_int
+        lib.ddto_plan_budget.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_double, i32p, f64p, f64p, i32p, i32p, i32p,
+                                         i32p, ctypes.c_int, ctypes.c_double, ctypes.c_double,
+                                         i32p, f64p, ctypes.POINTER(ctypes.c_int32)]
+        lib.ddto_plan_budget.restype = ctypes.c_int
         for f in (lib.ddto_topk, lib.ddto_build_tree, lib.ddto_tree_attn, lib.ddto_tree_walk,
                   lib.ddto_sample_row, lib.ddto_tree_walk_sample):
             f.restype = ctypes.c_int
@@ -462,3 +471,30 @@ def walk_row_tokens(row_tok, tok, parent, depth, n_nodes, L):
         res["acc_tok"][b] = at[:L]
         res["bonus"][b] = bo.value
     return res
+
+
+def plan_budget(ids, zk, lse, tree, L, inv_temperature, total_budget=-1, cost_fixed=0.0,
+                cost_per_node=0.0):
+    """Node budgets across a batch from trees built with each sequence's
+    largest budget (``tree``: dict with tok, parent, depth, n_nodes);
+    ``total_budget`` < 0: no cap on the nodes taken.
+    ``ids``/``zk`` [batch, L, k], ``lse`` [batch, L].  Returns (budget int32
+    [batch], expected_tokens f64 [batch], n_taken)."""
+    ids = np.ascontiguousarray(ids, np.int32)
+    zk = np.ascontiguousarray(zk, np.float64)
+    lse = np.ascontiguousarray(lse, np.float64)
+    bsz, Lx, kk = ids.shape
+    n_max = tree["tok"].shape[1]
+    budget = np.empty(bsz, np.int32)
+    exp_tok = np.empty(bsz, np.float64)
+    taken = ctypes.c_int32()
+    rc = _load().ddto_plan_budget(bsz, L, kk, n_max, _f32(inv_temperature), ids, zk, lse,
+                                  np.ascontiguousarray(tree["tok"], np.int32),
+                                  np.ascontiguousarray(tree["parent"], np.int32),
+                                  np.ascontiguousarray(tree["depth"], np.int32),
+                                  np.ascontiguousarray(tree["n_nodes"], np.int32),
+                                  int(total_budget), float(cost_fixed), float(cost_per_node),
+                                  budget, exp_tok, ctypes.byref(taken))
+    if rc != 0:
+        raise ValueError("ddto_plan_budget failed (%d)" % rc)
+    return budget, exp_tok, int(taken.value)

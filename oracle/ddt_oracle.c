@@ -811,3 +811,119 @@ int ddto_walk_row_tokens(const int32_t* row_tok, const int32_t* tok, const int32
   *acc_len = a;
   return DDTO_OK;
 }
+
+/* ------------------------------------------------------------------ */
+/* Node budgets across a batch (after step 2)                          */
+/* ------------------------------------------------------------------ */
+/*
+ * The page's trade-off (section 實驗結果與權衡): a larger node budget raises
+ * the expected acceptance but the verifier's cost grows with it.  By
+ * Proposition 1 (section 理論基礎) a tree's expected acceptance length is the
+ * sum of its nodes' prefix probabilities, and the best tree of any smaller
+ * budget is the K-first part of the best tree of a larger one.  So, given
+ * for every sequence the tree built with its largest budget, the nodes of
+ * the whole batch ranked by prefix probability (ties: smaller sequence
+ * index, then smaller row) give the allocation that maximises the summed
+ * expected acceptance for any total number of nodes n: the first n nodes.
+ * With a round cost of c0 + c1 * n for n draft nodes, the round emits
+ * (batch + accepted) tokens, so the plan takes the n that maximises
+ * (batch + sum of the first n probabilities) / (c0 + c1 * n) (the smallest
+ * such n), up to `total_budget` nodes (< 0: no cap).  With c1 <= 0 it takes
+ * all the nodes up to the cap.  Outputs: budget[b], the number of sequence
+ * b's nodes among those taken, and expected_tokens[b] = 1 + the sum of their
+ * probabilities (the tokens sequence b is expected to emit).
+ *
+ * Node probabilities: a row j of sequence b at depth d with tokens
+ * t_1..t_d on its path has score invT * (z_1 + ... + z_d) - (lse_1 + ... +
+ * lse_d), each sum in depth order (z_i the candidate logit of t_i at
+ * position i from the top-k lists ids / zk [L][kstride], lse [L]); the
+ * probability is exp(score).
+ */
+typedef struct {
+  double p;
+  int b, j;
+} pnode_t;
+
+static int cmp_pnode(const void* pa, const void* pb) {
+  const pnode_t* a = (const pnode_t*)pa;
+  const pnode_t* b = (const pnode_t*)pb;
+  if (a->p > b->p) return -1;
+  if (a->p < b->p) return 1;
+  if (a->b != b->b) return a->b < b->b ? -1 : 1;
+  return a->j < b->j ? -1 : (a->j > b->j);
+}
+
+int ddto_plan_budget(int batch, int L, int kstride, int n_max, double invT, const int32_t* ids,
+                     const double* zk, const double* lse, const int32_t* tok,
+                     const int32_t* parent, const int32_t* depth, const int32_t* n_nodes,
+                     int total_budget, double c0, double c1, int32_t* budget,
+                     double* expected_tokens, int32_t* n_taken) {
+  if (batch < 0 || L < 1 || L > DDTO_LMAX || kstride < 1 || n_max < 1 || !(invT > 0.0))
+    return DDTO_ERR_ARG;
+  if (c1 > 0.0 && !(c0 > 0.0)) return DDTO_ERR_ARG;
+  int total = 0;
+  for (int b = 0; b < batch; ++b)
+    if (n_nodes[b] > 1) total += n_nodes[b] - 1;
+  pnode_t* nodes = (pnode_t*)malloc(sizeof(pnode_t) * (size_t)(total > 0 ? total : 1));
+  if (!nodes) return DDTO_ERR_NOMEM;
+  int m = 0;
+  for (int b = 0; b < batch; ++b) {
+    const int32_t* bt = tok + (int64_t)b * n_max;
+    const int32_t* bp = parent + (int64_t)b * n_max;
+    const int32_t* bd = depth + (int64_t)b * n_max;
+    for (int j = 1; j < n_nodes[b]; ++j) {
+      /* the path's tokens, root excluded, from depth 1 down to depth d */
+      int path[DDTO_LMAX];
+      const int d = bd[j];
+      if (d < 1 || d > L) {
+        free(nodes);
+        return DDTO_ERR_ARG;
+      }
+      for (int x = j, t = d; t >= 1; x = bp[x], --t) path[t - 1] = bt[x];
+      double sz = 0.0, S = 0.0;
+      for (int t = 0; t < d; ++t) {
+        const int64_t row = ((int64_t)b * L + t) * kstride;
+        int r = 0;
+        while (r < kstride && ids[row + r] != path[t]) ++r;
+        if (r == kstride) {
+          free(nodes);
+          return DDTO_ERR_ARG;
+        }
+        sz = sz + zk[row + r];
+        S = S + lse[(int64_t)b * L + t];
+      }
+      const double a = invT * sz;
+      nodes[m].p = exp(a - S);
+      nodes[m].b = b;
+      nodes[m].j = j;
+      ++m;
+    }
+  }
+  qsort(nodes, (size_t)m, sizeof(pnode_t), cmp_pnode);
+  int cap = m;
+  if (total_budget >= 0 && total_budget < cap) cap = total_budget;
+  int best_n = cap;
+  if (c1 > 0.0) {
+    double P = 0.0, best = (double)batch / c0;
+    best_n = 0;
+    for (int n = 1; n <= cap; ++n) {
+      P += nodes[n - 1].p;
+      const double f = ((double)batch + P) / (c0 + c1 * (double)n);
+      if (f > best) {
+        best = f;
+        best_n = n;
+      }
+    }
+  }
+  for (int b = 0; b < batch; ++b) {
+    budget[b] = 0;
+    expected_tokens[b] = 1.0;
+  }
+  for (int i = 0; i < best_n; ++i) {
+    budget[nodes[i].b] += 1;
+    expected_tokens[nodes[i].b] += nodes[i].p;
+  }
+  *n_taken = best_n;
+  free(nodes);
+  return DDTO_OK;
+}
