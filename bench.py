@@ -69,6 +69,10 @@ def parse():
     ap.add_argument("--extensions", action="store_true",
                     help="with --profile: also run the sampled walk and the KV commit after "
                          "each round")
+    ap.add_argument("--no-budget-sweep", action="store_true",
+                    help="skip the budget sweep and the adaptive round in the bench line")
+    ap.add_argument("--line-budgets", default="16,32,64,128,256")
+    ap.add_argument("--line-sweep-draws", type=int, default=16)
     ap.add_argument("--no-per-workload", action="store_true",
                     help="skip the rounds of the other workloads (b256, paged128, long512)")
     ap.add_argument("--per-workload", default="b256,paged128,long512")
@@ -817,6 +821,9 @@ def run_ours(args):
     per_wl = (measure_per_workload(args.per_workload.split(","), hbm_peak, tf_peak,
                                    max(10, args.steps))
               if rank == 0 and not args.no_per_workload else None)
+    sweep = (budget_sweep(w, [int(b) for b in args.line_budgets.split(",")], args.sweep_batch,
+                          args.line_sweep_draws, args.sweep_invt)
+             if rank == 0 and not args.no_budget_sweep else None)
 
     # end to end: pinned host inputs -> H2D -> round -> D2H of the result, every step
     e2e = None
@@ -893,7 +900,7 @@ def run_ours(args):
             "roofline": roof, "stages": stages, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps, "clocks": clk,
             "mean_accepted": round(statistics.mean(acc), 3), "extensions": ext,
-            "per_workload": per_wl,
+            "per_workload": per_wl, "budget_sweep": sweep,
             "parallelism": "dp%d (independent sequences per GPU)" % world}
     print(json.dumps(line), flush=True)
     if world > 1:
@@ -964,44 +971,49 @@ def plant_targets(target, probs, depth, n_nodes, L, gen):
     return tok
 
 
-def run_sweep(args):
+def budget_sweep(w0, budgets, batch, draws, invt, spread=(0.5, 1.5), seed=2024, adaptive=True):
     """Budget sweep (DDTree page, 實驗結果與權衡: acceptance grows with the node
-    budget B while the verifier's cost grows too).  For each B: device time of
-    one round (CUDA graph, median of launches after an L2 flush), and the mean
-    accepted length over target resamplings planted from the drafter's own
-    marginals, next to the tree's surrogate (their expectation)."""
+    budget B while the verifier's cost grows too) on a batch whose sequences
+    draft with different confidence (sequence b's draft logits scaled by a
+    factor from ``spread``).  For each B: device time of one round (CUDA
+    graph, median of launches after an L2 flush) and the mean accepted
+    length over target resamplings planted from the drafter's own marginals
+    (so that its expectation is the tree's surrogate, Proposition 1).  A
+    linear fit of round time against the batch's draft nodes gives a cost
+    model, and the adaptive round (ddt_plan_budget between two builds, the
+    largest B as every sequence's cap) is measured the same way."""
     import torch
-    from block_draft_tree_b200 import synth
     from block_draft_tree_b200.round import VerifyRound
 
-    w0 = synth.WORKLOADS[args.workload or WORKLOAD]
-    budgets = [int(x) for x in args.budgets.split(",")]
-    batch = args.sweep_batch
     gen = torch.Generator(device="cuda")
-    gen.manual_seed(2024)
+    gen.manual_seed(seed)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
-    rows_out = []
-    for B in budgets:
-        w = w0.scaled(batch=batch, B=B, inv_temperature=args.sweep_invt)
-        rnd = VerifyRound(batch=w.batch, L=w.L, V=w.V, k=w.k, B_max=w.B, hq=w.hq, hkv=w.hkv,
-                          d=w.d, max_ctx=w.ctx, draft_dtype=torch.bfloat16,
-                          target_dtype=torch.float32, inv_temperature=w.inv_temperature)
-        xh, _ = make_inputs(w, 0, 0)
-        xd = to_device(xh, w, torch)
-        xd["target"] = torch.randn((w.batch, w.n_max, w.V), dtype=torch.float32, device="cuda",
-                                   generator=gen)
+    Bmax = max(budgets)
+    wmax = w0.scaled(batch=batch, B=Bmax, inv_temperature=invt)
+    x, _ = device_inputs(wmax, seed)
+    scale = torch.linspace(spread[0], spread[1], batch, device="cuda")
+    x["draft"] = (x["draft"].float() * scale[:, None, None]).to(torch.bfloat16)
+    probs = torch.softmax(x["draft"].float() * invt, dim=-1)
+
+    def inputs_for(n_max):
+        xd = dict(x)
+        for key in ("q", "k_tree", "v_tree", "target"):
+            xd[key] = x[key][:, :n_max].contiguous()
+        return xd
+
+    def measure(rnd, xd, n_max):
         rnd.bind(xd)
         rnd.launch()
         torch.cuda.synchronize()
         o = rnd.out
-        probs = torch.softmax(xd["draft"].float() * w.inv_temperature, dim=-1)
-        acc, surr = [], []
-        for r in range(args.sweep_draws):
+        acc, surr, nodes = [], [], []
+        for _ in range(draws):
             xd["target"].normal_(generator=gen)
-            plant_targets(xd["target"], probs, o["depth"], o["n_nodes"], w.L, gen)
+            plant_targets(xd["target"], probs, o["depth"], o["n_nodes"], w0.L, gen)
             rnd.launch()
             acc.append(o["acc_len"].double().mean().item())
             surr.append(o["surrogate"].mean().item())
+            nodes.append(int(o["n_nodes"].sum().item()) - batch)
         g = rnd.capture()
         times = []
         for rep in range(23):
@@ -1013,20 +1025,58 @@ def run_sweep(args):
             torch.cuda.synchronize()
             if rep >= 3:
                 times.append(a.elapsed_time(e) * 1e3)
+        assert int(o["status"].item()) == 0, "device status raised"
         us = statistics.median(times)
         mean_acc = statistics.mean(acc)
-        rows_out.append({"B": B, "round_us": round(us, 2), "mean_accepted": round(mean_acc, 3),
-                         "surrogate": round(statistics.mean(surr), 3),
-                         "accepted_se": round(statistics.pstdev(acc) / max(1, len(acc)) ** 0.5, 3),
-                         "tokens_per_round": round(mean_acc + 1, 3),
-                         "tokens_per_s": round(w.batch * (mean_acc + 1) / (us * 1e-6), 1)})
-        print("# sweep row", json.dumps(rows_out[-1]), file=sys.stderr, flush=True)
-        del g, rnd, xd, probs
-        torch.cuda.empty_cache()
-    print(json.dumps({"sweep": w0.name, "batch": batch, "draws": args.sweep_draws,
-                      "draft_inv_temperature": args.sweep_invt,
-                      "target": "argmax planted from the drafter's marginals per row",
-                      "rows": rows_out}), flush=True)
+        row = {"round_us": round(us, 2), "draft_nodes": round(statistics.mean(nodes), 1),
+               "mean_accepted": round(mean_acc, 3), "surrogate": round(statistics.mean(surr), 3),
+               "accepted_se": round(statistics.pstdev(acc) / max(1, len(acc)) ** 0.5, 3),
+               "tokens_per_s": round(batch * (mean_acc + 1) / (us * 1e-6), 1)}
+        del g
+        return row
+
+    rows = []
+    for B in budgets:
+        w = w0.scaled(batch=batch, B=B, inv_temperature=invt)
+        rnd = VerifyRound(batch=batch, L=w.L, V=w.V, k=w.k, B_max=B, hq=w.hq, hkv=w.hkv, d=w.d,
+                          max_ctx=w.ctx, inv_temperature=invt)
+        row = dict(B=B, **measure(rnd, inputs_for(B + 1), B + 1))
+        rows.append(row)
+        print("# sweep row", json.dumps(row), file=sys.stderr, flush=True)
+        del rnd
+    # round time against draft nodes: least squares c0 + c1 * nodes
+    xs = np.array([r["draft_nodes"] for r in rows])
+    ys = np.array([r["round_us"] for r in rows])
+    c1, c0 = np.polyfit(xs, ys, 1)
+    out = {"workload": "%s shapes at batch %d" % (w0.name, batch), "draws": draws,
+           "draft_inv_temperature": invt,
+           "confidence_spread": "draft logits of sequence b scaled by %.2f .. %.2f" % spread,
+           "target": "argmax planted from the drafter's marginals per row", "rows": rows,
+           "cost_model": {"c0_us": round(float(c0), 2), "c1_us_per_node": round(float(c1), 4)}}
+    if adaptive and c1 > 0 and c0 > 0:
+        rnd = VerifyRound(batch=batch, L=w0.L, V=w0.V, k=w0.k, B_max=Bmax, hq=w0.hq, hkv=w0.hkv,
+                          d=w0.d, max_ctx=w0.ctx, inv_temperature=invt,
+                          adaptive_budget={"total": -1, "cost_fixed": float(c0),
+                                           "cost_per_node": float(c1)})
+        row = measure(rnd, inputs_for(Bmax + 1), Bmax + 1)
+        row["budgets"] = rnd.out["budget"].cpu().tolist()
+        out["adaptive"] = dict(cap=Bmax, **row)
+        best = max(rows, key=lambda r: r["tokens_per_s"])
+        out["best_fixed"] = {"B": best["B"], "tokens_per_s": best["tokens_per_s"]}
+        print("# adaptive", json.dumps(out["adaptive"]), file=sys.stderr, flush=True)
+        del rnd
+    del x, probs
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_sweep(args):
+    """The budget sweep alone (see budget_sweep), one JSON line."""
+    from block_draft_tree_b200 import synth
+    w0 = synth.WORKLOADS[args.workload or WORKLOAD]
+    budgets = [int(x) for x in args.budgets.split(",")]
+    res = budget_sweep(w0, budgets, args.sweep_batch, args.sweep_draws, args.sweep_invt)
+    print(json.dumps({"sweep": res}), flush=True)
     return 0
 
 

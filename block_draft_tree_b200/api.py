@@ -31,13 +31,14 @@ EXPORTED = ("ddt_status_string", "ddt_mask_words", "ddt_topk_workspace_size", "d
             "ddt_tree_walk_workspace_size", "ddt_tree_walk", "ddt_tree_walk_sample",
             "ddt_kv_commit", "ddt_lm_head_max_rows", "ddt_lm_head_walk_workspace_size",
             "ddt_lm_head_walk", "ddt_tree_attn_plan", "ddt_debug_set_wait_limit",
-            "ddt_topk_noalloc", "ddt_tree_walk_resolve_mode")
+            "ddt_topk_noalloc", "ddt_tree_walk_resolve_mode", "ddt_plan_budget")
 
 # ddt_tree_walk's modes
 WALK_ALL_ROWS, WALK_LAZY, WALK_AUTO = 0, 1, 2
 
 # ddt_tree_attn_plan's paths
 ATTN_PATH_SIMT, ATTN_PATH_TC, ATTN_PATH_TC_CLUSTER, ATTN_PATH_TC_COMBINE = 0, 1, 2, 3
+ATTN_PATH_TC_PAIRS, ATTN_PATH_TC_PAIRS_COMBINE = 4, 5
 
 
 class KVCommitArgs(ctypes.Structure):
@@ -125,6 +126,9 @@ def load_library():
         lib.ddt_tree_walk.restype = i32
         lib.ddt_tree_walk.argtypes = [vp, i32, i32, i32, i32, i64, vp, vp, vp, vp, i32, i32,
                                       vp, vp, vp, vp, vp, sz, vp, vp]
+        lib.ddt_plan_budget.restype = i32
+        lib.ddt_plan_budget.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, f32, i32,
+                                        ctypes.c_double, ctypes.c_double, vp, vp, vp, vp]
         lib.ddt_tree_walk_resolve_mode.restype = i32
         lib.ddt_tree_walk_resolve_mode.argtypes = [i32, i32, i32, i32, i32, i32]
         lib.ddt_lm_head_max_rows.restype = i32
@@ -265,6 +269,30 @@ def build_tree(ids: torch.Tensor, zk: torch.Tensor, lse: torch.Tensor, B_max: in
                                 _stream(dev))
     _check(rc, "ddt_build_tree")
     return out
+
+
+def plan_budget(tree: dict, ids: torch.Tensor, zk: torch.Tensor, lse: torch.Tensor,
+                inv_temperature: float = 1.0, total_budget: int = -1, cost_fixed: float = 0.0,
+                cost_per_node: float = 0.0, dev_status: Optional[torch.Tensor] = None):
+    """``ddt_plan_budget``: each sequence's share of the batch's node budget,
+    from ``tree`` (tok, parent, depth, n_nodes of a build with the largest
+    budgets) and the candidates ``ids``/``zk`` [batch, L, k], ``lse`` [batch, L]
+    it was built from.  Returns (budget int32 [batch], expected_tokens f64
+    [batch]); pass ``budget`` to :func:`build_tree` as its per-sequence budget."""
+    lib = load_library()
+    dev = _need_cuda(ids, zk, lse, tree["tok"], dev_status)
+    b, L, k = ids.shape
+    n_max = tree["tok"].shape[1]
+    budget = torch.empty(b, dtype=torch.int32, device=dev)
+    exp_tok = torch.empty(b, dtype=torch.float64, device=dev)
+    with torch.cuda.device(dev):
+        rc = lib.ddt_plan_budget(_ptr(tree["tok"]), _ptr(tree["parent"]), _ptr(tree["depth"]),
+                                 _ptr(tree["n_nodes"]), _ptr(ids), _ptr(zk), _ptr(lse), b, L, k,
+                                 n_max, float(inv_temperature), int(total_budget),
+                                 float(cost_fixed), float(cost_per_node), _ptr(budget),
+                                 _ptr(exp_tok), _ptr(dev_status), _stream(dev))
+    _check(rc, "ddt_plan_budget")
+    return budget, exp_tok
 
 
 def _attn_args(q, k_cache, v_cache, k_tree, v_tree, mask, n_nodes, ctx_len, max_ctx, scale,

@@ -75,6 +75,7 @@ int attn_simt_rows_per_cta();
 bool attn_tc_eligible(const ddt_attn_args* a);
 void attn_tc_plan(const ddt_attn_args* a, int sms, int* qtiles, int* nsplit, int* tps);
 bool attn_tc_cluster(int nsplit, long clusters);
+bool attn_pair_plan(const ddt_attn_args* a, int sms, int* qtiles, int* nsplit, int* tps);
 size_t attn_tc_workspace_size(const ddt_attn_args* a, int sms);
 ddt_status launch_attn_tc(const ddt_attn_args* a, void* ws, int sms, cudaStream_t stream);
 
@@ -255,6 +256,30 @@ ddt_status ddt_build_tree(const int32_t* ids, const float* zk, const float* lse,
                            surrogate, dev_status, stream);
 }
 
+ddt_status ddt_plan_budget(const int32_t* tok, const int32_t* parent, const int32_t* depth,
+                           const int32_t* n_nodes, const int32_t* ids, const float* zk,
+                           const float* lse, int batch, int L, int k, int n_max,
+                           float inv_temperature, int total_budget, double cost_fixed,
+                           double cost_per_node, int32_t* budget_per_seq, double* expected_tokens,
+                           int32_t* dev_status, cudaStream_t stream) {
+  const NvtxRange nvtx("ddt_plan_budget");
+  if (batch < 0 || L < 1 || k < 1 || n_max < 1) return DDT_ERR_INVALID_ARG;
+  if (L > DDT_TREE_L_MAX || k > DDT_TOPK_K_MAX || n_max > DDT_TREE_B_MAX + 1)
+    return DDT_ERR_UNSUPPORTED;
+  if ((int64_t)batch * (n_max - 1) > plan_budget_max_nodes()) return DDT_ERR_UNSUPPORTED;
+  if (!(inv_temperature > 0.f) || !(inv_temperature < INFINITY)) return DDT_ERR_INVALID_ARG;
+  if (!(cost_fixed >= 0.0) || !(cost_fixed < INFINITY) || !(cost_per_node < INFINITY) ||
+      cost_per_node != cost_per_node)
+    return DDT_ERR_INVALID_ARG;
+  if (cost_per_node > 0.0 && !(cost_fixed > 0.0)) return DDT_ERR_INVALID_ARG;
+  if (batch > 0 && (!tok || !parent || !depth || !n_nodes || !ids || !zk || !lse ||
+                    !budget_per_seq))
+    return DDT_ERR_INVALID_ARG;
+  return launch_plan_budget(tok, parent, depth, n_nodes, ids, zk, lse, batch, L, k, n_max,
+                            inv_temperature, total_budget, cost_fixed, cost_per_node,
+                            budget_per_seq, expected_tokens, dev_status, stream);
+}
+
 static ddt_status check_attn(const ddt_attn_args* a) {
   if (!a) return DDT_ERR_INVALID_ARG;
   if (a->batch < 0 || a->n_max < 1 || a->hq < 1 || a->hkv < 1 || a->max_ctx < 0)
@@ -306,10 +331,14 @@ ddt_status ddt_tree_attn_plan(const ddt_attn_args* a, int* path, int* kv_splits)
   int pth, ns;
   if (attn_tc_eligible(a)) {
     int qt, tps;
-    attn_tc_plan(a, sm_count(), &qt, &ns, &tps);
-    if (ns <= 1) pth = DDT_ATTN_PATH_TC;
-    else if (attn_tc_cluster(ns, (long)qt * a->batch * a->hkv)) pth = DDT_ATTN_PATH_TC_CLUSTER;
-    else pth = DDT_ATTN_PATH_TC_COMBINE;
+    if (attn_pair_plan(a, sm_count(), &qt, &ns, &tps)) {
+      pth = ns <= 1 ? DDT_ATTN_PATH_TC_PAIRS : DDT_ATTN_PATH_TC_PAIRS_COMBINE;
+    } else {
+      attn_tc_plan(a, sm_count(), &qt, &ns, &tps);
+      if (ns <= 1) pth = DDT_ATTN_PATH_TC;
+      else if (attn_tc_cluster(ns, (long)qt * a->batch * a->hkv)) pth = DDT_ATTN_PATH_TC_CLUSTER;
+      else pth = DDT_ATTN_PATH_TC_COMBINE;
+    }
   } else {
     int rt, tps;
     attn_plan(a, attn_simt_rows_per_cta(), &rt, &ns, &tps);

@@ -256,11 +256,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   fence_after();
   const uint32_t tmem = bars->tmem_base;
 
-  if (ntiles == 0 && !p.cluster) {  // nothing in this split: an empty partial (or zero rows)
-    if (tid >= 64 && tid < 64 + BM) {
+  // nothing to compute: an empty split, or a tile whose rows are all past
+  // n_nodes (zero rows, written once: by split 0 of a cluster)
+  const bool dead = q0 / g >= n;
+  if ((ntiles == 0 && !p.cluster) || dead) {
+    if (tid >= 64 && tid < 64 + BM && !(p.cluster && split != 0)) {
       const int row = tid - 64;
       const int qr = q0 + row;
-      if (p.nsplit > 1) {
+      if (p.nsplit > 1 && !p.cluster) {
         float4* po = (float4*)(p.part_o + (part_row0 + row) * D);
         for (int i = 0; i < D / 4; ++i) po[i] = make_float4(0.f, 0.f, 0.f, 0.f);
         p.part_ml[part_row0 + row] = make_float2(-INFINITY, 0.f);
@@ -497,23 +500,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) continue;
       }
       fence_after();
-      if (move) {
-        if (i > 0 && m_used != -INFINITY) {
-          const float alpha = ex2(m_used - m_new);
-          uint32_t o[32];
+      // rows whose maximum moved rescale O; the whole warp takes part in the
+      // TMEM accesses (they are warp-collective), the other rows by 1
+      const bool resc = move && i > 0 && m_used != -INFINITY;
+      if (__any_sync(0xFFFFFFFFu, resc)) {
+        const float alpha = resc ? ex2(m_used - m_new) : 1.f;
+        uint32_t o[32];
 #pragma unroll
-          for (int c = 0; c < D / 64; ++c) {
-            const uint32_t oc = kColO + half * (D / 2) + 32 * c;
-            tmem_ld32(lane_base + oc, o);
-            tmem_ld_wait();
+        for (int c = 0; c < D / 64; ++c) {
+          const uint32_t oc = kColO + half * (D / 2) + 32 * c;
+          tmem_ld32(lane_base + oc, o);
+          tmem_ld_wait();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st32(lane_base + oc, o);
-          }
-          l *= alpha;
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(lane_base + oc, o);
         }
-        m_used = m_new;
+        l *= alpha;
       }
+      if (move) m_used = m_new;
       l += rs;
       tmem_st32(lane_base + kColP + half * (BN / 4), r);
       // token row `row` of a partial tile: zero its V row (this half's 64
@@ -673,6 +677,453 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   cluster_sync();  // peers' shared memory stays alive until every CTA has read it
 }
+
+// ---------------------------------------------------------------------------
+// Two query tiles per CTA
+// ---------------------------------------------------------------------------
+// Where a kv head has at least two query tiles, one CTA takes a pair of them
+// (A and B: 256 query rows) over its KV range: every K/V tile is loaded once
+// for both, so each byte staged feeds twice the MMA work, and the two tiles'
+// softmax work overlaps the other tile's MMAs.  Warp 0 loads (Q_A and Q_B
+// once; K_i and V_i into a ring of four 32 KB slots, two tiles ahead), warp 1
+// issues the MMAs, warps 2-5 are tile A's softmax and warps 6-9 tile B's, one
+// query row per thread (the thread's TMEM lane), all 128 scores of a tile
+// in registers.  TMEM: S_A, S_B (128 columns each), O_A, O_B (128 each); a
+// tile's P (bf16 pairs, 64 columns) overwrites the first half of its S.
+// MMA order per KV tile i:  [P_A(i) ready] PV_A(i), QK_A(i+1);
+// [P_B(i) ready] PV_B(i), QK_B(i+1): while one tile's softmax runs, the
+// tensor cores work for the other.  A commit after QK_t(i+1) completes after
+// PV_t(i) too (commits cover every earlier MMA of the thread), so the softmax
+// of tile i+1 may rescale O_t without another wait.
+constexpr int kPairThreads = 320;
+constexpr uint32_t kColSA = 0, kColSB = 128, kColOA = 256, kColOB = 384;
+
+struct __align__(8) PairBars {
+  uint64_t q_full;
+  uint64_t kv_full[4];
+  uint64_t kv_empty[4];
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t o_full;
+  uint64_t drain;
+  long long wait_cycles;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ __forceinline__ bool pair_wait(uint64_t* b, uint32_t parity, PairBars* bars) {
+  return mbar_wait_bounded(b, parity, &bars->abort, bars->wait_cycles);
+}
+
+// Load the K (kind 0) or V (kind 1) rows of KV tile `ti` into `dst`.
+__device__ __forceinline__ void pair_load_kv(const Params& p, const TileInfo& ti, int b, int kvh, int T,
+                                             int kind, unsigned char* dst, uint64_t* bar,
+                                             const CUtensorMap* tm_c, const CUtensorMap* tm_t) {
+  if (ti.tree) {
+    const int row = b * p.n_max + ti.base;
+    mbar_expect_tx(bar, (uint32_t)kTile);
+    for (int h = 0; h < 2; ++h) tma_load_3d(dst + h * kHalf, tm_t, 64 * h, kvh, row, bar);
+  } else if (!p.paged) {
+    const int row = (int)((int64_t)b * p.t_max + ti.base);
+    mbar_expect_tx(bar, (uint32_t)kTile);
+    for (int h = 0; h < 2; ++h) tma_load_3d(dst + h * kHalf, tm_c, 64 * h, kvh, row, bar);
+  } else {
+    const int rpb = p.rows_per_box;
+    int nbox = 0;
+    for (int bx = 0; bx < p.boxes_per_tile; ++bx)
+      if (ti.base + bx * rpb < T) ++nbox;
+    mbar_expect_tx(bar, (uint32_t)(nbox * rpb * 128 * 2));
+    for (int bx = 0; bx < nbox; ++bx) {
+      const int tok = ti.base + bx * rpb;
+      const int page = p.page_table[(int64_t)b * p.max_pages + tok / p.page_size];
+      const int slot = tok % p.page_size;
+      for (int h = 0; h < 2; ++h)
+        tma_load_4d(dst + h * kHalf + bx * rpb * 128, tm_c, 64 * h, kvh, slot, page, bar);
+    }
+  }
+  (void)kind;
+}
+
+__global__ void __launch_bounds__(kPairThreads, 1)
+    attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kt,
+                     const __grid_constant__ CUtensorMap tm_vt, const Params p) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  unsigned char* sQ = smem;                 // [2 tiles][2 halves][128][128 B]
+  unsigned char* sKV = smem + 2 * kTile;    // [4 slots][2 halves][128][128 B]
+  PairBars* bars = (PairBars*)(sKV + 4 * kTile);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int pair = blockIdx.x, split = blockIdx.y, grp = blockIdx.z;
+  const int b = grp / p.hkv, kvh = grp % p.hkv;
+  if (tid == 0) {
+    mbar_init(&bars->q_full, 1);
+    for (int s = 0; s < 4; ++s) {
+      mbar_init(&bars->kv_full[s], 1);
+      mbar_init(&bars->kv_empty[s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bars->s_full[t], 1);
+      mbar_init(&bars->p_full[t], 128);
+    }
+    mbar_init(&bars->o_full, 1);
+    mbar_init(&bars->drain, 1);
+    bars->wait_cycles = p.wait_cycles;
+    bars->abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      prefetch_tmap(&tm_kt);
+      prefetch_tmap(&tm_vt);
+    }
+    __syncwarp();
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&bars->tmem_base)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  pdl_wait();
+  const int g = p.g;
+  const int R = p.n_max * g;
+  const int q0 = pair * 2 * BM;
+  int n = p.n_nodes[b];
+  n = min(max(n, 1), p.n_max);
+  // tile B exists when it holds query rows; a tile works when one of its
+  // rows belongs to a tree row (rows past n_nodes only get zeros)
+  const bool a_work = q0 / g < n;
+  const bool b_exists = q0 + BM < R;
+  const bool has_b = b_exists && (q0 + BM) / g < n;
+  int T = p.ctx_len[b];
+  if (T < 0 || T > p.max_ctx) {
+    if (pair == 0 && split == 0 && kvh == 0 && tid == 0) raise_status(p.status, DDT_ERR_INVALID_ARG);
+    T = min(max(T, 0), p.max_ctx);
+  }
+  const int nct = (T + BN - 1) / BN;
+  const int ntt = (n + BN - 1) / BN;
+  const int t_lo = min(split * p.tiles_per_split, nct + ntt);
+  const int t_hi = min(t_lo + p.tiles_per_split, nct + ntt);
+  const int ntiles = a_work ? t_hi - t_lo : 0;  // KV tiles this CTA processes
+
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && ntiles > 0) {
+      const int j0 = q0 / g;
+      mbar_expect_tx(&bars->q_full, (uint32_t)((has_b ? 2 : 1) * kTile));
+      for (int t = 0; t < (has_b ? 2 : 1); ++t)
+        for (int h = 0; h < 2; ++h)
+          tma_load_3d(sQ + t * kTile + h * kHalf, &tm_q, 64 * h, kvh * g, b * p.n_max + j0 + t * (BM / g),
+                      &bars->q_full);
+      int issued = 0;  // K/V loads issued (two per tile)
+      for (int i = 0; i < ntiles; ++i) {
+        const TileInfo ti = tile_info(t_lo + i, nct, T, n);
+        bool ok = true;
+        for (int kind = 0; kind < 2 && ok; ++kind) {
+          const int s = (2 * i + kind) & 3;
+          if (!pair_wait(&bars->kv_empty[s], ((uint32_t)(i >> 1) & 1u) ^ 1u, bars)) {
+            ok = false;
+            break;
+          }
+          pair_load_kv(p, ti, b, kvh, T, kind, sKV + s * kTile, &bars->kv_full[s],
+                       kind ? &tm_v : &tm_k, kind ? &tm_vt : &tm_kt);
+          ++issued;
+        }
+        if (!ok) break;
+      }
+      if (*(volatile int*)&bars->abort) {
+        // a wait gave up: let the loads in flight land before the CTA (and
+        // its shared memory) goes away; only the Q tiles and the last four
+        // K/V loads can be outstanding, each on a slot with one phase pending
+        int keep_going = 0;
+        mbar_wait_bounded(&bars->q_full, 0u, &keep_going, kDrainCycles);
+        for (int c = issued > 4 ? issued - 4 : 0; c < issued; ++c)
+          mbar_wait_bounded(&bars->kv_full[c & 3], (uint32_t)(c >> 2) & 1u, &keep_going, kDrainCycles);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && ntiles > 0) {
+      constexpr uint32_t kIdQK = idesc_bf16(false);
+      constexpr uint32_t kIdPV = idesc_bf16(true);
+      const int nt = has_b ? 2 : 1;
+      auto qk = [&](int t, int i) {  // S_t = Q_t K_i^T
+        const uint32_t q_addr = smem_u32(sQ + t * kTile);
+        const uint32_t k_addr = smem_u32(sKV + ((2 * i) & 3) * kTile);
+        const uint32_t d_tm = tmem + (t ? kColSB : kColSA);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (uint32_t)((kk >> 2) * kHalf + (kk & 3) * 32);
+          mma_ss(d_tm, sdesc(q_addr + off, 16, 1024), sdesc(k_addr + off, 16, 1024), kIdQK,
+                 kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&bars->s_full[t]);
+      };
+      auto pv = [&](int t, int i) {  // O_t += P_t V_i, P_t in the first half of S_t
+        const uint32_t v_addr = smem_u32(sKV + ((2 * i + 1) & 3) * kTile);
+        const uint32_t s_col = t ? kColSB : kColSA, o_col = t ? kColOB : kColOA;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_ts(tmem + o_col, tmem + s_col + kk * 8, sdesc(v_addr + kk * 2048, kHalf, 1024), kIdPV,
+                 (i > 0 || kk > 0) ? 1u : 0u);
+      };
+      bool ok = pair_wait(&bars->q_full, 0, bars) && pair_wait(&bars->kv_full[0], 0, bars);
+      if (ok) {
+        fence_after();
+        for (int t = 0; t < nt; ++t) qk(t, 0);
+      }
+      for (int i = 0; ok && i < ntiles; ++i) {
+        const int ks = (2 * i) & 3, vs = (2 * i + 1) & 3;
+        const uint32_t ph = (uint32_t)(i >> 1) & 1u;
+        const bool next = i + 1 < ntiles;
+        const int ks1 = (2 * i + 2) & 3;
+        const uint32_t ph1 = (uint32_t)((i + 1) >> 1) & 1u;
+        if (!pair_wait(&bars->kv_full[vs], ph, bars)) break;
+        for (int t = 0; t < nt; ++t) {
+          if (!pair_wait(&bars->p_full[t], (uint32_t)i & 1u, bars) ||
+              (next && t == 0 && !pair_wait(&bars->kv_full[ks1], ph1, bars))) {
+            ok = false;
+            break;
+          }
+          fence_after();
+          pv(t, i);
+          if (next) qk(t, i + 1);
+        }
+        if (!ok) break;
+        mma_commit(&bars->kv_empty[ks]);  // K_i and V_i are free once every MMA so far is done
+        mma_commit(&bars->kv_empty[vs]);
+      }
+      if (ok) mma_commit(&bars->o_full);
+      if (*(volatile int*)&bars->abort) {
+        int keep_going = 0;
+        mma_commit(&bars->drain);
+        mbar_wait_bounded(&bars->drain, 0u, &keep_going, kDrainCycles);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warps
+    const int t = (warp - 2) >> 2;         // tile 0 (A) or 1 (B)
+    const int quarter = warp & 3;          // TMEM lanes 32*quarter .. +31
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t s_col = t ? kColSB : kColSA, o_col = t ? kColOB : kColOA;
+    const int qr = q0 + t * BM + row;
+    const int j = qr / g;
+    const bool tile_live = t == 0 || has_b;     // the tile has tree rows to compute
+    const bool tile_rows = t == 0 || b_exists;  // the tile has query rows to write
+    const bool row_valid = tile_live && qr < R && j < n;
+    const uint32_t* mrow = p.mask + ((int64_t)b * p.n_max + (j < p.n_max ? j : 0)) * p.W;
+    const float c_log2 = p.scale_log2;
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int i = 0; tile_live && i < ntiles; ++i) {
+      const TileInfo ti = tile_info(t_lo + i, nct, T, n);
+      if (ok) ok = __all_sync(0xFFFFFFFFu, pair_wait(&bars->s_full[t], (uint32_t)i & 1u, bars));
+      if (!ok) break;
+      fence_after();
+      // the tile's mask words for this row (all ones for full context tiles)
+      uint32_t mw[BN / 32];
+      const bool masked = ti.tree || ti.cnt < BN || !row_valid;
+#pragma unroll
+      for (int w = 0; w < BN / 32; ++w) {
+        mw[w] = 0xFFFFFFFFu;
+        if (masked) {
+          mw[w] = 0u;
+          if (row_valid) {
+            if (ti.tree) {
+              const int word = (ti.base >> 5) + w;
+              mw[w] = word < p.W ? mrow[word] : 0u;
+            } else {
+              const int lo = 32 * w;
+              mw[w] = ti.cnt >= lo + 32 ? 0xFFFFFFFFu : (ti.cnt > lo ? ((1u << (ti.cnt - lo)) - 1u) : 0u);
+            }
+          }
+        }
+      }
+      // pass 1: the row maximum, 32 scores at a time (the scores stay in TMEM)
+      float mx = -INFINITY;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(lane_base + s_col + 32 * c, r);
+        tmem_ld_wait();
+        if (masked) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (!((mw[c] >> e) & 1u)) r[e] = 0xFF800000u;  // -inf
+        }
+        float m4[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) m4[e] = __uint_as_float(r[e]);
+#pragma unroll
+        for (int e = 4; e < 32; e += 2)
+          m4[(e >> 1) & 3] = fmax3(m4[(e >> 1) & 3], __uint_as_float(r[e]), __uint_as_float(r[e + 1]));
+        mx = fmaxf(mx, fmax3(fmax3(m4[0], m4[1], m4[2]), m4[3], mx));
+      }
+      mx *= c_log2;
+      const float m_new = fmaxf(m_used, mx);
+      const bool move = m_new > m_used + kRescaleLog2 || (m_used == -INFINITY && m_new != -INFINITY);
+      const float m_tgt = move ? m_new : m_used;
+      // pass 2: p = 2^(s*c - m), two scores at a time: a packed FFMA for the
+      // exponents, then MUFU ex2 -- or, for 3 pairs in 8, exp2_poly2 on the
+      // FMA pipe; packed sums; bf16 pairs stored over the scores already read
+      uint64_t rs2[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) rs2[e] = 0ull;
+      const uint64_t c2 = pack2(c_log2, c_log2), nm2 = pack2(-m_tgt, -m_tgt);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32], pk[16];
+        tmem_ld32(lane_base + s_col + 32 * c, r);  // every lane: tcgen05.ld is warp-collective
+        tmem_ld_wait();
+        if (m_tgt == -INFINITY) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pk[e] = 0u;
+        } else {
+          if (masked) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (!((mw[c] >> e) & 1u)) r[e] = 0xFF800000u;
+          }
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const uint64_t x2 = ffma2(pack2(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), c2, nm2);
+            float a, bb;
+            if (((e >> 1) & 7) < 3) {
+              exp2_poly2(x2, a, bb);
+            } else {
+              float xa, xb;
+              unpack2(x2, xa, xb);
+              a = ex2(xa);
+              bb = ex2(xb);
+            }
+            rs2[(e >> 1) & 3] = fadd2(rs2[(e >> 1) & 3], pack2(a, bb));
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(a, bb);
+            pk[e >> 1] = *(uint32_t*)&h2;
+          }
+        }
+        tmem_st16(lane_base + s_col + 16 * c, pk);
+      }
+      float rs8[8];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) unpack2(rs2[e], rs8[2 * e], rs8[2 * e + 1]);
+      const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+      // O_t already holds PV_t(i-1) (complete: the commit behind s_full covers
+      // it); rows whose maximum moved rescale it -- the whole warp takes part
+      // in the TMEM accesses (they are warp-collective), the others by 1
+      const bool resc = move && i > 0 && m_used != -INFINITY;
+      if (__any_sync(0xFFFFFFFFu, resc)) {
+        const float alpha = resc ? ex2(m_used - m_new) : 1.f;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(lane_base + o_col + 32 * c, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(lane_base + o_col + 32 * c, o);
+        }
+        l *= alpha;
+      }
+      if (move) m_used = m_new;
+      l += rs;
+      // token row `row` of a partial KV tile: zero its V row (both halves)
+      // so that 0 * garbage cannot turn into NaN in the PV product; tile A's
+      // threads do it, once V_i has landed, before PV_A(i), which comes first
+      if (t == 0 && ti.cnt < BN &&
+          !__all_sync(0xFFFFFFFFu, pair_wait(&bars->kv_full[(2 * i + 1) & 3], (uint32_t)(i >> 1) & 1u, bars))) {
+        ok = false;
+        break;
+      }
+      if (t == 0 && row >= ti.cnt) {
+        unsigned char* vt = sKV + ((2 * i + 1) & 3) * kTile;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint4* vrow = (uint4*)(vt + h * kHalf + row * 128);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) vrow[e] = make_uint4(0, 0, 0, 0);
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      }
+      tmem_st_wait();
+      fence_before();
+      mbar_arrive(&bars->p_full[t]);
+    }
+    if (tile_live && ok && ntiles > 0)
+      ok = __all_sync(0xFFFFFFFFu, pair_wait(&bars->o_full, 0, bars));
+    // epilogue: the O row -> final output or a split partial
+    const bool final_out = p.nsplit == 1;
+    const int qt = 2 * pair + t;  // query tile index of this tile
+    const int64_t prow = (((int64_t)grp * p.qtiles + qt) * p.nsplit + split) * BM + row;
+    const bool has = ok && row_valid && l > 0.f && ntiles > 0;
+    const float inv = has ? 1.f / l : 0.f;
+    // (TMEM loads by every lane of the warp: they are warp-collective)
+    const bool writes = final_out ? qr < R : qt < p.qtiles;
+    if (tile_rows) {
+      fence_after();
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        if (tile_live && ntiles > 0) {
+          tmem_ld32(lane_base + o_col + 32 * c, o);
+          tmem_ld_wait();
+        }
+        if (!has) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = 0u;
+        }
+        if (!writes) {
+        } else if (final_out) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(o[2 * e]) * inv,
+                                                     __uint_as_float(o[2 * e + 1]) * inv);
+            pk[e] = *(uint32_t*)&h2;
+          }
+          uint4* d4 = (uint4*)(p.out + (((int64_t)b * p.n_max + j) * p.hq + (kvh * g + qr % g)) * D + 32 * c);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) d4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+        } else {
+          float4* q4 = (float4*)(p.part_o + prow * D + 32 * c);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            q4[e] = make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
+                                __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]));
+        }
+      }
+      if (writes && final_out) {
+        if (p.lse_out)
+          p.lse_out[((int64_t)b * p.n_max + j) * p.hq + (kvh * g + qr % g)] =
+              has ? (m_used + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+      } else if (writes) {
+        p.part_ml[prow] = has ? make_float2(m_used, l) : make_float2(-INFINITY, 0.f);
+      }
+    }
+  }
+
+  pdl_trigger();
+  fence_before();
+  __syncthreads();
+  if (bars->abort && tid == 0) raise_status(p.status, DDT_ERR_TIMEOUT);
+  if (warp == 0) {
+    __syncwarp();
+    fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+size_t pair_smem_bytes() { return 1024 + (size_t)6 * kTile + sizeof(PairBars) + 64; }
 
 // Merge the per-split partials: one warp per query row, 4 dims per lane.
 __global__ void __launch_bounds__(256) attn_tc_combine(const Params p) {
@@ -863,10 +1314,42 @@ bool attn_tc_cluster(int nsplit, long clusters) {
   return known[nsplit] > 0 && clusters <= known[nsplit];
 }
 
+// The two-query-tile kernel serves every call with at least two query tiles
+// per kv head whose splits would not merge on chip.  Its KV-split plan
+// minimises waves x tiles per split (plus the combine's cost when split).
+bool attn_pair_plan(const ddt_attn_args* a, int sms, int* qtiles, int* nsplit, int* tps) {
+  int qt, ns, t;
+  attn_tc_plan(a, sms, &qt, &ns, &t);
+  if (qt < 2 || (ns > 1 && attn_tc_cluster(ns, (long)qt * a->batch * a->hkv))) return false;
+  const long base = (long)((qt + 1) / 2) * a->batch * a->hkv;
+  const int tiles = (a->max_ctx + tc::BN - 1) / tc::BN + (a->n_max + tc::BN - 1) / tc::BN;
+  constexpr int kMergeTiles = 3;
+  long best_cost = -1;
+  int best_s = 1;
+  for (int s = 1; s <= 16 && s <= tiles; ++s) {
+    const int ts = (tiles + s - 1) / s;
+    const int sp = (tiles + ts - 1) / ts;
+    const long waves = (base * sp + sms - 1) / sms;
+    const long cost = waves * ts + (sp > 1 ? kMergeTiles : 0);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best_s = s;
+    }
+  }
+  *qtiles = qt;
+  *tps = (tiles + best_s - 1) / best_s;
+  *nsplit = (tiles + *tps - 1) / *tps;
+  return true;
+}
+
 size_t attn_tc_workspace_size(const ddt_attn_args* a, int sms) {
   int qt, ns, tps;
-  attn_tc_plan(a, sms, &qt, &ns, &tps);
-  if (ns <= 1 || attn_tc_cluster(ns, (long)qt * a->batch * a->hkv)) return 0;
+  if (!attn_pair_plan(a, sms, &qt, &ns, &tps)) {
+    attn_tc_plan(a, sms, &qt, &ns, &tps);
+    if (ns <= 1 || attn_tc_cluster(ns, (long)qt * a->batch * a->hkv)) return 0;
+  } else if (ns <= 1) {
+    return 0;
+  }
   const size_t rows = (size_t)a->batch * a->hkv * qt * ns * tc::BM;
   return ((rows * tc::D * sizeof(float) + 255) & ~(size_t)255) + rows * sizeof(float2);
 }
@@ -896,8 +1379,9 @@ ddt_status launch_attn_tc(const ddt_attn_args* a, void* ws, int sms, cudaStream_
   p.lse_out = a->lse_out;
   p.status = a->dev_status;
   p.wait_cycles = wait_limit_cycles();
-  attn_tc_plan(a, sms, &p.qtiles, &p.nsplit, &p.tiles_per_split);
-  p.cluster = attn_tc_cluster(p.nsplit, (long)p.qtiles * a->batch * a->hkv) ? 1 : 0;
+  const bool pairs = attn_pair_plan(a, sms, &p.qtiles, &p.nsplit, &p.tiles_per_split);
+  if (!pairs) attn_tc_plan(a, sms, &p.qtiles, &p.nsplit, &p.tiles_per_split);
+  p.cluster = !pairs && attn_tc_cluster(p.nsplit, (long)p.qtiles * a->batch * a->hkv) ? 1 : 0;
   if (p.nsplit > 1 && !p.cluster) {
     const size_t rows = (size_t)a->batch * a->hkv * p.qtiles * p.nsplit * BM;
     p.part_o = (float*)ws;
@@ -938,12 +1422,21 @@ ddt_status launch_attn_tc(const ddt_attn_args* a, void* ws, int sms, cudaStream_
     mk = mkt;  // no context: never read
     mv = mvt;
   }
-  const size_t smem = smem_bytes();
-  if (ensure_smem_attr((const void*)attn_tc_kernel, smem) != cudaSuccess) return DDT_ERR_CUDA;
-  dim3 grid(p.qtiles, p.nsplit, a->batch * a->hkv);
-  if (launch_pdl(attn_tc_kernel, grid, dim3(kThreads), smem, stream, p.cluster ? p.nsplit : 0, mq, mk, mv, mkt,
-                 mvt, p) != cudaSuccess)
-    return DDT_ERR_CUDA;
+  if (pairs) {
+    const size_t smem = pair_smem_bytes();
+    if (ensure_smem_attr((const void*)attn_pair_kernel, smem) != cudaSuccess) return DDT_ERR_CUDA;
+    dim3 grid((p.qtiles + 1) / 2, p.nsplit, a->batch * a->hkv);
+    if (launch_pdl(attn_pair_kernel, grid, dim3(kPairThreads), smem, stream, 0, mq, mk, mv, mkt, mvt, p) !=
+        cudaSuccess)
+      return DDT_ERR_CUDA;
+  } else {
+    const size_t smem = smem_bytes();
+    if (ensure_smem_attr((const void*)attn_tc_kernel, smem) != cudaSuccess) return DDT_ERR_CUDA;
+    dim3 grid(p.qtiles, p.nsplit, a->batch * a->hkv);
+    if (launch_pdl(attn_tc_kernel, grid, dim3(kThreads), smem, stream, p.cluster ? p.nsplit : 0, mq, mk, mv,
+                   mkt, mvt, p) != cudaSuccess)
+      return DDT_ERR_CUDA;
+  }
   if (p.nsplit > 1 && !p.cluster) {
     if (launch_pdl(attn_tc_combine, dim3(p.qtiles * BM / 8, a->batch * a->hkv), dim3(256), 0, stream, 0, p) !=
         cudaSuccess)

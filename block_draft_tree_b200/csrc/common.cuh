@@ -124,6 +124,13 @@ __device__ __forceinline__ void raise_status(int32_t* st, int code) {
 
 // L2-coherent loads for data written by other CTAs of the same grid.
 __device__ __forceinline__ uint64_t ld_cg_u64(const uint64_t* p) { return __ldcg((const unsigned long long*)p); }
+// Atomic add, acquire-release at device scope (a ticket that publishes what
+// the CTA wrote before its barrier and sees what earlier holders wrote).
+__device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
 __device__ __forceinline__ float2 ld_cg_f2(const float2* p) { return __ldcg(p); }
 
 // Programmatic dependent launch: every kernel of the library is launched

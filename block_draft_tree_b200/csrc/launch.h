@@ -84,6 +84,14 @@ ddt_status launch_kv_commit(const ddt_kv_commit_args* a, cudaStream_t stream);
 ddt_status launch_lm_head_walk(const ddt_lm_head_walk_args* a, void* ws, cudaStream_t stream);
 int lm_head_max_rows();
 
+int plan_budget_max_nodes();
+ddt_status launch_plan_budget(const int32_t* tok, const int32_t* parent, const int32_t* depth,
+                              const int32_t* n_nodes, const int32_t* ids, const float* zk,
+                              const float* lse, int batch, int L, int k, int n_max,
+                              float inv_temperature, int total_budget, double c0, double c1,
+                              int32_t* budget, double* expected_tokens, int32_t* dev_status,
+                              cudaStream_t stream);
+
 struct AttnParams;
 size_t attn_workspace_size(const ddt_attn_args* a);
 ddt_status launch_attn(const ddt_attn_args* a, void* ws, size_t ws_bytes, cudaStream_t stream);

@@ -8,25 +8,27 @@
 // Design (an HBM-bound stream over the logits):
 //   * the rows are cut into 16 KB chunks and the chunks, in row order, into
 //     one contiguous range per CTA, as many CTAs as fit on the device at
-//     once; every CTA streams its range through a 4-deep ring of shared
+//     once; every CTA streams its range through a 3-deep ring of shared
 //     memory filled by 16-byte asynchronous copies (each thread copies and
 //     later reads the same 64 bytes of a chunk, so no barrier guards the
-//     ring), so that 48 KB per CTA are always in flight;
+//     ring), so that two chunks per CTA are always in flight;
 //   * per chunk, each thread folds its 32 (bf16) or 16 (f32) logits into a
 //     running (max, sum of 2^((z - max) * c)) and compares its chunk maximum
-//     with the CTA's current k-th best key: only a thread whose maximum beats
-//     it looks at its logits again and appends the ones that do to a
-//     candidate list, which is ranked exactly against the current k best.
-//     After the first chunk of a row almost no logit qualifies;
-//   * the first chunk of each row a CTA sees starts from a threshold that k
-//     logits are sure to reach: the k-th largest of the per-lane maxima of
-//     the warp that has the largest one (a sort of 32 keys inside the warp);
+//     with the CTA's current bound on the k-th best key: only a thread whose
+//     maximum beats it looks at its logits again and appends the ones that
+//     do to a shared candidate buffer.  The buffer is ranked (exactly, by
+//     the 64-bit keys) only when it fills past half its size -- which also
+//     raises the bound -- and at the end of the CTA's part of the row;
+//   * the first chunk of each row a CTA sees starts from a bound k logits
+//     are sure to reach: the largest over warps of the k-th largest lane
+//     maximum (a sort of 32 keys inside each warp);
 //   * a CTA's part of a row ends in a partial (k best keys, max, sum) in the
 //     workspace; the last CTA of the row (atomic ticket, no waiting) merges
 //     the partials, writes the row's outputs and returns its ticket to zero.
 // The order key is 64 bits: the float's order-preserving bits, then the
 // complement of the token id, so ties go to the smaller id and every key is
 // distinct.  No CTA ever waits for another, so nothing can hang.
+#include <climits>
 #include <mutex>
 
 #include "common.cuh"
@@ -38,7 +40,7 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kChunkBytes = 16384;             // one chunk: 64 bytes per thread
 constexpr int kVecPerThread = kChunkBytes / 16 / kThreads;  // 4 vectors of 16 bytes
-constexpr int kStages = 4;                     // chunks of the ring
+constexpr int kStages = 3;                     // chunks of the ring
 constexpr int kCandCap = 1024;
 
 struct TopkParams {
@@ -181,7 +183,7 @@ struct Smem {
   uint64_t top2[DDT_TOPK_K_MAX];
   uint64_t red[kThreads / 32];
   float wm[kThreads / 32], wsum[kThreads / 32];
-  int count, last;
+  int count, last, overflow;
 };
 
 // Issue this thread's copies of chunk ch into ring slot `slot` (vectors
@@ -206,9 +208,11 @@ __device__ __forceinline__ void prefetch_chunk(const TopkParams& p, unsigned cha
 }
 
 template <bool BF16>
-__global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkParams p) {
+__global__ void __launch_bounds__(kThreads, 3) topk_kernel(TopkParams p) {
   constexpr int ES = BF16 ? 2 : 4, EPV = 16 / ES, EPC = kChunkBytes / ES;
   constexpr int NW = kVecPerThread * 4;  // 32-bit words of logits per thread per chunk
+  constexpr int PER = EPV / 4;           // elements per word
+  constexpr int NE = NW * PER;           // elements per thread per chunk
   extern __shared__ __align__(16) unsigned char ring[];
   __shared__ Smem sm;
 
@@ -219,17 +223,19 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkParams p) {
   pdl_trigger();
 
   float m = -INFINITY, s = 0.f;  // this thread's running (max, sum) for the current row
-  uint64_t tau = 0;              // the CTA's current k-th best key (0: fewer than k seen)
+  uint64_t tau = 0;              // a lower bound of the segment's k-th best key (0: none yet)
   bool first = true;             // next chunk is the first of a row for this CTA
-  if (tid < DDT_TOPK_K_MAX) sm.top[tid] = 0;
-  for (int64_t ch = c_lo; ch < c_hi; ++ch) {
-    const int slot = (int)((ch - c_lo) % kStages);
-    const int row = (int)(ch / p.S), cidx = (int)(ch % p.S);
+  int row = (int)(c_lo / p.S), cidx = (int)(c_lo % p.S), slot = 0;
+  for (int64_t ch = c_lo; ch < c_hi; ++ch, slot = slot == kStages - 1 ? 0 : slot + 1) {
+    if (ch > c_lo && ++cidx == p.S) {  // the next chunk (no division per chunk)
+      cidx = 0;
+      ++row;
+    }
     const int e0 = cidx * EPC;
     const char* rowp = (const char*)p.logits + (int64_t)row * p.row_stride * ES;
     cp_async_wait<kStages - 1>();
     // this thread's logits: word j of vector q holds elements
-    // e0 + (q*kThreads + tid)*EPV + j*(EPV/4) ...; absent ones read as -inf
+    // e0 + (q*kThreads + tid)*EPV + j*PER ...; absent ones read as -inf
     uint32_t w[NW];
 #pragma unroll
     for (int q = 0; q < kVecPerThread; ++q) {
@@ -244,7 +250,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkParams p) {
       } else {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const int ej = e + j * (EPV / 4);
+          const int ej = e + j * PER;
           if (BF16) {
             const uint32_t lo = ej < p.V ? ((const uint16_t*)rowp)[ej] : 0xFF80u;
             const uint32_t hi = ej + 1 < p.V ? ((const uint16_t*)rowp)[ej + 1] : 0xFF80u;
@@ -255,19 +261,15 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkParams p) {
         }
       }
     }
-    // the slot is free again: refill it with the chunk kStages ahead
-    prefetch_chunk<BF16>(p, ring, slot, ch + kStages < c_hi ? ch + kStages : p.T);
-
-    auto index_of = [&](int i) -> int {  // element i (0..NW*(EPV/4)) of this thread
-      const int per = EPV / 4;           // elements per word
-      const int q = i / (4 * per), r = i % (4 * per);
+    // element i (0..NE) of this thread: vector i / (4 PER), in increasing index order
+    auto index_of = [&](int i) -> int {
+      const int q = i / (4 * PER), r = i % (4 * PER);
       return e0 + (q * kThreads + tid) * EPV + r;
     };
     auto value_of = [&](int i) -> float {
       if (BF16) return (i & 1) ? bf16_hi(w[i >> 1]) : bf16_lo(w[i >> 1]);
       return __uint_as_float(w[i]);
     };
-    constexpr int NE = BF16 ? 2 * NW : NW;  // elements per thread per chunk
 
     // chunk maximum of this thread (-inf pads never exceed a real logit)
     float mc;
@@ -302,45 +304,105 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkParams p) {
       s += (a0 + a1) + (b0 + b1);
     }
 
+    // Candidates: every logit of the row segment that can still be among
+    // the k best goes to a shared buffer, which is only ranked when it
+    // fills past half its size and at the end of the segment.  The first
+    // chunk of a row starts from a threshold k logits of the CTA reach: the
+    // largest over warps of the k-th largest lane maximum (a lane maximum's
+    // key: its value at the smallest index holding it); later chunks take
+    // the logits above the current k-th best key's value (a logit equal to
+    // it comes later, so it ranks below it).
+    float tv;
+    int ti;
+    bool take_all;
     if (first) {
-      // a threshold k logits of this chunk reach: the k-th largest lane
-      // maximum of the best warp (exact 64-bit keys)
       uint64_t kmax = 0;
 #pragma unroll
-      for (int i = 0; i < NE; ++i) {
-        const int idx = index_of(i);
-        if (idx < p.V) {
-          const uint64_t key = cand_key(value_of(i), (uint32_t)idx);
-          kmax = key > kmax ? key : kmax;
-        }
-      }
+      for (int i = NE - 1; i >= 0; --i)
+        if (value_of(i) == mc && index_of(i) < p.V) kmax = cand_key(mc, (uint32_t)index_of(i));
       const uint64_t tw = warp_kth_key(kmax, p.k);
-      const uint64_t t0 = block_max_u64(tw, sm.red);  // barriers
-      if (tid == 0) sm.count = 0;
-      __syncthreads();
-      if (kmax >= t0 || t0 == 0) {
-#pragma unroll
-        for (int i = 0; i < NE; ++i) {
-          const int idx = index_of(i);
-          if (idx >= p.V) continue;
-          const uint64_t key = cand_key(value_of(i), (uint32_t)idx);
-          if (key >= t0) {
-            const int pos = atomicAdd(&sm.count, 1);
-            if (pos < kCandCap) sm.cand[pos] = key;
-          }
-        }
+      tau = block_max_u64(tw, sm.red);  // barriers; a lower bound of the k-th best
+      if (tid == 0) {
+        sm.count = 0;
+        sm.overflow = 0;
       }
       __syncthreads();
-      const int n = sm.count;
+      tv = tau ? key_val(tau) : -INFINITY;
+      ti = tau ? (int)key_id(tau) : INT_MAX;
+      take_all = tau == 0;  // fewer than k lanes hold logits
+    } else {
+      tv = tau ? key_val(tau) : -INFINITY;
+      ti = -1;
+      take_all = tau == 0;
+    }
+    // this thread's candidates as a bit mask over its elements; only a
+    // thread whose chunk maximum reaches the bound looks at them again
+    uint32_t mask = 0;
+    if (take_all || mc > tv || (mc == tv && ti >= 0)) {
+#pragma unroll
+      for (int i = 0; i < NE; ++i) {
+        const float v = value_of(i);
+        const bool c = take_all ? index_of(i) < p.V
+                                : (v > tv || (v == tv && ti >= 0 && index_of(i) <= ti));
+        mask |= (uint32_t)c << i;
+      }
+    }
+    // append them: one reservation per warp (a warp scan of the threads'
+    // counts and one atomic); each set bit re-reads its logit from this
+    // thread's own bytes of the ring (or from global memory for a vector
+    // the ring does not hold), so no register array is indexed at run time
+    if (__ballot_sync(0xFFFFFFFFu, mask != 0u)) {
+      const int lane = tid & 31;
+      const int cnt = __popc(mask);
+      int incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += u;
+      }
+      int base = 0;
+      if (lane == 31) base = atomicAdd(&sm.count, incl);
+      base = __shfl_sync(0xFFFFFFFFu, base, 31);
+      int pos = base + incl - cnt;
+      while (mask) {
+        const int i = __ffs(mask) - 1;
+        mask &= mask - 1u;
+        const int vq = (i / EPV) * kThreads + tid, r = i % EPV;  // vector of the chunk, element in it
+        const int e = e0 + vq * EPV + r;
+        float v;
+        if (p.vec_ok && e - r + EPV <= p.V) {
+          const unsigned char* src = ring + slot * kChunkBytes + vq * 16 + r * ES;
+          v = BF16 ? __uint_as_float((uint32_t)(*(const uint16_t*)src) << 16) : *(const float*)src;
+        } else {
+          v = BF16 ? __uint_as_float((uint32_t)((const uint16_t*)rowp)[e] << 16) : ((const float*)rowp)[e];
+        }
+        if (pos < kCandCap) sm.cand[pos] = cand_key(v, (uint32_t)e);
+        else sm.overflow = 1;
+        ++pos;
+      }
+    }
+    // this thread is done with its bytes of the slot: refill it with the
+    // chunk kStages ahead
+    prefetch_chunk<BF16>(p, ring, slot, ch + kStages < c_hi ? ch + kStages : p.T);
+    __syncthreads();
+    const int n = sm.count;
+    // the first chunk ranks at once, so that later chunks compare with the
+    // exact k-th best so far; later ones only when the buffer is half full
+    if (first || sm.overflow || n > kCandCap / 2) {
+      // compact the buffer to the k best (when it overflowed, this chunk's
+      // logits join by k rounds of block-wide argmax)
       if (tid < DDT_TOPK_K_MAX) sm.top2[tid] = 0;
       __syncthreads();
-      if (n <= kCandCap) {
+      if (!sm.overflow) {
         rank_select2(sm.cand, n, nullptr, 0, p.k, sm.top2);
       } else {
-        // degenerate chunk: k rounds of block-wide argmax below the previous pick
         uint64_t prev = ~0ull;
         for (int r = 0; r < p.k; ++r) {
           uint64_t best = 0;
+          for (int i = tid; i < kCandCap; i += kThreads) {
+            const uint64_t key = sm.cand[i];
+            if (key < prev && key > best) best = key;
+          }
 #pragma unroll
           for (int i = 0; i < NE; ++i) {
             const int idx = index_of(i);
@@ -354,66 +416,33 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkParams p) {
         }
       }
       __syncthreads();
-      if (tid < DDT_TOPK_K_MAX) sm.top[tid] = sm.top2[tid];
+      if (tid < p.k) sm.cand[tid] = sm.top2[tid];
+      if (tid == 0) {
+        sm.count = p.k;
+        sm.overflow = 0;
+      }
       __syncthreads();
-      tau = sm.top[p.k - 1];
-      first = false;
-    } else {
-      // later chunks: only logits beating the current k-th best key (a
-      // logit equal to its value comes later, so it ranks below it)
-      const bool need = tau == 0 || mc > key_val(tau);
-      if (__syncthreads_or(need)) {
-        if (tid == 0) sm.count = 0;
-        __syncthreads();
-        if (need) {
-#pragma unroll
-          for (int i = 0; i < NE; ++i) {
-            const int idx = index_of(i);
-            if (idx >= p.V) continue;
-            const uint64_t key = cand_key(value_of(i), (uint32_t)idx);
-            if (key > tau) {
-              const int pos = atomicAdd(&sm.count, 1);
-              if (pos < kCandCap) sm.cand[pos] = key;
-            }
-          }
-        }
-        if (tid < DDT_TOPK_K_MAX) sm.top2[tid] = 0;
-        __syncthreads();
-        const int n = sm.count;
-        if (n <= kCandCap) {
-          rank_select2(sm.top, p.k, sm.cand, n, p.k, sm.top2);
-        } else {
-          // degenerate: the previous k best and this chunk, k rounds of argmax
-          uint64_t prev = ~0ull;
-          for (int r = 0; r < p.k; ++r) {
-            uint64_t best = 0;
-            for (int i = tid; i < p.k; i += kThreads) {
-              const uint64_t key = sm.top[i];
-              if (key < prev && key > best) best = key;
-            }
-#pragma unroll
-            for (int i = 0; i < NE; ++i) {
-              const int idx = index_of(i);
-              if (idx >= p.V) continue;
-              const uint64_t key = cand_key(value_of(i), (uint32_t)idx);
-              if (key < prev && key > best) best = key;
-            }
-            best = block_max_u64(best, sm.red);
-            if (tid == 0) sm.top2[r] = best;
-            prev = best;
-          }
+      tau = sm.top2[p.k - 1];
+      if (tau == 0) {  // fewer than k logits so far: keep them all
+        if (tid == 0) {
+          int c = 0;
+          while (c < p.k && sm.top2[c] != 0) ++c;
+          sm.count = c;
         }
         __syncthreads();
-        if (tid < DDT_TOPK_K_MAX) sm.top[tid] = sm.top2[tid];
-        __syncthreads();
-        tau = sm.top[p.k - 1];
       }
     }
+    first = false;
 
-    // end of this CTA's part of the row: publish it (or finish the row)
+    // end of this CTA's part of the row: rank the buffer, publish (or
+    // finish the row)
     if (cidx == p.S - 1 || ch == c_hi - 1) {
       float M = m, Ssum = s;
-      block_ms_reduce(M, Ssum, p.c, sm.wm, sm.wsum);
+      block_ms_reduce(M, Ssum, p.c, sm.wm, sm.wsum);  // barriers
+      if (tid < DDT_TOPK_K_MAX) sm.top[tid] = 0;
+      __syncthreads();
+      rank_select2(sm.cand, min(sm.count, kCandCap), nullptr, 0, p.k, sm.top);
+      __syncthreads();
       const int64_t g_first = owner_of((int64_t)row * p.S, p.T, p.G);
       const int64_t g_last = owner_of((int64_t)row * p.S + p.S - 1, p.T, p.G);
       if (g_first == g_last) {
@@ -423,13 +452,13 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkParams p) {
         const int64_t pb = (int64_t)row * p.pmax + slot_p;
         for (int r = tid; r < p.k; r += kThreads) p.part_keys[pb * p.k + r] = sm.top[r];
         if (tid == 0) p.part_ms[pb] = make_float2(M, Ssum);
-        __threadfence();
         __syncthreads();
+        // one acquire-release ticket for the CTA: it releases the partial the
+        // barrier ordered before it and, for the last CTA, acquires the others
         const int np = (int)(g_last - g_first + 1);
-        if (tid == 0) sm.last = (atomicAdd(&p.tickets[row], 1u) == (unsigned)(np - 1));
+        if (tid == 0) sm.last = (atom_add_acq_rel_gpu(&p.tickets[row], 1u) == (unsigned)(np - 1));
         __syncthreads();
         if (sm.last) {
-          __threadfence();
           // every partial's keys and (max, sum) in one round of loads, then
           // the row's k best ranked directly
           const int tot = np * p.k;
@@ -473,8 +502,6 @@ __global__ void __launch_bounds__(kThreads, 2) topk_kernel(TopkParams p) {
       s = 0.f;
       tau = 0;
       first = true;
-      if (tid < DDT_TOPK_K_MAX) sm.top[tid] = 0;
-      __syncthreads();
     }
   }
   cp_async_wait<0>();

@@ -38,6 +38,7 @@
 // fair share of them to a neighbour.
 #include <climits>
 #include <cmath>
+#include <mutex>
 
 #include "common.cuh"
 #include "launch.h"
@@ -852,32 +853,44 @@ __global__ void __launch_bounds__(kLazyThreads) walk_lazy_kernel(WalkParams p, i
   }
 }
 
-// Largest cluster (16, else 8) of path-only walk CTAs the device can run.
-int lazy_cluster_size() {
-  static int cached = 0;
-  if (cached) return cached;
-  int best = 8;
+// Largest cluster (16, else 8) of path-only walk CTAs the device can run,
+// and how many such clusters it runs at once.
+struct LazyShape {
+  int csize, active;
+};
+LazyShape lazy_shape() {
+  static std::mutex mu;
+  static LazyShape cached = {0, 0};
+  std::lock_guard<std::mutex> lock(mu);
+  if (cached.csize) return cached;
   auto* fn = (const void*)walk_lazy_kernel<false>;
   auto* fn2 = (const void*)walk_lazy_kernel<true>;
-  if (cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess &&
-      cudaFuncSetAttribute(fn2, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
+  const bool big = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess &&
+                   cudaFuncSetAttribute(fn2, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+  LazyShape r = {8, 1};
+  for (int cs : {16, 8}) {
+    if (cs == 16 && !big) continue;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(16, 1, 1);
+    cfg.gridDim = dim3(cs, 1, 1);
     cfg.blockDim = dim3(kLazyThreads, 1, 1);
     cudaLaunchAttribute attr;
     attr.id = cudaLaunchAttributeClusterDimension;
-    attr.val.clusterDim.x = 16;
+    attr.val.clusterDim.x = cs;
     attr.val.clusterDim.y = 1;
     attr.val.clusterDim.z = 1;
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
     int nc = 0;
-    if (cudaOccupancyMaxActiveClusters(&nc, fn, &cfg) == cudaSuccess && nc > 0) best = 16;
+    if (cudaOccupancyMaxActiveClusters(&nc, fn, &cfg) == cudaSuccess && nc > 0) {
+      r = {cs, nc};
+      break;
+    }
   }
   cudaGetLastError();  // a refused query must not leave a sticky error behind
-  cached = best;
-  return best;
+  cached = r;
+  return r;
 }
+int lazy_cluster_size() { return lazy_shape().csize; }
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
@@ -890,21 +903,22 @@ size_t walk_workspace_size(int batch, int n_max, int V) {
          align256(2 * sizeof(uint64_t) * rows * S);
 }
 
-// Path-only or all-rows for DDT_WALK_AUTO.  The all-rows scan costs its
-// bytes at the rate it reaches on B200 plus its fixed part (tickets, the
-// merge, the walk); the path-only walk costs up to L + 1 dependent steps
-// (measured per step on B200, per wave of clusters).  AUTO takes the
-// path-only walk when even its worst case (every row down to depth L
-// accepted) is the cheaper.
-constexpr double kAllRowsGBs = 6000.0, kAllRowsFixedUs = 9.0;
-constexpr double kLazyStepUs = 2.0;
+// Path-only or all-rows for DDT_WALK_AUTO, from times measured on B200: the
+// all-rows scan costs its bytes at about 5.8 TB/s plus a few microseconds of
+// merging; the path-only walk costs about 3.5 us per dependent step (one
+// row per sequence), per wave of clusters the device runs at once, and up
+// to L + 1 steps.  AUTO takes the path-only walk when even its worst case
+// (every row down to depth L accepted) is the cheaper.  (Both pay the same
+// launch latency, which cancels.)
+constexpr double kAllRowsGBs = 5800.0, kAllRowsMergeUs = 4.0;
+constexpr double kLazyStepUs = 3.5;
 
 int walk_mode_for(int mode, ddt_dtype dt, int batch, int n_max, int V, int L) {
   if (mode != DDT_WALK_AUTO) return mode;
   const double bytes = (double)batch * n_max * V * (dt == DDT_BF16 ? 2 : 4);
-  const double all_us = bytes / (kAllRowsGBs * 1e3) + kAllRowsFixedUs;
-  const int csize = lazy_cluster_size();
-  const double waves = std::ceil((double)batch * csize / (2.0 * device_sm_count()));
+  const double all_us = bytes / (kAllRowsGBs * 1e3) + kAllRowsMergeUs;
+  const LazyShape ls = lazy_shape();
+  const double waves = std::ceil((double)batch / (double)(ls.active > 0 ? ls.active : 1));
   const double lazy_us = (L + 1) * kLazyStepUs * waves;
   return lazy_us < all_us ? DDT_WALK_LAZY : DDT_WALK_ALL_ROWS;
 }

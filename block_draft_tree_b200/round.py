@@ -27,6 +27,12 @@ class VerifyRound:
     head; no logits are stored).  With ``commit`` the round ends with
     ``ddt_kv_commit``: the root's and the accepted rows' K/V join the bound
     cache and ``ctx_len`` advances in place.
+
+    With ``adaptive_budget`` (a dict of ``total``, ``cost_fixed``,
+    ``cost_per_node``) stage 2 builds every sequence's tree with its largest
+    budget, splits the batch's nodes with ``ddt_plan_budget`` under that cost
+    model, and builds the trees again with those budgets; ``out["budget"]``
+    and ``out["expected_tokens"]`` hold the split.
     """
 
     def __init__(self, *, batch: int, L: int, V: int, k: int, B_max: int, hq: int, hkv: int,
@@ -34,10 +40,12 @@ class VerifyRound:
                  target_dtype: torch.dtype = torch.float32, inv_temperature: float = 1.0,
                  paged: bool = False, page_size: int = 64, max_pages: int = 0,
                  decode: str = "greedy", sample_inv_temperature: float = 1.0, seed: int = 0,
-                 commit: bool = False, walk_mode: int = api.WALK_AUTO, device: str = "cuda"):
+                 commit: bool = False, walk_mode: int = api.WALK_AUTO,
+                 adaptive_budget: Optional[dict] = None, device: str = "cuda"):
         if decode not in ("greedy", "sample", "lm_head"):
             raise ValueError("decode must be 'greedy', 'sample' or 'lm_head'")
         self.decode, self.commit, self.walk_mode = decode, commit, int(walk_mode)
+        self.adaptive = dict(adaptive_budget) if adaptive_budget else None
         self.sample_inv_t, self.seed = float(sample_inv_temperature), int(seed)
         self.lib = api.load_library()
         self.dev = torch.device(device)
@@ -61,6 +69,7 @@ class VerifyRound:
             "attn": e(batch, self.n_max, hq, d, dt=torch.bfloat16),
             "acc_len": e(batch), "acc_nodes": e(batch, L), "acc_tok": e(batch, L), "bonus": e(batch),
             "status": torch.zeros(1, dtype=torch.int32, device=dev),
+            "budget": e(batch), "expected_tokens": e(batch, dt=torch.float64),
         }
         self.ws_topk_n = int(self.lib.ddt_topk_workspace_size(batch, L, V, k))
         self.ws_walk_n = int(self.lib.ddt_tree_walk_workspace_size(batch, self.n_max, V))
@@ -148,12 +157,25 @@ class VerifyRound:
                               None, P(o["lse"]), P(self.ws_topk), self.ws_topk_n, s)
             api._check(rc, "ddt_topk")
         elif i == 1:
-            rc = lib.ddt_build_tree(P(o["ids"]), P(o["zk"]), P(o["lse"]), self.batch, self.L,
-                                    self.k, self.inv_t, P(x.get("k_per_seq")), P(x.get("budget")),
-                                    self.B_max, P(x["root"]), P(x["ctx_len"]), P(o["tok"]),
-                                    P(o["parent"]), P(o["depth"]), P(o["pos"]), P(o["mask"]),
-                                    P(o["n_nodes"]), P(o["surrogate"]), P(o["status"]), s)
-            api._check(rc, "ddt_build_tree")
+            def build(budget):
+                rc = lib.ddt_build_tree(P(o["ids"]), P(o["zk"]), P(o["lse"]), self.batch, self.L,
+                                        self.k, self.inv_t, P(x.get("k_per_seq")), P(budget),
+                                        self.B_max, P(x["root"]), P(x["ctx_len"]), P(o["tok"]),
+                                        P(o["parent"]), P(o["depth"]), P(o["pos"]), P(o["mask"]),
+                                        P(o["n_nodes"]), P(o["surrogate"]), P(o["status"]), s)
+                api._check(rc, "ddt_build_tree")
+
+            build(x.get("budget"))
+            if self.adaptive:
+                a = self.adaptive
+                rc = lib.ddt_plan_budget(P(o["tok"]), P(o["parent"]), P(o["depth"]),
+                                         P(o["n_nodes"]), P(o["ids"]), P(o["zk"]), P(o["lse"]),
+                                         self.batch, self.L, self.k, self.n_max, self.inv_t,
+                                         int(a.get("total", -1)), float(a.get("cost_fixed", 0.0)),
+                                         float(a.get("cost_per_node", 0.0)), P(o["budget"]),
+                                         P(o["expected_tokens"]), P(o["status"]), s)
+                api._check(rc, "ddt_plan_budget")
+                build(o["budget"])
         elif i == 2:
             rc = lib.ddt_tree_attn(ctypes.byref(self.attn_args), P(self.ws_attn), self.ws_attn_n, s)
             api._check(rc, "ddt_tree_attn")

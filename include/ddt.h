@@ -20,6 +20,8 @@
  *                            hidden states (LM head on the tensor cores);
  *   5. ddt_kv_commit   appends the root's and the accepted rows' K/V to the
  *                      committed context for the next round.
+ *   ddt_plan_budget    splits a batch's node budget between its sequences
+ *                      (between a first and a second ddt_build_tree).
  *
  * Conventions shared by every entry point:
  *   - Every tensor pointer is a DEVICE pointer owned by the caller.  The
@@ -200,6 +202,39 @@ ddt_status ddt_build_tree(const int32_t* ids, const float* zk, const float* lse,
                           int32_t* dev_status, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Between stage 2 and a second build: node budgets across the batch.
+ * DDTree page, section 實驗結果與權衡: acceptance grows with the node budget
+ * and so does the verifier's cost; section 理論基礎, Proposition 1: a tree's
+ * expected acceptance length is the sum of its nodes' prefix probabilities,
+ * and a smaller budget's best tree is the best-first part of a larger one's.
+ *
+ * Input: every sequence's tree built with the largest budget it may get
+ * (tok, parent, depth, n_nodes of ddt_build_tree, n_max rows) and the
+ * candidates it was built from (ids, zk, lse of ddt_topk, [batch][L][k]).
+ * A draft node of depth d with tokens t_1..t_d on its path has the score
+ * invT*(z_1 + ... + z_d) - (lse_1 + ... + lse_d) (fp64, depth order) and the
+ * probability exp(score).  The batch's nodes ranked by score (ties: smaller
+ * sequence, then smaller row) give the split of any total n that maximises
+ * the expected acceptance: the first n.  The call takes the n in
+ * [0, total_budget] (total_budget < 0: every node) that maximises
+ * (batch + the first n probabilities) / (cost_fixed + cost_per_node * n),
+ * the expected emitted tokens per unit of round cost (smallest n on ties);
+ * with cost_per_node <= 0 it takes n = min(total_budget, all nodes).
+ * Outputs: budget_per_seq int32 [batch], sequence b's share (feed it to
+ * ddt_build_tree's budget_per_seq); expected_tokens double [batch] (may be
+ * NULL): 1 + the sum of the probabilities of its share.
+ * Limits: batch * (n_max - 1) <= 8192 nodes.  cost_per_node > 0 needs
+ * cost_fixed > 0.  A row that is not a node of these candidates raises
+ * DDT_ERR_INVALID_ARG in dev_status and counts for nothing.
+ * ------------------------------------------------------------------------ */
+ddt_status ddt_plan_budget(const int32_t* tok, const int32_t* parent, const int32_t* depth,
+                           const int32_t* n_nodes, const int32_t* ids, const float* zk,
+                           const float* lse, int batch, int L, int k, int n_max,
+                           float inv_temperature, int total_budget, double cost_fixed,
+                           double cost_per_node, int32_t* budget_per_seq, double* expected_tokens,
+                           int32_t* dev_status, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
  * Stage 3: tree attention.
  * DDTree page, 核心創新 third bullet and 運作流程 step 3: one target forward
  * scores the whole tree; each tree row attends to the committed context and
@@ -256,14 +291,17 @@ ddt_status ddt_tree_attn(const ddt_attn_args* a, void* workspace, size_t workspa
 
 /* How ddt_tree_attn would run this call on the current device (a query: it
  * launches nothing).  *path: DDT_ATTN_PATH_SIMT (CUDA cores), _TC (tensor
- * cores, one pass over the KV range per query tile), _TC_CLUSTER (KV splits
- * of a query tile run as one thread-block cluster and merge through
- * distributed shared memory) or _TC_COMBINE (KV splits write partials to the
- * workspace and a second kernel merges them); *kv_splits: the number of KV
- * splits per query tile (either pointer may be NULL).  Returns the status
- * ddt_tree_attn's argument check would return. */
+ * cores, one query tile of 128 rows per CTA, one pass over the KV range),
+ * _TC_CLUSTER (KV splits of a query tile run as one thread-block cluster and
+ * merge through distributed shared memory), _TC_COMBINE (KV splits write
+ * partials to the workspace and a second kernel merges them), _TC_PAIRS
+ * (two query tiles of one kv head per CTA, sharing every K/V tile, one pass)
+ * or _TC_PAIRS_COMBINE (the same with workspace-combined KV splits);
+ * *kv_splits: the number of KV splits per query tile (either pointer may be
+ * NULL).  Returns the status ddt_tree_attn's argument check would return. */
 enum { DDT_ATTN_PATH_SIMT = 0, DDT_ATTN_PATH_TC = 1, DDT_ATTN_PATH_TC_CLUSTER = 2,
-       DDT_ATTN_PATH_TC_COMBINE = 3 };
+       DDT_ATTN_PATH_TC_COMBINE = 3, DDT_ATTN_PATH_TC_PAIRS = 4,
+       DDT_ATTN_PATH_TC_PAIRS_COMBINE = 5 };
 ddt_status ddt_tree_attn_plan(const ddt_attn_args* a, int* path, int* kv_splits);
 
 /* ------------------------------------------------------------------------

@@ -822,8 +822,8 @@ int ddto_walk_row_tokens(const int32_t* row_tok, const int32_t* tok, const int32
  * sum of its nodes' prefix probabilities, and the best tree of any smaller
  * budget is the K-first part of the best tree of a larger one.  So, given
  * for every sequence the tree built with its largest budget, the nodes of
- * the whole batch ranked by prefix probability (ties: smaller sequence
- * index, then smaller row) give the allocation that maximises the summed
+ * the whole batch ranked by prefix probability (by its logarithm, the score;
+ * ties: smaller sequence index, then smaller row) give the allocation that maximises the summed
  * expected acceptance for any total number of nodes n: the first n nodes.
  * With a round cost of c0 + c1 * n for n draft nodes, the round emits
  * (batch + accepted) tokens, so the plan takes the n that maximises
@@ -840,15 +840,17 @@ int ddto_walk_row_tokens(const int32_t* row_tok, const int32_t* tok, const int32
  * probability is exp(score).
  */
 typedef struct {
-  double p;
+  double score, p;
   int b, j;
 } pnode_t;
 
+/* by score (the probability's logarithm, so that no two distinct scores
+   tie through the rounding of exp), then sequence, then row */
 static int cmp_pnode(const void* pa, const void* pb) {
   const pnode_t* a = (const pnode_t*)pa;
   const pnode_t* b = (const pnode_t*)pb;
-  if (a->p > b->p) return -1;
-  if (a->p < b->p) return 1;
+  if (a->score > b->score) return -1;
+  if (a->score < b->score) return 1;
   if (a->b != b->b) return a->b < b->b ? -1 : 1;
   return a->j < b->j ? -1 : (a->j > b->j);
 }
@@ -893,7 +895,8 @@ int ddto_plan_budget(int batch, int L, int kstride, int n_max, double invT, cons
         S = S + lse[(int64_t)b * L + t];
       }
       const double a = invT * sz;
-      nodes[m].p = exp(a - S);
+      nodes[m].score = a - S;
+      nodes[m].p = exp(nodes[m].score);
       nodes[m].b = b;
       nodes[m].j = j;
       ++m;

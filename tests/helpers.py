@@ -191,3 +191,20 @@ def check_sampled_walk(logits, tree, L, invT, seed, step, got, count=None):
             for key in ("acc_len", "acc_nodes", "acc_tok", "bonus"):
                 np.testing.assert_array_equal(got[key][b], ref[key][b], err_msg="%s[%d]" % (key, b))
     return ref
+
+
+# Shapes (batch, budget, context; b64 heads, L=6, V=400, k=4) that take each
+# attention path on a B200; the plan depends on the device (SM count,
+# co-resident clusters), so a test takes the first shape whose plan matches.
+# Keys: the suffix of the binding's ATTN_PATH_* constant.
+ATTN_PATH_SHAPES = {
+    "TC_CLUSTER": [dict(batch=1, B=64, ctx=4096), dict(batch=1, B=40, ctx=2000),
+                   dict(batch=2, B=30, ctx=3000)],
+    "TC_COMBINE": [dict(batch=b, B=31, ctx=8192) for b in (20, 24, 30, 12)] +
+                  [dict(batch=5, B=20, ctx=16384)],
+    "TC": [dict(batch=37, B=31, ctx=500), dict(batch=74, B=20, ctx=300)],
+    "TC_PAIRS": [dict(batch=37, B=63, ctx=500), dict(batch=37, B=127, ctx=500)],
+    "TC_PAIRS_COMBINE": [dict(batch=2, B=63, ctx=16384), dict(batch=3, B=100, ctx=8192),
+                         dict(batch=8, B=256, ctx=1000), dict(batch=16, B=63, ctx=16384)],
+    "SIMT": [dict(batch=3, B=8, ctx=900)],
+}

@@ -19,7 +19,7 @@ import torch
 import oracle
 from block_draft_tree_b200 import api, synth
 
-from helpers import assert_attn_close, bf16_tensor, i32, oracle_tree_inputs
+from helpers import ATTN_PATH_SHAPES, assert_attn_close, bf16_tensor, i32, oracle_tree_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -202,14 +202,7 @@ def _plan(w, max_ctx):
 
 
 # candidate shapes per path; the test takes the first whose plan is that path
-_PATH_CANDIDATES = {
-    api.ATTN_PATH_TC_CLUSTER: [dict(batch=1, B=64, ctx=4096), dict(batch=1, B=40, ctx=2000),
-                               dict(batch=2, B=30, ctx=3000)],
-    api.ATTN_PATH_TC_COMBINE: [dict(batch=b, B=32, ctx=8192) for b in (5, 6, 8, 10, 12)] +
-                              [dict(batch=3, B=64, ctx=16384), dict(batch=7, B=40, ctx=6000)],
-    api.ATTN_PATH_TC: [dict(batch=37, B=127, ctx=500), dict(batch=74, B=63, ctx=300)],
-    api.ATTN_PATH_SIMT: [dict(batch=3, B=8, ctx=900)],
-}
+_PATH_CANDIDATES = {getattr(api, "ATTN_PATH_" + k): v for k, v in ATTN_PATH_SHAPES.items()}
 
 
 @pytest.mark.parametrize("path", sorted(_PATH_CANDIDATES))
@@ -222,7 +215,7 @@ def test_each_attention_path(path):
             break
     else:
         pytest.fail("no candidate shape takes path %d" % path)
-    if path in (api.ATTN_PATH_TC_CLUSTER, api.ATTN_PATH_TC_COMBINE):
+    if path in (api.ATTN_PATH_TC_CLUSTER, api.ATTN_PATH_TC_COMBINE, api.ATTN_PATH_TC_PAIRS_COMBINE):
         assert splits > 1
     tree = _tree_for(w)
     a = synth.attention_inputs(w)
@@ -232,7 +225,7 @@ def test_each_attention_path(path):
             torch.from_numpy(tree["mask"].view(np.int32)).cuda(), i32(tree["n_nodes"]))
     assert api.tree_attn_plan(*args, kw_t["ctx_len"], kw_t["max_ctx"]) == (got_path, splits)
     nb = api.tree_attn_workspace_size(*args, kw_t["ctx_len"], kw_t["max_ctx"])
-    assert (nb > 0) == (path == api.ATTN_PATH_TC_COMBINE or
+    assert (nb > 0) == (path in (api.ATTN_PATH_TC_COMBINE, api.ATTN_PATH_TC_PAIRS_COMBINE) or
                         (path == api.ATTN_PATH_SIMT and splits > 1))
     out, lse = _gpu_attn(a, tree, w)
     seqs = [0, w.batch - 1] if w.batch > 1 else [0]
