@@ -31,7 +31,8 @@ EXPORTED = ("ddt_status_string", "ddt_mask_words", "ddt_topk_workspace_size", "d
             "ddt_tree_walk_workspace_size", "ddt_tree_walk", "ddt_tree_walk_sample",
             "ddt_kv_commit", "ddt_lm_head_max_rows", "ddt_lm_head_walk_workspace_size",
             "ddt_lm_head_walk", "ddt_tree_attn_plan", "ddt_debug_set_wait_limit",
-            "ddt_topk_noalloc", "ddt_tree_walk_resolve_mode", "ddt_plan_budget")
+            "ddt_topk_noalloc", "ddt_tree_walk_resolve_mode", "ddt_plan_budget",
+            "ddt_debug_set_attn_kernel")
 
 # ddt_tree_walk's modes
 WALK_ALL_ROWS, WALK_LAZY, WALK_AUTO = 0, 1, 2
@@ -121,6 +122,8 @@ def load_library():
                                            ctypes.POINTER(i32)]
         lib.ddt_debug_set_wait_limit.restype = ctypes.c_longlong
         lib.ddt_debug_set_wait_limit.argtypes = [ctypes.c_longlong]
+        lib.ddt_debug_set_attn_kernel.restype = ctypes.c_int
+        lib.ddt_debug_set_attn_kernel.argtypes = [ctypes.c_int]
         lib.ddt_tree_walk_workspace_size.restype = sz
         lib.ddt_tree_walk_workspace_size.argtypes = [i32, i32, i32]
         lib.ddt_tree_walk.restype = i32
@@ -360,6 +363,18 @@ def set_wait_limit(cycles: int) -> int:
     kernels' on-chip waits for later launches; <= 0 restores the default of
     about one second.  Returns the previous setting.  A test hook."""
     return int(load_library().ddt_debug_set_wait_limit(int(cycles)))
+
+
+# ddt_debug_set_attn_kernel's choices
+ATTN_KERNEL_AUTO, ATTN_KERNEL_ONE_TILE, ATTN_KERNEL_PAIRS = 0, 1, 2
+
+
+def set_attn_kernel(which: int) -> int:
+    """``ddt_debug_set_attn_kernel``: the tensor-core attention kernel later
+    calls use (ATTN_KERNEL_AUTO, _ONE_TILE or _PAIRS).  Returns the previous
+    choice (-1 for a value out of range, which changes nothing).  A tuning and
+    test hook."""
+    return int(load_library().ddt_debug_set_attn_kernel(int(which)))
 
 
 def tree_attn(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,

@@ -51,6 +51,10 @@ constexpr long long kDefaultWaitCycles = 2000000000LL;  // about one second at 1
 std::atomic<long long> g_wait_override{0};
 }  // namespace
 
+std::atomic<int> g_attn_kernel{0};
+
+int attn_kernel_choice() { return g_attn_kernel.load(std::memory_order_relaxed); }
+
 long long wait_limit_cycles() {
   const long long v = g_wait_override.load(std::memory_order_relaxed);
   return v > 0 ? v : kDefaultWaitCycles;
@@ -215,6 +219,11 @@ int ddt_mask_words(int n_max) { return n_max > 0 ? (n_max + 31) / 32 : 0; }
 
 long long ddt_debug_set_wait_limit(long long cycles) {
   return g_wait_override.exchange(cycles > 0 ? cycles : 0);
+}
+
+int ddt_debug_set_attn_kernel(int which) {
+  if (which < 0 || which > 2) return -1;
+  return g_attn_kernel.exchange(which);
 }
 
 size_t ddt_topk_workspace_size(int batch, int L, int V, int k) {

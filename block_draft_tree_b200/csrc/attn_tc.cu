@@ -949,54 +949,46 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           }
         }
       }
-      // pass 1: the row maximum, 32 scores at a time (the scores stay in TMEM)
-      float mx = -INFINITY;
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(lane_base + s_col + 32 * c, r);
-        tmem_ld_wait();
-        if (masked) {
+      // the row's 128 scores in registers: four TMEM loads, one wait
+      uint32_t r[BN];
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (!((mw[c] >> e) & 1u)) r[e] = 0xFF800000u;  // -inf
-        }
-        float m4[4];
+      for (int c = 0; c < BN / 32; ++c) tmem_ld32(lane_base + s_col + 32 * c, r + 32 * c);
+      tmem_ld_wait();
+      if (masked) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) m4[e] = __uint_as_float(r[e]);
-#pragma unroll
-        for (int e = 4; e < 32; e += 2)
-          m4[(e >> 1) & 3] = fmax3(m4[(e >> 1) & 3], __uint_as_float(r[e]), __uint_as_float(r[e + 1]));
-        mx = fmaxf(mx, fmax3(fmax3(m4[0], m4[1], m4[2]), m4[3], mx));
+        for (int e = 0; e < BN; ++e)
+          if (!((mw[e >> 5] >> (e & 31)) & 1u)) r[e] = 0xFF800000u;  // -inf
       }
-      mx *= c_log2;
+      // the row maximum (three-input max, four independent chains)
+      float m4[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) m4[e] = __uint_as_float(r[e]);
+#pragma unroll
+      for (int e = 4; e < BN; e += 2)
+        m4[(e >> 1) & 3] = fmax3(m4[(e >> 1) & 3], __uint_as_float(r[e]), __uint_as_float(r[e + 1]));
+      const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * c_log2;
       const float m_new = fmaxf(m_used, mx);
       const bool move = m_new > m_used + kRescaleLog2 || (m_used == -INFINITY && m_new != -INFINITY);
       const float m_tgt = move ? m_new : m_used;
-      // pass 2: p = 2^(s*c - m), two scores at a time: a packed FFMA for the
+      // p = 2^(s*c - m), two scores at a time: a packed FFMA for the
       // exponents, then MUFU ex2 -- or, for 3 pairs in 8, exp2_poly2 on the
-      // FMA pipe; packed sums; bf16 pairs stored over the scores already read
+      // FMA pipe; packed sums; bf16 pairs stored over the scores, 32 scores
+      // (16 columns) per store
       uint64_t rs2[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) rs2[e] = 0ull;
       const uint64_t c2 = pack2(c_log2, c_log2), nm2 = pack2(-m_tgt, -m_tgt);
-#pragma unroll 1
+#pragma unroll
       for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32], pk[16];
-        tmem_ld32(lane_base + s_col + 32 * c, r);  // every lane: tcgen05.ld is warp-collective
-        tmem_ld_wait();
+        uint32_t pk[16];
         if (m_tgt == -INFINITY) {
 #pragma unroll
           for (int e = 0; e < 16; ++e) pk[e] = 0u;
         } else {
-          if (masked) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (!((mw[c] >> e) & 1u)) r[e] = 0xFF800000u;
-          }
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            const uint64_t x2 = ffma2(pack2(__uint_as_float(r[e]), __uint_as_float(r[e + 1])), c2, nm2);
+            const uint64_t x2 = ffma2(pack2(__uint_as_float(r[32 * c + e]), __uint_as_float(r[32 * c + e + 1])),
+                                      c2, nm2);
             float a, bb;
             if (((e >> 1) & 7) < 3) {
               exp2_poly2(x2, a, bb);
@@ -1314,13 +1306,19 @@ bool attn_tc_cluster(int nsplit, long clusters) {
   return known[nsplit] > 0 && clusters <= known[nsplit];
 }
 
-// The two-query-tile kernel serves every call with at least two query tiles
-// per kv head whose splits would not merge on chip.  Its KV-split plan
+// The two-query-tile kernel serves every call on a dense cache with at least
+// two query tiles per kv head whose splits would not merge on chip.  Its KV-split plan
 // minimises waves x tiles per split (plus the combine's cost when split).
 bool attn_pair_plan(const ddt_attn_args* a, int sms, int* qtiles, int* nsplit, int* tps) {
   int qt, ns, t;
   attn_tc_plan(a, sms, &qt, &ns, &t);
-  if (qt < 2 || (ns > 1 && attn_tc_cluster(ns, (long)qt * a->batch * a->hkv))) return false;
+  const int choice = attn_kernel_choice();
+  if (qt < 2 || choice == 1) return false;
+  if (choice == 0 && ns > 1 && attn_tc_cluster(ns, (long)qt * a->batch * a->hkv)) return false;
+  // paged caches: the pair kernel's ring holds two K/V tiles (the one-tile
+  // kernel's three), too shallow for page gathers in random order (measured
+  // on a B200: 32 ragged sequences, 64-token pages, 2.27 ms against 1.85 ms)
+  if (choice == 0 && a->page_table) return false;
   const long base = (long)((qt + 1) / 2) * a->batch * a->hkv;
   const int tiles = (a->max_ctx + tc::BN - 1) / tc::BN + (a->n_max + tc::BN - 1) / tc::BN;
   constexpr int kMergeTiles = 3;

@@ -21,6 +21,8 @@ int device_sm_count();
 // gives up (about one second by default; see ddt_debug_set_wait_limit), and
 // the bound of each wait that drains loads and MMAs in flight after that.
 long long wait_limit_cycles();
+// The tensor-core attention kernel override (0 auto, 1 one-tile, 2 pairs).
+int attn_kernel_choice();
 constexpr long long kDrainCycles = 200000000LL;
 
 // Launch with programmatic stream serialization (see pdl_wait/pdl_trigger),

@@ -99,6 +99,17 @@ int ddt_mask_words(int n_max);
  * synchronised with launches on other host threads. */
 long long ddt_debug_set_wait_limit(long long cycles);
 
+/* Tuning and test hook: which tensor-core attention kernel ddt_tree_attn
+ * uses.  0 (default): the planner chooses; 1: the one-query-tile kernel
+ * only; 2: the two-query-tile kernel wherever a kv head has at least two
+ * query tiles (the one-tile kernel elsewhere).  The KV split is planned for
+ * the chosen kernel as usual, and ddt_tree_attn_plan and
+ * ddt_tree_attn_workspace_size follow the same choice.  Applies to every
+ * later call in the process; returns the previous setting, or -1 (nothing
+ * changed) for a value outside 0..2.  Not synchronised with calls on other
+ * host threads. */
+int ddt_debug_set_attn_kernel(int which);
+
 /* ------------------------------------------------------------------------
  * Stage 1: per-position softmax normaliser and top-k.
  * DDTree page, 運作流程 step 1: the drafter returns one marginal q_i per

@@ -213,3 +213,13 @@ def test_walk_rejects_an_unknown_mode(lib):
                            dummy, dummy, dummy, dummy, None, 0, None, None)
     assert rc == 1
     assert lib.ddt_tree_walk_resolve_mode(7, 1, 1, 9, 100, 4) == -1
+
+
+def test_attention_kernel_override_is_a_setting(lib):
+    prev = api.set_attn_kernel(api.ATTN_KERNEL_PAIRS)
+    try:
+        assert api.set_attn_kernel(api.ATTN_KERNEL_ONE_TILE) == api.ATTN_KERNEL_PAIRS
+        assert api.set_attn_kernel(3) == -1 and api.set_attn_kernel(-1) == -1
+        assert api.set_attn_kernel(api.ATTN_KERNEL_AUTO) == api.ATTN_KERNEL_ONE_TILE
+    finally:
+        api.set_attn_kernel(prev)

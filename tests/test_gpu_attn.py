@@ -243,3 +243,25 @@ def test_workload_paths(name, path):
     assert _plan(w, w.ctx)[0] == path
     for big in ("b256", "paged128", "long512"):
         assert _plan(synth.WORKLOADS[big], synth.WORKLOADS[big].ctx)[0] != api.ATTN_PATH_SIMT
+
+
+@pytest.mark.parametrize("paged", [False, True], ids=["dense", "paged"])
+@pytest.mark.parametrize("kernel", ["ONE_TILE", "PAIRS"])
+def test_each_kernel_family(kernel, paged):
+    """Both tensor-core kernels, chosen through the library's override, on the
+    same inputs: a dense cache and a paged one (ragged contexts, partial last
+    pages), with two query tiles per kv head, match the oracle; the planner's
+    own choice is restored afterwards."""
+    base = synth.WORKLOADS["paged128" if paged else "b64"]
+    w = base.scaled(batch=3, L=6, V=400, k=4, B=63, ctx=1500, hq=32, hkv=8, d=128,
+                    **(dict(ctx_min=200) if paged else {}))
+    prev = api.set_attn_kernel(getattr(api, "ATTN_KERNEL_" + kernel))
+    try:
+        got_path, _ = _plan(w, int(synth.context_lengths(w).max()))
+        if kernel == "PAIRS":
+            assert got_path in (api.ATTN_PATH_TC_PAIRS, api.ATTN_PATH_TC_PAIRS_COMBINE)
+        else:
+            assert got_path in (api.ATTN_PATH_TC, api.ATTN_PATH_TC_CLUSTER, api.ATTN_PATH_TC_COMBINE)
+        _check(w, sample=400, seed=3)
+    finally:
+        api.set_attn_kernel(prev)
