@@ -915,12 +915,13 @@ def run_profile(args):
     from block_draft_tree_b200.round import VerifyRound
 
     w = synth.WORKLOADS[args.workload or WORKLOAD]
-    rnd = VerifyRound(batch=w.batch, L=w.L, V=w.V, k=w.k, B_max=w.B, hq=w.hq, hkv=w.hkv, d=w.d,
-                      max_ctx=w.ctx, draft_dtype=torch.bfloat16, target_dtype=torch.float32,
-                      inv_temperature=w.inv_temperature, paged=w.page_size > 0,
-                      page_size=w.page_size or 64,
-                      max_pages=(w.ctx + (w.page_size or 64) - 1) // (w.page_size or 64))
     xh, seed = make_inputs(w, 0, 0)
+    ps = w.page_size or 64
+    max_ctx = int(xh["ctx_len"].max())  # the page table covers the longest context drawn
+    rnd = VerifyRound(batch=w.batch, L=w.L, V=w.V, k=w.k, B_max=w.B, hq=w.hq, hkv=w.hkv, d=w.d,
+                      max_ctx=max_ctx, draft_dtype=torch.bfloat16, target_dtype=torch.float32,
+                      inv_temperature=w.inv_temperature, paged=w.page_size > 0, page_size=ps,
+                      max_pages=(max_ctx + ps - 1) // ps)
     xd = to_device(xh, w, torch)
     xd["target"] = torch.randn((w.batch, w.n_max, w.V), dtype=torch.float32, device="cuda")
     rnd.bind(xd)

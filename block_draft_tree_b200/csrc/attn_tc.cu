@@ -876,13 +876,18 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           mma_ts(tmem + o_col, tmem + s_col + kk * 8, sdesc(v_addr + kk * 2048, kHalf, 1024), kIdPV,
                  (i > 0 || kk > 0) ? 1u : 0u);
       };
+      // Each K/V slot is released (a commit on its kv_empty) as soon as the
+      // last MMA that reads it is issued: K_i after the QKs of step i - 1,
+      // V_i after the PVs of step i, so the producer refills K slots a step
+      // earlier than it could if both waited for the end of step i.
       bool ok = pair_wait(&bars->q_full, 0, bars) && pair_wait(&bars->kv_full[0], 0, bars);
       if (ok) {
         fence_after();
         for (int t = 0; t < nt; ++t) qk(t, 0);
+        mma_commit(&bars->kv_empty[0]);  // K_0
       }
       for (int i = 0; ok && i < ntiles; ++i) {
-        const int ks = (2 * i) & 3, vs = (2 * i + 1) & 3;
+        const int vs = (2 * i + 1) & 3;
         const uint32_t ph = (uint32_t)(i >> 1) & 1u;
         const bool next = i + 1 < ntiles;
         const int ks1 = (2 * i + 2) & 3;
@@ -899,8 +904,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           if (next) qk(t, i + 1);
         }
         if (!ok) break;
-        mma_commit(&bars->kv_empty[ks]);  // K_i and V_i are free once every MMA so far is done
-        mma_commit(&bars->kv_empty[vs]);
+        mma_commit(&bars->kv_empty[vs]);  // V_i: every PV of step i issued
+        if (next) mma_commit(&bars->kv_empty[ks1]);  // K_{i+1}: every QK of step i + 1 issued
       }
       if (ok) mma_commit(&bars->o_full);
       if (*(volatile int*)&bars->abort) {
@@ -971,7 +976,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       const bool move = m_new > m_used + kRescaleLog2 || (m_used == -INFINITY && m_new != -INFINITY);
       const float m_tgt = move ? m_new : m_used;
       // p = 2^(s*c - m), two scores at a time: a packed FFMA for the
-      // exponents, then MUFU ex2 -- or, for 3 pairs in 8, exp2_poly2 on the
+      // exponents, then MUFU ex2 -- or, for 2 pairs in 8, exp2_poly2 on the
       // FMA pipe; packed sums; bf16 pairs stored over the scores, 32 scores
       // (16 columns) per store
       uint64_t rs2[4];
@@ -990,7 +995,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             const uint64_t x2 = ffma2(pack2(__uint_as_float(r[32 * c + e]), __uint_as_float(r[32 * c + e + 1])),
                                       c2, nm2);
             float a, bb;
-            if (((e >> 1) & 7) < 3) {
+            if (((e >> 1) & 7) < 2) {
               exp2_poly2(x2, a, bb);
             } else {
               float xa, xb;
