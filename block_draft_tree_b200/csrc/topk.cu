@@ -173,9 +173,10 @@ __device__ __forceinline__ uint64_t warp_sort_desc(uint64_t v) {
 }
 
 // The k-th largest nonzero key over the CTA's lanes (0 when fewer than k
-// lanes hold one), from each warp's k largest, sorted: a key's rank is its
-// place in its warp's list plus a binary search in every other warp's list.
-// Barriers: two.  wtop: kWarps * k keys of shared scratch.
+// lanes hold one; keys may repeat), from each warp's k largest, sorted: a
+// key is the k-th when fewer than k keys lie above it and at least k at or
+// above it, both counted by binary searches in every warp's list.  Barriers:
+// two.  wtop: kWarps * k keys of shared scratch.
 __device__ uint64_t block_kth_key(uint64_t v, int k, uint64_t* wtop, uint64_t* result) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const uint64_t sorted = warp_sort_desc(v);
@@ -184,21 +185,26 @@ __device__ uint64_t block_kth_key(uint64_t v, int k, uint64_t* wtop, uint64_t* r
   __syncthreads();
   if ((int)threadIdx.x < kWarps * k) {
     const uint64_t key = wtop[threadIdx.x];
-    const int own = threadIdx.x / k;
-    int r = threadIdx.x - own * k;
     if (key != 0) {
+      int gt = 0, ge = 0;
       for (int w = 0; w < kWarps; ++w) {
-        if (w == own) continue;
         const uint64_t* l = wtop + w * k;
-        int lo = 0, hi = k;
+        int lo = 0, hi = k;  // first position not above key
         while (lo < hi) {
           const int mid = (lo + hi) >> 1;
           if (l[mid] > key) lo = mid + 1;
           else hi = mid;
         }
-        r += lo;
+        gt += lo;
+        hi = k;  // first position below key
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          if (l[mid] >= key) lo = mid + 1;
+          else hi = mid;
+        }
+        ge += lo;
       }
-      if (r == k - 1) *result = key;
+      if (gt < k && ge >= k) *result = key;  // equal keys write the same value
     }
   }
   __syncthreads();
@@ -482,10 +488,13 @@ __global__ void __launch_bounds__(kThreads, 3) topk_kernel(TopkParams p) {
     int ti;
     bool take_all;
     if (first) {
+      // the lane's bound: the smallest key a logit of value mc can have (its
+      // maximum's key is at least that); 0 for a lane past the row's end
       uint64_t kmax = 0;
-#pragma unroll
-      for (int i = NE - 1; i >= 0; --i)
-        if (value_of(i) == mc && index_of(i) < p.V) kmax = cand_key(mc, (uint32_t)index_of(i));
+      if (index_of(0) < p.V) {
+        kmax = cand_key(mc, 0xFFFFFFFFu);
+        if (kmax == 0) kmax = 1;
+      }
       if (tid == 0) {
         sm.count = 0;
         sm.overflow = 0;
@@ -494,7 +503,7 @@ __global__ void __launch_bounds__(kThreads, 3) topk_kernel(TopkParams p) {
       // lower bound of the k-th best (barriers)
       tau = block_kth_key(kmax, p.k, sm.wtop, &sm.kth);
       tv = tau ? key_val(tau) : -INFINITY;
-      ti = tau ? (int)key_id(tau) : INT_MAX;
+      ti = INT_MAX;         // a logit equal to the bound may rank above it
       take_all = tau == 0;  // fewer than k lanes hold logits
     } else {
       tv = tau ? key_val(tau) : -INFINITY;
