@@ -264,9 +264,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row = tid - 64;
       const int qr = q0 + row;
       if (p.nsplit > 1 && !p.cluster) {
-        float4* po = (float4*)(p.part_o + (part_row0 + row) * D);
-        for (int i = 0; i < D / 4; ++i) po[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-        p.part_ml[part_row0 + row] = make_float2(-INFINITY, 0.f);
+        // an empty partial (m = -inf: the combine never reads its O) for the
+        // tree's rows; the combine writes rows past the tree by itself
+        if (qr < R && qr / g < n) p.part_ml[part_row0 + row] = make_float2(-INFINITY, 0.f);
       } else if (qr < R) {
         const int j = qr / g, h = kvh * g + qr % g;
         uint4* dst = (uint4*)(p.out + (((int64_t)b * p.n_max + j) * p.hq + h) * D);
@@ -1064,7 +1064,9 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     const bool has = ok && row_valid && l > 0.f && ntiles > 0;
     const float inv = has ? 1.f / l : 0.f;
     // (TMEM loads by every lane of the warp: they are warp-collective)
-    const bool writes = final_out ? qr < R : qt < p.qtiles;
+    // final rows: every query row (zeros past the tree); partials: the tree's
+    // rows only (the combine writes the others without reading partials)
+    const bool writes = final_out ? qr < R : (qt < p.qtiles && qr < R && j < n);
     if (tile_rows) {
       fence_after();
 #pragma unroll 1
@@ -1138,6 +1140,12 @@ __global__ void __launch_bounds__(256) attn_tc_combine(const Params p) {
   int n = p.n_nodes[b];
   n = min(max(n, 1), p.n_max);
   const int j = qr / g, h = kvh * g + qr % g;
+  if (j >= n) {  // a row past the tree: zeros, and no partial to read (none was written)
+    uint2* dst = (uint2*)(p.out + (((int64_t)b * p.n_max + j) * p.hq + h) * D);
+    dst[lane] = make_uint2(0u, 0u);
+    if (lane == 0 && p.lse_out) p.lse_out[((int64_t)b * p.n_max + j) * p.hq + h] = -INFINITY;
+    return;
+  }
   const int64_t base = (((int64_t)grp * p.qtiles + qtile) * p.nsplit) * BM + r;
   float M = -INFINITY;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);

@@ -265,3 +265,35 @@ def test_each_kernel_family(kernel, paged):
         _check(w, sample=400, seed=3)
     finally:
         api.set_attn_kernel(prev)
+
+
+@pytest.mark.parametrize("path", ["TC_COMBINE", "TC_PAIRS_COMBINE", "TC_CLUSTER", "TC_PAIRS"])
+def test_small_budgets_leave_dead_tiles(path):
+    """Per-sequence budgets far below B_max (an adaptive split of the nodes):
+    whole query tiles and pairs hold no tree row, and split partials exist
+    only for the tree's rows.  Rows of the tree match the oracle; rows past
+    n_nodes are zero with lse = -inf, on every path that splits or pairs."""
+    base = synth.WORKLOADS["b64"].scaled(L=6, V=400, k=4, hq=32, hkv=8, d=128)
+    want = getattr(api, "ATTN_PATH_" + path)
+    for kw in ATTN_PATH_SHAPES[path]:
+        w = base.scaled(**kw)
+        if _plan(w, w.ctx)[0] == want:
+            break
+    else:
+        pytest.fail("no candidate shape takes path " + path)
+    ids, zk, lse = oracle_tree_inputs(w, synth.draft_logits(w))
+    budgets = np.array([[w.B, 0, 3, max(1, w.B // 3)][b % 4] for b in range(w.batch)], np.int32)
+    tree = oracle.build_tree(ids, zk, lse.astype(np.float64), budgets, w.inv_temperature,
+                             root_token=synth.root_tokens(w), ctx_len=synth.context_lengths(w),
+                             k_per_seq=w.k_per_seq(), n_max=w.n_max)
+    a = synth.attention_inputs(w)
+    out, lse_g = _gpu_attn(a, tree, w)
+    seqs = sorted({0, 1, 2, 3, w.batch - 1} & set(range(w.batch)))
+    items = np.array([(b, j, h) for b in seqs for j in range(int(tree["n_nodes"][b]))
+                      for h in range(0, w.hq, 5)], np.int32)
+    ref, ref_lse = _oracle_attn(a, tree, w, items)
+    assert_attn_close(out[items[:, 0], items[:, 1], items[:, 2]], ref, "path %s, small budgets" % path)
+    np.testing.assert_allclose(lse_g[items[:, 0], items[:, 1], items[:, 2]], ref_lse, atol=2e-3)
+    for b in range(w.batch):
+        n = int(tree["n_nodes"][b])
+        assert np.all(out[b, n:] == 0) and np.all(np.isneginf(lse_g[b, n:]))
