@@ -578,12 +578,10 @@ __global__ void __launch_bounds__(kThreads) walk_kernel(WalkParams p) {
     if (p.S > 1) {
       if (tid == 0) {
         ((double2*)p.part)[row * p.S + chunk] = rs;
-        __threadfence();
-        s_flag = (atomicAdd(&p.row_ticket[row], 1u) == (unsigned)(p.S - 1));
+        s_flag = (atom_add_acq_rel_gpu(&p.row_ticket[row], 1u) == (unsigned)(p.S - 1));
       }
       __syncthreads();
       if (!s_flag) return;
-      __threadfence();
     } else {
       if (tid == 0) ((double2*)p.part)[row] = rs;
       __syncthreads();
@@ -619,12 +617,12 @@ __global__ void __launch_bounds__(kThreads) walk_kernel(WalkParams p) {
     } else {
       if (tid == 0) {
         p.part[row * p.S + chunk] = key;
-        __threadfence();
-        s_flag = (atomicAdd(&p.row_ticket[row], 1u) == (unsigned)(p.S - 1));
+        // acquire-release ticket: releases this thread's partial, and for the
+        // last CTA acquires the others' (its barrier then orders the block)
+        s_flag = (atom_add_acq_rel_gpu(&p.row_ticket[row], 1u) == (unsigned)(p.S - 1));
       }
       __syncthreads();
       if (!s_flag) return;
-      __threadfence();
       uint64_t m = 0;
       for (int c = tid; c < p.S; c += kThreads) {
         const uint64_t u = ld_cg_u64(&p.part[row * p.S + c]);
@@ -639,13 +637,10 @@ __global__ void __launch_bounds__(kThreads) walk_kernel(WalkParams p) {
     }
   }
   // the row is done; the last row of the sequence walks it
-  if (tid == 0) {
-    __threadfence();
-    s_flag = (atomicAdd(&p.seq_count[b], 1u) == (unsigned)(n - 1));
-  }
+  if (tid == 0)  // thread 0 wrote the row's token: the ticket releases it
+    s_flag = (atom_add_acq_rel_gpu(&p.seq_count[b], 1u) == (unsigned)(n - 1));
   __syncthreads();
   if (!s_flag) return;
-  __threadfence();
   for (int r = tid; r < n; r += kThreads) {
     s_amax[r] = __ldcg(&p.amax[(int64_t)b * p.n_max + r]);
     s_tok[r] = p.tok[(int64_t)b * p.n_max + r];
