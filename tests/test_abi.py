@@ -223,3 +223,24 @@ def test_attention_kernel_override_is_a_setting(lib):
         assert api.set_attn_kernel(api.ATTN_KERNEL_AUTO) == api.ATTN_KERNEL_ONE_TILE
     finally:
         api.set_attn_kernel(prev)
+
+
+def test_plan_budget_rejects_bad_arguments(lib):
+    d = ctypes.c_void_p(256)  # any non-null address: nothing is launched
+
+    def call(batch=4, L=16, k=8, n_max=65, inv_t=1.0, total=128, c0=1.0, c1=0.01, **ptrs):
+        p = dict(tok=d, parent=d, depth=d, n_nodes=d, ids=d, zk=d, lse=d, budget=d)
+        p.update(ptrs)
+        return lib.ddt_plan_budget(p["tok"], p["parent"], p["depth"], p["n_nodes"], p["ids"],
+                                   p["zk"], p["lse"], batch, L, k, n_max, inv_t, total, c0, c1,
+                                   p["budget"], None, None, None)
+
+    assert call(batch=-1) == 1 and call(L=0) == 1 and call(k=0) == 1 and call(n_max=0) == 1
+    assert call(L=65) == 2 and call(k=33) == 2 and call(n_max=1025) == 2
+    assert call(batch=129, n_max=65) == 2            # 129 * 64 nodes > 8192
+    assert call(inv_t=0.0) == 1 and call(inv_t=float("inf")) == 1 and call(inv_t=float("nan")) == 1
+    assert call(c0=-1.0) == 1 and call(c0=float("inf")) == 1
+    assert call(c1=float("nan")) == 1 and call(c1=float("inf")) == 1
+    assert call(c0=0.0, c1=0.5) == 1                  # a per-node cost needs a fixed cost
+    for name in ("tok", "parent", "depth", "n_nodes", "ids", "zk", "lse", "budget"):
+        assert call(**{name: None}) == 1, name
