@@ -14,7 +14,7 @@
 //   being captured uses the remembered address, so the first call on a
 //   device must come before any capture.  A device reset (or a new primary
 //   context) reloads the library's device code at another address: the next
-//   call outside capture picks that up, so capture again after a reset.
+//   call outside capture picks that up.
 // * The array is shared by every call on that device and keeps whatever the
 //   last call left in it.  Each call checks its arguments exactly as
 //   ddt_topk does (same status codes) and only then clears the part it

@@ -154,8 +154,9 @@ ddt_status ddt_topk(const void* logits, ddt_dtype dtype, int batch, int L, int V
  * A call made outside stream capture (with its device current) looks up the
  * array's device address and remembers it for that device; a call made
  * during capture uses the remembered address, so make the first call on a
- * device before any stream capture (and capture again after a device reset,
- * which moves the array).
+ * device before any stream capture.  A device reset (or a new primary
+ * context) moves the array; the next call made outside capture looks up the
+ * new address.
  * Every call on a device shares the array; each call clears the part it uses
  * (an asynchronous memset on `stream`), so consecutive calls on one stream
  * are independent, while calls that overlap on the GPU race on the array.
