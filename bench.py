@@ -38,6 +38,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "verify rounds/sec and tree-attn HBM GB/s (% of B200 peak) at B=64–512"
 WORKLOAD = "b64"
+PER_WORKLOAD_MAX_STEPS = 2000  # graph replays per workload of `per_workload` (long512: ~5 s)
 
 
 def parse():
@@ -816,14 +817,6 @@ def run_ours(args):
             "peak_kind": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind if peak_kind == "measured"
             else "fallback"}
     acc = [r.out["acc_len"].float().mean().item() for _, r in graphs]
-    ext = (measure_extensions(w, sets, graphs, hbm_peak)
-           if rank == 0 and not args.no_extensions else None)
-    per_wl = (measure_per_workload(args.per_workload.split(","), hbm_peak, tf_peak,
-                                   max(10, args.steps))
-              if rank == 0 and not args.no_per_workload else None)
-    sweep = (budget_sweep(w, [int(b) for b in args.line_budgets.split(",")], args.sweep_batch,
-                          args.line_sweep_draws, args.sweep_invt)
-             if rank == 0 and not args.no_budget_sweep else None)
 
     # end to end: pinned host inputs -> H2D -> round -> D2H of the result, every step
     e2e = None
@@ -871,6 +864,16 @@ def run_ours(args):
                 del g
             dist.destroy_process_group()
         return 0
+
+    # Rank 0 alone, after the last collective: the other ranks never wait on
+    # these in a collective, whatever the process group's timeout.
+    ext = measure_extensions(w, sets, graphs, hbm_peak) if not args.no_extensions else None
+    per_wl = (measure_per_workload(args.per_workload.split(","), hbm_peak, tf_peak,
+                                   max(10, min(args.steps, PER_WORKLOAD_MAX_STEPS)))
+              if not args.no_per_workload else None)
+    sweep = (budget_sweep(w, [int(b) for b in args.line_budgets.split(",")], args.sweep_batch,
+                          args.line_sweep_draws, args.sweep_invt)
+             if not args.no_budget_sweep else None)
 
     cpu = None
     if not args.no_cpu_baseline and world == 1:
