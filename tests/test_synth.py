@@ -95,8 +95,8 @@ def test_zipf_drafts_are_a_permuted_profile():
 
 def test_planted_target_agrees_with_one_child():
     """A planted row's maximum is one of its children's tokens, at least 2
-    above the rest of the row; with agreement 1 and no decay every row with children is
-    planted, with agreement 0 none is."""
+    above the rest of the row; with agreement 1 and no decay every row with
+    children is planted, with agreement 0 none is."""
     w = W["tiny"].scaled(batch=1, V=300, plant_p0=1.0, plant_decay=0.0)
     tok = np.array([[7, 11, 12, 13, 21, 22, 0, 0, 0]], np.int32)
     parent = np.array([[-1, 0, 0, 0, 1, 1, 0, 0, 0]], np.int32)
