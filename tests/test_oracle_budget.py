@@ -13,7 +13,9 @@ the best n.  These tests tie it to things other than itself:
 * the cost model: brute force over n of (batch + best acceptance(n)) /
   (c0 + c1 * n) picks the plan's n;
 * each sequence's expected tokens equal 1 + the surrogate of its tree rebuilt
-  with the planned budget (Proposition 1 through the tree builder).
+  with the planned budget (Proposition 1 through the tree builder);
+* a hand-worked batch of two sequences (tests/golden/budget_two_seqs.json):
+  caps and two cost models, worked out on paper.
 """
 import itertools
 
@@ -90,3 +92,25 @@ def test_confident_sequences_get_more_nodes():
     ids, zk, lse, tree = _case(5, 2, 4, 30, 4, 20)  # sequence 1's logits are 3x sequence 0's
     budget, _, _ = oracle.plan_budget(ids, zk, lse, tree, 4, 1.0, total_budget=20)
     assert budget[1] > budget[0]
+
+
+def test_golden_two_sequences():
+    """The hand-worked budgets of tests/golden/budget_two_seqs.json (its
+    derivation is in the file): caps and two cost models over a batch of two
+    sequences of different confidence."""
+    import json
+    import os
+    d = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "budget_two_seqs.json")))
+    z = np.log(np.asarray(d["q"], np.float64)).astype(np.float32)
+    invT = d["inv_temperature"]
+    ids, zk, logp, lse = oracle.topk(z, d["k"], invT)
+    tree = oracle.build_tree(ids, zk, lse, d["B"], invT, n_max=d["B"] + 1)
+    assert list(tree["n_nodes"]) == [d["B"] + 1] * 2
+    for c in d["cases"]:
+        budget, exp_tok, taken = oracle.plan_budget(ids, zk, lse, tree, d["L"], invT,
+                                                    total_budget=c["total_budget"],
+                                                    cost_fixed=c["cost_fixed"],
+                                                    cost_per_node=c["cost_per_node"])
+        assert taken == c["taken"], c
+        assert list(budget) == c["budget"], c
+        np.testing.assert_allclose(exp_tok, c["expected_tokens"], rtol=0, atol=1e-6)
