@@ -244,3 +244,15 @@ def test_plan_budget_rejects_bad_arguments(lib):
     assert call(c0=0.0, c1=0.5) == 1                  # a per-node cost needs a fixed cost
     for name in ("tok", "parent", "depth", "n_nodes", "ids", "zk", "lse", "budget"):
         assert call(**{name: None}) == 1, name
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """Without libddt.so every call raises: there is no other implementation
+    to fall back to."""
+    import torch
+    monkeypatch.setattr(api, "_lib", None)
+    monkeypatch.setattr(api, "_LIB_PATH", str(tmp_path / "libddt.so"))
+    with pytest.raises(api.DDTError, match="not built"):
+        api.load_library()
+    with pytest.raises(api.DDTError):
+        api.topk(torch.zeros(1, 2, 64), 4)
