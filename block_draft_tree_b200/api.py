@@ -178,6 +178,14 @@ def _need_cuda(*ts):
     return dev
 
 
+def _check_types(fn: str, *pairs):
+    """Raise unless every given tensor (None skipped) is contiguous with its
+    dtype: the kernels read plain int32 / float32 arrays."""
+    for t, dt in pairs:
+        if t is not None and (t.dtype != dt or not t.is_contiguous()):
+            raise DDTError("%s: expected contiguous %s tensors, got %s" % (fn, dt, t.dtype))
+
+
 def _dtype_code(t: torch.Tensor) -> int:
     if t.dtype == torch.bfloat16:
         return DDT_BF16
@@ -283,7 +291,12 @@ def plan_budget(tree: dict, ids: torch.Tensor, zk: torch.Tensor, lse: torch.Tens
     it was built from.  Returns (budget int32 [batch], expected_tokens f64
     [batch]); pass ``budget`` to :func:`build_tree` as its per-sequence budget."""
     lib = load_library()
-    dev = _need_cuda(ids, zk, lse, tree["tok"], dev_status)
+    _check_types("plan_budget", *[(tree[n], torch.int32) for n in ("tok", "parent", "depth",
+                                                                   "n_nodes")],
+                 (ids, torch.int32), (zk, torch.float32), (lse, torch.float32),
+                 (dev_status, torch.int32))
+    dev = _need_cuda(ids, zk, lse, tree["tok"], tree["parent"], tree["depth"], tree["n_nodes"],
+                     dev_status)
     b, L, k = ids.shape
     n_max = tree["tok"].shape[1]
     budget = torch.empty(b, dtype=torch.int32, device=dev)
@@ -428,6 +441,8 @@ def tree_walk(logits: torch.Tensor, tok: torch.Tensor, parent: torch.Tensor,
     stride); ``mode`` one of WALK_ALL_ROWS, WALK_LAZY, WALK_AUTO.  Returns dict
     acc_len [batch], acc_nodes/acc_tok [batch, L], bonus [batch]."""
     lib = load_library()
+    _check_types("tree_walk", (tok, torch.int32), (parent, torch.int32), (depth, torch.int32),
+                 (n_nodes, torch.int32), (dev_status, torch.int32))
     dev = _need_cuda(logits, tok, parent, depth, n_nodes, dev_status)
     if logits.dim() != 3 or logits.stride(2) != 1 or logits.stride(0) != logits.stride(1) * logits.shape[1]:
         raise DDTError("logits must be [batch, n_max, V] with contiguous rows and a uniform row stride")
@@ -458,6 +473,8 @@ def tree_walk_sample(logits: torch.Tensor, tok: torch.Tensor, parent: torch.Tens
     and advanced by one per call, for replays of a captured graph.
     Arguments and outputs otherwise as :func:`tree_walk`."""
     lib = load_library()
+    _check_types("tree_walk_sample", (tok, torch.int32), (parent, torch.int32),
+                 (depth, torch.int32), (n_nodes, torch.int32), (dev_status, torch.int32))
     dev = _need_cuda(logits, tok, parent, depth, n_nodes, dev_status, step_counter)
     if step_counter is not None and (step_counter.dtype != torch.int64 or step_counter.numel() != 1):
         raise DDTError("step_counter must be a one-element int64 tensor")

@@ -256,3 +256,29 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
         api.load_library()
     with pytest.raises(api.DDTError):
         api.topk(torch.zeros(1, 2, 64), 4)
+
+
+def test_binding_checks_tree_tensor_types(lib):
+    """The walk and budget bindings refuse tree tensors the kernels would
+    misread (int64, float, non-contiguous) before anything else."""
+    import torch
+    logits = torch.zeros(1, 3, 16)
+    ok = [torch.zeros(1, 3, dtype=torch.int32) for _ in range(3)] + [torch.ones(1, dtype=torch.int32)]
+    bad64 = [t.long() for t in ok]
+    strided = torch.zeros(1, 6, dtype=torch.int32)[:, ::2]
+    for fn, extra in ((api.tree_walk, ()), (api.tree_walk_sample, (1.0, 1, 0))):
+        with pytest.raises(api.DDTError, match="contiguous"):
+            fn(logits, *bad64, 2, *extra)
+        with pytest.raises(api.DDTError, match="contiguous"):
+            fn(logits, strided, *ok[1:], 2, *extra)
+        with pytest.raises(api.DDTError, match="CUDA tensors only"):
+            fn(logits, *ok, 2, *extra)
+    tree = dict(zip(("tok", "parent", "depth", "n_nodes"), ok))
+    ids = torch.zeros(1, 2, 2, dtype=torch.int32)
+    zk, lse = torch.zeros(1, 2, 2), torch.zeros(1, 2)
+    with pytest.raises(api.DDTError, match="contiguous"):
+        api.plan_budget(tree, ids, zk.double(), lse)
+    with pytest.raises(api.DDTError, match="contiguous"):
+        api.plan_budget(dict(tree, parent=bad64[1]), ids, zk, lse)
+    with pytest.raises(api.DDTError, match="CUDA tensors only"):
+        api.plan_budget(tree, ids, zk, lse)
