@@ -186,6 +186,17 @@ def _check_types(fn: str, *pairs):
             raise DDTError("%s: expected contiguous %s tensors, got %s" % (fn, dt, t.dtype))
 
 
+def _check_tree_shapes(fn: str, b: int, n_max: int, tok, parent, depth, n_nodes):
+    """Raise unless tok/parent/depth are [b, n_max] and n_nodes is [b]: the
+    kernels index them with those extents."""
+    for t in (tok, parent, depth):
+        if tuple(t.shape) != (b, n_max):
+            raise DDTError("%s: tree tensors must be [%d, %d], got %s"
+                           % (fn, b, n_max, tuple(t.shape)))
+    if tuple(n_nodes.shape) != (b,):
+        raise DDTError("%s: n_nodes must be [%d], got %s" % (fn, b, tuple(n_nodes.shape)))
+
+
 def _dtype_code(t: torch.Tensor) -> int:
     if t.dtype == torch.bfloat16:
         return DDT_BF16
@@ -295,10 +306,14 @@ def plan_budget(tree: dict, ids: torch.Tensor, zk: torch.Tensor, lse: torch.Tens
                                                                    "n_nodes")],
                  (ids, torch.int32), (zk, torch.float32), (lse, torch.float32),
                  (dev_status, torch.int32))
-    dev = _need_cuda(ids, zk, lse, tree["tok"], tree["parent"], tree["depth"], tree["n_nodes"],
-                     dev_status)
+    if ids.dim() != 3 or zk.shape != ids.shape or lse.shape != ids.shape[:2] or tree["tok"].dim() != 2:
+        raise DDTError("plan_budget: ids/zk must be [batch, L, k], lse [batch, L], tree [batch, n_max]")
     b, L, k = ids.shape
     n_max = tree["tok"].shape[1]
+    _check_tree_shapes("plan_budget", b, n_max, tree["tok"], tree["parent"], tree["depth"],
+                       tree["n_nodes"])
+    dev = _need_cuda(ids, zk, lse, tree["tok"], tree["parent"], tree["depth"], tree["n_nodes"],
+                     dev_status)
     budget = torch.empty(b, dtype=torch.int32, device=dev)
     exp_tok = torch.empty(b, dtype=torch.float64, device=dev)
     with torch.cuda.device(dev):
@@ -443,10 +458,11 @@ def tree_walk(logits: torch.Tensor, tok: torch.Tensor, parent: torch.Tensor,
     lib = load_library()
     _check_types("tree_walk", (tok, torch.int32), (parent, torch.int32), (depth, torch.int32),
                  (n_nodes, torch.int32), (dev_status, torch.int32))
-    dev = _need_cuda(logits, tok, parent, depth, n_nodes, dev_status)
     if logits.dim() != 3 or logits.stride(2) != 1 or logits.stride(0) != logits.stride(1) * logits.shape[1]:
         raise DDTError("logits must be [batch, n_max, V] with contiguous rows and a uniform row stride")
     b, n_max, V = logits.shape
+    _check_tree_shapes("tree_walk", b, n_max, tok, parent, depth, n_nodes)
+    dev = _need_cuda(logits, tok, parent, depth, n_nodes, dev_status)
     res = {"acc_len": torch.empty(b, dtype=torch.int32, device=dev),
            "acc_nodes": torch.empty((b, L), dtype=torch.int32, device=dev),
            "acc_tok": torch.empty((b, L), dtype=torch.int32, device=dev),
@@ -475,12 +491,13 @@ def tree_walk_sample(logits: torch.Tensor, tok: torch.Tensor, parent: torch.Tens
     lib = load_library()
     _check_types("tree_walk_sample", (tok, torch.int32), (parent, torch.int32),
                  (depth, torch.int32), (n_nodes, torch.int32), (dev_status, torch.int32))
-    dev = _need_cuda(logits, tok, parent, depth, n_nodes, dev_status, step_counter)
     if step_counter is not None and (step_counter.dtype != torch.int64 or step_counter.numel() != 1):
         raise DDTError("step_counter must be a one-element int64 tensor")
     if logits.dim() != 3 or logits.stride(2) != 1 or logits.stride(0) != logits.stride(1) * logits.shape[1]:
         raise DDTError("logits must be [batch, n_max, V] with contiguous rows and a uniform row stride")
     b, n_max, V = logits.shape
+    _check_tree_shapes("tree_walk_sample", b, n_max, tok, parent, depth, n_nodes)
+    dev = _need_cuda(logits, tok, parent, depth, n_nodes, dev_status, step_counter)
     res = {"acc_len": torch.empty(b, dtype=torch.int32, device=dev),
            "acc_nodes": torch.empty((b, L), dtype=torch.int32, device=dev),
            "acc_tok": torch.empty((b, L), dtype=torch.int32, device=dev),

@@ -282,3 +282,22 @@ def test_binding_checks_tree_tensor_types(lib):
         api.plan_budget(dict(tree, parent=bad64[1]), ids, zk, lse)
     with pytest.raises(api.DDTError, match="CUDA tensors only"):
         api.plan_budget(tree, ids, zk, lse)
+
+
+def test_binding_checks_tree_tensor_shapes(lib):
+    """Tree tensors whose extents differ from the logits' [batch, n_max] (or
+    the candidates' batch) are refused before anything is launched."""
+    import torch
+    i32 = lambda *s: torch.zeros(*s, dtype=torch.int32)
+    logits = torch.zeros(2, 3, 16)
+    for fn, extra in ((api.tree_walk, ()), (api.tree_walk_sample, (1.0, 1, 0))):
+        with pytest.raises(api.DDTError, match=r"\[2, 3\]"):
+            fn(logits, i32(2, 2), i32(2, 3), i32(2, 3), i32(2), 2, *extra)
+        with pytest.raises(api.DDTError, match=r"n_nodes must be \[2\]"):
+            fn(logits, i32(2, 3), i32(2, 3), i32(2, 3), i32(1), 2, *extra)
+    tree = {"tok": i32(2, 3), "parent": i32(2, 3), "depth": i32(1, 3), "n_nodes": i32(2)}
+    ids, zk, lse = i32(2, 4, 2), torch.zeros(2, 4, 2), torch.zeros(2, 4)
+    with pytest.raises(api.DDTError, match=r"\[2, 3\]"):
+        api.plan_budget(tree, ids, zk, lse)
+    with pytest.raises(api.DDTError, match="lse"):
+        api.plan_budget(dict(tree, depth=i32(2, 3)), ids, zk, torch.zeros(2, 3))
