@@ -197,6 +197,35 @@ def _check_tree_shapes(fn: str, b: int, n_max: int, tok, parent, depth, n_nodes)
         raise DDTError("%s: n_nodes must be [%d], got %s" % (fn, b, tuple(n_nodes.shape)))
 
 
+def _check_kv_shapes(fn: str, b: int, n_max: int, d: int, k_tree, v_tree, k_cache, v_cache,
+                     page_table, page_size=None):
+    """Raise unless the tree K/V are [b, n_max, hkv, d] and a non-empty cache
+    is dense [b, t_max, hkv, d] or, with ``page_table`` [b, max_pages], a page
+    pool [pages, page_size, hkv, d]: the kernels index them with those
+    extents.  Returns hkv."""
+    if k_tree.dim() != 4 or tuple(k_tree.shape[:2]) != (b, n_max) or k_tree.shape[3] != d:
+        raise DDTError("%s: tree K must be [%d, %d, hkv, %d], got %s"
+                       % (fn, b, n_max, d, tuple(k_tree.shape)))
+    if v_tree.shape != k_tree.shape:
+        raise DDTError("%s: tree V must have tree K's shape" % fn)
+    hkv = k_tree.shape[2]
+    if k_cache is not None and k_cache.numel():
+        if v_cache is None or v_cache.shape != k_cache.shape:
+            raise DDTError("%s: the V cache must have the K cache's shape" % fn)
+        if k_cache.dim() != 4 or tuple(k_cache.shape[2:]) != (hkv, d):
+            raise DDTError("%s: caches must be [.., .., %d, %d], got %s"
+                           % (fn, hkv, d, tuple(k_cache.shape)))
+        if page_table is None and k_cache.shape[0] != b:
+            raise DDTError("%s: a dense cache must have %d sequences" % (fn, b))
+        if page_table is not None:
+            if page_table.dim() != 2 or page_table.shape[0] != b:
+                raise DDTError("%s: page_table must be [%d, max_pages]" % (fn, b))
+            if page_size is not None and k_cache.shape[1] != page_size:
+                raise DDTError("%s: the page pool's pages hold %d tokens, page_size is %d"
+                               % (fn, k_cache.shape[1], page_size))
+    return hkv
+
+
 def _dtype_code(t: torch.Tensor) -> int:
     if t.dtype == torch.bfloat16:
         return DDT_BF16
@@ -268,6 +297,12 @@ def build_tree(ids: torch.Tensor, zk: torch.Tensor, lse: torch.Tensor, B_max: in
     int32 (bit pattern of the uint32 words), n_nodes [batch] int32,
     surrogate [batch] float64."""
     lib = load_library()
+    if ids.dim() != 3 or zk.shape != ids.shape or lse.shape != ids.shape[:2]:
+        raise DDTError("build_tree: ids/zk must be [batch, L, k] and lse [batch, L]")
+    for t in (root_token, k_per_seq, budget, ctx_len):
+        if t is not None and tuple(t.shape) != (ids.shape[0],):
+            raise DDTError("build_tree: root_token / k_per_seq / budget / ctx_len must be [%d]"
+                           % ids.shape[0])
     dev = _need_cuda(ids, zk, lse, root_token, k_per_seq, budget, ctx_len, dev_status)
     for t, dt in ((ids, torch.int32), (zk, torch.float32), (lse, torch.float32),
                   (root_token, torch.int32), (k_per_seq, torch.int32), (budget, torch.int32),
@@ -415,6 +450,15 @@ def tree_attn(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
     tree K/V [batch, n_max, hkv, d]; mask [batch, n_max, W].  Returns out bf16
     [batch, n_max, hq, d] (and lse f32 [batch, n_max, hq] when asked)."""
     lib = load_library()
+    if q.dim() != 4:
+        raise DDTError("tree_attn: q must be [batch, n_max, hq, d]")
+    bq, nq, _, dq = q.shape
+    _check_kv_shapes("tree_attn", bq, nq, dq, k_tree, v_tree, k_cache, v_cache, page_table)
+    if tuple(mask.shape) != (bq, nq, mask_words(nq)):
+        raise DDTError("tree_attn: mask must be [%d, %d, %d], got %s"
+                       % (bq, nq, mask_words(nq), tuple(mask.shape)))
+    if tuple(n_nodes.shape) != (bq,) or tuple(ctx_len.shape) != (bq,):
+        raise DDTError("tree_attn: n_nodes and ctx_len must be [%d]" % bq)
     dev = _need_cuda(q, k_cache, v_cache, k_tree, v_tree, mask, n_nodes, ctx_len, page_table,
                      dev_status)
     for t in (q, k_cache, v_cache, k_tree, v_tree):
@@ -526,6 +570,15 @@ def kv_commit(k_tree: torch.Tensor, v_tree: torch.Tensor, acc_len: torch.Tensor,
     hkv, d] or a page pool [pages, page_size, hkv, d] with ``page_table``) and
     advance ``ctx_len`` (int32, in place) by acc_len + 1."""
     lib = load_library()
+    if k_tree.dim() != 4:
+        raise DDTError("kv_commit: tree K must be [batch, n_max, hkv, d]")
+    bk, nk, _, dk = k_tree.shape
+    _check_kv_shapes("kv_commit", bk, nk, dk, k_tree, v_tree, k_cache, v_cache, page_table,
+                     page_size)
+    if tuple(acc_len.shape) != (bk,) or tuple(ctx_len.shape) != (bk,):
+        raise DDTError("kv_commit: acc_len and ctx_len must be [%d]" % bk)
+    if acc_nodes.dim() != 2 or acc_nodes.shape[0] != bk:
+        raise DDTError("kv_commit: acc_nodes must be [%d, L]" % bk)
     dev = _need_cuda(k_tree, v_tree, acc_len, acc_nodes, ctx_len, k_cache, v_cache, page_table,
                      dev_status)
     for t in (k_tree, v_tree, k_cache, v_cache):
@@ -566,6 +619,10 @@ def lm_head_walk(hidden: torch.Tensor, weight: torch.Tensor, tok: torch.Tensor,
     walk outputs of :func:`tree_walk` (plus ``row_token`` [batch, n_max] when
     asked)."""
     lib = load_library()
+    if hidden.dim() != 3 or weight.dim() != 2:
+        raise DDTError("lm_head_walk: hidden must be [batch, n_max, K] and weight [V, K]")
+    _check_tree_shapes("lm_head_walk", hidden.shape[0], hidden.shape[1], tok, parent, depth,
+                       n_nodes)
     dev = _need_cuda(hidden, weight, tok, parent, depth, n_nodes, dev_status)
     for t in (hidden, weight):
         if t.dtype != torch.bfloat16 or not t.is_contiguous():

@@ -301,3 +301,72 @@ def test_binding_checks_tree_tensor_shapes(lib):
         api.plan_budget(tree, ids, zk, lse)
     with pytest.raises(api.DDTError, match="lse"):
         api.plan_budget(dict(tree, depth=i32(2, 3)), ids, zk, torch.zeros(2, 3))
+
+
+def test_binding_checks_attention_and_commit_extents(lib):
+    """tree_attn and kv_commit refuse K/V, caches, masks and per-sequence
+    arrays whose extents disagree with q / the tree K/V, before any launch."""
+    import torch
+    bf = lambda *s: torch.zeros(*s, dtype=torch.bfloat16)
+    i32 = lambda *s: torch.zeros(*s, dtype=torch.int32)
+    b, n, hq, hkv, d, T = 2, 5, 4, 2, 64, 16
+    good = dict(q=bf(b, n, hq, d), k_cache=bf(b, T, hkv, d), v_cache=bf(b, T, hkv, d),
+                k_tree=bf(b, n, hkv, d), v_tree=bf(b, n, hkv, d), mask=i32(b, n, 1),
+                n_nodes=i32(b), ctx_len=i32(b), max_ctx=T)
+
+    def attn(**kw):
+        return api.tree_attn(**dict(good, **kw))
+
+    with pytest.raises(api.DDTError, match="CUDA tensors only"):
+        attn()
+    for kw, msg in ((dict(k_tree=bf(b, n + 1, hkv, d)), "tree K"),
+                    (dict(v_tree=bf(b, n, hkv, d + 64)), "tree V"),
+                    (dict(k_cache=bf(b + 1, T, hkv, d), v_cache=bf(b + 1, T, hkv, d)), "dense"),
+                    (dict(v_cache=bf(b, T - 1, hkv, d)), "V cache"),
+                    (dict(k_cache=bf(b, T, 1, d), v_cache=bf(b, T, 1, d)), "caches"),
+                    (dict(mask=i32(b, n, 2)), "mask"),
+                    (dict(n_nodes=i32(b + 1)), "n_nodes"),
+                    (dict(k_cache=bf(9, 16, hkv, d), v_cache=bf(9, 16, hkv, d),
+                          page_table=i32(b + 1, 3)), "page_table")):
+        with pytest.raises(api.DDTError, match=msg):
+            attn(**kw)
+
+    kt, acc_len, acc_nodes, cl = bf(b, n, hkv, d), i32(b), i32(b, 3), i32(b)
+    with pytest.raises(api.DDTError, match="CUDA tensors only"):
+        api.kv_commit(kt, kt.clone(), acc_len, acc_nodes, cl, bf(b, T, hkv, d), bf(b, T, hkv, d))
+    with pytest.raises(api.DDTError, match="dense"):
+        api.kv_commit(kt, kt.clone(), acc_len, acc_nodes, cl, bf(1, T, hkv, d), bf(1, T, hkv, d))
+    with pytest.raises(api.DDTError, match="page_size"):
+        api.kv_commit(kt, kt.clone(), acc_len, acc_nodes, cl, bf(8, 32, hkv, d), bf(8, 32, hkv, d),
+                      page_table=i32(b, 4), page_size=64)
+    with pytest.raises(api.DDTError, match="acc_nodes"):
+        api.kv_commit(kt, kt.clone(), acc_len, i32(b), cl, bf(b, T, hkv, d), bf(b, T, hkv, d))
+    with pytest.raises(api.DDTError, match="acc_len"):
+        api.kv_commit(kt, kt.clone(), i32(b + 1), acc_nodes, cl, bf(b, T, hkv, d), bf(b, T, hkv, d))
+
+
+def test_binding_checks_tree_builder_extents(lib):
+    import torch
+    i32 = lambda *s: torch.zeros(*s, dtype=torch.int32)
+    ids, zk, lse = i32(2, 3, 4), torch.zeros(2, 3, 4), torch.zeros(2, 3)
+    with pytest.raises(api.DDTError, match="CUDA tensors only"):
+        api.build_tree(ids, zk, lse, 8, i32(2))
+    with pytest.raises(api.DDTError, match="lse"):
+        api.build_tree(ids, zk, torch.zeros(2, 4), 8, i32(2))
+    with pytest.raises(api.DDTError, match="root_token"):
+        api.build_tree(ids, zk, lse, 8, i32(3))
+    with pytest.raises(api.DDTError, match="budget"):
+        api.build_tree(ids, zk, lse, 8, i32(2), budget=i32(1))
+
+
+def test_binding_checks_lm_head_extents(lib):
+    import torch
+    i32 = lambda *s: torch.zeros(*s, dtype=torch.int32)
+    h, wt = torch.zeros(2, 5, 64, dtype=torch.bfloat16), torch.zeros(100, 64, dtype=torch.bfloat16)
+    tree = (i32(2, 5), i32(2, 5), i32(2, 5), i32(2))
+    with pytest.raises(api.DDTError, match="CUDA tensors only"):
+        api.lm_head_walk(h, wt, *tree, 4)
+    with pytest.raises(api.DDTError, match=r"\[2, 5\]"):
+        api.lm_head_walk(h, wt, i32(2, 4), *tree[1:], 4)
+    with pytest.raises(api.DDTError, match="weight"):
+        api.lm_head_walk(h, wt.reshape(-1), *tree, 4)
