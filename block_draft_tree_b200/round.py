@@ -89,6 +89,7 @@ class VerifyRound:
         """Bind device input tensors: draft [b,L,V], root [b], ctx_len [b],
         q [b,n,hq,d], k_cache/v_cache, optional page_table, k_tree/v_tree
         [b,n,hkv,d], target [b,n,V]; optional k_per_seq / budget [b]."""
+        self._check_inputs(inputs)
         self.inputs = inputs
         o = self.out
         a = api._attn_args(inputs["q"], inputs["k_cache"], inputs["v_cache"], inputs["k_tree"],
@@ -133,6 +134,52 @@ class VerifyRound:
             ca.batch, ca.n_max, ca.hkv, ca.d, ca.L = self.batch, self.n_max, self.hkv, self.d, self.L
             ca.dev_status = o["status"].data_ptr()
             self.commit_args = ca
+
+    def _check_inputs(self, x: dict):
+        """Refuse inputs whose shapes, dtypes or layouts differ from this
+        round's sizes: the calls index the bound memory with those sizes."""
+        b, L, V, n = self.batch, self.L, self.V, self.n_max
+
+        def need(name, shape, dtype):
+            t = x.get(name)
+            if t is None:
+                raise api.DDTError("bind: input %r is missing" % name)
+            if tuple(t.shape) != tuple(shape) or t.dtype != dtype:
+                raise api.DDTError("bind: %r must be %s %s, got %s %s"
+                                   % (name, tuple(shape), dtype, tuple(t.shape), t.dtype))
+            return t
+
+        def rows(name, t, r):  # [b, r, V] with contiguous rows and a uniform row stride
+            if t.stride(2) != 1 or t.stride(0) != t.stride(1) * r:
+                raise api.DDTError("bind: %r needs contiguous rows and a uniform row stride" % name)
+
+        rows("draft", need("draft", (b, L, V), torch.bfloat16 if self.draft_code == api.DDT_BF16
+                           else torch.float32), L)
+        need("root", (b,), torch.int32)
+        need("ctx_len", (b,), torch.int32)
+        for name in ("k_per_seq", "budget"):
+            if x.get(name) is not None:
+                need(name, (b,), torch.int32)
+        for name, shape in (("q", (b, n, self.hq, self.d)), ("k_tree", (b, n, self.hkv, self.d)),
+                            ("v_tree", (b, n, self.hkv, self.d))):
+            if not need(name, shape, torch.bfloat16).is_contiguous():
+                raise api.DDTError("bind: %r must be contiguous" % name)
+        api._check_types("bind", (x.get("k_cache"), torch.bfloat16),
+                         (x.get("v_cache"), torch.bfloat16), (x.get("page_table"), torch.int32))
+        pt = x.get("page_table")
+        api._check_kv_shapes("bind", b, n, self.d, x["k_tree"], x["v_tree"], x.get("k_cache"),
+                             x.get("v_cache"), pt,
+                             self.page_size if self.commit and pt is not None else None)
+        if self.decode == "lm_head":
+            hid, head = x.get("hidden"), x.get("head")
+            if hid is None or head is None:
+                raise api.DDTError("bind: decode='lm_head' needs 'hidden' and 'head'")
+            need("hidden", (b, n, hid.shape[-1]), torch.bfloat16)
+            need("head", (V, hid.shape[-1]), torch.bfloat16)
+            api._check_types("bind", (hid, torch.bfloat16), (head, torch.bfloat16))
+        else:
+            rows("target", need("target", (b, n, V), torch.bfloat16
+                                if self.target_code == api.DDT_BF16 else torch.float32), n)
 
     def launch(self, stream: Optional[torch.cuda.Stream] = None, marks=None):
         """Enqueue the four stages (and the commit) on ``stream``.  ``marks(i)``

@@ -370,3 +370,40 @@ def test_binding_checks_lm_head_extents(lib):
         api.lm_head_walk(h, wt, i32(2, 4), *tree[1:], 4)
     with pytest.raises(api.DDTError, match="weight"):
         api.lm_head_walk(h, wt.reshape(-1), *tree, 4)
+
+
+def test_round_driver_checks_bound_inputs():
+    """VerifyRound.bind refuses inputs that disagree with the round's sizes
+    (shape, dtype, row layout), before any pointer reaches the library."""
+    import torch
+    from block_draft_tree_b200.round import VerifyRound
+    b, L, V, k, B, hq, hkv, d, T = 2, 4, 64, 4, 8, 4, 1, 64, 32
+    n = B + 1
+    rnd = VerifyRound(batch=b, L=L, V=V, k=k, B_max=B, hq=hq, hkv=hkv, d=d, max_ctx=T,
+                      draft_dtype=torch.float32, device="cpu")
+    bf = lambda *s: torch.zeros(*s, dtype=torch.bfloat16)
+    i32 = lambda *s: torch.zeros(*s, dtype=torch.int32)
+    good = {"draft": torch.zeros(b, L, V), "root": i32(b), "ctx_len": i32(b),
+            "q": bf(b, n, hq, d), "k_tree": bf(b, n, hkv, d), "v_tree": bf(b, n, hkv, d),
+            "k_cache": bf(b, T, hkv, d), "v_cache": bf(b, T, hkv, d),
+            "target": torch.zeros(b, n, V)}
+    rnd._check_inputs(good)   # consistent inputs pass
+    bad = [(dict(draft=torch.zeros(b, L, V, dtype=torch.bfloat16)), "draft"),
+           (dict(draft=torch.zeros(b, L + 1, V)), "draft"),
+           (dict(draft=torch.zeros(b, L, 2 * V)[:, :, ::2]), "row stride"),
+           (dict(root=i32(b + 1)), "root"),
+           (dict(ctx_len=torch.zeros(b, dtype=torch.int64)), "ctx_len"),
+           (dict(q=bf(b, n, hq, 128)), "'q'"),
+           (dict(k_tree=bf(b, n - 1, hkv, d)), "k_tree"),
+           (dict(k_cache=bf(b + 1, T, hkv, d), v_cache=bf(b + 1, T, hkv, d)), "dense"),
+           (dict(target=torch.zeros(b, n - 1, V)), "target"),
+           (dict(budget=i32(b + 1)), "budget")]
+    for kw, msg in bad:
+        with pytest.raises(api.DDTError, match=msg):
+            rnd.bind(dict(good, **kw))
+    lm = VerifyRound(batch=b, L=L, V=V, k=k, B_max=B, hq=hq, hkv=hkv, d=d, max_ctx=T,
+                     draft_dtype=torch.float32, decode="lm_head", device="cpu")
+    with pytest.raises(api.DDTError, match="hidden"):
+        lm.bind(good)
+    with pytest.raises(api.DDTError, match="head"):
+        lm.bind(dict(good, hidden=bf(b, n, 128), head=bf(V, 64)))
