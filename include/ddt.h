@@ -418,8 +418,9 @@ ddt_status ddt_lm_head_walk(const ddt_lm_head_walk_args* a, void* workspace,
  * negative page id or one >= num_pages when num_pages > 0), an acc_len
  * outside [0, L] or an accepted row outside [0, n_max) is not written and
  * raises DDT_ERR_INVALID_ARG in dev_status; ctx_len still advances by
- * acc_len + 1.  Limits: hkv * d a multiple of 8; all base pointers 16-byte
- * aligned.  No workspace.
+ * acc_len + 1.  Limits: hkv * d a multiple of 8 and at most 2^20, and
+ * L <= DDT_TREE_L_MAX (DDT_ERR_UNSUPPORTED otherwise); all base pointers
+ * 16-byte aligned (DDT_ERR_INVALID_ARG otherwise).  No workspace.
  * ------------------------------------------------------------------------ */
 typedef struct ddt_kv_commit_args {
   const void* k_tree;
