@@ -343,7 +343,7 @@ ddt_status ddt_tree_attn_plan(const ddt_attn_args* a, int* path, int* kv_splits)
  * Outputs: acc_len int32 [batch] (0..L), acc_nodes / acc_tok int32
  * [batch][L] (accepted rows and their tokens in walk order; unused -1),
  * bonus int32 [batch].  Tokens emitted this round = acc_len + 1.
- * Limits: row_stride >= V, an unknown mode or a null pointer give
+ * Limits: row_stride < V, an unknown mode or a null pointer give
  * DDT_ERR_INVALID_ARG; L <= DDT_TREE_L_MAX, n_max <= DDT_TREE_B_MAX + 1,
  * batch <= 65535 and batch * (n_max + 1) + 1 <= DDT_WS_COUNTER_BYTES / 4
  * (the tickets) give DDT_ERR_UNSUPPORTED otherwise.
