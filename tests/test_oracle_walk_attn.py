@@ -10,7 +10,9 @@ lossless), 運作流程 steps 3-4.  Pins:
 * rows that are not ancestors do not influence a row;
 * losslessness: with a deterministic toy target, the walk emits exactly the
   tokens that token-by-token greedy decoding emits, computed without a tree;
-* the hand-worked walk in tests/golden/tree_b5.json.
+* the hand-worked walk in tests/golden/tree_b5.json;
+* a hand-worked tree attention (tests/golden/attn_hand_tree.json): every
+  row and head of a four-row tree, as sums of powers of e.
 """
 import json
 import os
@@ -234,3 +236,32 @@ def test_golden_walk():
     assert list(res["acc_nodes"][0, :w["acc_len"]]) == w["acc_nodes"]
     assert list(res["acc_tok"][0, :w["acc_len"]]) == w["acc_tok"]
     assert res["bonus"][0] == w["bonus"]
+
+
+def test_attention_golden_hand_tree():
+    """tests/golden/attn_hand_tree.json: every row and head of a four-row
+    tree over a two-token context, worked out by hand (sums of powers of e;
+    the derivation is in the file), including siblings that must not see
+    each other and a grouped-query pair of heads."""
+    d = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "attn_hand_tree.json")))
+    D, n, T = d["d"], len(d["parent"]), d["ctx_len"]
+
+    def bits(rows, shape):
+        a = np.zeros(shape, np.float32)
+        a.reshape(-1, D)[:len(rows), :2] = np.asarray(rows, np.float32)
+        return (a.view(np.uint32) >> 16).astype(np.uint16)
+
+    q = np.zeros((1, n, 2, D), np.float32)
+    for h, qh in enumerate(d["q_heads"]):
+        q[0, :, h, :2] = qh
+    q = (q.view(np.uint32) >> 16).astype(np.uint16)
+    kc, vc = bits(d["k_ctx"], (1, T, 1, D)), bits(d["v_ctx"], (1, T, 1, D))
+    kt, vt = bits(d["k_tree"], (1, n, 1, D)), bits(d["v_tree"], (1, n, 1, D))
+    mask = np.asarray(d["mask"], np.uint32).reshape(1, n, 1)
+    items = np.array([(0, e["row"], e["head"]) for e in d["expected"]], np.int32)
+    out, lse = oracle.tree_attn(items, q, kc, vc, np.array([T], np.int32), kt, vt, mask,
+                                np.array([n], np.int32), d["scale"])
+    for i, e in enumerate(d["expected"]):
+        np.testing.assert_allclose(out[i, :2], e["out"], rtol=1e-13, atol=0, err_msg=str(e))
+        assert np.all(out[i, 2:] == 0.0)
+        assert lse[i] == pytest.approx(e["lse"], rel=1e-13)
